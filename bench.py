@@ -1,0 +1,410 @@
+"""WKV-7 benchmark on B200: tokens/s for forward and forward+backward at H=32, N=64.
+
+Default workload (one "step" = one forward with checkpoints + one backward over
+one batch): the packed-document training batch B=8, T=4096, H=32, N=64, bf16,
+geometric document lengths (mean 512) with state resets, seeded synthetic
+data shaped like a 1.5B-model layer (32 heads of 64).  Its inputs (>0.9 GB)
+exceed the 126 MB L2, so no flush is needed between timed steps.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints ONE JSON line (rank 0).  ``value`` is fwd+bwd tokens/s over all ranks
+(weak scaling: every rank runs its own batch, no data-path collective);
+timing is CUDA events on the launching stream, max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+from linear_recurrent_lm_b200 import inputs as I   # noqa: E402
+
+METRIC = "WKV-7 tokens/s fwd and fwd+bwd (H=32,N=64) + % of HBM roofline, 1xB200"
+WORKLOAD = 3
+# algorithmic bytes per token-head (bf16): inputs 6x64x2, y or dy 64x2, one fp32 64x64
+# checkpoint per 16 tokens (16 KiB / 16), gradients 6x64x2
+BYTES_FWD_TRAIN = 768 + 128 + 1024
+BYTES_BWD = 768 + 128 + 1024 + 768
+BYTES_PREFILL = 768 + 128
+BYTES_DECODE = 64 * 64 * 4 * 2 + 768 + 128
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_traffic(kernel: str, workload: str):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
+    if not os.path.exists(path):
+        return None
+    text = open(path).read()
+    m_src = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_src or not m_tr:
+        return None
+    src = re.search(r"source_file:\s*(\S+)", text)
+    if not src:
+        return None
+    try:
+        cur = hashlib.sha256(open(os.path.join(ROOT, src.group(1)), "rb").read()).hexdigest()
+    except OSError:
+        return None
+    return float(m_tr.group(1)) if cur == m_src.group(1) else None
+
+
+class Clocks:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
+             "clocks_event_reasons.sw_power_cap"
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+
+    def __enter__(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.index)], stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.f.close()
+
+    def summary(self):
+        if self.proc is None:
+            return None
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) != 7:
+                continue
+            try:
+                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+            except ValueError:
+                continue
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        loaded = [s for s, _, _ in rows if s > 500] or [s for s, _, _ in rows]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(m for _, m, _ in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def cpu_oracle_sample(wl, budget_s: float = 10.0):
+    """The CPU oracle (C, fp64, all host cores) on a bounded sample of whole (b,h) units of the
+    workload, forward + backward.  Returns tokens/s scaled to the workload's H heads."""
+    import oracle
+    cores = os.cpu_count() or 1
+    units = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+    rng = np.random.default_rng(0)
+    rng.shuffle(units)
+
+    def run(us):
+        t0 = time.perf_counter()
+        for b in sorted({u[0] for u in us}):
+            hs = [u[1] for u in us if u[0] == b]
+            part = {n: I.to_f64(wl.inputs[n][b:b + 1, :, hs]) for n in I.NAMES}
+            reset = wl.reset[b:b + 1] if wl.reset is not None else None
+            oracle.forward(*(part[n] for n in I.NAMES), reset=reset)
+            oracle.backward(*(part[n] for n in I.NAMES), I.to_f64(wl.dy[b:b + 1, :, hs]), reset=reset)
+        return time.perf_counter() - t0
+
+    t_one = run(units[:1])
+    n = int(min(len(units), max(1, budget_s / max(t_one, 1e-3)) * min(cores, len(units)) / 2))
+    n = max(1, min(n, len(units)))
+    t = run(units[:n])
+    tokens = n * wl.T / wl.H          # unit-tokens expressed as tokens of the H-head layer
+    return {"value": tokens / t, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{n} of {wl.B * wl.H} (b,h) units x T={wl.T}, fwd+bwd, fp64 C oracle, {t:.1f} s"}
+
+
+def run_reference(args):
+    """The oracle as the reference arm: same workload/metric, bounded sample per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    wl = I.make_workload(WORKLOAD)
+    cores = os.cpu_count() or 1
+    import oracle
+    units = [(b, h) for b in range(wl.B) for h in range(wl.H)][: max(1, min(cores, 32))]
+    part_b = {}
+    for b, h in units:
+        part_b.setdefault(b, []).append(h)
+
+    def step():
+        for b, hs in part_b.items():
+            part = {n: I.to_f64(wl.inputs[n][b:b + 1, :, hs]) for n in I.NAMES}
+            reset = wl.reset[b:b + 1]
+            oracle.forward(*(part[n] for n in I.NAMES), reset=reset)
+            oracle.backward(*(part[n] for n in I.NAMES), I.to_f64(wl.dy[b:b + 1, :, hs]), reset=reset)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = (time.perf_counter() - t0) / max(args.steps, 1)
+    tokens = len(units) * wl.T / wl.H
+    value = tokens / dt
+    sample = f"{len(units)} of {wl.B * wl.H} (b,h) units x T={wl.T} per step, fwd+bwd, fp64 C oracle"
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "N": wl.N},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "scan", "chunked"])
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-secondary", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    from linear_recurrent_lm_b200 import wkv7
+
+    dev = torch.device("cuda", local)
+    wl = I.make_workload(WORKLOAD, seed=1000 + WORKLOAD + rank)
+    B, T, H = wl.B, wl.T, wl.H
+
+    def d(x):
+        x = np.ascontiguousarray(x)
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(x).to(dev)
+
+    xs = [d(wl.inputs[n]) for n in I.NAMES]
+    dy = d(wl.dy)
+    reset = d(wl.reset)
+    y = torch.empty_like(xs[0])
+    s_out = torch.empty((B, H, 64, 64), device=dev, dtype=torch.float32)
+    ws = torch.empty(wkv7.workspace_bytes(B, T, H), device=dev, dtype=torch.uint8)
+    grads = {n: torch.empty_like(xs[0]) for n in ("dr", "dw", "dk", "dv", "da", "db")}
+    stream = torch.cuda.current_stream()
+
+    def step(evs=None):
+        if evs is not None:
+            evs[0].record(stream)
+        wkv7.forward(*xs, reset=reset, y=y, s_out=s_out, workspace=ws, algo=args.algo)
+        if evs is not None:
+            evs[1].record(stream)
+        wkv7.backward(*xs, dy, ws, reset=reset, grads=grads, want_ds0=False, algo=args.algo)
+        if evs is not None:
+            evs[2].record(stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    with Clocks(local) as clk:
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        start = torch.cuda.Event(enable_timing=True)
+        end = torch.cuda.Event(enable_timing=True)
+        start.record(stream)
+        for s in range(args.steps):
+            step(evs[s])
+        end.record(stream)
+        torch.cuda.synchronize()
+    total_ms = start.elapsed_time(end)
+    fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    t = torch.tensor([total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    total_ms, fwd_avg, bwd_avg = (float(v) for v in t.tolist())
+    ms_per_step = total_ms / args.steps
+    tokens_step = B * T * world
+    value = tokens_step / (ms_per_step / 1e3)
+
+    # ---- e2e: through the public API with host buffers, copies inside the timed region
+    host_in = [x.cpu().pin_memory() for x in xs] + [dy.cpu().pin_memory(), reset.cpu().pin_memory()]
+    host_out = [torch.empty(xs[0].shape, dtype=xs[0].dtype, pin_memory=True) for _ in range(7)]
+    dev_in = [torch.empty_like(x) for x in xs] + [torch.empty_like(dy), torch.empty_like(reset)]
+    h2d = sum(x.numel() * x.element_size() for x in host_in)
+    d2h = sum(x.numel() * x.element_size() for x in host_out)
+
+    def e2e_step():
+        for hsrc, dd in zip(host_in, dev_in):
+            dd.copy_(hsrc, non_blocking=True)
+        wkv7.forward(*dev_in[:6], reset=dev_in[7], y=y, s_out=s_out, workspace=ws, algo=args.algo)
+        wkv7.backward(*dev_in[:6], dev_in[6], ws, reset=dev_in[7], grads=grads, want_ds0=False, algo=args.algo)
+        outs = [y] + [grads[n] for n in ("dr", "dw", "dk", "dv", "da", "db")]
+        for o, hdst in zip(outs, host_out):
+            hdst.copy_(o, non_blocking=True)
+
+    e2e_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item()) / args.e2e_steps
+    e2e_value = tokens_step / (e2e_ms / 1e3)
+
+    secondary = {}
+    if rank == 0 and not args.no_secondary:
+        secondary = measure_secondary(wkv7, dev, args.algo)
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        peak, peak_kind = measured_peaks()
+        units = B * T * H
+        fwd_gbs = BYTES_FWD_TRAIN * units / (fwd_avg / 1e3) / 1e9
+        bwd_gbs = BYTES_BWD * units / (bwd_avg / 1e3) / 1e9
+        dominant = ("bwd", bwd_avg, bwd_gbs, BYTES_BWD) if bwd_avg >= fwd_avg else ("fwd", fwd_avg, fwd_gbs, BYTES_FWD_TRAIN)
+        kname = {"fwd": "chunk_fwd" if args.algo != "scan" else "scan_fwd", "bwd": "scan_bwd"}[dominant[0]]
+        traffic = kernel_traffic(kname, "packed_train_B8_T4096_H32")
+        cpu = None
+        if not args.no_cpu_baseline and world == 1:
+            cpu = cpu_oracle_sample(wl)
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": wl.name, "B": B, "T": T, "H": H, "N": 64, "algo": args.algo,
+                       "l2": "inputs larger than L2 (no flush)", "parallelism": f"dp{world} (independent batches)"},
+            "fwd": {"tokens_per_s": tokens_step / (fwd_avg / 1e3), "ms": fwd_avg, "achieved_gbs": fwd_gbs,
+                    "frac": fwd_gbs / peak},
+            "fwd_bwd": {"tokens_per_s": value, "ms": ms_per_step,
+                        "achieved_gbs": (BYTES_FWD_TRAIN + BYTES_BWD) * units / (ms_per_step / 1e3) / 1e9,
+                        "frac": (BYTES_FWD_TRAIN + BYTES_BWD) * units / (ms_per_step / 1e3) / 1e9 / peak},
+            "roofline": {"bound": "hbm", "kernel": kname, "achieved": dominant[2], "peak": peak, "unit": "GB/s",
+                         "frac": dominant[2] / peak, "peak_kind": peak_kind,
+                         "bytes_per_launch": dominant[3] * units,
+                         "traffic": traffic},
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clk.summary(),
+            "secondary": secondary,
+        }
+        print(json.dumps(line))
+    if world > 1:
+        dist.destroy_process_group()
+
+
+def measure_secondary(wkv7, dev, algo):
+    """Stateful prefill (B=1, T=1024, H=32) and the 128-step ragged decode (256 x 32 states)."""
+    import torch
+    out = {}
+    peak, _ = measured_peaks()
+    flush = torch.empty(512 * 1024 * 1024 // 4, device=dev, dtype=torch.float32)
+
+    def d(x):
+        x = np.ascontiguousarray(x)
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(x).to(dev)
+
+    wl = I.make_workload(2)
+    prior = [d(wl.prior[n]) for n in I.NAMES]
+    _, s0, _ = wkv7.forward(*prior, algo=algo, need_workspace=False)
+    xs = [d(wl.inputs[n]) for n in I.NAMES]
+    y = torch.empty_like(xs[0])
+    s_out = torch.empty_like(s0)
+    times = []
+    for rep in range(25):
+        flush.fill_(float(rep))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        wkv7.forward(*xs, s0=s0, y=y, s_out=s_out, need_workspace=False, algo=algo)
+        e1.record()
+        torch.cuda.synchronize()
+        if rep >= 5:
+            times.append(e0.elapsed_time(e1))
+    ms = statistics.median(times)
+    units = wl.B * wl.T * wl.H
+    gbs = BYTES_PREFILL * units / (ms / 1e3) / 1e9
+    out["prefill_B1_T1024_H32"] = {"tokens_per_s": wl.B * wl.T / (ms / 1e3), "ms": ms, "achieved_gbs": gbs,
+                                   "frac": gbs / peak, "l2": "flushed (512 MB write) before each rep"}
+
+    wl = I.make_workload(4)
+    state = d(wl.state0)
+    steps = [[d(s[n]) for n in I.NAMES] for s in wl.steps]
+    acts = [d(wl.active(s)) for s in range(len(wl.steps))]
+    yb = torch.empty_like(steps[0][0])
+    for s in range(len(steps)):            # warm-up pass (state keeps evolving; the timing is per byte)
+        wkv7.step(*steps[s], state, acts[s], y=yb)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for s in range(len(steps)):
+        wkv7.step(*steps[s], state, acts[s], y=yb)
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    active_tok = int(sum(int(wl.active(s).sum()) for s in range(len(wl.steps))))
+    gbs = BYTES_DECODE * active_tok * wl.H / (ms / 1e3) / 1e9
+    out["decode_B256_H32_128steps"] = {"tokens_per_s": active_tok / (ms / 1e3), "ms_128_steps": ms,
+                                       "achieved_gbs": gbs, "frac": gbs / peak, "active_tokens": active_tok}
+    return out
+
+
+if __name__ == "__main__":
+    main()

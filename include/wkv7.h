@@ -1,0 +1,163 @@
+/*
+ * wkv7.h -- C ABI of the B200 (sm_100a) WKV-7 library (libwkv7.so).
+ *
+ * WKV-7 is the recurrence at the core of RWKV-7 "Goose": the part of the
+ * model that "doesn't map onto standard ops" and that the rwkv-metal page runs
+ * as a hand-written kernel with a checkpointed backward ("The Metal WKV-7
+ * kernel").  Per (batch b, head h) it keeps an fp32 N x N state S (row i =
+ * value channel, column j = key channel) and, for each token t,
+ *
+ *     sa[i]   = sum_j S[i][j] * a_t[j]                 (S before the update)
+ *     S[i][j] = S[i][j] * w_t[j] + sa[i] * b_t[j] + v_t[i] * k_t[j]
+ *     y_t[i]  = sum_j S[i][j] * r_t[j]                 (S after the update)
+ *
+ * i.e. S_t = S_{t-1} (diag(w_t) + a_t b_t^T) + v_t k_t^T, y_t = S_t r_t: a
+ * diagonal-plus-rank-one ("generalised delta rule") transition.  The
+ * rwkv-lab page ("GDN subset of RWKV-7") shows the gated delta rule as the
+ * special case w = exp(g), a = -k, b = k exp(g) beta, k_write = beta k.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Head size N must be 64 (the HF model card page: "the kernel supports
+ *   64-wide heads and FP32 WKV state"); anything else -> WKV7_ERR_UNSUPPORTED.
+ * - Activations r,w,k,v,a,b,y,dy and the gradients dr..db are [B,T,H,64],
+ *   contiguous, row-major, all in the one dtype of the descriptor (f32, bf16
+ *   or f16; "accepts BF16/FP16/FP32 activations", same page).  Outputs in a
+ *   16-bit dtype are rounded to nearest even.  w is the multiplicative decay
+ *   (normally in (0,1]).
+ * - States s0, s_out, dsT, ds0 and the decode state are fp32 [B,H,64,64],
+ *   contiguous, S[i][j] at offset i*64+j.
+ * - reset is [B,T] bytes: reset[b][t] != 0 zeroes the incoming state before
+ *   token t (packed sequences: "Packed sequences are run with a state reset
+ *   at each boundary", HF model card page).  At t = 0 it overrides s0.  No
+ *   gradient crosses a reset.
+ * - Every pointer is a DEVICE pointer, 16-byte aligned (reset and active may
+ *   have any alignment).  The caller allocates and owns every buffer; the
+ *   library allocates nothing, keeps no per-call state and may be called from
+ *   several host threads on different streams.
+ * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
+ *   asynchronous on it.  The returned status covers argument validation and
+ *   the launch itself (cudaGetLastError); on any validation error nothing is
+ *   launched and no output is touched.
+ * - Any T >= 0 is accepted.  T need not be a multiple of 16 (the checkpoint
+ *   interval): "pads independent sequences to its 16-token checkpoint
+ *   interval" (HF model card page) -- here the padding is internal.
+ */
+#ifndef WKV7_H
+#define WKV7_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  WKV7_OK = 0,
+  WKV7_ERR_NULL = 1,        /* a required pointer is NULL                                    */
+  WKV7_ERR_SHAPE = 2,       /* B, T or H negative, or the element count overflows int64       */
+  WKV7_ERR_DTYPE = 3,       /* dtype code is not a wkv7_dtype_t                               */
+  WKV7_ERR_ALIGN = 4,       /* a tensor pointer is not 16-byte aligned                        */
+  WKV7_ERR_WORKSPACE = 5,   /* backward without a checkpoint workspace                        */
+  WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, non-zero flags, or T != 1 for a step   */
+  WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
+  WKV7_ERR_TIMEOUT = 8      /* reserved for device-side bounded waits (see wkv7_device_status) */
+} wkv7_status_t;
+
+typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
+
+/*
+ * Algorithm.  SCAN: token-order scan on FP32 cores, state in registers.
+ * CHUNKED: 16-token chunks with the intra-chunk products on tensor cores
+ * (the chunk-parallel form the HF model card page mentions as its
+ * "chunk-parallel path").  AUTO: CHUNKED for 16-bit inputs, SCAN for f32.
+ * Both produce the same result up to floating-point rounding order.
+ */
+typedef enum { WKV7_ALGO_AUTO = 0, WKV7_ALGO_SCAN = 1, WKV7_ALGO_CHUNKED = 2 } wkv7_algo_t;
+
+typedef struct {
+  int64_t B;      /* batch rows                                  */
+  int64_t T;      /* tokens per row (for wkv7_step: must be 1)   */
+  int64_t H;      /* heads                                       */
+  int32_t N;      /* head size: must be 64                       */
+  int32_t dtype;  /* wkv7_dtype_t of every activation/gradient   */
+  int32_t algo;   /* wkv7_algo_t                                 */
+  uint32_t flags; /* reserved, must be 0                         */
+} wkv7_desc_t;
+
+/* Library version, major*10000 + minor*100 + patch. */
+int wkv7_version(void);
+
+/* Static string for a status code (never NULL). */
+const char* wkv7_status_string(wkv7_status_t status);
+
+/*
+ * Bytes of checkpoint workspace that wkv7_forward writes and wkv7_backward
+ * reads: one fp32 64x64 state per (b, h) every 16 tokens, i.e.
+ * B*H*ceil(T/16)*64*64*4 bytes (rwkv-metal page: "checkpointing the hidden
+ * state every 16 tokens"; RWKV-MLX page, "Key Design Decisions" 2: "~12MB
+ * extra memory" at B=2, T=512, 12 heads -- this formula gives 12.58 MB).
+ * Checkpoint c holds the state after token min(16(c+1), T) - 1.
+ * Returns 0 for an invalid descriptor.
+ */
+size_t wkv7_workspace_bytes(const wkv7_desc_t* desc);
+
+/*
+ * Forward pass over T tokens (rwkv-metal page, "The Metal WKV-7 kernel":
+ * "handles the whole sequence in one forward dispatch ... checkpointing the
+ * hidden state every 16 tokens"; entry points wkv7_train / wkv7_train_with_state).
+ *
+ *   r,w,k,v,a,b  in   [B,T,H,64] desc->dtype
+ *   s0           in   [B,H,64,64] fp32 initial state, or NULL for zeros
+ *   reset        in   [B,T] u8, or NULL for no resets
+ *   y            out  [B,T,H,64] desc->dtype
+ *   s_out        out  [B,H,64,64] fp32 final state, or NULL
+ *   workspace    out  wkv7_workspace_bytes(desc) bytes of checkpoints for the
+ *                     backward, or NULL (inference: no checkpoints written)
+ */
+wkv7_status_t wkv7_forward(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
+                           const void* v, const void* a, const void* b, const float* s0,
+                           const uint8_t* reset, void* y, float* s_out, void* workspace, void* stream);
+
+/*
+ * Backward pass (rwkv-metal page: "one backward dispatch", reconstructing
+ * each 16-token chunk from its checkpoint; "differentiable through h_in").
+ * Inputs are those of the forward call that wrote `workspace` (same
+ * descriptor, r..b, s0, reset), plus
+ *
+ *   dy           in   [B,T,H,64] gradient of the loss w.r.t. y
+ *   dsT          in   [B,H,64,64] fp32 gradient w.r.t. the final state, or NULL
+ *   dr..db       out  [B,T,H,64] desc->dtype gradients w.r.t. r,w,k,v,a,b
+ *   ds0          out  [B,H,64,64] fp32 gradient w.r.t. s0, or NULL
+ *
+ * dw is the derivative with respect to the multiplicative decay w itself.
+ * `workspace` must not be NULL when T > 0 (WKV7_ERR_WORKSPACE).
+ */
+wkv7_status_t wkv7_backward(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
+                            const void* v, const void* a, const void* b, const float* s0,
+                            const uint8_t* reset, const void* dy, const float* dsT,
+                            const void* workspace, void* dr, void* dw, void* dk, void* dv, void* da,
+                            void* db, float* ds0, void* stream);
+
+/*
+ * One decode token for B*H resident states, in place (rwkv-metal page:
+ * "wkv7_step(..., h_in) one token"; "exact right-padding for ragged batches").
+ *
+ *   desc         B, H, N=64, dtype; T must be 1; algo is ignored
+ *   r..b         in      [B,H,64] desc->dtype (one token per row)
+ *   state        in/out  [B,H,64,64] fp32
+ *   active       in      [B] u8, or NULL for all rows active.  A row with
+ *                        active[b] == 0 leaves its state bitwise unchanged
+ *                        and gets y = 0.
+ *   y            out     [B,H,64] desc->dtype
+ */
+wkv7_status_t wkv7_step(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
+                        const void* v, const void* a, const void* b, float* state,
+                        const uint8_t* active, void* y, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* WKV7_H */

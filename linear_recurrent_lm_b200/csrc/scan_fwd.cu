@@ -1,0 +1,171 @@
+// WKV-7 forward, token-order scan on the FP32 cores (algo SCAN).
+//
+// One CTA per (b,h) unit, 64 threads, thread i owns row i of the 64x64 fp32
+// state in registers.  Rows of S never interact in the forward (sa[i] and
+// y[i] only read row i), so the scan needs no cross-thread reduction.  Each
+// 16-token slab of r,w,k,v,a,b is copied to shared memory with cp.async while
+// the previous slab is being consumed, widened once to fp32, and then read by
+// all threads as broadcasts.  After every 16 tokens (and after the last
+// token) the state is written to the checkpoint workspace, the
+// "checkpointing the hidden state every 16 tokens" of the rwkv-metal page
+// ("The Metal WKV-7 kernel").
+#include "common.cuh"
+#include "kernels.h"
+
+namespace wkv7 {
+namespace {
+
+constexpr int kThreads = 64;
+constexpr int kInputs = 6;   // slab order: r, w, k, v, a, b
+
+template <typename T>
+struct FwdSmem {
+  static constexpr size_t raw_bytes = size_t(kInputs) * kChunk * kN * sizeof(T);
+  static constexpr size_t f32_bytes = size_t(kInputs) * kChunk * kN * sizeof(float);
+  static constexpr size_t total = raw_bytes + f32_bytes;
+};
+
+template <typename T>
+__device__ __forceinline__ void stage_slab(const FwdArgs& p, const T* const* src, unsigned char* raw,
+                                           int64_t b, int64_t h, int64_t t0, int len) {
+  constexpr int VPT = kN / Vec16<T>::n;  // 16-byte vectors per token vector
+  const int total = kInputs * len * VPT;
+  for (int idx = threadIdx.x; idx < total; idx += kThreads) {
+    const int in = idx / (len * VPT);
+    const int rem = idx - in * len * VPT;
+    const int tt = rem / VPT;
+    const int vec = rem - tt * VPT;
+    const T* g = src[in] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * Vec16<T>::n;
+    unsigned char* s = raw + ((size_t(in) * kChunk + tt) * kN + vec * Vec16<T>::n) * sizeof(T);
+    cp_async16(s, g);
+  }
+  cp_async_commit();
+}
+
+template <typename T>
+__device__ __forceinline__ void widen_slab(const unsigned char* raw, float* f32, int len) {
+  const T* src = reinterpret_cast<const T*>(raw);
+  for (int in = 0; in < kInputs; ++in)
+    for (int e = threadIdx.x; e < len * kN; e += kThreads)
+      f32[in * kChunk * kN + e] = Elt<T>::to_f32(src[in * kChunk * kN + e]);
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
+  extern __shared__ __align__(16) unsigned char smem[];
+  unsigned char* raw = smem;
+  float* f32 = reinterpret_cast<float*>(smem + FwdSmem<T>::raw_bytes);
+
+  const int64_t unit = blockIdx.x;
+  const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
+  const int i = threadIdx.x;
+  const int64_t nc = (p.T + kChunk - 1) / kChunk;
+  const T* src[kInputs] = {static_cast<const T*>(p.r), static_cast<const T*>(p.w), static_cast<const T*>(p.k),
+                           static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b)};
+
+  float S[kN];
+  if (p.s0) {
+    const float4* row = reinterpret_cast<const float4*>(p.s0 + (unit * kN + i) * kN);
+#pragma unroll
+    for (int q = 0; q < kN / 4; ++q) {
+      float4 v4 = row[q];
+      S[4 * q] = v4.x; S[4 * q + 1] = v4.y; S[4 * q + 2] = v4.z; S[4 * q + 3] = v4.w;
+    }
+  } else {
+#pragma unroll
+    for (int j = 0; j < kN; ++j) S[j] = 0.f;
+  }
+
+  if (nc > 0) {
+    stage_slab<T>(p, src, raw, b, h, 0, int(min64(kChunk, p.T)));
+    cp_async_wait_all();
+    __syncthreads();
+    widen_slab<T>(raw, f32, int(min64(kChunk, p.T)));
+    __syncthreads();
+  }
+
+  T* y = static_cast<T*>(p.y);
+  for (int64_t c = 0; c < nc; ++c) {
+    const int64_t t0 = c * kChunk;
+    const int len = int(min64(kChunk, p.T - t0));
+    if (c + 1 < nc) stage_slab<T>(p, src, raw, b, h, t0 + kChunk, int(min64(kChunk, p.T - t0 - kChunk)));
+
+    for (int tt = 0; tt < len; ++tt) {
+      const int64_t t = t0 + tt;
+      if (p.reset && p.reset[b * p.T + t]) {
+#pragma unroll
+        for (int j = 0; j < kN; ++j) S[j] = 0.f;
+      }
+      const float4* r4 = reinterpret_cast<const float4*>(f32 + (0 * kChunk + tt) * kN);
+      const float4* w4 = reinterpret_cast<const float4*>(f32 + (1 * kChunk + tt) * kN);
+      const float4* k4 = reinterpret_cast<const float4*>(f32 + (2 * kChunk + tt) * kN);
+      const float vi = f32[(3 * kChunk + tt) * kN + i];
+      const float4* a4 = reinterpret_cast<const float4*>(f32 + (4 * kChunk + tt) * kN);
+      const float4* b4 = reinterpret_cast<const float4*>(f32 + (5 * kChunk + tt) * kN);
+      float s0 = 0.f, s1 = 0.f, s2 = 0.f, s3 = 0.f;
+#pragma unroll
+      for (int q = 0; q < kN / 4; ++q) {
+        const float4 av = a4[q];
+        s0 = fmaf(S[4 * q], av.x, s0);
+        s1 = fmaf(S[4 * q + 1], av.y, s1);
+        s2 = fmaf(S[4 * q + 2], av.z, s2);
+        s3 = fmaf(S[4 * q + 3], av.w, s3);
+      }
+      const float sa = (s0 + s1) + (s2 + s3);
+      float y0 = 0.f, y1 = 0.f, y2 = 0.f, y3 = 0.f;
+#pragma unroll
+      for (int q = 0; q < kN / 4; ++q) {
+        const float4 wv = w4[q], bv = b4[q], kv = k4[q], rv = r4[q];
+        S[4 * q] = fmaf(S[4 * q], wv.x, fmaf(sa, bv.x, vi * kv.x));
+        S[4 * q + 1] = fmaf(S[4 * q + 1], wv.y, fmaf(sa, bv.y, vi * kv.y));
+        S[4 * q + 2] = fmaf(S[4 * q + 2], wv.z, fmaf(sa, bv.z, vi * kv.z));
+        S[4 * q + 3] = fmaf(S[4 * q + 3], wv.w, fmaf(sa, bv.w, vi * kv.w));
+        y0 = fmaf(S[4 * q], rv.x, y0);
+        y1 = fmaf(S[4 * q + 1], rv.y, y1);
+        y2 = fmaf(S[4 * q + 2], rv.z, y2);
+        y3 = fmaf(S[4 * q + 3], rv.w, y3);
+      }
+      y[tok_off(b, t, h, p.T, p.H) + i] = Elt<T>::from_f32((y0 + y1) + (y2 + y3));
+    }
+
+    if (p.ckpt) {
+      float4* dst = reinterpret_cast<float4*>(p.ckpt + ((unit * nc + c) * kN + i) * kN);
+#pragma unroll
+      for (int q = 0; q < kN / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    if (c + 1 < nc) {
+      widen_slab<T>(raw, f32, int(min64(kChunk, p.T - t0 - kChunk)));
+      __syncthreads();
+    }
+  }
+
+  if (p.s_out) {
+    float4* dst = reinterpret_cast<float4*>(p.s_out + (unit * kN + i) * kN);
+#pragma unroll
+    for (int q = 0; q < kN / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+  }
+}
+
+template <typename T>
+cudaError_t launch(const FwdArgs& p, cudaStream_t stream) {
+  const size_t smem = FwdSmem<T>::total;
+  cudaError_t e = cudaFuncSetAttribute(scan_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  if (e != cudaSuccess) return e;
+  scan_fwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream) {
+  switch (dtype) {
+    case 0: return launch<float>(p, stream);
+    case 1: return launch<__nv_bfloat16>(p, stream);
+    case 2: return launch<__half>(p, stream);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace wkv7

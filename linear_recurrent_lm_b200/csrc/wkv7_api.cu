@@ -1,0 +1,140 @@
+// C ABI of libwkv7 (declared in include/wkv7.h): argument validation and
+// dispatch to the sm_100a kernels.  Nothing here allocates memory or keeps
+// state between calls; every kernel runs on the caller's stream.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kernels.h"
+#include "wkv7.h"
+
+namespace {
+
+constexpr int64_t kMaxGrid = 2147483647;   // grid.x limit: one CTA per (b,h)
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool mul_ok(int64_t a, int64_t b, int64_t* out) {
+  if (a < 0 || b < 0) return false;
+  if (a != 0 && b > INT64_MAX / a) return false;
+  *out = a * b;
+  return true;
+}
+
+// Common descriptor checks.  On success fills the element counts.
+wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
+  if (!d) return WKV7_ERR_NULL;
+  if (d->N != 64 || d->flags != 0u) return WKV7_ERR_UNSUPPORTED;
+  if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
+  if (d->algo != WKV7_ALGO_AUTO && d->algo != WKV7_ALGO_SCAN && d->algo != WKV7_ALGO_CHUNKED)
+    return WKV7_ERR_UNSUPPORTED;
+  if (d->B < 0 || d->T < 0 || d->H < 0) return WKV7_ERR_SHAPE;
+  int64_t bh, bth, e;
+  if (!mul_ok(d->B, d->H, &bh) || bh > kMaxGrid) return WKV7_ERR_SHAPE;
+  if (!mul_ok(bh, d->T, &bth) || !mul_ok(bth, 64 * 4, &e)) return WKV7_ERR_SHAPE;   // byte count fits
+  int64_t st;
+  if (!mul_ok(bh, 64 * 64 * 4, &st)) return WKV7_ERR_SHAPE;
+  *units = bh;
+  *tok_elems = bth * 64;
+  return WKV7_OK;
+}
+
+// Every listed pointer must be non-null (when `need`) and 16-byte aligned (when non-null).
+wkv7_status_t check_ptrs(bool need, std::initializer_list<const void*> ptrs) {
+  for (const void* p : ptrs) {
+    if (!p) {
+      if (need) return WKV7_ERR_NULL;
+      continue;
+    }
+    if (!aligned16(p)) return WKV7_ERR_ALIGN;
+  }
+  return WKV7_OK;
+}
+
+wkv7_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA; }
+
+bool use_chunked(const wkv7_desc_t* d) {
+  if (d->algo == WKV7_ALGO_CHUNKED) return true;
+  if (d->algo == WKV7_ALGO_SCAN) return false;
+  return d->dtype != WKV7_F32;
+}
+
+}  // namespace
+
+extern "C" {
+
+int wkv7_version(void) { return 100; }
+
+const char* wkv7_status_string(wkv7_status_t s) {
+  switch (s) {
+    case WKV7_OK: return "ok";
+    case WKV7_ERR_NULL: return "a required pointer is NULL";
+    case WKV7_ERR_SHAPE: return "invalid or overflowing shape";
+    case WKV7_ERR_DTYPE: return "unknown dtype";
+    case WKV7_ERR_ALIGN: return "tensor pointer is not 16-byte aligned";
+    case WKV7_ERR_WORKSPACE: return "checkpoint workspace is required";
+    case WKV7_ERR_UNSUPPORTED: return "unsupported head size, algorithm, flags or step length";
+    case WKV7_ERR_CUDA: return "CUDA launch failed";
+    case WKV7_ERR_TIMEOUT: return "device-side wait timed out";
+  }
+  return "unknown status";
+}
+
+size_t wkv7_workspace_bytes(const wkv7_desc_t* d) {
+  int64_t units = 0, te = 0;
+  if (check_desc(d, &units, &te) != WKV7_OK) return 0;
+  const int64_t nc = (d->T + 15) / 16;
+  int64_t n1, n2;
+  if (!mul_ok(units, nc, &n1) || !mul_ok(n1, 64 * 64 * 4, &n2)) return 0;
+  return static_cast<size_t>(n2);
+}
+
+wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
+                           const void* a, const void* b, const float* s0, const uint8_t* reset, void* y,
+                           float* s_out, void* workspace, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(te > 0, {r, w, k, v, a, b, y});
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(false, {s0, s_out, workspace});
+  if (st != WKV7_OK) return st;
+  if (units == 0) return WKV7_OK;
+  wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace)};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_fwd(p, d->dtype, s));
+  return from_cuda(wkv7::launch_chunk_fwd(p, d->dtype, s));
+}
+
+wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
+                            const void* a, const void* b, const float* s0, const uint8_t* reset, const void* dy,
+                            const float* dsT, const void* workspace, void* dr, void* dw, void* dk, void* dv,
+                            void* da, void* db, float* ds0, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(te > 0, {r, w, k, v, a, b, dy, dr, dw, dk, dv, da, db});
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(false, {s0, dsT, ds0, workspace});
+  if (st != WKV7_OK) return st;
+  if (te > 0 && !workspace) return WKV7_ERR_WORKSPACE;
+  if (units == 0) return WKV7_OK;
+  wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
+                  dr, dw, dk, dv, da, db, ds0};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, s));
+}
+
+wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
+                        const void* a, const void* b, float* state, const uint8_t* active, void* y, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  if (d->T != 1) return WKV7_ERR_UNSUPPORTED;
+  st = check_ptrs(units > 0, {r, w, k, v, a, b, state, y});
+  if (st != WKV7_OK) return st;
+  if (units == 0) return WKV7_OK;
+  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y};
+  return from_cuda(wkv7::launch_step(p, d->dtype, static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

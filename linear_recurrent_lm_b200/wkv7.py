@@ -1,0 +1,152 @@
+"""Python binding of libwkv7 (the C ABI in include/wkv7.h).
+
+Argument marshalling only: every step of the WKV-7 path runs in the CUDA
+kernels of ``libwkv7.so``.  PyTorch provides device memory and the current
+stream.  The same entry points as the C ABI:
+
+* ``forward(r, w, k, v, a, b, s0=None, reset=None, ...)``  -> (y, s_out, workspace)
+* ``backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, ...)``
+  -> dict(dr, dw, dk, dv, da, db, ds0)
+* ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
+* ``workspace_bytes(B, T, H, dtype)``
+
+Tensors are [B,T,H,64] (token inputs), [B,H,64,64] fp32 (states), [B,T] uint8
+(reset), [B] uint8 (active), all on one CUDA device and contiguous.  If the
+library is missing, importing this module raises: there is no fallback.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Dict, Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libwkv7.so")
+
+OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(9)
+DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
+ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2}
+N_HEAD = 64
+CHUNK = 16
+
+
+class Desc(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64), ("N", ctypes.c_int32),
+                ("dtype", ctypes.c_int32), ("algo", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class WKV7Error(RuntimeError):
+    def __init__(self, status: int, where: str):
+        super().__init__(f"{where}: {lib().wkv7_status_string(status).decode()} (status {status})")
+        self.status = status
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded libwkv7.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_recurrent_lm_b200.build` "
+                              "(or __graft_entry__.build()); the WKV-7 path has no CPU fallback")
+        L = ctypes.CDLL(LIB_PATH)
+        vp = ctypes.c_void_p
+        dp = ctypes.POINTER(Desc)
+        L.wkv7_version.restype = ctypes.c_int
+        L.wkv7_status_string.restype = ctypes.c_char_p
+        L.wkv7_status_string.argtypes = [ctypes.c_int]
+        L.wkv7_workspace_bytes.restype = ctypes.c_size_t
+        L.wkv7_workspace_bytes.argtypes = [dp]
+        L.wkv7_forward.restype = ctypes.c_int
+        L.wkv7_forward.argtypes = [dp] + [vp] * 12
+        L.wkv7_backward.restype = ctypes.c_int
+        L.wkv7_backward.argtypes = [dp] + [vp] * 19
+        L.wkv7_step.restype = ctypes.c_int
+        L.wkv7_step.argtypes = [dp] + [vp] * 10
+        _lib = L
+    return _lib
+
+
+lib()   # fail at import time if the CUDA library is absent
+
+
+def make_desc(B: int, T: int, H: int, dtype, algo: str = "auto", N: int = N_HEAD, flags: int = 0) -> Desc:
+    code = DTYPE_CODE[dtype] if isinstance(dtype, torch.dtype) else int(dtype)
+    return Desc(int(B), int(T), int(H), int(N), code, ALGO_CODE[algo] if isinstance(algo, str) else int(algo), int(flags))
+
+
+def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16) -> int:
+    return int(lib().wkv7_workspace_bytes(ctypes.byref(make_desc(B, T, H, dtype))))
+
+
+def _ptr(x: Optional[torch.Tensor]):
+    return None if x is None else ctypes.c_void_p(x.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != OK:
+        raise WKV7Error(status, where)
+
+
+def _token_shape(x: torch.Tensor):
+    if x.dim() != 4 or x.shape[-1] != N_HEAD:
+        raise ValueError(f"expected [B,T,H,{N_HEAD}], got {tuple(x.shape)}")
+    return tuple(int(s) for s in x.shape[:3])
+
+
+def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, workspace=None,
+            need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None):
+    """WKV-7 forward over [B,T,H,64] inputs.  Returns (y, s_out, workspace)."""
+    B, T, H = _token_shape(r)
+    dev = r.device
+    if y is None:
+        y = torch.empty_like(r)
+    if s_out is None and want_state:
+        s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=dev, dtype=torch.float32)
+    if workspace is None and need_workspace:
+        workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype), 16), device=dev, dtype=torch.uint8)
+    d = make_desc(B, T, H, r.dtype, algo)
+    st = lib().wkv7_forward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, workspace)),
+                            _stream(stream))
+    _check(st, "wkv7_forward")
+    return y, s_out, workspace
+
+
+def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, grads=None,
+             want_ds0: bool = True, algo: str = "auto", stream=None) -> Dict[str, torch.Tensor]:
+    """WKV-7 backward from the checkpoints written by ``forward``."""
+    B, T, H = _token_shape(r)
+    g = dict(grads) if grads is not None else {}
+    for n in ("dr", "dw", "dk", "dv", "da", "db"):
+        if g.get(n) is None:
+            g[n] = torch.empty_like(r)
+    if g.get("ds0") is None and want_ds0:
+        g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
+    d = make_desc(B, T, H, r.dtype, algo)
+    st = lib().wkv7_backward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, dy, dsT, workspace)),
+                             *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
+                             _stream(stream))
+    _check(st, "wkv7_backward")
+    return g
+
+
+def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None):
+    """One decode token on ``state`` [B,H,64,64] (in place).  Inputs [B,H,64].  Returns y."""
+    if r.dim() != 3 or r.shape[-1] != N_HEAD:
+        raise ValueError(f"expected [B,H,{N_HEAD}], got {tuple(r.shape)}")
+    B, H = int(r.shape[0]), int(r.shape[1])
+    if y is None:
+        y = torch.empty_like(r)
+    d = make_desc(B, 1, H, r.dtype)
+    st = lib().wkv7_step(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, state, active, y)), _stream(stream))
+    _check(st, "wkv7_step")
+    return y

@@ -1,0 +1,114 @@
+"""The C ABI without a GPU: the library loads, exports every function the
+header declares, and rejects bad arguments before launching anything."""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "wkv7.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    from linear_recurrent_lm_b200 import build
+    build.build()
+    from linear_recurrent_lm_b200 import wkv7
+    return wkv7
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(wkv7_[a-z_0-9]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = declared_functions()
+    assert {"wkv7_forward", "wkv7_backward", "wkv7_step", "wkv7_workspace_bytes"} <= set(names)
+    lib = ctypes.CDLL(L.LIB_PATH)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings(L):
+    lib = L.lib()
+    assert lib.wkv7_version() >= 100
+    for s in range(9):
+        assert lib.wkv7_status_string(s)
+    assert lib.wkv7_status_string(12345) == b"unknown status"
+
+
+def test_workspace_matches_checkpoint_memory_on_rwkv_mlx_page(L):
+    """RWKV-MLX page ("Key Design Decisions" 2): checkpoints every 16 tokens cost
+    about 12 MB at the 184M-model layer shape (B=2, T=512, 12 heads of 64)."""
+    n = L.workspace_bytes(2, 512, 12)
+    assert n == 2 * 12 * (512 // 16) * 64 * 64 * 4 == 12_582_912
+    assert L.workspace_bytes(1, 17, 1) == 2 * 64 * 64 * 4        # ceil(17/16) = 2 checkpoints
+    assert L.workspace_bytes(1, 0, 1) == 0
+
+
+FAKE = 0x10000       # 16-byte aligned address that is never dereferenced (validation fails first)
+
+
+def call_fwd(L, desc, ptrs=None, **over):
+    p = dict(r=FAKE, w=FAKE, k=FAKE, v=FAKE, a=FAKE, b=FAKE, s0=None, reset=None, y=FAKE, s_out=None, ws=None)
+    p.update(over)
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    return L.lib().wkv7_forward(None if desc is None else ctypes.byref(desc),
+                                *(vp(p[n]) for n in ("r", "w", "k", "v", "a", "b", "s0", "reset", "y", "s_out", "ws")),
+                                None)
+
+
+def test_forward_validation_codes(L):
+    import torch
+    d = L.make_desc(1, 16, 1, torch.bfloat16)
+    assert call_fwd(L, None) == L.ERR_NULL
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.N = 32
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 1
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = 7
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.dtype = 9
+    assert call_fwd(L, bad) == L.ERR_DTYPE
+    assert call_fwd(L, L.make_desc(-1, 16, 1, torch.bfloat16)) == L.ERR_SHAPE
+    assert call_fwd(L, L.make_desc(1, -3, 1, torch.bfloat16)) == L.ERR_SHAPE
+    assert call_fwd(L, L.make_desc(1 << 40, 1 << 20, 1 << 10, torch.bfloat16)) == L.ERR_SHAPE
+    assert call_fwd(L, L.make_desc(1 << 20, 1, 1 << 12, torch.bfloat16)) == L.ERR_SHAPE   # grid > 2^31-1
+    assert call_fwd(L, d, k=None) == L.ERR_NULL
+    assert call_fwd(L, d, y=None) == L.ERR_NULL
+    assert call_fwd(L, d, v=FAKE + 2) == L.ERR_ALIGN
+    assert call_fwd(L, d, s0=FAKE + 8) == L.ERR_ALIGN
+    assert call_fwd(L, d, ws=FAKE + 4) == L.ERR_ALIGN
+    # empty problems launch nothing and succeed
+    assert call_fwd(L, L.make_desc(0, 16, 4, torch.bfloat16), r=None, w=None, k=None, v=None, a=None, b=None, y=None) == L.OK
+    assert call_fwd(L, L.make_desc(3, 16, 0, torch.bfloat16), r=None, w=None, k=None, v=None, a=None, b=None, y=None) == L.OK
+
+
+def test_backward_and_step_validation_codes(L):
+    import torch
+    lib = L.lib()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    d = L.make_desc(1, 16, 1, torch.bfloat16)
+    base = [FAKE] * 6 + [None, None, FAKE, None]     # r..b, s0, reset, dy, dsT
+    grads = [FAKE] * 6 + [None]
+    assert lib.wkv7_backward(ctypes.byref(d), *map(vp, base), None, *map(vp, grads), None) == L.ERR_WORKSPACE
+    assert lib.wkv7_backward(ctypes.byref(d), *map(vp, base), vp(FAKE), *map(vp, [FAKE] * 5 + [None, None]), None) == L.ERR_NULL
+    assert lib.wkv7_backward(ctypes.byref(d), *map(vp, base), vp(FAKE + 1), *map(vp, grads), None) == L.ERR_ALIGN
+    s = L.make_desc(4, 2, 1, torch.bfloat16)      # a step takes exactly one token
+    assert lib.wkv7_step(ctypes.byref(s), *map(vp, [FAKE] * 7), None, vp(FAKE), None) == L.ERR_UNSUPPORTED
+    s = L.make_desc(4, 1, 1, torch.bfloat16)
+    assert lib.wkv7_step(ctypes.byref(s), *map(vp, [FAKE] * 6), None, None, vp(FAKE), None) == L.ERR_NULL
+
+
+def test_no_cpu_fallback_without_gpu(L):
+    """On a host with no GPU a valid call must fail loudly (ERR_CUDA), never compute on the CPU."""
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("host has a GPU")
+    d = L.make_desc(1, 16, 1, torch.bfloat16)
+    assert call_fwd(L, d) == L.ERR_CUDA

@@ -1,0 +1,150 @@
+"""GPU forward parity against the CPU oracle (both algorithms, all dtypes)."""
+from __future__ import annotations
+
+import numpy as np
+import pytest
+
+import oracle
+from linear_recurrent_lm_b200 import inputs as I
+from tests.gpu_util import f64, inputs_dev, inputs_f64, sample_units, to_dev
+from tests.metrics import err_rms, err_rms_excess
+
+pytestmark = pytest.mark.gpu
+
+TOL = {"f32": 1e-4, "bf16": 2e-2, "f16": 5e-3}
+ALGOS = ("scan", "chunked")
+
+
+@pytest.fixture(scope="module")
+def W():
+    import torch
+    from linear_recurrent_lm_b200 import wkv7
+    torch.cuda.set_device(0)
+    return wkv7
+
+
+def run_fwd(W, d, s0=None, reset=None, algo="auto"):
+    y, s, ws = W.forward(*inputs_dev(d), s0=None if s0 is None else to_dev(s0),
+                         reset=None if reset is None else to_dev(reset), algo=algo)
+    return y, s, ws
+
+
+def check_fwd(y, s, yo, so, dtype):
+    ey = err_rms_excess(f64(y), yo, dtype)
+    es = err_rms(f64(s), so)
+    assert ey <= TOL[dtype], ("y", ey)
+    assert es <= TOL[dtype], ("s_out", es)
+    return ey, es
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_config0_fp32(W, algo):
+    """B=1, T=64, H=2, fp32 inputs, zero initial state: max|err|/RMS <= 1e-4."""
+    wl = I.make_workload(0)
+    y, s, _ = run_fwd(W, wl.inputs, algo=algo)
+    yo, so, _ = oracle.forward(*inputs_f64(wl.inputs))
+    assert err_rms(f64(y), yo) <= 1e-4
+    assert err_rms(f64(s), so) <= 1e-4
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_config1_forward_and_checkpoints(W, algo):
+    import torch
+    wl = I.make_workload(1)
+    y, s, ws = run_fwd(W, wl.inputs, algo=algo)
+    yo, so, _ = oracle.forward(*inputs_f64(wl.inputs))
+    check_fwd(y, s, yo, so, "bf16")
+    # checkpoint c holds the state after token 16c+15: compare with the oracle run to that token
+    ck = ws.view(torch.float32).view(2, 12, 32, 64, 64)
+    for c in (0, 7, 31):
+        part = {n: wl.inputs[n][:, : 16 * (c + 1)] for n in I.NAMES}
+        _, sc, _ = oracle.forward(*inputs_f64(part))
+        assert err_rms(f64(ck[:, :, c]), sc) <= 2e-2
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_config2_prefill_chained_equals_single(W, algo):
+    """1.5B-model shape: s0 from 256 prior tokens, then 1024 tokens; equals one 1280-token call."""
+    import torch
+    wl = I.make_workload(2)
+    _, s_prior, _ = run_fwd(W, wl.prior, algo=algo)
+    y, s, _ = W.forward(*inputs_dev(wl.inputs), s0=s_prior, algo=algo, need_workspace=False)
+    full = {n: np.concatenate([wl.prior[n], wl.inputs[n]], axis=1) for n in I.NAMES}
+    yf, sf, _ = run_fwd(W, full, algo=algo)
+    # split at a multiple of 16: the same arithmetic in the same order
+    assert torch.equal(yf[:, 256:], y) and torch.equal(sf, s)
+    yo, so, _ = oracle.forward(*inputs_f64(full))
+    check_fwd(y, s, yo[:, 256:], so, "bf16")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_config3_full_size_sampled_units(W, algo):
+    """B=8, T=4096, H=32 packed documents with resets, at full size on the GPU; the oracle
+    recomputes a sample of (b,h) units exactly (units are independent)."""
+    wl = I.make_workload(3)
+    y, s, _ = run_fwd(W, wl.inputs, reset=wl.reset, algo=algo)
+    yg, sg = f64(y), f64(s)
+    for (b, h) in sample_units(8, 32, 10, seed=3):
+        part = {n: wl.inputs[n][b:b + 1, :, h:h + 1] for n in I.NAMES}
+        yo, so, _ = oracle.forward(*inputs_f64(part), reset=wl.reset[b:b + 1])
+        check_fwd_arr = (err_rms_excess(yg[b:b + 1, :, h:h + 1], yo, "bf16"), err_rms(sg[b:b + 1, h:h + 1], so))
+        assert check_fwd_arr[0] <= 2e-2 and check_fwd_arr[1] <= 2e-2, ((b, h), check_fwd_arr)
+
+
+EDGE_T = [1, 15, 16, 17, 40, 100]
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("T", EDGE_T)
+def test_ragged_lengths_state_and_resets(W, algo, dtype, T):
+    rng = np.random.default_rng(T)
+    B, H = 2, 3
+    d = I.draw_inputs(rng, (B, T, H, 64), dtype)
+    s0 = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    reset = np.zeros((B, T), np.uint8)
+    reset[1, 0] = 1                                  # overrides s0 for row 1
+    for t in (5, 6, 16, T - 1):                      # consecutive resets, a chunk boundary, the last token
+        if 0 < t < T:
+            reset[0, t] = 1
+    y, s, _ = run_fwd(W, d, s0=s0, reset=reset, algo=algo)
+    yo, so, _ = oracle.forward(*inputs_f64(d), s0=s0, reset=reset)
+    check_fwd(y, s, yo, so, dtype)
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_zero_decay_and_identity_tokens(W, algo):
+    """w = 0 (keeps only the last write; the chunked path must not divide by the decay) and
+    identity tokens (w=1, a=b=k=0) that leave the state bitwise unchanged."""
+    import torch
+    rng = np.random.default_rng(9)
+    d = I.draw_inputs(rng, (1, 48, 2, 64), "bf16")
+    w = I.to_f64(d["w"])
+    w[:, 20:23] = 0.0
+    d["w"] = I.to_storage(w, "bf16")
+    y, s, _ = run_fwd(W, d, algo=algo)
+    yo, so, _ = oracle.forward(*inputs_f64(d))
+    check_fwd(y, s, yo, so, "bf16")
+    s0 = rng.standard_normal((1, 2, 64, 64)).astype(np.float32)
+    ident = {n: np.zeros((1, 32, 2, 64), np.uint16) for n in I.NAMES}
+    ident["w"][:] = I.f32_to_bf16_bits(np.ones(1, np.float32))[0]
+    _, s2, _ = run_fwd(W, ident, s0=s0, algo=algo)
+    assert torch.equal(s2.cpu(), torch.from_numpy(s0))
+
+
+@pytest.mark.parametrize("algo", ALGOS)
+def test_zero_tokens_and_single_unit(W, algo):
+    import torch
+    rng = np.random.default_rng(11)
+    d = I.draw_inputs(rng, (1, 0, 1, 64), "bf16")
+    s0 = rng.standard_normal((1, 1, 64, 64)).astype(np.float32)
+    _, s, _ = run_fwd(W, d, s0=s0, algo=algo)
+    assert torch.equal(s.cpu(), torch.from_numpy(s0))
+
+
+def test_forward_is_deterministic(W):
+    import torch
+    wl = I.make_workload(1)
+    a = run_fwd(W, wl.inputs)
+    b = run_fwd(W, wl.inputs)
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
