@@ -200,9 +200,14 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--only", choices=["fwd", "bwd", "prefill", "step"],
+                    help="time one kernel alone (profiling entry point); prints its own JSON line")
+    ap.add_argument("--B", type=int, default=None, help="batch override for --only")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.only:
+        return run_only(args)
 
     import torch
     import torch.distributed as dist
@@ -404,6 +409,57 @@ def measure_secondary(wkv7, dev, algo):
     out["decode_B256_H32_128steps"] = {"tokens_per_s": active_tok / (ms / 1e3), "ms_128_steps": ms,
                                        "achieved_gbs": gbs, "frac": gbs / peak, "active_tokens": active_tok}
     return out
+
+
+def run_only(args):
+    """Warm-up + timed launches of a single kernel on the default workload (or a smaller batch)."""
+    import torch
+    from linear_recurrent_lm_b200 import wkv7
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    idx = {"fwd": 3, "bwd": 3, "prefill": 2, "step": 4}[args.only]
+    wl = I.make_workload(idx, B=args.B)
+
+    def d(x):
+        x = np.ascontiguousarray(x)
+        if x.dtype == np.uint16:
+            return torch.from_numpy(x.view(np.int16)).view(torch.bfloat16).to(dev)
+        return torch.from_numpy(x).to(dev)
+
+    if args.only == "step":
+        state = d(wl.state0)
+        xs = [d(wl.steps[0][n]) for n in I.NAMES]
+        act = d(wl.active(0))
+        fn = lambda: wkv7.step(*xs, state, act)
+        units, per = int(wl.active(0).sum()) * wl.H, BYTES_DECODE
+    else:
+        xs = [d(wl.inputs[n]) for n in I.NAMES]
+        reset = d(wl.reset) if wl.reset is not None else None
+        y, s_out, ws = wkv7.forward(*xs, reset=reset, algo=args.algo, need_workspace=args.only != "prefill")
+        units = wl.B * wl.T * wl.H
+        if args.only in ("fwd", "prefill"):
+            fn = lambda: wkv7.forward(*xs, reset=reset, y=y, s_out=s_out, workspace=ws, algo=args.algo,
+                                      need_workspace=args.only == "fwd")
+            per = BYTES_FWD_TRAIN if args.only == "fwd" else BYTES_PREFILL
+        else:
+            dy = d(wl.dy)
+            grads = {n: torch.empty_like(xs[0]) for n in ("dr", "dw", "dk", "dv", "da", "db")}
+            fn = lambda: wkv7.backward(*xs, dy, ws, reset=reset, grads=grads, want_ds0=False, algo=args.algo)
+            per = BYTES_BWD
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    peak, _ = measured_peaks()
+    gbs = per * units / (ms / 1e3) / 1e9
+    print(json.dumps({"only": args.only, "workload": wl.name, "B": wl.B, "algo": args.algo, "ms": ms,
+                      "achieved_gbs": gbs, "frac": gbs / peak}))
 
 
 if __name__ == "__main__":
