@@ -93,13 +93,15 @@ int wkv7_version(void);
 const char* wkv7_status_string(wkv7_status_t status);
 
 /*
- * Bytes of checkpoint workspace that wkv7_forward writes and wkv7_backward
+ * Bytes of workspace that wkv7_forward writes and wkv7_backward
  * reads: one fp32 64x64 state per (b, h) every 16 tokens, i.e.
  * B*H*ceil(T/16)*64*64*4 bytes (rwkv-metal page: "checkpointing the hidden
  * state every 16 tokens"; RWKV-MLX page, "Key Design Decisions" 2: "~12MB
  * extra memory" at B=2, T=512, 12 heads -- this formula gives 12.58 MB).
- * Checkpoint c holds the state after token min(16(c+1), T) - 1.
- * Returns 0 for an invalid descriptor.
+ * Checkpoint c holds the state after token min(16(c+1), T) - 1.  After the
+ * checkpoints come B*H ints (rounded up to 16 bytes) that wkv7_backward uses
+ * to mark heads it must recompute with the exact scan.
+ * Returns 0 for an invalid descriptor or T == 0.
  */
 size_t wkv7_workspace_bytes(const wkv7_desc_t* desc);
 

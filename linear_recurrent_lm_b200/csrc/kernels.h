@@ -26,6 +26,7 @@ struct BwdArgs {
   const float* ckpt;
   void *dr, *dw, *dk, *dv, *da, *db;
   float* ds0;
+  int* unit_flags;   // [B*H] in the workspace tail: the chunked backward marks units it could not handle
 };
 
 struct StepArgs {
@@ -38,7 +39,8 @@ struct StepArgs {
 
 // dtype: 0 = f32, 1 = bf16, 2 = f16.  Each returns the launch status.
 cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
-cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, cudaStream_t stream);
+// only_flagged: run only the (b,h) units whose unit_flags entry is non-zero (others exit at once).
+cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_chunk_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_chunk_bwd(const BwdArgs& p, int dtype, cudaStream_t stream);

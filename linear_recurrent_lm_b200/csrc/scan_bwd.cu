@@ -79,11 +79,12 @@ __device__ __forceinline__ float row_reduce16(float (&v)[16], int lane) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p) {
+__global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only_flagged) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   BwdSmem& sm = *reinterpret_cast<BwdSmem*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
+  if (only_flagged && p.unit_flags[unit] == 0) return;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
   const int tid = threadIdx.x, lane = tid & 31;
   const int q = tid >> 6;          // row quarter
@@ -239,21 +240,21 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p) {
 }
 
 template <typename T>
-cudaError_t launch(const BwdArgs& p, cudaStream_t stream) {
+cudaError_t launch(const BwdArgs& p, bool only_flagged, cudaStream_t stream) {
   const size_t smem = sizeof(BwdSmem);
   cudaError_t e = cudaFuncSetAttribute(scan_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  scan_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p);
+  scan_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, only_flagged);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, cudaStream_t stream) {
+cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream) {
   switch (dtype) {
-    case 0: return launch<float>(p, stream);
-    case 1: return launch<__nv_bfloat16>(p, stream);
-    case 2: return launch<__half>(p, stream);
+    case 0: return launch<float>(p, only_flagged, stream);
+    case 1: return launch<__nv_bfloat16>(p, only_flagged, stream);
+    case 2: return launch<__half>(p, only_flagged, stream);
     default: return cudaErrorInvalidValue;
   }
 }

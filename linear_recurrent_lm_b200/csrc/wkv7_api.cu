@@ -79,13 +79,22 @@ const char* wkv7_status_string(wkv7_status_t s) {
   return "unknown status";
 }
 
+// Checkpoint bytes (one fp32 64x64 state per head per 16 tokens), or -1 on overflow.
+int64_t checkpoint_bytes(const wkv7_desc_t* d, int64_t units) {
+  const int64_t nc = (d->T + 15) / 16;
+  int64_t n1, n2;
+  if (!mul_ok(units, nc, &n1) || !mul_ok(n1, 64 * 64 * 4, &n2)) return -1;
+  return n2;
+}
+
+// Workspace = checkpoints, then one int per (b,h) for the chunked backward's
+// "recompute this unit exactly" marks, rounded up to 16 bytes.
 size_t wkv7_workspace_bytes(const wkv7_desc_t* d) {
   int64_t units = 0, te = 0;
   if (check_desc(d, &units, &te) != WKV7_OK) return 0;
-  const int64_t nc = (d->T + 15) / 16;
-  int64_t n1, n2;
-  if (!mul_ok(units, nc, &n1) || !mul_ok(n1, 64 * 64 * 4, &n2)) return 0;
-  return static_cast<size_t>(n2);
+  const int64_t ck = checkpoint_bytes(d, units);
+  if (ck < 0 || d->T == 0) return 0;
+  return static_cast<size_t>(ck + ((units * 4 + 15) / 16) * 16);
 }
 
 wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
@@ -118,10 +127,17 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   if (st != WKV7_OK) return st;
   if (te > 0 && !workspace) return WKV7_ERR_WORKSPACE;
   if (units == 0) return WKV7_OK;
+  int* flags = d->T > 0 ? reinterpret_cast<int*>(static_cast<char*>(const_cast<void*>(workspace)) +
+                                                 checkpoint_bytes(d, units))
+                        : nullptr;
   wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
-                  dr, dw, dk, dv, da, db, ds0};
+                  dr, dw, dk, dv, da, db, ds0, flags};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, s));
+  if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, false, s));
+  // Chunked pass, then the exact scan for the units it marked (decays too small for 1/L scaling).
+  cudaError_t e = wkv7::launch_chunk_bwd(p, d->dtype, s);
+  if (e != cudaSuccess) return WKV7_ERR_CUDA;
+  return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, true, s));
 }
 
 wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,

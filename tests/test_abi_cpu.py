@@ -45,9 +45,11 @@ def test_version_and_status_strings(L):
 def test_workspace_matches_checkpoint_memory_on_rwkv_mlx_page(L):
     """RWKV-MLX page ("Key Design Decisions" 2): checkpoints every 16 tokens cost
     about 12 MB at the 184M-model layer shape (B=2, T=512, 12 heads of 64)."""
-    n = L.workspace_bytes(2, 512, 12)
-    assert n == 2 * 12 * (512 // 16) * 64 * 64 * 4 == 12_582_912
-    assert L.workspace_bytes(1, 17, 1) == 2 * 64 * 64 * 4        # ceil(17/16) = 2 checkpoints
+    ckpt = 2 * 12 * (512 // 16) * 64 * 64 * 4
+    assert ckpt == 12_582_912
+    # checkpoints, then one int per head (rounded up to 16 bytes) for the backward's marks
+    assert L.workspace_bytes(2, 512, 12) == ckpt + 96
+    assert L.workspace_bytes(1, 17, 1) == 2 * 64 * 64 * 4 + 16        # ceil(17/16) = 2 checkpoints
     assert L.workspace_bytes(1, 0, 1) == 0
 
 
