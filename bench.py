@@ -323,7 +323,8 @@ def main():
         fwd_gbs = BYTES_FWD_TRAIN * units / (fwd_avg / 1e3) / 1e9
         bwd_gbs = BYTES_BWD * units / (bwd_avg / 1e3) / 1e9
         dominant = ("bwd", bwd_avg, bwd_gbs, BYTES_BWD) if bwd_avg >= fwd_avg else ("fwd", fwd_avg, fwd_gbs, BYTES_FWD_TRAIN)
-        kname = {"fwd": "chunk_fwd" if args.algo != "scan" else "scan_fwd", "bwd": "scan_bwd"}[dominant[0]]
+        kname = {"fwd": "chunk_fwd" if args.algo != "scan" else "scan_fwd",
+                 "bwd": "chunk_bwd" if args.algo != "scan" else "scan_bwd"}[dominant[0]]
         traffic = kernel_traffic(kname, "packed_train_B8_T4096_H32")
         cpu = None
         if not args.no_cpu_baseline and world == 1:
