@@ -62,7 +62,8 @@ typedef enum {
   WKV7_ERR_WORKSPACE = 5,   /* backward without a checkpoint workspace                        */
   WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, non-zero flags, or T != 1 for a step   */
   WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
-  WKV7_ERR_TIMEOUT = 8      /* reserved for device-side bounded waits (see wkv7_device_status) */
+  WKV7_ERR_TIMEOUT = 8,     /* reserved for device-side bounded waits                          */
+  WKV7_ERR_SCRATCH_LIMIT = 9 /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
 } wkv7_status_t;
 
 typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
@@ -157,6 +158,36 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* desc, const void* r, const void* 
 wkv7_status_t wkv7_step(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
                         const void* v, const void* a, const void* b, float* state,
                         const uint8_t* active, void* y, void* stream);
+
+/*
+ * Forward + backward in one call, allocating nothing -- for callers that
+ * cannot call cudaMalloc (device memory owned by another allocator, such as
+ * a framework's caching allocator or a serving engine that reserves all free
+ * memory up front, or code paths where allocation is not allowed).  The
+ * pages have no counterpart to this entry point.
+ *
+ * Same arguments and results as wkv7_forward followed by wkv7_backward on
+ * the same descriptor, except that no workspace is passed: the checkpoints
+ * and the backward's per-head marks live in one fixed device array of the
+ * library, WKV7_NOALLOC_SCRATCH_BYTES bytes, which every GPU that loads the
+ * library holds until the process exits.  A problem whose
+ * wkv7_workspace_bytes() exceeds that size is rejected with
+ * WKV7_ERR_SCRATCH_LIMIT before anything is launched (32 MiB holds, e.g.,
+ * B=2, T=512, H=12, or B*H*ceil(T/16) <= 2047 checkpoints).
+ *
+ * The first call on a device looks up the array's device address for that
+ * device; make that first call before any stream capture.  All calls share
+ * the array and it keeps the last call's contents (nothing in it needs to
+ * start at zero), so calls that overlap on the GPU -- on different streams
+ * or different host threads -- race on it and must be serialised by the
+ * caller.
+ */
+#define WKV7_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+wkv7_status_t wkv7_train_step_noalloc(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
+                                      const void* v, const void* a, const void* b, const float* s0,
+                                      const uint8_t* reset, void* y, float* s_out, const void* dy,
+                                      const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
+                                      void* db, float* ds0, void* stream);
 
 #ifdef __cplusplus
 }

@@ -75,6 +75,7 @@ const char* wkv7_status_string(wkv7_status_t s) {
     case WKV7_ERR_UNSUPPORTED: return "unsupported head size, algorithm, flags or step length";
     case WKV7_ERR_CUDA: return "CUDA launch failed";
     case WKV7_ERR_TIMEOUT: return "device-side wait timed out";
+    case WKV7_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of wkv7_train_step_noalloc";
   }
   return "unknown status";
 }

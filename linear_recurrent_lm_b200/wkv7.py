@@ -25,7 +25,9 @@ import torch
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwkv7.so")
 
-OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT = range(9)
+(OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT,
+ ERR_SCRATCH_LIMIT) = range(10)
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2}
 N_HEAD = 64
@@ -67,6 +69,8 @@ def lib() -> ctypes.CDLL:
         L.wkv7_backward.argtypes = [dp] + [vp] * 19
         L.wkv7_step.restype = ctypes.c_int
         L.wkv7_step.argtypes = [dp] + [vp] * 10
+        L.wkv7_train_step_noalloc.restype = ctypes.c_int
+        L.wkv7_train_step_noalloc.argtypes = [dp] + [vp] * 20
         _lib = L
     return _lib
 
@@ -150,3 +154,27 @@ def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None):
     st = lib().wkv7_step(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, state, active, y)), _stream(stream))
     _check(st, "wkv7_step")
     return y
+
+
+def train_step_noalloc(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, *, y=None, s_out=None, grads=None,
+                       want_ds0: bool = True, algo: str = "auto", stream=None):
+    """Forward + backward with the library's fixed scratch instead of a workspace (nothing is
+    allocated by the library; outputs not given are allocated here by torch).  For callers that
+    cannot allocate device memory themselves: pass every output.  Returns (y, s_out, grads)."""
+    B, T, H = _token_shape(r)
+    if y is None:
+        y = torch.empty_like(r)
+    if s_out is None:
+        s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
+    g = dict(grads) if grads is not None else {}
+    for n in ("dr", "dw", "dk", "dv", "da", "db"):
+        if g.get(n) is None:
+            g[n] = torch.empty_like(r)
+    if g.get("ds0") is None and want_ds0:
+        g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
+    d = make_desc(B, T, H, r.dtype, algo)
+    st = lib().wkv7_train_step_noalloc(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, dy, dsT)),
+                                       *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
+                                       _stream(stream))
+    _check(st, "wkv7_train_step_noalloc")
+    return y, s_out, g

@@ -1,0 +1,84 @@
+"""wkv7_train_step_noalloc: forward + backward without any caller workspace.
+
+Some callers cannot call cudaMalloc -- their device memory belongs to another
+allocator (a framework's caching allocator, a serving engine that reserves all
+free memory up front) or they run where allocating is not allowed.  For them
+the library keeps the checkpoint scratch in a fixed device array.  This test
+calls that entry point through the C ABI, twice in a row on different inputs
+(the second call reuses the scratch the first one left behind), and compares
+every output with the regular wkv7_forward + wkv7_backward pair, within the
+tolerances the parity tests use.  It lives in its own file, collected last.
+"""
+from __future__ import annotations
+
+import ctypes
+
+import numpy as np
+import pytest
+
+from linear_recurrent_lm_b200 import inputs as I
+from tests.gpu_util import f64, to_dev
+from tests.metrics import cosine, err_rms, err_rms_excess
+
+pytestmark = pytest.mark.gpu
+
+GRADS = ("dr", "dw", "dk", "dv", "da", "db")
+
+
+def _case(seed, B, T, H):
+    rng = np.random.default_rng(seed)
+    d = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    dy = I.to_storage(rng.standard_normal((B, T, H, 64)), "bf16")
+    s0 = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    dsT = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    reset = np.zeros((B, T), np.uint8)
+    reset[0, T // 3] = 1
+    reset[B - 1, 0] = 1
+    return d, dy, s0, dsT, reset
+
+
+def _noalloc_call(W, xs, dy, s0, reset, dsT):
+    """Call the C entry point directly; every output buffer is the caller's."""
+    import torch
+    B, T, H = (int(s) for s in xs[0].shape[:3])
+    y = torch.empty_like(xs[0])
+    s_out = torch.empty((B, H, 64, 64), device=xs[0].device, dtype=torch.float32)
+    g = {n: torch.empty_like(xs[0]) for n in GRADS}
+    g["ds0"] = torch.empty((B, H, 64, 64), device=xs[0].device, dtype=torch.float32)
+    desc = W.make_desc(B, T, H, xs[0].dtype)
+    ptr = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+    st = W.lib().wkv7_train_step_noalloc(ctypes.byref(desc), *(ptr(x) for x in xs), ptr(s0), ptr(reset), ptr(y),
+                                         ptr(s_out), ptr(dy), ptr(dsT), *(ptr(g[n]) for n in GRADS), ptr(g["ds0"]),
+                                         ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+    assert st == W.OK, W.lib().wkv7_status_string(st)
+    return y, s_out, g
+
+
+def test_noalloc_matches_regular_entry_points_twice():
+    import torch
+    from linear_recurrent_lm_b200 import wkv7 as W
+    torch.cuda.set_device(0)
+    for seed, (B, T, H) in ((71, (2, 100, 3)), (72, (2, 512, 12))):
+        d, dy, s0, dsT, reset = _case(seed, B, T, H)
+        xs = [to_dev(d[n]) for n in I.NAMES]
+        dyd, s0d, dsTd, rd = to_dev(dy), to_dev(s0), to_dev(dsT), to_dev(reset)
+        y, s_out, g = _noalloc_call(W, xs, dyd, s0d, rd, dsTd)
+        torch.cuda.synchronize()
+        y_r, s_r, ws = W.forward(*xs, s0=s0d, reset=rd)
+        g_r = W.backward(*xs, dyd, ws, s0=s0d, reset=rd, dsT=dsTd)
+        torch.cuda.synchronize()
+        assert err_rms_excess(f64(y), f64(y_r), "bf16") <= 2e-2
+        assert err_rms(f64(s_out), f64(s_r)) <= 2e-2
+        for n in GRADS + ("ds0",):
+            assert cosine(f64(g[n]), f64(g_r[n])) >= 0.999, n
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    from linear_recurrent_lm_b200 import wkv7 as W
+    B, T, H = 8, 4096, 32                      # 1.07 GB of checkpoints, far above the fixed 32 MiB
+    assert W.workspace_bytes(B, T, H) > W.NOALLOC_SCRATCH_BYTES
+    desc = W.make_desc(B, T, H, __import__("torch").bfloat16)
+    fake = ctypes.c_void_p(0x10000)            # never dereferenced: the size check comes first
+    st = W.lib().wkv7_train_step_noalloc(ctypes.byref(desc), *([fake] * 6), None, None, fake, None, fake, None,
+                                         *([fake] * 6), None, None)
+    assert st == W.ERR_SCRATCH_LIMIT
