@@ -10,30 +10,31 @@
 // Unrolling it gives, for the 16 x 64 blocks SA (rows sa_t) and Y (rows y_t),
 //   (I - Lab) SA = At S0^T + Lak V,    Y = Rt S0^T + Mrb SA + Mrk V,
 // where Lab[t,tau] = at_t . bh_tau, Lak[t,tau] = at_t . kh_tau (tau < t) and
-// Mrb, Mrk are the same with rt_t (tau <= t).  Solving the unit lower
-// triangular system by substitution (the triangular solve the rwkv-lab page
-// names for chunked delta rules):
+// Mrb, Mrk are the same with rt_t (tau <= t).  With T = (I - Lab)^-1 (unit
+// lower triangular, by substitution -- the triangular solve the rwkv-lab page
+// names for chunked delta rules) and M = Mrb T:
 //   SA = W S0^T + X V,  Y = Q S0^T + Z V,
-//   W = (I - Lab)^-1 At,  X = (I - Lab)^-1 Lak,  Q = Rt + Mrb W,  Z = Mrb X + Mrk,
+//   W = T At,  X = T Lak,  Q = Rt + M At,  Z = Mrk + M Lak,
 //   S_16 = S0 diag(L_15) + (SA^T Bh + V^T Kh) diag(L_15).
 // Reset flags inside a chunk become masks: pairs (t, tau) separated by a
 // reset are dropped from Lab..Mrk, S0 only reaches tokens before the first
-// reset (rows of At, Rt masked), only the last segment feeds S_16, and S0
-// drops out of S_16 if the chunk holds any reset.
+// reset (At and Rt rows masked, i.e. columns of T and M), only the last
+// segment feeds S_16, and S0 drops out of S_16 if the chunk holds any reset.
 //
-// Precision: every product with an fp32 operand uses the 3-term bf16 split
-// (hi*hi + hi*lo + lo*hi, about 2^-16 relative); v enters exactly when the
-// inputs are bf16.  A chunk whose decay product leaves [2^-40, 2^40] (e.g.
-// w = 0) cannot use the 1/L scaling and is run token by token instead.
+// Precision: all products are tf32 mma.sync (m16n8k8) with fp32 accumulation;
+// operands are rounded to tf32 (nearest).  An emulation of exactly these
+// roundings against the fp64 oracle stays ~6x inside the bf16 tolerance.  A
+// chunk whose decay product leaves [2^-40, 2^40] (e.g. w = 0) cannot use the
+// 1/L scaling and is run token by token instead.
 //
-// Work split (one CTA of 8 warps per (b,h)):
-//   warps 0-3 ("state"): warp w owns rows 16w..16w+15 of S as mma
-//     accumulator fragments for the whole sequence; per chunk they do the
-//     two state products above, write y and the chunk-end checkpoint;
-//   warps 4-7 ("context"): meanwhile build everything the NEXT chunk's
-//     state products need (decay-scaled operands, Gram, W, X, Q, Z) into the
-//     other half of a double buffer, and stage the chunk after that with
-//     cp.async.
+// Work split (one CTA of 8 warps per (b,h)), pipelined over chunks:
+//   warps 4-7 ("context") for chunk c+1: stage the inputs (cp.async), build
+//     the decay-scaled operands, the masked Gram of [At; Rt] and [Bh; Kh] and
+//     T into one half of a double-buffered context;
+//   warps 0-3 ("state") for chunk c: warp w owns rows 16w..16w+15 of S as
+//     accumulator fragments for the whole sequence; they form W, X, M, Q, Z
+//     from the context, then the two state products, write y and the
+//     chunk-end checkpoint.
 // One CTA barrier per chunk hands the context over.
 #include <type_traits>
 
@@ -45,60 +46,42 @@ namespace wkv7 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStr = 72;    // padded row stride (elements) of 64-wide tiles: conflict-free ldmatrix
-constexpr int kStrS = 24;   // padded row stride of 16-wide tiles
-constexpr int kIn = 6;      // staged inputs: r, w, k, v, a, b
+constexpr int kIn = 6;       // staged inputs: r, w, k, v, a, b
+constexpr int kStrIn = 72;   // staged input row stride (elements)
+constexpr int S68 = 68, S72 = 72, S20 = 20, S24 = 24;
 using bf16 = __nv_bfloat16;
 
-// Everything the state warps need for one chunk.
+// Produced by the context warps for one chunk, consumed by the state warps one iteration later.
 struct __align__(16) Ctx {
-  bf16 Wh[kChunk][kStr], Wl[kChunk][kStr];   // W [t][j]
-  bf16 Qh[kChunk][kStr], Ql[kChunk][kStr];   // Q [t][j]
-  bf16 Bh[32][kStr], Bl[32][kStr];           // rows 0..15 bh_tau, 16..31 kh_tau  [tau][j]
-  bf16 Vh[kChunk][kStr], Vl[kChunk][kStr];   // v [tau][i]  (Vl unused for bf16 inputs)
-  bf16 Xh[kChunk][kStrS], Xl[kChunk][kStrS]; // X [t][tau]
-  bf16 Zh[kChunk][kStrS], Zl[kChunk][kStrS]; // Z [t][tau]
+  float Rt[kChunk][S68];    // m0 . rt  [t][j]   (fp32, initial value of Q)
+  float AtT[kN][S20];       // at       [j][tau]
+  float BhT[kN][S24];       // bh       [j][tau]
+  float KhT[kN][S20];       // kh       [j][tau]
+  float VT[kN][S20];        // v        [i][tau]
+  float Tm[kChunk][S20];    // T        [t][tau]
+  float TT[kChunk][S20];    // T^T      [tau][t]
+  float LakT[kChunk][S20];  // Lak^T    [tau][t]
+  float Mrb[kChunk][S20];   // Mrb      [t][tau]
+  float Mrk[kChunk][S20];   // Mrk      [t][tau] (fp32, initial value of Z)
   float lam15[kN];
-  int mask;     // reset bits of the chunk
-  int unsafe;   // decay product out of range: run this chunk token by token
+  int mask;                 // reset bits of the chunk
+  int unsafe;               // decay product out of range: run this chunk token by token
 };
 
 template <typename T>
-struct __align__(16) FwdSmem2 {
+struct __align__(16) FwdSmem3 {
   Ctx ctx[2];
-  T in[2][kIn][kChunk][kStr];                 // staged inputs of two chunks
-  bf16 GAh[32][kStr], GAl[32][kStr];          // rows 0..15 at_t, 16..31 rt_t
-  __align__(16) float LT[4][kChunk][20];      // masked Gram blocks, transposed [tau][t]: Lab, Lak, Mrb, Mrk
-  bf16 Mrbh[kChunk][kStrS], Mrbl[kChunk][kStrS];
-  float ybuf[kChunk][kN + 4];
-  int kmask;
+  float GA[32][S68];        // rows 0..15 at_t, 16..31 rt_t   [t][j]
+  float GB[32][S68];        // rows 0..15 bh_t, 16..31 kh_t   [tau][j]
+  __align__(16) float LabT[kChunk][S20];
+  float W[kChunk][S72], Q[kChunk][S72];      // [t][j]
+  float X[kChunk][S20], Z[kChunk][S20], M[kChunk][S20];
+  T in[kIn][kChunk][kStrIn];                 // staged inputs of the chunk being built
   int kbad[4];
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
-}
-
-template <typename T>
-__device__ __forceinline__ float2 ld2(const T* p);
-template <>
-__device__ __forceinline__ float2 ld2<bf16>(const bf16* p) {
-  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
-}
-template <>
-__device__ __forceinline__ float2 ld2<__half>(const __half* p) {
-  return __half22float2(*reinterpret_cast<const __half2*>(p));
-}
-template <>
-__device__ __forceinline__ float2 ld2<float>(const float* p) {
-  return *reinterpret_cast<const float2*>(p);
-}
-
-__device__ __forceinline__ void st_split2(bf16* hi, bf16* lo, float x0, float x1) {
-  uint32_t h, l;
-  split2(x0, x1, h, l);
-  *reinterpret_cast<uint32_t*>(hi) = h;
-  *reinterpret_cast<uint32_t*>(lo) = l;
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -107,35 +90,32 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-// Keep only the bf16 halves of an A fragment whose k index is set in `keep_bits`.
-__device__ __forceinline__ void mask_a_k(uint32_t (&a)[4], int c4, unsigned keep_bits) {
-  const int k0 = 2 * c4, k1 = 8 + 2 * c4;
-  const uint32_t m0 = ((keep_bits >> k0) & 1u ? 0x0000ffffu : 0u) | ((keep_bits >> (k0 + 1)) & 1u ? 0xffff0000u : 0u);
-  const uint32_t m1 = ((keep_bits >> k1) & 1u ? 0x0000ffffu : 0u) | ((keep_bits >> (k1 + 1)) & 1u ? 0xffff0000u : 0u);
-  a[0] &= m0;
-  a[1] &= m0;
-  a[2] &= m1;
-  a[3] &= m1;
+// Keep the A-fragment entries of a natural-k fragment (k = 8s+c and 8s+c+4) whose bit is set.
+__device__ __forceinline__ void mask_nat(uint32_t (&a)[4], int s, int c4, unsigned bits) {
+  const bool k0 = (bits >> (8 * s + c4)) & 1u, k1 = (bits >> (8 * s + c4 + 4)) & 1u;
+  if (!k0) { a[0] = 0u; a[1] = 0u; }
+  if (!k1) { a[2] = 0u; a[3] = 0u; }
 }
 
 template <typename T>
-__device__ __forceinline__ void stage_chunk(const FwdArgs& p, T (*dst)[kChunk][kStr], int64_t b, int64_t h,
+__device__ __forceinline__ void stage_chunk(const FwdArgs& p, T (*dst)[kChunk][kStrIn], int64_t b, int64_t h,
                                             int64_t t0, int len, int ktid) {
   constexpr int n = Vec16<T>::n;
   constexpr int VPT = kN / n;
   const T* src[kIn] = {static_cast<const T*>(p.r), static_cast<const T*>(p.w), static_cast<const T*>(p.k),
                        static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b)};
-  for (int idx = ktid; idx < kIn * kChunk * VPT; idx += 128) {
-    const int m = idx / (kChunk * VPT);
-    const int rem = idx - m * kChunk * VPT;
-    const int tt = rem / VPT, vec = rem - (rem / VPT) * VPT;
-    T* s = &dst[m][tt][vec * n];
-    if (tt < len) {
-      cp_async16(s, src[m] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * n);
-    } else {   // padding token: w = 1, everything else 0 -> leaves the state unchanged
-      const T fill = Elt<T>::from_f32(m == 1 ? 1.f : 0.f);
 #pragma unroll
-      for (int e = 0; e < n; ++e) s[e] = fill;
+  for (int m = 0; m < kIn; ++m) {
+    for (int idx = ktid; idx < kChunk * VPT; idx += 128) {
+      const int tt = idx / VPT, vec = idx - (idx / VPT) * VPT;
+      T* s = &dst[m][tt][vec * n];
+      if (tt < len) {
+        cp_async16(s, src[m] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * n);
+      } else {   // padding token: w = 1, everything else 0 -> leaves the state unchanged
+        const T fill = Elt<T>::from_f32(m == 1 ? 1.f : 0.f);
+#pragma unroll
+        for (int e = 0; e < n; ++e) s[e] = fill;
+      }
     }
   }
   cp_async_commit();
@@ -143,64 +123,51 @@ __device__ __forceinline__ void stage_chunk(const FwdArgs& p, T (*dst)[kChunk][k
 
 // ------------------------------------------------------------------ context warps
 template <typename T>
-__device__ __forceinline__ void build_context(FwdSmem2<T>& sm, Ctx& cx, const T (*X)[kChunk][kStr], unsigned mask,
-                                              int ktid) {
-  constexpr bool kVExact = std::is_same<T, bf16>::value;
+__device__ __forceinline__ void build_context(const FwdArgs& p, FwdSmem3<T>& sm, Ctx& cx, unsigned mask, int64_t b,
+                                              int64_t h, int64_t c, int64_t nc, int ktid) {
   const int kw = ktid >> 5, lane = ktid & 31;
   const int g = lane >> 2, c4 = lane & 3;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
+  const T (*X)[kChunk][kStrIn] = sm.in;
 
-  // ---- K1: decay products and the decay-scaled operands (hi/lo bf16)
+  // ---- K1: decay products and decay-scaled operands; thread = (column j, token half)
   bool bad = false;
   {
-    const int j = 2 * lane;   // this thread's column pair
-    float la[kChunk], lb[kChunk];
-    float l0 = 1.f, l1 = 1.f;
+    const int j = ktid & 63, half = ktid >> 6;
+    float lam[kChunk];
+    float l = 1.f;
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) {
-      const float2 w2 = ld2<T>(&X[1][t][j]);
-      l0 *= w2.x;
-      l1 *= w2.y;
-      la[t] = l0;
-      lb[t] = l1;
-      bad |= !(l0 >= 0x1p-40f && l0 <= 0x1p40f && l1 >= 0x1p-40f && l1 <= 0x1p40f);
+      l *= Elt<T>::to_f32(X[1][t][j]);
+      lam[t] = l;
+      bad |= !(l >= 0x1p-40f && l <= 0x1p40f);
     }
-    if (kw == 0) {            // at_t = a_t L_{t-1}
-      float p0 = 1.f, p1 = 1.f;
 #pragma unroll
-      for (int t = 0; t < kChunk; ++t) {
-        const float2 a2 = ld2<T>(&X[4][t][j]);
-        st_split2(&sm.GAh[t][j], &sm.GAl[t][j], a2.x * p0, a2.y * p1);
-        p0 = la[t];
-        p1 = lb[t];
-      }
-    } else if (kw == 1) {     // rt_t = r_t L_t
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) {
-        const float2 r2 = ld2<T>(&X[0][t][j]);
-        st_split2(&sm.GAh[16 + t][j], &sm.GAl[16 + t][j], r2.x * la[t], r2.y * lb[t]);
-      }
-    } else if (kw == 2) {     // bh_t = b_t / L_t ; L_15
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) {
-        const float2 b2 = ld2<T>(&X[5][t][j]);
-        st_split2(&cx.Bh[t][j], &cx.Bl[t][j], b2.x * rcp_approx(la[t]), b2.y * rcp_approx(lb[t]));
-      }
-      cx.lam15[j] = la[kChunk - 1];
-      cx.lam15[j + 1] = lb[kChunk - 1];
-    } else {                  // kh_t = k_t / L_t ; v
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) {
-        const float2 k2 = ld2<T>(&X[2][t][j]);
-        st_split2(&cx.Bh[16 + t][j], &cx.Bl[16 + t][j], k2.x * rcp_approx(la[t]), k2.y * rcp_approx(lb[t]));
-        if constexpr (kVExact) {
-          *reinterpret_cast<uint32_t*>(&cx.Vh[t][j]) = *reinterpret_cast<const uint32_t*>(&X[3][t][j]);
-        } else {
-          const float2 v2 = ld2<T>(&X[3][t][j]);
-          st_split2(&cx.Vh[t][j], &cx.Vl[t][j], v2.x, v2.y);
-        }
-      }
+    for (int tp = 0; tp < 8; tp += 2) {
+      const int t = 8 * half + tp;
+      const float lp0 = t > 0 ? lam[t - 1] : 1.f, l0 = lam[t], l1 = lam[t + 1];
+      const float i0 = rcp_approx(l0), i1 = rcp_approx(l1);
+      const float at0 = Elt<T>::to_f32(X[4][t][j]) * lp0, at1 = Elt<T>::to_f32(X[4][t + 1][j]) * l0;
+      const float rt0 = Elt<T>::to_f32(X[0][t][j]) * l0, rt1 = Elt<T>::to_f32(X[0][t + 1][j]) * l1;
+      const float bh0 = Elt<T>::to_f32(X[5][t][j]) * i0, bh1 = Elt<T>::to_f32(X[5][t + 1][j]) * i1;
+      const float kh0 = Elt<T>::to_f32(X[2][t][j]) * i0, kh1 = Elt<T>::to_f32(X[2][t + 1][j]) * i1;
+      const float v0 = Elt<T>::to_f32(X[3][t][j]), v1 = Elt<T>::to_f32(X[3][t + 1][j]);
+      sm.GA[t][j] = tf32f(at0);
+      sm.GA[t + 1][j] = tf32f(at1);
+      sm.GA[16 + t][j] = tf32f(rt0);
+      sm.GA[16 + t + 1][j] = tf32f(rt1);
+      sm.GB[t][j] = tf32f(bh0);
+      sm.GB[t + 1][j] = tf32f(bh1);
+      sm.GB[16 + t][j] = tf32f(kh0);
+      sm.GB[16 + t + 1][j] = tf32f(kh1);
+      cx.Rt[t][j] = t < fr ? rt0 : 0.f;
+      cx.Rt[t + 1][j] = t + 1 < fr ? rt1 : 0.f;
+      *reinterpret_cast<float2*>(&cx.AtT[j][t]) = make_float2(tf32f(at0), tf32f(at1));
+      *reinterpret_cast<float2*>(&cx.BhT[j][t]) = make_float2(tf32f(bh0), tf32f(bh1));
+      *reinterpret_cast<float2*>(&cx.KhT[j][t]) = make_float2(tf32f(kh0), tf32f(kh1));
+      *reinterpret_cast<float2*>(&cx.VT[j][t]) = make_float2(tf32f(v0), tf32f(v1));
     }
+    if (half == 0) cx.lam15[j] = lam[kChunk - 1];
   }
   const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
   if (lane == 0) sm.kbad[kw] = any_bad ? 1 : 0;
@@ -210,25 +177,25 @@ __device__ __forceinline__ void build_context(FwdSmem2<T>& sm, Ctx& cx, const T 
     cx.mask = int(mask);
     cx.unsafe = unsafe ? 1 : 0;
   }
+
+  // the staged inputs are consumed: fetch the next chunk while the rest is built
+  if (c + 1 < nc) {
+    const int64_t t1 = (c + 1) * kChunk;
+    stage_chunk<T>(p, sm.in, b, h, t1, int(min64(kChunk, p.T - t1)), ktid);
+  }
   if (unsafe) return;
 
-  // ---- K2: 32x32 Gram of [at; rt] and [bh; kh] on tensor cores (3-term split), masked
+  // ---- K2: 32x32 Gram of [at; rt] and [bh; kh] (tf32), masked
   {
     const int m0 = (kw >> 1) * 16, n0 = (kw & 1) * 16;
     float gr[2][4] = {};
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t ah[4], al[4], bh[4], bl[4];
-      ldsm_x4(ah, a_rowmajor_addr(&sm.GAh[0][0], kStr, m0, 16 * ks, lane));
-      ldsm_x4(al, a_rowmajor_addr(&sm.GAl[0][0], kStr, m0, 16 * ks, lane));
-      ldsm_x4(bh, b_nmajor_addr(&cx.Bh[0][0], kStr, n0, 16 * ks, lane));
-      ldsm_x4(bl, b_nmajor_addr(&cx.Bl[0][0], kStr, n0, 16 * ks, lane));
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        mma16816(gr[nt], al, bh[2 * nt], bh[2 * nt + 1]);
-        mma16816(gr[nt], ah, bl[2 * nt], bl[2 * nt + 1]);
-        mma16816(gr[nt], ah, bh[2 * nt], bh[2 * nt + 1]);
-      }
+    for (int ks = 0; ks < 8; ++ks) {
+      uint32_t a[4], bb[4];
+      ldsm_x4(a, a32_addr(&sm.GA[0][0], S68, m0, 8 * ks, lane));
+      ldsm_x4(bb, b32_2n_addr(&sm.GB[0][0], S68, n0, 8 * ks, lane));
+      mma1688(gr[0], a, bb[0], bb[1]);
+      mma1688(gr[1], a, bb[2], bb[3]);
     }
     const bool strict = kw < 2;   // Lab, Lak strictly lower; Mrb, Mrk include the diagonal
 #pragma unroll
@@ -240,31 +207,23 @@ __device__ __forceinline__ void build_context(FwdSmem2<T>& sm, Ctx& cx, const T 
         bool ok = strict ? (tau < t) : (tau <= t);
         ok = ok && ((mask & ((2u << t) - (2u << tau))) == 0u);   // no reset in (tau, t]
         const float v = ok ? gr[nt][e] : 0.f;
-        sm.LT[kw][tau][t] = v;
-        if (kw == 2) split1(v, sm.Mrbh[t][tau], sm.Mrbl[t][tau]);
+        if (kw == 0) sm.LabT[tau][t] = v;
+        else if (kw == 1) cx.LakT[tau][t] = tf32f(v);
+        else if (kw == 2) cx.Mrb[t][tau] = tf32f(v);
+        else cx.Mrk[t][tau] = v;
       }
   }
   named_bar(1, 128);
 
-  // ---- K3: W = (I - Lab)^-1 diag(m0) At (threads 0..63), X = (I - Lab)^-1 Lak (threads 64..79)
-  if (ktid < 80) {
+  // ---- K3: T = (I - Lab)^-1 by forward substitution, one column per lane (warp kw == 0)
+  if (kw == 0 && lane < kChunk) {
+    const int cc = lane;
     float u[kChunk];
-    const int cc = ktid < 64 ? ktid : ktid - 64;
-    if (ktid < 64) {
 #pragma unroll
-      for (int t = 0; t < kChunk; ++t)
-        u[t] = t < fr ? __bfloat162float(sm.GAh[t][cc]) + __bfloat162float(sm.GAl[t][cc]) : 0.f;
-    } else {
-      const float4* col = reinterpret_cast<const float4*>(&sm.LT[1][cc][0]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 f = col[q];
-        u[4 * q] = f.x; u[4 * q + 1] = f.y; u[4 * q + 2] = f.z; u[4 * q + 3] = f.w;
-      }
-    }
+    for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
 #pragma unroll
     for (int tau = 0; tau < kChunk - 1; ++tau) {
-      const float4* lrow = reinterpret_cast<const float4*>(&sm.LT[0][tau][0]);
+      const float4* lrow = reinterpret_cast<const float4*>(&sm.LabT[tau][0]);
       float lv[kChunk];
 #pragma unroll
       for (int q = (tau + 1) / 4; q < 4; ++q) {
@@ -274,185 +233,218 @@ __device__ __forceinline__ void build_context(FwdSmem2<T>& sm, Ctx& cx, const T 
 #pragma unroll
       for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
     }
-    if (ktid < 64) {
 #pragma unroll
-      for (int t = 0; t < kChunk; ++t) split1(u[t], cx.Wh[t][cc], cx.Wl[t][cc]);
-    } else {
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) split1(u[t], cx.Xh[t][cc], cx.Xl[t][cc]);
-    }
-  }
-  named_bar(1, 128);
-
-  // ---- K4: Q = m0.Rt + Mrb W (columns 16kw..16kw+15), Z = Mrk + Mrb X (warp kw == 0)
-  {
-    uint32_t mh[4], ml[4];
-    ldsm_x4(mh, a_rowmajor_addr(&sm.Mrbh[0][0], kStrS, 0, 0, lane));
-    ldsm_x4(ml, a_rowmajor_addr(&sm.Mrbl[0][0], kStrS, 0, 0, lane));
-    const int j0 = 16 * kw;
-    float q[2][4];
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int t = g + 8 * hh;
-        const int j = j0 + 8 * nt + 2 * c4;
-        float2 r2 = make_float2(0.f, 0.f);
-        if (t < fr) {
-          const float2 h2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sm.GAh[16 + t][j]));
-          const float2 l2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&sm.GAl[16 + t][j]));
-          r2 = make_float2(h2.x + l2.x, h2.y + l2.y);
-        }
-        q[nt][2 * hh] = r2.x;
-        q[nt][2 * hh + 1] = r2.y;
-      }
-    uint32_t wh[4], wl[4];
-    ldsm_x4_t(wh, b_kmajor_addr(&cx.Wh[0][0], kStr, 0, j0, lane));
-    ldsm_x4_t(wl, b_kmajor_addr(&cx.Wl[0][0], kStr, 0, j0, lane));
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      mma16816(q[nt], ml, wh[2 * nt], wh[2 * nt + 1]);
-      mma16816(q[nt], mh, wl[2 * nt], wl[2 * nt + 1]);
-      mma16816(q[nt], mh, wh[2 * nt], wh[2 * nt + 1]);
-    }
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        st_split2(&cx.Qh[g + 8 * hh][j0 + 8 * nt + 2 * c4], &cx.Ql[g + 8 * hh][j0 + 8 * nt + 2 * c4],
-                  q[nt][2 * hh], q[nt][2 * hh + 1]);
-    if (kw == 0) {
-      float z[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) z[nt][e] = sm.LT[3][8 * nt + 2 * c4 + (e & 1)][g + 8 * (e >> 1)];
-      uint32_t xh[4], xl[4];
-      ldsm_x4_t(xh, b_kmajor_addr(&cx.Xh[0][0], kStrS, 0, 0, lane));
-      ldsm_x4_t(xl, b_kmajor_addr(&cx.Xl[0][0], kStrS, 0, 0, lane));
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        mma16816(z[nt], ml, xh[2 * nt], xh[2 * nt + 1]);
-        mma16816(z[nt], mh, xl[2 * nt], xl[2 * nt + 1]);
-        mma16816(z[nt], mh, xh[2 * nt], xh[2 * nt + 1]);
-      }
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-          st_split2(&cx.Zh[g + 8 * hh][8 * nt + 2 * c4], &cx.Zl[g + 8 * hh][8 * nt + 2 * c4], z[nt][2 * hh],
-                    z[nt][2 * hh + 1]);
+    for (int t = 0; t < kChunk; ++t) {
+      const float v = tf32f(u[t]);
+      cx.Tm[t][cc] = v;
+      cx.TT[cc][t] = v;
     }
   }
 }
 
 // ------------------------------------------------------------------ state warps
 template <typename T>
-__device__ __forceinline__ void state_chunk(FwdSmem2<T>& sm, const Ctx& cx, float (&acc)[8][4], int warp, int lane) {
-  constexpr bool kVExact = std::is_same<T, bf16>::value;
+__device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, const Ctx& cx, float (&acc)[8][4],
+                                            int64_t b, int64_t h, int64_t t0, int len, int warp, int lane) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
+  const int j0 = 16 * warp;
   const unsigned mask = unsigned(cx.mask);
-  // SA^T, Y^T (rows i, columns t) = S0 [W^T | Q^T] + V^T [X^T | Z^T]
+  const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
+  const unsigned m0bits = (1u << fr) - 1u;   // tokens that S0 reaches
+
+  // ---- step a: W = T diag(m0) At (columns j0..j0+15), M = Mrb T (warp 0), X = T Lak (warp 1)
+  uint32_t bat[2][4];   // At^T fragments of this warp's columns: [n-tile][k-step pair]
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) ldsm_x4(bat[nt], b32_2k_addr(&cx.AtT[0][0], S20, j0 + 8 * nt, 0, lane));
+  {
+    uint32_t at[2][4];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) ldsm_x4(at[s], a32_addr(&cx.Tm[0][0], S20, 0, 8 * s, lane));
+    if (warp == 1) {   // X = T Lak (unmasked T)
+      float xx[2][4] = {};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bl[4];
+        ldsm_x4(bl, b32_2k_addr(&cx.LakT[0][0], S20, 8 * nt, 0, lane));
+        mma1688(xx[nt], at[0], bl[0], bl[1]);
+        mma1688(xx[nt], at[1], bl[2], bl[3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<float2*>(&sm.X[g + 8 * hh][8 * nt + 2 * c4]) =
+              make_float2(tf32f(xx[nt][2 * hh]), tf32f(xx[nt][2 * hh + 1]));
+    }
+    mask_nat(at[0], 0, c4, m0bits);
+    mask_nat(at[1], 1, c4, m0bits);
+    float ww[2][4] = {};
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      mma1688(ww[nt], at[0], bat[nt][0], bat[nt][1]);
+      mma1688(ww[nt], at[1], bat[nt][2], bat[nt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        *reinterpret_cast<float2*>(&sm.W[g + 8 * hh][j0 + 8 * nt + 2 * c4]) =
+            make_float2(tf32f(ww[nt][2 * hh]), tf32f(ww[nt][2 * hh + 1]));
+    if (warp == 0) {   // M = Mrb T
+      uint32_t am[2][4];
+#pragma unroll
+      for (int s = 0; s < 2; ++s) ldsm_x4(am[s], a32_addr(&cx.Mrb[0][0], S20, 0, 8 * s, lane));
+      float mm[2][4] = {};
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bt[4];
+        ldsm_x4(bt, b32_2k_addr(&cx.TT[0][0], S20, 8 * nt, 0, lane));
+        mma1688(mm[nt], am[0], bt[0], bt[1]);
+        mma1688(mm[nt], am[1], bt[2], bt[3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<float2*>(&sm.M[g + 8 * hh][8 * nt + 2 * c4]) =
+              make_float2(tf32f(mm[nt][2 * hh]), tf32f(mm[nt][2 * hh + 1]));
+    }
+  }
+  named_bar(2, 128);
+
+  // ---- step b: Q = m0.Rt + M diag(m0) At (columns j0..j0+15), Z = Mrk + M Lak (warp 2)
+  {
+    uint32_t am[2][4];
+#pragma unroll
+    for (int s = 0; s < 2; ++s) ldsm_x4(am[s], a32_addr(&sm.M[0][0], S20, 0, 8 * s, lane));
+    if (warp == 2) {
+      float zz[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+          const float2 m2 = *reinterpret_cast<const float2*>(&cx.Mrk[g + 8 * hh][8 * nt + 2 * c4]);
+          zz[nt][2 * hh] = m2.x;
+          zz[nt][2 * hh + 1] = m2.y;
+        }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        uint32_t bl[4];
+        ldsm_x4(bl, b32_2k_addr(&cx.LakT[0][0], S20, 8 * nt, 0, lane));
+        mma1688(zz[nt], am[0], bl[0], bl[1]);
+        mma1688(zz[nt], am[1], bl[2], bl[3]);
+      }
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<float2*>(&sm.Z[g + 8 * hh][8 * nt + 2 * c4]) =
+              make_float2(tf32f(zz[nt][2 * hh]), tf32f(zz[nt][2 * hh + 1]));
+    }
+    mask_nat(am[0], 0, c4, m0bits);
+    mask_nat(am[1], 1, c4, m0bits);
+    float qq[2][4];
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const float2 r2 = *reinterpret_cast<const float2*>(&cx.Rt[g + 8 * hh][j0 + 8 * nt + 2 * c4]);
+        qq[nt][2 * hh] = r2.x;
+        qq[nt][2 * hh + 1] = r2.y;
+      }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) {
+      mma1688(qq[nt], am[0], bat[nt][0], bat[nt][1]);
+      mma1688(qq[nt], am[1], bat[nt][2], bat[nt][3]);
+    }
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh)
+        *reinterpret_cast<float2*>(&sm.Q[g + 8 * hh][j0 + 8 * nt + 2 * c4]) =
+            make_float2(tf32f(qq[nt][2 * hh]), tf32f(qq[nt][2 * hh + 1]));
+  }
+  named_bar(2, 128);
+
+  // ---- S1: SA^T, Y^T (rows i, columns t) = S0 [W^T | Q^T] + V^T [X^T | Z^T]
   float sa[2][4] = {}, yy[2][4] = {};
 #pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    uint32_t ah[4], al[4];
-    split2(acc[2 * ks][0], acc[2 * ks][1], ah[0], al[0]);
-    split2(acc[2 * ks][2], acc[2 * ks][3], ah[1], al[1]);
-    split2(acc[2 * ks + 1][0], acc[2 * ks + 1][1], ah[2], al[2]);
-    split2(acc[2 * ks + 1][2], acc[2 * ks + 1][3], ah[3], al[3]);
-    uint32_t wh[4], wl[4], qh[4], ql[4];
-    ldsm_x4(wh, b_nmajor_addr(&cx.Wh[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(wl, b_nmajor_addr(&cx.Wl[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(qh, b_nmajor_addr(&cx.Qh[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(ql, b_nmajor_addr(&cx.Ql[0][0], kStr, 0, 16 * ks, lane));
+  for (int ks = 0; ks < 8; ++ks) {
+    uint32_t a[4] = {to_tf32(acc[ks][0]), to_tf32(acc[ks][2]), to_tf32(acc[ks][1]), to_tf32(acc[ks][3])};
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt) {
-      mma16816(sa[nt], al, wh[2 * nt], wh[2 * nt + 1]);
-      mma16816(sa[nt], ah, wl[2 * nt], wl[2 * nt + 1]);
-      mma16816(sa[nt], ah, wh[2 * nt], wh[2 * nt + 1]);
-      mma16816(yy[nt], al, qh[2 * nt], qh[2 * nt + 1]);
-      mma16816(yy[nt], ah, ql[2 * nt], ql[2 * nt + 1]);
-      mma16816(yy[nt], ah, qh[2 * nt], qh[2 * nt + 1]);
+      const uint2 wb = *reinterpret_cast<const uint2*>(&sm.W[8 * nt + g][8 * ks + 2 * c4]);
+      const uint2 qb = *reinterpret_cast<const uint2*>(&sm.Q[8 * nt + g][8 * ks + 2 * c4]);
+      mma1688(sa[nt], a, wb.x, wb.y);
+      mma1688(yy[nt], a, qb.x, qb.y);
     }
   }
-  uint32_t vh[4], vl[4] = {0u, 0u, 0u, 0u};
-  ldsm_x4_t(vh, a_kmajor_addr(&cx.Vh[0][0], kStr, 0, row0, lane));
-  if constexpr (!kVExact) ldsm_x4_t(vl, a_kmajor_addr(&cx.Vl[0][0], kStr, 0, row0, lane));
+  uint32_t av[2][4];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) ldsm_x4(av[s], a32_addr(&cx.VT[0][0], S20, row0, 8 * s, lane));
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    uint32_t xb[4], zb[4];
+    ldsm_x4(xb, b32_2k_addr(&sm.X[0][0], S20, 8 * nt, 0, lane));
+    ldsm_x4(zb, b32_2k_addr(&sm.Z[0][0], S20, 8 * nt, 0, lane));
+    mma1688(sa[nt], av[0], xb[0], xb[1]);
+    mma1688(sa[nt], av[1], xb[2], xb[3]);
+    mma1688(yy[nt], av[0], zb[0], zb[1]);
+    mma1688(yy[nt], av[1], zb[2], zb[3]);
+  }
   {
-    uint32_t xh[4], xl[4], zh[4], zl[4];
-    ldsm_x4(xh, b_nmajor_addr(&cx.Xh[0][0], kStrS, 0, 0, lane));
-    ldsm_x4(xl, b_nmajor_addr(&cx.Xl[0][0], kStrS, 0, 0, lane));
-    ldsm_x4(zh, b_nmajor_addr(&cx.Zh[0][0], kStrS, 0, 0, lane));
-    ldsm_x4(zl, b_nmajor_addr(&cx.Zl[0][0], kStrS, 0, 0, lane));
+    T* y = static_cast<T*>(p.y);
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      mma16816(sa[nt], vh, xl[2 * nt], xl[2 * nt + 1]);
-      mma16816(sa[nt], vh, xh[2 * nt], xh[2 * nt + 1]);
-      mma16816(yy[nt], vh, zl[2 * nt], zl[2 * nt + 1]);
-      mma16816(yy[nt], vh, zh[2 * nt], zh[2 * nt + 1]);
-      if constexpr (!kVExact) {
-        mma16816(sa[nt], vl, xh[2 * nt], xh[2 * nt + 1]);
-        mma16816(yy[nt], vl, zh[2 * nt], zh[2 * nt + 1]);
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int t = 8 * nt + 2 * c4 + (e & 1);
+        if (t < len) y[tok_off(b, t0 + t, h, p.T, p.H) + row0 + g + 8 * (e >> 1)] = Elt<T>::from_f32(yy[nt][e]);
       }
-    }
   }
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-    for (int e = 0; e < 4; ++e) sm.ybuf[8 * nt + 2 * c4 + (e & 1)][row0 + g + 8 * (e >> 1)] = yy[nt][e];
 
-  // S_16 = keep.S0 diag(L_15) + (SA^T Bh + V^T Kh) diag(L_15); only the last segment's tokens
-  // contribute.  The products go to a separate accumulator so that S0 is scaled exactly and
-  // never added to the (1/L-sized) intermediate terms.
+  // ---- S3: S_16 = keep.S0 diag(L_15) + (SA^T Bh + V^T Kh) diag(L_15), last segment only
   const unsigned seg_last = __popc(mask & 0xfffeu);
   unsigned last_bits = 0u;
 #pragma unroll
   for (int t = 0; t < kChunk; ++t) last_bits |= (unsigned(__popc(mask & ((2u << t) - 2u))) == seg_last ? 1u : 0u) << t;
   const float keep = mask == 0u ? 1.f : 0.f;
-  uint32_t sh[4], sl[4];
-  split2(sa[0][0], sa[0][1], sh[0], sl[0]);
-  split2(sa[0][2], sa[0][3], sh[1], sl[1]);
-  split2(sa[1][0], sa[1][1], sh[2], sl[2]);
-  split2(sa[1][2], sa[1][3], sh[3], sl[3]);
-  if (last_bits != 0xffffu) {
-    mask_a_k(sh, c4, last_bits);
-    mask_a_k(sl, c4, last_bits);
-    mask_a_k(vh, c4, last_bits);
-    mask_a_k(vl, c4, last_bits);
+  uint32_t asa[2][4];
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const int k0 = 8 * s + 2 * c4;   // permuted k: a0,a1 <-> k0, a2,a3 <-> k0 + 1
+    const bool e0 = (last_bits >> k0) & 1u, e1 = (last_bits >> (k0 + 1)) & 1u;
+    asa[s][0] = e0 ? to_tf32(sa[s][0]) : 0u;
+    asa[s][1] = e0 ? to_tf32(sa[s][2]) : 0u;
+    asa[s][2] = e1 ? to_tf32(sa[s][1]) : 0u;
+    asa[s][3] = e1 ? to_tf32(sa[s][3]) : 0u;
+    mask_nat(av[s], s, c4, last_bits);
   }
 #pragma unroll
-  for (int np = 0; np < 4; ++np) {
-    uint32_t bbh[4], bbl[4], kbh[4], kbl[4];
-    ldsm_x4_t(bbh, b_kmajor_addr(&cx.Bh[0][0], kStr, 0, 16 * np, lane));
-    ldsm_x4_t(bbl, b_kmajor_addr(&cx.Bl[0][0], kStr, 0, 16 * np, lane));
-    ldsm_x4_t(kbh, b_kmajor_addr(&cx.Bh[0][0], kStr, 16, 16 * np, lane));
-    ldsm_x4_t(kbl, b_kmajor_addr(&cx.Bl[0][0], kStr, 16, 16 * np, lane));
+  for (int jt = 0; jt < 8; ++jt) {
+    float d[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int u = 0; u < 2; ++u) {
-      float d[4] = {0.f, 0.f, 0.f, 0.f};
-      mma16816(d, sl, bbh[2 * u], bbh[2 * u + 1]);
-      mma16816(d, sh, bbl[2 * u], bbl[2 * u + 1]);
-      mma16816(d, sh, bbh[2 * u], bbh[2 * u + 1]);
-      mma16816(d, vh, kbl[2 * u], kbl[2 * u + 1]);
-      mma16816(d, vh, kbh[2 * u], kbh[2 * u + 1]);
-      if constexpr (!kVExact) mma16816(d, vl, kbh[2 * u], kbh[2 * u + 1]);
-      const int nt = 2 * np + u;
-      const float2 l2 = *reinterpret_cast<const float2*>(&cx.lam15[8 * nt + 2 * c4]);
-      acc[nt][0] = fmaf(keep * acc[nt][0], l2.x, d[0] * l2.x);
-      acc[nt][1] = fmaf(keep * acc[nt][1], l2.y, d[1] * l2.y);
-      acc[nt][2] = fmaf(keep * acc[nt][2], l2.x, d[2] * l2.x);
-      acc[nt][3] = fmaf(keep * acc[nt][3], l2.y, d[3] * l2.y);
+    for (int s = 0; s < 2; ++s) {
+      const uint2 bb = *reinterpret_cast<const uint2*>(&cx.BhT[8 * jt + g][8 * s + 2 * c4]);
+      mma1688(d, asa[s], bb.x, bb.y);
     }
+    uint32_t kb[4];
+    ldsm_x4(kb, b32_2k_addr(&cx.KhT[0][0], S20, 8 * jt, 0, lane));
+    mma1688(d, av[0], kb[0], kb[1]);
+    mma1688(d, av[1], kb[2], kb[3]);
+    const float2 l2 = *reinterpret_cast<const float2*>(&cx.lam15[8 * jt + 2 * c4]);
+    acc[jt][0] = fmaf(keep * acc[jt][0], l2.x, d[0] * l2.x);
+    acc[jt][1] = fmaf(keep * acc[jt][1], l2.y, d[1] * l2.y);
+    acc[jt][2] = fmaf(keep * acc[jt][2], l2.x, d[2] * l2.x);
+    acc[jt][3] = fmaf(keep * acc[jt][3], l2.y, d[3] * l2.y);
   }
 }
 
 // Token-by-token update of one chunk on the state fragments (decay out of range), inputs read from global.
 template <typename T>
-__device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, FwdSmem2<T>& sm, unsigned mask,
-                                                   float (&acc)[8][4], int64_t b, int64_t h, int64_t t0, int len,
-                                                   int warp, int lane) {
+__device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned mask, float (&acc)[8][4], int64_t b,
+                                                   int64_t h, int64_t t0, int len, int warp, int lane) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
   const T* R = static_cast<const T*>(p.r);
@@ -461,6 +453,7 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, FwdSmem2<T>
   const T* V = static_cast<const T*>(p.v);
   const T* A = static_cast<const T*>(p.a);
   const T* Bb = static_cast<const T*>(p.b);
+  T* y = static_cast<T*>(p.y);
   for (int tt = 0; tt < len; ++tt) {
     const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H);
     if ((mask >> tt) & 1u) {
@@ -500,8 +493,8 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, FwdSmem2<T>
     y_hi += __shfl_xor_sync(0xffffffffu, y_hi, 1);
     y_hi += __shfl_xor_sync(0xffffffffu, y_hi, 2);
     if (c4 == 0) {
-      sm.ybuf[tt][row0 + g] = y_lo;
-      sm.ybuf[tt][row0 + g + 8] = y_hi;
+      y[o + row0 + g] = Elt<T>::from_f32(y_lo);
+      y[o + row0 + g + 8] = Elt<T>::from_f32(y_hi);
     }
   }
 }
@@ -509,7 +502,7 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, FwdSmem2<T>
 template <typename T>
 __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  FwdSmem2<T>& sm = *reinterpret_cast<FwdSmem2<T>*>(smem_raw);
+  FwdSmem3<T>& sm = *reinterpret_cast<FwdSmem3<T>*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
@@ -517,11 +510,11 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
   const bool is_state = warp < 4;
   const int ktid = tid - 128;
   const int64_t nc = (p.T + kChunk - 1) / kChunk;
+  const int g = lane >> 2, c4 = lane & 3;
+  const int row0 = 16 * warp;
 
   // state fragments: acc[nt][e] = S[16*warp + g + 8*(e>>1)][8*nt + 2*c4 + (e&1)]
   float acc[8][4];
-  const int g = lane >> 2, c4 = lane & 3;
-  const int row0 = 16 * warp;
   if (is_state) {
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
@@ -535,14 +528,12 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
   }
 
   // prologue: the context warps stage chunk 0 and fetch its reset flags
-  unsigned reset_bits_next = 0u;
+  unsigned reset_bits = 0u;
   if (!is_state) {
-    stage_chunk<T>(p, sm.in[0], b, h, 0, int(min64(kChunk, p.T)), ktid);
-    if (warp == 4) {
-      const int len0 = int(min64(kChunk, p.T));
-      const bool f = p.reset && lane < len0 && p.reset[b * p.T + lane] != 0;
-      reset_bits_next = __ballot_sync(0xffffffffu, f) & 0xffffu;
-    }
+    stage_chunk<T>(p, sm.in, b, h, 0, int(min64(kChunk, p.T)), ktid);
+    const int len0 = int(min64(kChunk, p.T));
+    const bool f = p.reset && lane < len0 && p.reset[b * p.T + lane] != 0;
+    reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
     cp_async_wait_all();
   }
   __syncthreads();
@@ -551,19 +542,14 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
     if (!is_state) {
       if (it < nc) {
         const int64_t c = it;
-        const int buf = int(c & 1);
-        if (warp == 4 && lane == 0) sm.kmask = int(reset_bits_next);
-        if (c + 1 < nc) {
+        const unsigned mask = reset_bits;
+        if (c + 1 < nc) {   // reset flags of the next chunk (used next iteration)
           const int64_t t1 = (c + 1) * kChunk;
           const int len1 = int(min64(kChunk, p.T - t1));
-          stage_chunk<T>(p, sm.in[buf ^ 1], b, h, t1, len1, ktid);
-          if (warp == 4) {
-            const bool f = p.reset && lane < len1 && p.reset[b * p.T + t1 + lane] != 0;
-            reset_bits_next = __ballot_sync(0xffffffffu, f) & 0xffffu;
-          }
+          const bool f = p.reset && lane < len1 && p.reset[b * p.T + t1 + lane] != 0;
+          reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
         }
-        named_bar(1, 128);
-        build_context<T>(sm, sm.ctx[buf], sm.in[buf], unsigned(sm.kmask), ktid);
+        build_context<T>(p, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid);
         cp_async_wait_all();
       }
     } else if (it >= 1) {
@@ -572,9 +558,9 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
       const int64_t t0 = c * kChunk;
       const int len = int(min64(kChunk, p.T - t0));
       if (!cx.unsafe) {
-        state_chunk<T>(sm, cx, acc, warp, lane);
+        state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane);
       } else {
-        state_chunk_tokens<T>(p, sm, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
+        state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
       }
       if (p.ckpt) {
         float* base = p.ckpt + (unit * nc + c) * kN * kN;
@@ -585,20 +571,8 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
             *reinterpret_cast<float2*>(base + (row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
                 make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
       }
-      named_bar(2, 128);   // ybuf complete
-      T* y = static_cast<T*>(p.y);
-      for (int e = tid; e < len * 8; e += 128) {
-        const int tt = e >> 3, part = e & 7;
-        alignas(16) T vals[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) vals[u] = Elt<T>::from_f32(sm.ybuf[tt][part * 8 + u]);
-        uint4* dst = reinterpret_cast<uint4*>(y + tok_off(b, t0 + tt, h, p.T, p.H) + part * 8);
-        const uint4* sv = reinterpret_cast<const uint4*>(vals);
-#pragma unroll
-        for (int u = 0; u < int(sizeof(vals) / 16); ++u) dst[u] = sv[u];
-      }
     }
-    __syncthreads();   // context of chunk it handed to the state warps; staged inputs rotate
+    __syncthreads();   // context of chunk it handed to the state warps
   }
 
   if (is_state && p.s_out) {
@@ -613,7 +587,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
 
 template <typename T>
 cudaError_t launch(const FwdArgs& p, cudaStream_t stream) {
-  const size_t smem = sizeof(FwdSmem2<T>);
+  const size_t smem = sizeof(FwdSmem3<T>);
   cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   chunk_fwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p);

@@ -12,9 +12,11 @@ from tests.metrics import err_rms, err_rms_excess
 pytestmark = pytest.mark.gpu
 
 TOL = {"f32": 1e-4, "bf16": 2e-2, "f16": 5e-3}
-# The tensor-core path represents each fp32 operand as two bf16 halves (~2^-17 relative), so on
-# fp32 inputs it lands near the 1e-4 bound (AUTO runs fp32 inputs on the exact-fp32 scan).
-TOL_CHUNKED_F32 = 2.5e-4
+# The tensor-core path computes its products in tf32 (operands rounded to 11 significant bits,
+# fp32 accumulation): on fp32 inputs it cannot reach the 1e-4 bound, which is why AUTO runs fp32
+# inputs on the exact-fp32 scan.  An emulation of the same roundings puts its error near 4e-3
+# of RMS; the explicit CHUNKED path on fp32 inputs is held to 1e-2.
+TOL_CHUNKED_F32 = 1e-2
 ALGOS = ("scan", "chunked")
 
 
