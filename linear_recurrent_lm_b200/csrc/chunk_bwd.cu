@@ -67,6 +67,7 @@ struct __align__(16) BCtx {
   bf16 Tb[kChunk][kStrS], Mrbb[kChunk][kStrS], Mrkb[kChunk][kStrS], Lakb[kChunk][kStrS];   // [t][tau]
   float lam[kChunk][kN + 4];   // L_t [t][j]
   int mask, unsafe;
+  unsigned ls_bits;            // tokens of the chunk's last segment
 };
 
 template <typename T>
@@ -80,9 +81,9 @@ struct __align__(16) BwdSmem2 {
   bf16 dSb[kN][kStr];         // dS16 [i][j]
   bf16 dG[32][kStrG];         // [dMrb dMrk; dLab dLak]
   bf16 dVs[kChunk][kStr];     // dv staging [tau][i]
-  float DL[kChunk][kN + 4];   // d log L_t without the chunk-end term
-  float e3[kN];
-  float dlam[4][kN];
+  __align__(16) float DL[kChunk][kN + 4];   // d log L_t without the chunk-end term
+  __align__(16) float e3[kN];
+  __align__(16) float dlam[4][kN];
   int kbad[4];
   int stop;
 };
@@ -123,13 +124,14 @@ __device__ __forceinline__ void stage7(const BwdArgs& p, T (*dst)[kChunk][kStr],
   const T* src[kIn] = {static_cast<const T*>(p.r), static_cast<const T*>(p.w), static_cast<const T*>(p.k),
                        static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b),
                        static_cast<const T*>(p.dy)};
+  for (int idx = ktid; idx < kChunk * VPT; idx += 128) {
+    const int tt = idx / VPT, vec = idx - (idx / VPT) * VPT;
+    const int64_t off = tok_off(b, t0 + tt, h, p.T, p.H) + vec * n;
 #pragma unroll
-  for (int m = 0; m < kIn; ++m) {
-    for (int idx = ktid; idx < kChunk * VPT; idx += 128) {
-      const int tt = idx / VPT, vec = idx - (idx / VPT) * VPT;
+    for (int m = 0; m < kIn; ++m) {
       T* s = &dst[m][tt][vec * n];
       if (tt < len) {
-        cp_async16(s, src[m] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * n);
+        cp_async16(s, src[m] + off);
       } else {   // padding token: w = 1, everything else (dy included) 0
         const T fill = Elt<T>::from_f32(m == 1 ? 1.f : 0.f);
 #pragma unroll
@@ -162,32 +164,42 @@ __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm,
   const int kw = ktid >> 5, lane = ktid & 31;
   const T (*X)[kChunk][kStr] = sm.in;
 
-  // ---- K1: decay products, scaled operands, v/dy copies, entering state in bf16
+  // ---- K1: decay products, scaled operands, v/dy copies, entering state in bf16.
+  // Thread = (column pair 2jp, 2jp+1; token quarter kw), two columns per packed fp32 op.
   bool bad = false;
   {
-    const int j = ktid & 63, half = ktid >> 6;
-    float lam[kChunk];
-    float l = 1.f;
+    const int j = 2 * lane, t0 = 4 * kw;
+    // L_{t0-1}: product of the earlier quarters' decays (warp-uniform trip count)
+    float2 lam = make_float2(1.f, 1.f);
+    for (int t = 0; t < t0; ++t) lam = mul2(lam, load2(&X[1][t][j]));
+    float2 wmin = make_float2(1.f, 1.f), lmin = make_float2(1.f, 1.f), lmax = lmin;
 #pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float w = Elt<T>::to_f32(X[1][t][j]);
-      l *= w;
-      lam[t] = l;
-      bad |= !(w >= 0.0625f && l >= 0x1p-40f && l <= 0x1p40f);
+    for (int u = 0; u < 4; ++u) {
+      const int t = t0 + u;
+      const float2 lp = lam, w2 = load2(&X[1][t][j]);
+      lam = mul2(lam, w2);
+      wmin = make_float2(fminf(wmin.x, w2.x), fminf(wmin.y, w2.y));
+      lmin = make_float2(fminf(lmin.x, lam.x), fminf(lmin.y, lam.y));
+      lmax = make_float2(fmaxf(lmax.x, lam.x), fmaxf(lmax.y, lam.y));
+      const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
+      const float2 at = mul2(load2(&X[4][t][j]), lp), rt = mul2(load2(&X[0][t][j]), lam);
+      const float2 bh = mul2(load2(&X[5][t][j]), inv), kh = mul2(load2(&X[2][t][j]), inv);
+      *reinterpret_cast<float2*>(&cx.lam[t][j]) = lam;
+      *reinterpret_cast<uint32_t*>(&cx.GA[t][j]) = pack_bf16(at.x, at.y);
+      *reinterpret_cast<uint32_t*>(&cx.GA[16 + t][j]) = pack_bf16(rt.x, rt.y);
+      *reinterpret_cast<uint32_t*>(&cx.GB[t][j]) = pack_bf16(bh.x, bh.y);
+      *reinterpret_cast<uint32_t*>(&cx.GB[16 + t][j]) = pack_bf16(kh.x, kh.y);
+      if constexpr (std::is_same<T, bf16>::value) {
+        *reinterpret_cast<uint32_t*>(&cx.Vb[t][j]) = *reinterpret_cast<const uint32_t*>(&X[3][t][j]);
+        *reinterpret_cast<uint32_t*>(&cx.DYb[t][j]) = *reinterpret_cast<const uint32_t*>(&X[6][t][j]);
+      } else {
+        const float2 v2 = load2(&X[3][t][j]), d2 = load2(&X[6][t][j]);
+        *reinterpret_cast<uint32_t*>(&cx.Vb[t][j]) = pack_bf16(v2.x, v2.y);
+        *reinterpret_cast<uint32_t*>(&cx.DYb[t][j]) = pack_bf16(d2.x, d2.y);
+      }
     }
-#pragma unroll
-    for (int tt = 0; tt < 8; ++tt) {
-      const int t = 8 * half + tt;
-      const float lp = t > 0 ? lam[t - 1] : 1.f, lt = lam[t];
-      const float inv = rcp_approx(lt);
-      cx.lam[t][j] = lt;
-      cx.GA[t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[4][t][j]) * lp);
-      cx.GA[16 + t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[0][t][j]) * lt);
-      cx.GB[t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[5][t][j]) * inv);
-      cx.GB[16 + t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[2][t][j]) * inv);
-      cx.Vb[t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[3][t][j]));
-      cx.DYb[t][j] = __float2bfloat16_rn(Elt<T>::to_f32(X[6][t][j]));
-    }
+    // every L_t of the chunk lies in exactly one quarter, so the CTA-wide ballot sees all of them
+    bad = !(fminf(wmin.x, wmin.y) >= 0.0625f && fminf(lmin.x, lmin.y) >= 0x1p-40f && fmaxf(lmax.x, lmax.y) <= 0x1p40f);
     const int row = ktid >> 1, col0 = (ktid & 1) * 32;
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
@@ -204,6 +216,7 @@ __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm,
   if (ktid == 0) {
     cx.mask = int(mask);
     cx.unsafe = unsafe ? 1 : 0;
+    cx.ls_bits = last_segment_bits(mask);
   }
 }
 
@@ -226,14 +239,14 @@ __device__ __forceinline__ void finish_context(BwdSmem2<T>& sm, BCtx& cx, unsign
       mma16816(gr[1], a, bb[2], bb[3]);
     }
     const bool strict = kw < 2;
+    const int st0 = seg_of(mask, g), st1 = seg_of(mask, g + 8);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int t = g + (e >> 1) * 8;
         const int tau = 8 * nt + 2 * c4 + (e & 1);
-        bool ok = strict ? (tau < t) : (tau <= t);
-        ok = ok && ((mask & ((2u << t) - (2u << tau))) == 0u);
+        const bool ok = (strict ? (tau < t) : (tau <= t)) && seg_of(mask, tau) == ((e >> 1) ? st1 : st0);
         const float v = ok ? gr[nt][e] : 0.f;
         if (kw == 0) sm.LabT[tau][t] = v;
         else if (kw == 1) { sm.LakT[tau][t] = v; cx.Lakb[t][tau] = __float2bfloat16_rn(v); }
@@ -323,19 +336,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
   const unsigned m0bits = (1u << fr) - 1u;
   const bool keep = mask == 0u;
-  const unsigned seg_last = __popc(mask & 0xfffeu);
-  unsigned ls_bits = 0u;
-#pragma unroll
-  for (int t = 0; t < kChunk; ++t) ls_bits |= (unsigned(__popc(mask & ((2u << t) - 2u))) == seg_last ? 1u : 0u) << t;
-
-  // L_15 for this thread's dS columns 8nt + 2c4 + {0,1}
-  float l15[8][2];
-#pragma unroll
-  for (int nt = 0; nt < 8; ++nt) {
-    const float2 v = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][8 * nt + 2 * c4]);
-    l15[nt][0] = v.x;
-    l15[nt][1] = v.y;
-  }
+  const unsigned ls_bits = cx.ls_bits;
 
   // ---- M1: [dSA^T | dV^T] = dSl [ls.Bh | ls.Kh]^T + dY^T [Mrb | Mrk]   (rows i of this warp)
   float acc4[4][4] = {};
@@ -343,11 +344,13 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
     const bool ls_lo = (ls_bits >> g) & 1u, ls_hi = (ls_bits >> (8 + g)) & 1u;
 #pragma unroll
     for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4];
-      a[0] = pack_bf16(dS[2 * ks][0] * l15[2 * ks][0], dS[2 * ks][1] * l15[2 * ks][1]);
-      a[1] = pack_bf16(dS[2 * ks][2] * l15[2 * ks][0], dS[2 * ks][3] * l15[2 * ks][1]);
-      a[2] = pack_bf16(dS[2 * ks + 1][0] * l15[2 * ks + 1][0], dS[2 * ks + 1][1] * l15[2 * ks + 1][1]);
-      a[3] = pack_bf16(dS[2 * ks + 1][2] * l15[2 * ks + 1][0], dS[2 * ks + 1][3] * l15[2 * ks + 1][1]);
+      const float2 la = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][16 * ks + 2 * c4]);
+      const float2 lb = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][16 * ks + 8 + 2 * c4]);
+      const float2 p0 = mul2(make_float2(dS[2 * ks][0], dS[2 * ks][1]), la);
+      const float2 p1 = mul2(make_float2(dS[2 * ks][2], dS[2 * ks][3]), la);
+      const float2 p2 = mul2(make_float2(dS[2 * ks + 1][0], dS[2 * ks + 1][1]), lb);
+      const float2 p3 = mul2(make_float2(dS[2 * ks + 1][2], dS[2 * ks + 1][3]), lb);
+      uint32_t a[4] = {pack_bf16(p0.x, p0.y), pack_bf16(p1.x, p1.y), pack_bf16(p2.x, p2.y), pack_bf16(p3.x, p3.y)};
       uint32_t bb[4], bk[4];
       ldsm_x4(bb, b_nmajor_addr(&cx.GB[0][0], kStr, 0, 16 * ks, lane));
       ldsm_x4(bk, b_nmajor_addr(&cx.GB[0][0], kStr, 16, 16 * ks, lane));
@@ -399,8 +402,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
       const int col = 8 * nt + 2 * c4;
       float2 s_lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.S0b[row0 + g][col]));
       float2 s_hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.S0b[row0 + g + 8][col]));
-      part[2 * nt] = s_lo.x * dS[nt][0] + s_hi.x * dS[nt][2];
-      part[2 * nt + 1] = s_lo.y * dS[nt][1] + s_hi.y * dS[nt][3];
+      const float2 pr = fma2(s_lo, make_float2(dS[nt][0], dS[nt][1]), mul2(s_hi, make_float2(dS[nt][2], dS[nt][3])));
+      part[2 * nt] = pr.x;
+      part[2 * nt + 1] = pr.y;
       *reinterpret_cast<uint32_t*>(&sm.dSb[row0 + g][col]) = pack_bf16(dS[nt][0], dS[nt][1]);
       *reinterpret_cast<uint32_t*>(&sm.dSb[row0 + g + 8][col]) = pack_bf16(dS[nt][2], dS[nt][3]);
     }
@@ -433,12 +437,17 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
 
   // ---- M5: gradient entering the chunk: keep.dSl + (m0.dY)^T Rt + (m0.dU)^T At
   {
+    if (keep) {
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      dS[nt][0] = keep ? dS[nt][0] * l15[nt][0] : 0.f;
-      dS[nt][1] = keep ? dS[nt][1] * l15[nt][1] : 0.f;
-      dS[nt][2] = keep ? dS[nt][2] * l15[nt][0] : 0.f;
-      dS[nt][3] = keep ? dS[nt][3] * l15[nt][1] : 0.f;
+      for (int nt = 0; nt < 8; ++nt) {
+        const float2 l = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][8 * nt + 2 * c4]);
+        const float2 u0 = mul2(make_float2(dS[nt][0], dS[nt][1]), l);
+        const float2 u1 = mul2(make_float2(dS[nt][2], dS[nt][3]), l);
+        dS[nt][0] = u0.x; dS[nt][1] = u0.y; dS[nt][2] = u1.x; dS[nt][3] = u1.y;
+      }
+    } else {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt) dS[nt][0] = dS[nt][1] = dS[nt][2] = dS[nt][3] = 0.f;
     }
     uint32_t ay[4], au[4];
     ldsm_x4_t(ay, a_kmajor_addr(&cx.DYb[0][0], kStr, 0, row0, lane));
@@ -485,14 +494,14 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
       mma16816(gr[1], a, bb[2], bb[3]);
     }
     const bool strict = (warp >> 1) != 0;
+    const int st0 = seg_of(mask, g), st1 = seg_of(mask, g + 8);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int t = g + (e >> 1) * 8;
         const int tau = 8 * nt + 2 * c4 + (e & 1);
-        bool ok = strict ? (tau < t) : (tau <= t);
-        ok = ok && ((mask & ((2u << t) - (2u << tau))) == 0u);
+        const bool ok = (strict ? (tau < t) : (tau <= t)) && seg_of(mask, tau) == ((e >> 1) ? st1 : st0);
         sm.dG[(warp >> 1) * 16 + t][(warp & 1) * 16 + tau] = __float2bfloat16_rn(ok ? gr[nt][e] : 0.f);
       }
   }
@@ -542,9 +551,10 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
     T* gdr = static_cast<T*>(p.dr);
     T* gdb = static_cast<T*>(p.db);
     T* gdk = static_cast<T*>(p.dk);
-    float e2v[2][2][2];   // [nt][hh][q]
-    float e1v[2][2][2];
-    float e3p[2][2] = {};
+    float2 e2v[2][2];   // [nt][hh], columns j, j+1
+    float2 e1v[2][2];
+    float2 e3p[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+    const float2 zero2 = make_float2(0.f, 0.f);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       const int t = g + 8 * hh;
@@ -554,74 +564,82 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         const int j = j0 + 8 * nt + 2 * c4;
-        const float2 Lt2 = *reinterpret_cast<const float2*>(&cx.lam[t][j]);
-        const float2 Lp2 = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
+        const int e = 2 * hh;
+        const float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[t][j]);
+        const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
         const float2 L15 = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]);
-        const float2 At2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[t][j]));
-        const float2 Rt2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[16 + t][j]));
-        const float2 Bh2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[t][j]));
-        const float2 Kh2 = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[16 + t][j]));
-        float oda[2], odr[2], odb[2], odk[2];
-#pragma unroll
-        for (int q = 0; q < 2; ++q) {
-          const int e = 2 * hh + q;
-          const float Lt = q ? Lt2.y : Lt2.x, Lp = q ? Lp2.y : Lp2.x, L = q ? L15.y : L15.x;
-          const float at = q ? At2.y : At2.x, rt = q ? Rt2.y : Rt2.x;
-          const float bh = q ? Bh2.y : Bh2.x, kh = q ? Kh2.y : Kh2.x;
-          const float dAt = dA[nt][e] + (m0t ? xa[nt][e] : 0.f);
-          const float dRt = dR[nt][e] + (m0t ? xr[nt][e] : 0.f);
-          const float dBt = dB[nt][e] + (ls ? L * xb[nt][e] : 0.f);
-          const float dKt = dK[nt][e] + (ls ? L * xk[nt][e] : 0.f);
-          const float inv = rcp_approx(Lt);
-          oda[q] = dAt * Lp;
-          odr[q] = dRt * Lt;
-          odb[q] = dBt * inv;
-          odk[q] = dKt * inv;
-          e1v[nt][hh][q] = dRt * rt - dBt * bh - dKt * kh;
-          e2v[nt][hh][q] = dAt * at;
-          if (ls) e3p[nt][q] += (xb[nt][e] * bh + xk[nt][e] * kh) * L;
-        }
+        const float2 at = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[t][j]));
+        const float2 rt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[16 + t][j]));
+        const float2 bh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[t][j]));
+        const float2 kh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[16 + t][j]));
+        const float2 xb2 = ls ? make_float2(xb[nt][e], xb[nt][e + 1]) : zero2;
+        const float2 xk2 = ls ? make_float2(xk[nt][e], xk[nt][e + 1]) : zero2;
+        const float2 dAt = add2(make_float2(dA[nt][e], dA[nt][e + 1]), m0t ? make_float2(xa[nt][e], xa[nt][e + 1]) : zero2);
+        const float2 dRt = add2(make_float2(dR[nt][e], dR[nt][e + 1]), m0t ? make_float2(xr[nt][e], xr[nt][e + 1]) : zero2);
+        const float2 dBt = fma2(L15, xb2, make_float2(dB[nt][e], dB[nt][e + 1]));
+        const float2 dKt = fma2(L15, xk2, make_float2(dK[nt][e], dK[nt][e + 1]));
+        const float2 inv = make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y));
+        e1v[nt][hh] = sub2(mul2(dRt, rt), fma2(dBt, bh, mul2(dKt, kh)));
+        e2v[nt][hh] = mul2(dAt, at);
+        e3p[nt] = fma2(fma2(xb2, bh, mul2(xk2, kh)), L15, e3p[nt]);
         if (t < len) {
-          gda[orow + j] = Elt<T>::from_f32(oda[0]); gda[orow + j + 1] = Elt<T>::from_f32(oda[1]);
-          gdr[orow + j] = Elt<T>::from_f32(odr[0]); gdr[orow + j + 1] = Elt<T>::from_f32(odr[1]);
-          gdb[orow + j] = Elt<T>::from_f32(odb[0]); gdb[orow + j + 1] = Elt<T>::from_f32(odb[1]);
-          gdk[orow + j] = Elt<T>::from_f32(odk[0]); gdk[orow + j + 1] = Elt<T>::from_f32(odk[1]);
+          store2(gda + orow + j, mul2(dAt, Lp));
+          store2(gdr + orow + j, mul2(dRt, Lt));
+          store2(gdb + orow + j, mul2(dBt, inv));
+          store2(gdk + orow + j, mul2(dKt, inv));
         }
       }
     }
     // d log L_t = E1_t + E2_{t+1}: E2 of row t+1 lives in lane+4 (same half) or, for row 7, in lane c4 (upper half)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int nt = 0; nt < 2; ++nt) {
+      float2 dn0, up0, dn1;
+      dn0.x = __shfl_down_sync(0xffffffffu, e2v[nt][0].x, 4);
+      dn0.y = __shfl_down_sync(0xffffffffu, e2v[nt][0].y, 4);
+      up0.x = __shfl_sync(0xffffffffu, e2v[nt][1].x, c4);
+      up0.y = __shfl_sync(0xffffffffu, e2v[nt][1].y, c4);
+      dn1.x = __shfl_down_sync(0xffffffffu, e2v[nt][1].x, 4);
+      dn1.y = __shfl_down_sync(0xffffffffu, e2v[nt][1].y, 4);
+      const int j = j0 + 8 * nt + 2 * c4;
+      *reinterpret_cast<float2*>(&sm.DL[g][j]) = add2(e1v[nt][0], g < 7 ? dn0 : up0);
+      *reinterpret_cast<float2*>(&sm.DL[g + 8][j]) = add2(e1v[nt][1], g < 7 ? dn1 : make_float2(0.f, 0.f));
+      float2 v = e3p[nt];
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const float dn0 = __shfl_down_sync(0xffffffffu, e2v[nt][0][q], 4);
-        const float up0 = __shfl_sync(0xffffffffu, e2v[nt][1][q], c4);
-        const float dn1 = __shfl_down_sync(0xffffffffu, e2v[nt][1][q], 4);
-        const int j = j0 + 8 * nt + 2 * c4 + q;
-        sm.DL[g][j] = e1v[nt][0][q] + (g < 7 ? dn0 : up0);
-        sm.DL[g + 8][j] = e1v[nt][1][q] + (g < 7 ? dn1 : 0.f);
-        float v = e3p[nt][q];
-        v += __shfl_xor_sync(0xffffffffu, v, 4);
-        v += __shfl_xor_sync(0xffffffffu, v, 8);
-        v += __shfl_xor_sync(0xffffffffu, v, 16);
-        if (g == 0) sm.e3[j] = v;
+      for (int o = 4; o < 32; o <<= 1) {
+        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
+        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
       }
+      if (g == 0) *reinterpret_cast<float2*>(&sm.e3[j]) = v;
+    }
   }
   named_bar(2, 128);   // DL, e3 complete
 
-  // ---- M11: dw = (reverse cumulative sum of d log L) / w, one column per thread
-  if (tid < kN) {
-    const int j = tid;
-    float fin = sm.e3[j];
-    if (keep) fin += cx.lam[kChunk - 1][j] * ((sm.dlam[0][j] + sm.dlam[1][j]) + (sm.dlam[2][j] + sm.dlam[3][j]));
-    T* gdw = static_cast<T*>(p.dw);
-    float cum = fin;
+  // ---- M11: dw = (reverse cumulative sum of d log L) / w.  Thread = (column pair, token half);
+  // the lower half adds the upper half's rows itself instead of waiting for it.
+  {
+    const int j = 2 * (tid & 31), th = tid >> 5;   // warps 0 and 1: token halves 0..7 and 8..15
+    if (th < 2) {
+      const int tlo = th ? 8 : 0;
+      float2 cum = *reinterpret_cast<const float2*>(&sm.e3[j]);
+      if (keep) {
+        const float2 d01 = add2(*reinterpret_cast<const float2*>(&sm.dlam[0][j]), *reinterpret_cast<const float2*>(&sm.dlam[1][j]));
+        const float2 d23 = add2(*reinterpret_cast<const float2*>(&sm.dlam[2][j]), *reinterpret_cast<const float2*>(&sm.dlam[3][j]));
+        cum = fma2(*reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]), add2(d01, d23), cum);
+      }
+      if (!th) {
 #pragma unroll
-    for (int t = kChunk - 1; t >= 0; --t) {
-      cum += sm.DL[t][j];
-      if (t < len) {
-        const float Lt = cx.lam[t][j], Lp = t > 0 ? cx.lam[t - 1][j] : 1.f;
-        gdw[tok_off(b, t0 + t, h, p.T, p.H) + j] = Elt<T>::from_f32(cum * Lp * rcp_approx(Lt));
+        for (int t = 8; t < kChunk; ++t) cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
+      }
+      T* gdw = static_cast<T*>(p.dw) + tok_off(b, t0, h, p.T, p.H) + j;
+      const int64_t rs = p.H * kN;
+      float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[tlo + 7][j]);
+#pragma unroll
+      for (int u = 7; u >= 0; --u) {
+        const int t = tlo + u;
+        cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
+        const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
+        if (t < len) store2(gdw + t * rs, mul2(cum, mul2(Lp, make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y)))));
+        Lt = Lp;
       }
     }
   }

@@ -27,6 +27,20 @@ template <> struct Elt<__half> {
   static __device__ __forceinline__ __half from_f32(float x) { return __float2half_rn(x); }
 };
 
+// Two adjacent elements of T (4- or 8-byte aligned) as fp32.
+__device__ __forceinline__ float2 load2(const float* p) { return *reinterpret_cast<const float2*>(p); }
+__device__ __forceinline__ float2 load2(const __nv_bfloat16* p) {
+  return __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(p));
+}
+__device__ __forceinline__ float2 load2(const __half* p) { return __half22float2(*reinterpret_cast<const __half2*>(p)); }
+
+// Store two fp32 values as adjacent elements of T (round to nearest).
+__device__ __forceinline__ void store2(float* p, float2 v) { *reinterpret_cast<float2*>(p) = v; }
+__device__ __forceinline__ void store2(__nv_bfloat16* p, float2 v) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(v.x, v.y);
+}
+__device__ __forceinline__ void store2(__half* p, float2 v) { *reinterpret_cast<__half2*>(p) = __floats2half2_rn(v.x, v.y); }
+
 // Number of elements of T in one 16-byte vector.
 template <typename T> struct Vec16 { static constexpr int n = 16 / sizeof(T); };
 
@@ -51,6 +65,54 @@ __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return
 // Offset (in elements) of x[b][t][h][0] in a [B,T,H,64] tensor.
 __device__ __forceinline__ int64_t tok_off(int64_t b, int64_t t, int64_t h, int64_t T, int64_t H) {
   return ((b * T + t) * H + h) * kN;
+}
+
+}  // namespace wkv7
+
+namespace wkv7 {
+
+// ------------------------------------------------------------------ packed fp32 pairs (sm_100 f32x2)
+// One instruction operates on two adjacent fp32 values; on sm_100a this issues half the
+// instructions of the scalar form at the same arithmetic throughput.
+__device__ __forceinline__ unsigned long long f2_pack(float2 v) {
+  unsigned long long r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(v.x), "f"(v.y));
+  return r;
+}
+__device__ __forceinline__ float2 f2_unpack(unsigned long long r) {
+  float2 v;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(v.x), "=f"(v.y) : "l"(r));
+  return v;
+}
+__device__ __forceinline__ float2 fma2(float2 a, float2 b, float2 c) {
+  unsigned long long d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)), "l"(f2_pack(c)));
+  return f2_unpack(d);
+}
+__device__ __forceinline__ float2 mul2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(d);
+}
+__device__ __forceinline__ float2 add2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(d);
+}
+__device__ __forceinline__ float2 sub2(float2 a, float2 b) {
+  unsigned long long d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(f2_pack(a)), "l"(f2_pack(b)));
+  return f2_unpack(d);
+}
+
+// Segment index of token t inside a chunk: number of resets among tokens 1..t.
+__device__ __forceinline__ int seg_of(unsigned mask, int t) { return __popc(mask & ((2u << t) - 2u)); }
+
+// Bits of the tokens that belong to the chunk's last segment.
+__device__ __forceinline__ unsigned last_segment_bits(unsigned mask) {
+  if (!(mask & 0xfffeu)) return 0xffffu;
+  const int last = 31 - __clz(mask & 0xfffeu);   // start of the last segment
+  return 0xffffu & ~((1u << last) - 1u);
 }
 
 }  // namespace wkv7
