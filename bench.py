@@ -20,8 +20,8 @@ import json
 import os
 import re
 import statistics
-import subprocess
 import sys
+import threading
 import time
 
 import numpy as np
@@ -73,54 +73,71 @@ def kernel_traffic(kernel: str, workload: str):
 
 
 class Clocks:
-    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
-    FIELDS = "clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown," \
-             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown," \
-             "clocks_event_reasons.sw_power_cap"
+    """Samples the SM clock and the clock-event (throttle) reasons through NVML every few
+    milliseconds on a background thread.  Only samples taken between mark_start() and
+    mark_end() -- the timed region -- are summarised; reading clocks changes nothing."""
+    REASONS = {0x8: "hw_slowdown", 0x40: "hw_thermal_slowdown", 0x20: "sw_thermal_slowdown",
+               0x4: "sw_power_cap", 0x80: "hw_power_brake_slowdown"}
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_{os.getpid()}.csv")
+    def __init__(self, index: int, period_s: float = 0.002):
+        self.index, self.period = index, period_s
+        self.samples, self.t0, self.t1 = [], None, None
+        self.handle, self.thread, self.max_mhz = None, None, None
+        self._stop = False
+
+    def _open(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            self.handle = pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM))
+        get = getattr(pynvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            pynvml.nvmlDeviceGetCurrentClocksThrottleReasons
+        return pynvml, get
+
+    def _run(self, pynvml, get_reasons):
+        while not self._stop:
+            try:
+                now = time.perf_counter()
+                mhz = pynvml.nvmlDeviceGetClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+                self.samples.append((now, float(mhz), int(get_reasons(self.handle))))
+            except Exception:
+                pass
+            time.sleep(self.period)
 
     def __enter__(self):
         try:
-            os.makedirs(os.path.dirname(self.path), exist_ok=True)
-            self.f = open(self.path, "w")
-            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                                          "-lms", "200", "-i", str(self.index)], stdout=self.f, stderr=subprocess.DEVNULL)
+            pynvml, get = self._open()
+            self.thread = threading.Thread(target=self._run, args=(pynvml, get), daemon=True)
+            self.thread.start()
         except Exception:
-            self.proc = None
+            self.thread = None
         return self
 
+    def mark_start(self):
+        self.t0 = time.perf_counter()
+
+    def mark_end(self):
+        self.t1 = time.perf_counter()
+
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            self.f.close()
+        self._stop = True
+        if self.thread is not None:
+            self.thread.join(timeout=5)
 
     def summary(self):
-        if self.proc is None:
+        if self.thread is None or self.t0 is None or self.t1 is None:
             return None
-        rows = []
-        for line in open(self.path):
-            parts = [p.strip() for p in line.split(",")]
-            if len(parts) != 7:
-                continue
-            try:
-                rows.append((float(parts[0]), float(parts[1]), parts[3:]))
-            except ValueError:
-                continue
+        rows = [(m, r) for t, m, r in list(self.samples) if self.t0 <= t <= self.t1]
         if not rows:
             return None
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
-        loaded = [s for s, _, _ in rows if s > 500] or [s for s, _, _ in rows]
-        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(m for _, m, _ in rows),
-                "reasons": reasons, "samples": len(rows)}
+        reasons = sorted({name for _, r in rows for bit, name in self.REASONS.items() if r & bit})
+        return {"sm_mhz": statistics.median(m for m, _ in rows), "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(rows), "source": "nvml"}
 
 
 def cpu_oracle_sample(wl, budget_s: float = 10.0):
@@ -193,7 +210,7 @@ def run_reference(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--algo", default="auto", choices=["auto", "scan", "chunked"])
@@ -257,16 +274,19 @@ def main():
         dist.barrier()
     evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     with Clocks(local) as clk:
+        time.sleep(0.05)   # let the sampler take its first readings
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
         start = torch.cuda.Event(enable_timing=True)
         end = torch.cuda.Event(enable_timing=True)
+        clk.mark_start()
         start.record(stream)
         for s in range(args.steps):
             step(evs[s])
         end.record(stream)
         torch.cuda.synchronize()
+        clk.mark_end()
     total_ms = start.elapsed_time(end)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]

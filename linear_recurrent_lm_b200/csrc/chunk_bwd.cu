@@ -91,6 +91,7 @@ struct __align__(16) BwdSmem2 {
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 0;\n" ::: "memory"); }
 
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
@@ -337,6 +338,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
   const unsigned m0bits = (1u << fr) - 1u;
   const bool keep = mask == 0u;
   const unsigned ls_bits = cx.ls_bits;
+  // staging of da, dr, db, dk [q][t][j] in bf16; reuses dSb, which is dead after M8
+  bf16 (*gst)[kChunk][kStr] = reinterpret_cast<bf16 (*)[kChunk][kStr]>(&sm.dSb[0][0]);
 
   // ---- M1: [dSA^T | dV^T] = dSl [ls.Bh | ls.Kh]^T + dY^T [Mrb | Mrk]   (rows i of this warp)
   float acc4[4][4] = {};
@@ -582,7 +585,12 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
         e1v[nt][hh] = sub2(mul2(dRt, rt), fma2(dBt, bh, mul2(dKt, kh)));
         e2v[nt][hh] = mul2(dAt, at);
         e3p[nt] = fma2(fma2(xb2, bh, mul2(xk2, kh)), L15, e3p[nt]);
-        if (t < len) {
+        if constexpr (std::is_same<T, bf16>::value) {   // staged, written coalesced after the barrier
+          store2(&gst[0][t][j], mul2(dAt, Lp));
+          store2(&gst[1][t][j], mul2(dRt, Lt));
+          store2(&gst[2][t][j], mul2(dBt, inv));
+          store2(&gst[3][t][j], mul2(dKt, inv));
+        } else if (t < len) {
           store2(gda + orow + j, mul2(dAt, Lp));
           store2(gdr + orow + j, mul2(dRt, Lt));
           store2(gdb + orow + j, mul2(dBt, inv));
@@ -612,7 +620,18 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
       if (g == 0) *reinterpret_cast<float2*>(&sm.e3[j]) = v;
     }
   }
-  named_bar(2, 128);   // DL, e3 complete
+  named_bar(2, 128);   // DL, e3, staged gradients complete
+
+  if constexpr (std::is_same<T, bf16>::value) {
+    T* const outs[4] = {static_cast<T*>(p.da), static_cast<T*>(p.dr), static_cast<T*>(p.db), static_cast<T*>(p.dk)};
+    const int tt = tid >> 3, part = tid & 7;
+    if (tt < len) {
+      const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + part * 8;
+#pragma unroll
+      for (int q = 0; q < 4; ++q)
+        *reinterpret_cast<uint4*>(outs[q] + o) = *reinterpret_cast<const uint4*>(&gst[q][tt][part * 8]);
+    }
+  }
 
   // ---- M11: dw = (reverse cumulative sum of d log L) / w.  Thread = (column pair, token half);
   // the lower half adds the upper half's rows itself instead of waiting for it.
@@ -659,8 +678,12 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(BwdArgs p) {
   const int row0 = 16 * warp;
   const int64_t nc = (p.T + kChunk - 1) / kChunk;
 
-  float dS[8][4];
+  if (tid == 0) sm.stop = 0;
+
+  // The two roles run separate loops so that their register sets never overlap; both meet
+  // at one CTA barrier per iteration (bar.sync 0, executed by all 256 threads).
   if (is_main) {
+    float dS[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -670,25 +693,48 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(BwdArgs p) {
         dS[nt][2 * hh] = v.x;
         dS[nt][2 * hh + 1] = v.y;
       }
-  }
-  if (tid == 0) sm.stop = 0;
-
-  // prologue: the context warps stage the last chunk, its entering state and reset flags
-  float4 s0rows[8];
-  unsigned mask_next = 0u;
-  if (!is_main) {
-    const int64_t c = nc - 1;
-    const int64_t t0 = c * kChunk;
-    stage7<T>(p, sm.in, b, h, t0, int(p.T - t0), ktid);
-    load_entry_rows(p, unit, nc, c, ktid, s0rows);
-    mask_next = reset_bits_of(p, b, t0, int(p.T - t0), lane);
-    cp_async_wait_all();
-  }
-  __syncthreads();
-
-  bool flagged = false;
-  for (int64_t it = 0; it <= nc; ++it) {
-    if (!is_main) {
+    cta_sync();   // prologue staged by the context warps
+    bool flagged = false;
+    for (int64_t it = 0; it <= nc; ++it) {
+      if (it >= 1) {
+        const int64_t c = nc - it;   // chunk whose gradients are computed now
+        const BCtx& cx = sm.ctx[c & 1];
+        if (cx.unsafe) {
+          if (tid == 0) sm.stop = 1;
+        } else {
+          const int64_t t0 = c * kChunk;
+          main_chunk<T>(p, sm, cx, dS, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane);
+        }
+      }
+      cta_sync();
+      if (sm.stop) {
+        flagged = true;
+        break;
+      }
+    }
+    if (tid == 0 && p.unit_flags) p.unit_flags[unit] = flagged ? 1 : 0;
+    if (!flagged && p.ds0) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<float2*>(p.ds0 + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
+              make_float2(dS[nt][2 * hh], dS[nt][2 * hh + 1]);
+    }
+  } else {
+    // prologue: stage the last chunk, its entering state and reset flags
+    float4 s0rows[8];
+    unsigned mask_next;
+    {
+      const int64_t c = nc - 1;
+      const int64_t t0 = c * kChunk;
+      stage7<T>(p, sm.in, b, h, t0, int(p.T - t0), ktid);
+      load_entry_rows(p, unit, nc, c, ktid, s0rows);
+      mask_next = reset_bits_of(p, b, t0, int(p.T - t0), lane);
+      cp_async_wait_all();
+    }
+    cta_sync();
+    for (int64_t it = 0; it <= nc; ++it) {
       const int64_t c = nc - 1 - it;   // chunk whose context is built now
       if (c >= 0) {
         BCtx& cx = sm.ctx[c & 1];
@@ -705,32 +751,10 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(BwdArgs p) {
         if (!unsafe) finish_context<T>(sm, cx, mask, ktid);
         cp_async_wait_all();
       }
-    } else if (it >= 1) {
-      const int64_t c = nc - it;       // chunk whose gradients are computed now
-      const BCtx& cx = sm.ctx[c & 1];
-      if (cx.unsafe) {
-        if (tid == 0) sm.stop = 1;
-      } else {
-        const int64_t t0 = c * kChunk;
-        main_chunk<T>(p, sm, cx, dS, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane);
-      }
+      cta_sync();
+      if (sm.stop) break;
     }
-    __syncthreads();
-    if (sm.stop) {
-      flagged = true;
-      break;
-    }
-  }
-
-  cp_async_wait_all();
-  if (tid == 0 && p.unit_flags) p.unit_flags[unit] = flagged ? 1 : 0;
-  if (!flagged && is_main && p.ds0) {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float2*>(p.ds0 + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-            make_float2(dS[nt][2 * hh], dS[nt][2 * hh + 1]);
+    cp_async_wait_all();
   }
 }
 
