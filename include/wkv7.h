@@ -99,7 +99,10 @@ const char* wkv7_status_string(wkv7_status_t status);
  * B*H*ceil(T/16)*64*64*4 bytes (rwkv-metal page: "checkpointing the hidden
  * state every 16 tokens"; RWKV-MLX page, "Key Design Decisions" 2: "~12MB
  * extra memory" at B=2, T=512, 12 heads -- this formula gives 12.58 MB).
- * Checkpoint c holds the state after token min(16(c+1), T) - 1.  After the
+ * Checkpoint c holds the state after token min(16(c+1), T) - 1, its element
+ * (i, j) at offset (i/16)*1024 + (j/8)*128 + (4*(i%8) + (j%8)/2)*4
+ * + 2*((i/8)%2) + j%2 (the order of the kernels' mma accumulator fragments, so
+ * that every warp moves 512 contiguous bytes per store).  After the
  * checkpoints come B*H ints (rounded up to 16 bytes) that wkv7_backward uses
  * to mark heads it must recompute with the exact scan.
  * Returns 0 for an invalid descriptor or T == 0.

@@ -143,14 +143,27 @@ __device__ __forceinline__ void stage7(const BwdArgs& p, T (*dst)[kChunk][kStr],
   cp_async_commit();
 }
 
-// State entering chunk c (checkpoint c-1, s0 or zero): thread ktid holds row ktid/2, half ktid%2.
+// State entering chunk c (checkpoint c-1, s0 or zero) as accumulator fragments: context thread
+// (warp kw, lane 4g + c4) holds s[nt] = S[16kw + g][8nt + 2c4 + {0,1}], S[16kw + g + 8][same].
 __device__ __forceinline__ void load_entry_rows(const BwdArgs& p, int64_t unit, int64_t nc, int64_t c, int ktid,
                                                 float4 (&s)[8]) {
-  const float* src = c > 0 ? p.ckpt + (unit * nc + (c - 1)) * kN * kN : (p.s0 ? p.s0 + unit * kN * kN : nullptr);
-  const int row = ktid >> 1, col0 = (ktid & 1) * 32;
+  if (c > 0) {   // tiled checkpoint order: one contiguous 512-byte row of float4 per warp and nt
+    const float* src = p.ckpt + (unit * nc + (c - 1)) * kN * kN + (ktid >> 5) * 1024 + (ktid & 31) * 4;
 #pragma unroll
-  for (int q = 0; q < 8; ++q)
-    s[q] = src ? *reinterpret_cast<const float4*>(src + row * kN + col0 + 4 * q) : make_float4(0.f, 0.f, 0.f, 0.f);
+    for (int nt = 0; nt < 8; ++nt) s[nt] = *reinterpret_cast<const float4*>(src + nt * 128);
+  } else if (p.s0) {
+    const int lane = ktid & 31;
+    const float* src = p.s0 + unit * kN * kN + (16 * (ktid >> 5) + (lane >> 2)) * kN + 2 * (lane & 3);
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) {
+      const float2 lo = *reinterpret_cast<const float2*>(src + 8 * nt);
+      const float2 hi = *reinterpret_cast<const float2*>(src + 8 * kN + 8 * nt);
+      s[nt] = make_float4(lo.x, lo.y, hi.x, hi.y);
+    }
+  } else {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt) s[nt] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
 }
 
 __device__ __forceinline__ unsigned reset_bits_of(const BwdArgs& p, int64_t b, int64_t t0, int len, int lane) {
@@ -201,13 +214,11 @@ __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm,
     }
     // every L_t of the chunk lies in exactly one quarter, so the CTA-wide ballot sees all of them
     bad = !(fminf(wmin.x, wmin.y) >= 0.0625f && fminf(lmin.x, lmin.y) >= 0x1p-40f && fmaxf(lmax.x, lmax.y) <= 0x1p40f);
-    const int row = ktid >> 1, col0 = (ktid & 1) * 32;
+    const int row = 16 * kw + (lane >> 2), col = 2 * (lane & 3);
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      uint2 v;
-      v.x = pack_bf16(s0rows[q].x, s0rows[q].y);
-      v.y = pack_bf16(s0rows[q].z, s0rows[q].w);
-      *reinterpret_cast<uint2*>(&cx.S0b[row][col0 + 4 * q]) = v;
+    for (int nt = 0; nt < 8; ++nt) {
+      *reinterpret_cast<uint32_t*>(&cx.S0b[row][8 * nt + col]) = pack_bf16(s0rows[nt].x, s0rows[nt].y);
+      *reinterpret_cast<uint32_t*>(&cx.S0b[row + 8][8 * nt + col]) = pack_bf16(s0rows[nt].z, s0rows[nt].w);
     }
   }
   const unsigned any_bad = __ballot_sync(0xffffffffu, bad);

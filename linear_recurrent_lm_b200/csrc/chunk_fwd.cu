@@ -77,11 +77,29 @@ struct __align__(16) FwdSmem3 {
   float W[kChunk][S72], Q[kChunk][S72];      // [t][j]
   float X[kChunk][S20], Z[kChunk][S20], M[kChunk][S20];
   T in[kIn][kChunk][kStrIn];                 // staged inputs of the chunk being built
+  __align__(16) uint16_t Ys[kChunk][kStrIn]; // y of the last chunk [t][i] (16-bit outputs), written next iteration
   int kbad[4];
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
+__device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 0;\n" ::: "memory"); }
+
+// Store four 8x8 b16 matrices from accumulator-fragment registers, transposed.
+__device__ __forceinline__ void stsm_x4_t(void* row_ptr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
+  asm volatile("stmatrix.sync.aligned.m8n8.x4.trans.shared.b16 [%0], {%1, %2, %3, %4};\n"
+               ::"r"(smem_u32(row_ptr)), "r"(r0), "r"(r1), "r"(r2), "r"(r3) : "memory");
+}
+
+template <typename T>
+__device__ __forceinline__ uint32_t pack16(float lo, float hi) {
+  if constexpr (std::is_same<T, __half>::value) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  } else {
+    return pack_bf16(lo, hi);
+  }
 }
 
 __device__ __forceinline__ float rcp_approx(float x) {
@@ -130,44 +148,51 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, FwdSmem3<T>& sm,
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
   const T (*X)[kChunk][kStrIn] = sm.in;
 
-  // ---- K1: decay products and decay-scaled operands; thread = (column j, token half)
+  // ---- K1: decay products and decay-scaled operands.  Thread = (token quarter kw; columns lane
+  // and lane + 32, as one packed fp32 pair); the transposed copies go out as one float4 per column.
   bool bad = false;
   {
-    const int j = ktid & 63, half = ktid >> 6;
-    float lam[kChunk];
-    float l = 1.f;
+    const int tq = 4 * kw, ja = lane, jb = lane + 32;
+    auto ld2 = [&](int m, int t) { return make_float2(Elt<T>::to_f32(X[m][t][ja]), Elt<T>::to_f32(X[m][t][jb])); };
+    float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
+    for (int t = 0; t < tq; ++t) lam = mul2(lam, ld2(1, t));
+    float at[2][4], bh[2][4], kh[2][4], vv[2][4];
 #pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      l *= Elt<T>::to_f32(X[1][t][j]);
-      lam[t] = l;
-      bad |= !(l >= 0x1p-40f && l <= 0x1p40f);
+    for (int u = 0; u < 4; ++u) {
+      const int t = tq + u;
+      const float2 lp = lam;
+      lam = mul2(lam, ld2(1, t));
+      bad |= !(lam.x >= 0x1p-40f && lam.x <= 0x1p40f) || !(lam.y >= 0x1p-40f && lam.y <= 0x1p40f);
+      const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
+      const float2 a2 = mul2(ld2(4, t), lp), r2 = mul2(ld2(0, t), lam);
+      const float2 b2 = mul2(ld2(5, t), inv), k2 = mul2(ld2(2, t), inv), v2 = ld2(3, t);
+      at[0][u] = tf32f(a2.x); at[1][u] = tf32f(a2.y);
+      bh[0][u] = tf32f(b2.x); bh[1][u] = tf32f(b2.y);
+      kh[0][u] = tf32f(k2.x); kh[1][u] = tf32f(k2.y);
+      vv[0][u] = tf32f(v2.x); vv[1][u] = tf32f(v2.y);
+      sm.GA[t][ja] = at[0][u];
+      sm.GA[t][jb] = at[1][u];
+      sm.GA[16 + t][ja] = tf32f(r2.x);
+      sm.GA[16 + t][jb] = tf32f(r2.y);
+      sm.GB[t][ja] = bh[0][u];
+      sm.GB[t][jb] = bh[1][u];
+      sm.GB[16 + t][ja] = kh[0][u];
+      sm.GB[16 + t][jb] = kh[1][u];
+      cx.Rt[t][ja] = t < fr ? r2.x : 0.f;
+      cx.Rt[t][jb] = t < fr ? r2.y : 0.f;
     }
 #pragma unroll
-    for (int tp = 0; tp < 8; tp += 2) {
-      const int t = 8 * half + tp;
-      const float lp0 = t > 0 ? lam[t - 1] : 1.f, l0 = lam[t], l1 = lam[t + 1];
-      const float i0 = rcp_approx(l0), i1 = rcp_approx(l1);
-      const float at0 = Elt<T>::to_f32(X[4][t][j]) * lp0, at1 = Elt<T>::to_f32(X[4][t + 1][j]) * l0;
-      const float rt0 = Elt<T>::to_f32(X[0][t][j]) * l0, rt1 = Elt<T>::to_f32(X[0][t + 1][j]) * l1;
-      const float bh0 = Elt<T>::to_f32(X[5][t][j]) * i0, bh1 = Elt<T>::to_f32(X[5][t + 1][j]) * i1;
-      const float kh0 = Elt<T>::to_f32(X[2][t][j]) * i0, kh1 = Elt<T>::to_f32(X[2][t + 1][j]) * i1;
-      const float v0 = Elt<T>::to_f32(X[3][t][j]), v1 = Elt<T>::to_f32(X[3][t + 1][j]);
-      sm.GA[t][j] = tf32f(at0);
-      sm.GA[t + 1][j] = tf32f(at1);
-      sm.GA[16 + t][j] = tf32f(rt0);
-      sm.GA[16 + t + 1][j] = tf32f(rt1);
-      sm.GB[t][j] = tf32f(bh0);
-      sm.GB[t + 1][j] = tf32f(bh1);
-      sm.GB[16 + t][j] = tf32f(kh0);
-      sm.GB[16 + t + 1][j] = tf32f(kh1);
-      cx.Rt[t][j] = t < fr ? rt0 : 0.f;
-      cx.Rt[t + 1][j] = t + 1 < fr ? rt1 : 0.f;
-      *reinterpret_cast<float2*>(&cx.AtT[j][t]) = make_float2(tf32f(at0), tf32f(at1));
-      *reinterpret_cast<float2*>(&cx.BhT[j][t]) = make_float2(tf32f(bh0), tf32f(bh1));
-      *reinterpret_cast<float2*>(&cx.KhT[j][t]) = make_float2(tf32f(kh0), tf32f(kh1));
-      *reinterpret_cast<float2*>(&cx.VT[j][t]) = make_float2(tf32f(v0), tf32f(v1));
+    for (int q = 0; q < 2; ++q) {
+      const int j = q ? jb : ja;
+      *reinterpret_cast<float4*>(&cx.AtT[j][tq]) = make_float4(at[q][0], at[q][1], at[q][2], at[q][3]);
+      *reinterpret_cast<float4*>(&cx.BhT[j][tq]) = make_float4(bh[q][0], bh[q][1], bh[q][2], bh[q][3]);
+      *reinterpret_cast<float4*>(&cx.KhT[j][tq]) = make_float4(kh[q][0], kh[q][1], kh[q][2], kh[q][3]);
+      *reinterpret_cast<float4*>(&cx.VT[j][tq]) = make_float4(vv[q][0], vv[q][1], vv[q][2], vv[q][3]);
     }
-    if (half == 0) cx.lam15[j] = lam[kChunk - 1];
+    if (kw == 3) {
+      cx.lam15[ja] = lam.x;
+      cx.lam15[jb] = lam.y;
+    }
   }
   const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
   if (lane == 0) sm.kbad[kw] = any_bad ? 1 : 0;
@@ -393,7 +418,11 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     mma1688(yy[nt], av[0], zb[0], zb[1]);
     mma1688(yy[nt], av[1], zb[2], zb[3]);
   }
-  {
+  if constexpr (sizeof(T) == 2) {   // Y^T fragments -> Ys[t][i]; written out after the next CTA barrier
+    const int m = lane >> 3;
+    stsm_x4_t(&sm.Ys[8 * (m >> 1) + (lane & 7)][row0 + 8 * (m & 1)], pack16<T>(yy[0][0], yy[0][1]),
+              pack16<T>(yy[0][2], yy[0][3]), pack16<T>(yy[1][0], yy[1][1]), pack16<T>(yy[1][2], yy[1][3]));
+  } else {
     T* y = static_cast<T*>(p.y);
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
@@ -513,9 +542,11 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
 
-  // state fragments: acc[nt][e] = S[16*warp + g + 8*(e>>1)][8*nt + 2*c4 + (e&1)]
-  float acc[8][4];
+  // The two roles run separate loops so that their register sets never overlap; both meet
+  // at one CTA barrier per iteration (bar.sync 0, executed by all 256 threads).
   if (is_state) {
+    // state fragments: acc[nt][e] = S[16*warp + g + 8*(e>>1)][8*nt + 2*c4 + (e&1)]
+    float acc[8][4];
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
@@ -525,21 +556,56 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
         acc[nt][2 * hh] = v2.x;
         acc[nt][2 * hh + 1] = v2.y;
       }
-  }
-
-  // prologue: the context warps stage chunk 0 and fetch its reset flags
-  unsigned reset_bits = 0u;
-  if (!is_state) {
-    stage_chunk<T>(p, sm.in, b, h, 0, int(min64(kChunk, p.T)), ktid);
-    const int len0 = int(min64(kChunk, p.T));
-    const bool f = p.reset && lane < len0 && p.reset[b * p.T + lane] != 0;
-    reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
-    cp_async_wait_all();
-  }
-  __syncthreads();
-
-  for (int64_t it = 0; it <= nc; ++it) {
-    if (!is_state) {
+    cta_sync();   // chunk 0 staged
+    // y of the previous chunk (16-bit outputs): this thread's 16-byte piece of token row tid/8
+    T* ydst = nullptr;
+    const int ytt = tid >> 3, ypart = tid & 7;
+    for (int64_t it = 0; it <= nc; ++it) {
+      if (ydst) {
+        *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+        ydst = nullptr;
+      }
+      if (it >= 1) {
+        const int64_t c = it - 1;
+        const Ctx& cx = sm.ctx[c & 1];
+        const int64_t t0 = c * kChunk;
+        const int len = int(min64(kChunk, p.T - t0));
+        if (!cx.unsafe) {
+          state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane);
+          if (sizeof(T) == 2 && ytt < len) ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
+        } else {
+          state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
+        }
+        if (p.ckpt) {   // tiled checkpoint order: 512 contiguous bytes per warp and nt
+          float* base = p.ckpt + (unit * nc + c) * kN * kN + warp * 1024 + lane * 4;
+#pragma unroll
+          for (int nt = 0; nt < 8; ++nt)
+            *reinterpret_cast<float4*>(base + nt * 128) = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+        }
+      }
+      cta_sync();   // context of chunk it handed over; Ys complete
+    }
+    if (ydst) *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+    if (p.s_out) {
+#pragma unroll
+      for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          *reinterpret_cast<float2*>(p.s_out + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
+              make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+    }
+  } else {
+    // prologue: stage chunk 0 and fetch its reset flags
+    unsigned reset_bits;
+    {
+      const int len0 = int(min64(kChunk, p.T));
+      stage_chunk<T>(p, sm.in, b, h, 0, len0, ktid);
+      const bool f = p.reset && lane < len0 && p.reset[b * p.T + lane] != 0;
+      reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
+      cp_async_wait_all();
+    }
+    cta_sync();
+    for (int64_t it = 0; it <= nc; ++it) {
       if (it < nc) {
         const int64_t c = it;
         const unsigned mask = reset_bits;
@@ -552,36 +618,8 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
         build_context<T>(p, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid);
         cp_async_wait_all();
       }
-    } else if (it >= 1) {
-      const int64_t c = it - 1;
-      const Ctx& cx = sm.ctx[c & 1];
-      const int64_t t0 = c * kChunk;
-      const int len = int(min64(kChunk, p.T - t0));
-      if (!cx.unsafe) {
-        state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane);
-      } else {
-        state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
-      }
-      if (p.ckpt) {
-        float* base = p.ckpt + (unit * nc + c) * kN * kN;
-#pragma unroll
-        for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-          for (int hh = 0; hh < 2; ++hh)
-            *reinterpret_cast<float2*>(base + (row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-                make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
-      }
+      cta_sync();
     }
-    __syncthreads();   // context of chunk it handed to the state warps
-  }
-
-  if (is_state && p.s_out) {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float2*>(p.s_out + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-            make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
   }
 }
 

@@ -62,6 +62,14 @@ __device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wai
 
 __host__ __device__ __forceinline__ int64_t min64(int64_t a, int64_t b) { return a < b ? a : b; }
 
+// Offset of element (i, j) inside one checkpointed 64x64 fp32 state.  The order is the one
+// in which the chunked kernels hold the state as m16n8 accumulator fragments (warp i/16,
+// lane 4(i%8) + (j%8)/2, register 4(j/8) + 2((i/8)%2) + j%2), so that each warp stores and
+// loads 512 contiguous bytes per instruction.
+__host__ __device__ __forceinline__ int ckpt_off(int i, int j) {
+  return (i >> 4) * 1024 + (j >> 3) * 128 + ((i & 7) * 4 + ((j & 7) >> 1)) * 4 + ((i >> 3) & 1) * 2 + (j & 1);
+}
+
 // Offset (in elements) of x[b][t][h][0] in a [B,T,H,64] tensor.
 __device__ __forceinline__ int64_t tok_off(int64_t b, int64_t t, int64_t h, int64_t T, int64_t H) {
   return ((b * T + t) * H + h) * kN;

@@ -118,9 +118,15 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
     // state entering the chunk (before the reset of its first token applies)
     float E[16];
     {
-      const float* es = c > 0 ? p.ckpt + ((unit * nc + (c - 1)) * kN) * kN : (p.s0 ? p.s0 + unit * kN * kN : nullptr);
+      if (c > 0) {   // checkpoint c-1, in the tiled checkpoint order
+        const float* es = p.ckpt + (unit * nc + (c - 1)) * kN * kN;
 #pragma unroll
-      for (int ii = 0; ii < 16; ++ii) E[ii] = es ? es[(q * 16 + ii) * kN + j] : 0.f;
+        for (int ii = 0; ii < 16; ++ii) E[ii] = es[ckpt_off(q * 16 + ii, j)];
+      } else {       // the caller's s0, row-major
+        const float* es = p.s0 ? p.s0 + unit * kN * kN : nullptr;
+#pragma unroll
+        for (int ii = 0; ii < 16; ++ii) E[ii] = es ? es[(q * 16 + ii) * kN + j] : 0.f;
+      }
     }
 
     int seg_end = len;

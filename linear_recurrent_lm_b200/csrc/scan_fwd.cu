@@ -129,9 +129,9 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
     }
 
     if (p.ckpt) {
-      float4* dst = reinterpret_cast<float4*>(p.ckpt + ((unit * nc + c) * kN + i) * kN);
+      float* dst = p.ckpt + (unit * nc + c) * kN * kN;
 #pragma unroll
-      for (int q = 0; q < kN / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);
+      for (int q = 0; q < kN / 2; ++q) *reinterpret_cast<float2*>(dst + ckpt_off(i, 2 * q)) = make_float2(S[2 * q], S[2 * q + 1]);
     }
     cp_async_wait_all();
     __syncthreads();

@@ -33,3 +33,19 @@ def sample_units(B, H, k, seed=0):
     while len(units) < min(k, B * H):
         units.add((int(rng.integers(B)), int(rng.integers(H))))
     return sorted(units)
+
+
+def checkpoint_states(ws, B, H, n_ck) -> np.ndarray:
+    """Checkpoints of a forward workspace as [B, H, n_ck, 64, 64] fp64 states.
+
+    Inside one checkpoint, element (i, j) sits at the documented tiled offset
+    (i//16)*1024 + (j//8)*128 + (4*(i%8) + (j%8)//2)*4 + 2*((i//8)%2) + j%2."""
+    import torch
+    raw = ws[: B * H * n_ck * 64 * 64 * 4].view(torch.float32).view(B, H, n_ck, 4096)
+    raw = raw.double().cpu().numpy()
+    i = np.arange(64)[:, None]
+    j = np.arange(64)[None, :]
+    off = (i // 16) * 1024 + (j // 8) * 128 + (4 * (i % 8) + (j % 8) // 2) * 4 + 2 * ((i // 8) % 2) + j % 2
+    assert len(np.unique(off)) == 4096
+    return raw[..., off]
+

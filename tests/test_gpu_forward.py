@@ -6,7 +6,7 @@ import pytest
 
 import oracle
 from linear_recurrent_lm_b200 import inputs as I
-from tests.gpu_util import f64, inputs_dev, inputs_f64, sample_units, to_dev
+from tests.gpu_util import checkpoint_states, f64, inputs_dev, inputs_f64, sample_units, to_dev
 from tests.metrics import err_rms, err_rms_excess
 
 pytestmark = pytest.mark.gpu
@@ -62,11 +62,11 @@ def test_config1_forward_and_checkpoints(W, algo):
     yo, so, _ = oracle.forward(*inputs_f64(wl.inputs))
     check_fwd(y, s, yo, so, "bf16")
     # checkpoint c holds the state after token 16c+15: compare with the oracle run to that token
-    ck = ws[: 2 * 12 * 32 * 64 * 64 * 4].view(torch.float32).view(2, 12, 32, 64, 64)
+    ck = checkpoint_states(ws, 2, 12, 32)
     for c in (0, 7, 31):
         part = {n: wl.inputs[n][:, : 16 * (c + 1)] for n in I.NAMES}
         _, sc, _ = oracle.forward(*inputs_f64(part))
-        assert err_rms(f64(ck[:, :, c]), sc) <= 2e-2
+        assert err_rms(ck[:, :, c], sc) <= 2e-2
 
 
 @pytest.mark.parametrize("algo", ALGOS)
