@@ -60,7 +60,7 @@ typedef enum {
   WKV7_ERR_DTYPE = 3,       /* dtype code is not a wkv7_dtype_t                               */
   WKV7_ERR_ALIGN = 4,       /* a tensor pointer is not 16-byte aligned                        */
   WKV7_ERR_WORKSPACE = 5,   /* backward without a checkpoint workspace                        */
-  WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, non-zero flags, or T != 1 for a step   */
+  WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, unknown flags, or T != 1 for a step     */
   WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
   WKV7_ERR_TIMEOUT = 8,     /* reserved for device-side bounded waits                          */
   WKV7_ERR_SCRATCH_LIMIT = 9 /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
@@ -84,8 +84,30 @@ typedef struct {
   int32_t N;      /* head size: must be 64                       */
   int32_t dtype;  /* wkv7_dtype_t of every activation/gradient   */
   int32_t algo;   /* wkv7_algo_t                                 */
-  uint32_t flags; /* reserved, must be 0                         */
+  uint32_t flags; /* 0, or WKV7_FLAG_TEST_WAIT_TIMEOUT (below)     */
 } wkv7_desc_t;
+
+/*
+ * desc->flags bit (no page counterpart: a test hook for the device status
+ * word).  With it, the chunked kernels' staging of input rows expects 16
+ * bytes that are never copied, so the bounded wait for them runs out after
+ * about one second; the chunk is then computed from global memory instead
+ * (forward: token by token; backward: the exact scan), the results stay
+ * correct, and wkv7_get_device_status() reports WKV7_ERR_TIMEOUT.  Accepted
+ * only with T <= 16; every other flag bit must be 0 (WKV7_ERR_UNSUPPORTED).
+ */
+#define WKV7_FLAG_TEST_WAIT_TIMEOUT 0x80000000u
+
+/*
+ * Device status word (the device-side error channel of the boundary).
+ * Kernels record errors they cannot return from an asynchronous launch --
+ * today a bounded wait on staged inputs that ran out -- in one word per
+ * device.  This call synchronises the current device, reads the word and,
+ * if `clear` is non-zero, resets it.  Returns WKV7_OK, WKV7_ERR_TIMEOUT if a
+ * wait ran out since the last clear, or WKV7_ERR_CUDA if synchronising or
+ * reading failed (e.g. no device).
+ */
+wkv7_status_t wkv7_get_device_status(int clear);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int wkv7_version(void);

@@ -71,9 +71,9 @@ struct __align__(16) BCtx {
 };
 
 template <typename T>
-struct __align__(16) BwdSmem2 {
+struct __align__(128) BwdSmem2 {
   BCtx ctx[2];
-  T in[kIn][kChunk][kStr];    // staged inputs of the chunk being built
+  __align__(128) T in[kIn][kChunk][kN];   // staged inputs of the chunk being built (TMA boxes)
   __align__(16) float LabT[kChunk][20];
   __align__(16) float LakT[kChunk][20];
   bf16 Wb[kChunk][kStr], Xb[kChunk][kStrS];
@@ -84,6 +84,7 @@ struct __align__(16) BwdSmem2 {
   __align__(16) float DL[kChunk][kN + 4];   // d log L_t without the chunk-end term
   __align__(16) float e3[kN];
   __align__(16) float dlam[4][kN];
+  unsigned long long in_bar;   // completion of the bulk copies into `in` (one phase per staged chunk)
   int kbad[4];
   int stop;
 };
@@ -117,30 +118,16 @@ __device__ __forceinline__ void mask_k16(uint32_t (&a)[4], int c4, unsigned bits
   a[3] &= m1;
 }
 
+// Stage the seven inputs (r, w, k, v, a, b, dy) of chunk tokens t0..t0+15 into sm.in: one TMA box
+// per input, issued by one thread; rows past T arrive as zeros (K1 reads w there as 1).
 template <typename T>
-__device__ __forceinline__ void stage7(const BwdArgs& p, T (*dst)[kChunk][kStr], int64_t b, int64_t h, int64_t t0,
-                                       int len, int ktid) {
-  constexpr int n = Vec16<T>::n;
-  constexpr int VPT = kN / n;
-  const T* src[kIn] = {static_cast<const T*>(p.r), static_cast<const T*>(p.w), static_cast<const T*>(p.k),
-                       static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b),
-                       static_cast<const T*>(p.dy)};
-  for (int idx = ktid; idx < kChunk * VPT; idx += 128) {
-    const int tt = idx / VPT, vec = idx - (idx / VPT) * VPT;
-    const int64_t off = tok_off(b, t0 + tt, h, p.T, p.H) + vec * n;
+__device__ __forceinline__ void stage7(const BwdArgs& p, const InputMaps& tm, BwdSmem2<T>& sm, int64_t b, int64_t h,
+                                       int64_t t0, int ktid) {
+  if (ktid == 0) {
+    mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + p.extra_tx);
 #pragma unroll
-    for (int m = 0; m < kIn; ++m) {
-      T* s = &dst[m][tt][vec * n];
-      if (tt < len) {
-        cp_async16(s, src[m] + off);
-      } else {   // padding token: w = 1, everything else (dy included) 0
-        const T fill = Elt<T>::from_f32(m == 1 ? 1.f : 0.f);
-#pragma unroll
-        for (int e = 0; e < n; ++e) s[e] = fill;
-      }
-    }
+    for (int m = 0; m < kIn; ++m) tma_load_4d(&sm.in[m][0][0], &tm.m[m], 0, int(h), int(t0), int(b), &sm.in_bar);
   }
-  cp_async_commit();
 }
 
 // State entering chunk c (checkpoint c-1, s0 or zero) as accumulator fragments: context thread
@@ -172,11 +159,15 @@ __device__ __forceinline__ unsigned reset_bits_of(const BwdArgs& p, int64_t b, i
 }
 
 // ------------------------------------------------------------------ context warps
+// A wait for staged inputs that runs out marks the chunk unsafe (the unit is then recomputed by the
+// exact scan, which reads global memory) and sets `timed_out`, after which nothing more is staged.
 template <typename T>
 __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm, BCtx& cx, unsigned mask,
-                                              const float4 (&s0rows)[8], int ktid, bool& unsafe) {
+                                              const float4 (&s0rows)[8], int ktid, int len, unsigned parity,
+                                              bool& unsafe, bool& timed_out) {
   const int kw = ktid >> 5, lane = ktid & 31;
-  const T (*X)[kChunk][kStr] = sm.in;
+  const bool to = !mbar_wait_bounded(&sm.in_bar, parity, kWaitLimitNs);
+  const T (*X)[kChunk][kN] = sm.in;
 
   // ---- K1: decay products, scaled operands, v/dy copies, entering state in bf16.
   // Thread = (column pair 2jp, 2jp+1; token quarter kw), two columns per packed fp32 op.
@@ -185,12 +176,13 @@ __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm,
     const int j = 2 * lane, t0 = 4 * kw;
     // L_{t0-1}: product of the earlier quarters' decays (warp-uniform trip count)
     float2 lam = make_float2(1.f, 1.f);
-    for (int t = 0; t < t0; ++t) lam = mul2(lam, load2(&X[1][t][j]));
+    auto ldw = [&](int t) { return t < len ? load2(&X[1][t][j]) : make_float2(1.f, 1.f); };   // padding: w = 1
+    for (int t = 0; t < t0; ++t) lam = mul2(lam, ldw(t));
     float2 wmin = make_float2(1.f, 1.f), lmin = make_float2(1.f, 1.f), lmax = lmin;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = t0 + u;
-      const float2 lp = lam, w2 = load2(&X[1][t][j]);
+      const float2 lp = lam, w2 = ldw(t);
       lam = mul2(lam, w2);
       wmin = make_float2(fminf(wmin.x, w2.x), fminf(wmin.y, w2.y));
       lmin = make_float2(fminf(lmin.x, lam.x), fminf(lmin.y, lam.y));
@@ -221,10 +213,13 @@ __device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm,
       *reinterpret_cast<uint32_t*>(&cx.S0b[row + 8][8 * nt + col]) = pack_bf16(s0rows[nt].z, s0rows[nt].w);
     }
   }
-  const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
-  if (lane == 0) sm.kbad[kw] = any_bad ? 1 : 0;
+  const unsigned any_bad = __ballot_sync(0xffffffffu, bad), any_to = __ballot_sync(0xffffffffu, to);
+  if (lane == 0) sm.kbad[kw] = (any_bad ? 1 : 0) | (any_to ? 2 : 0);
   named_bar(1, 128);
-  unsafe = (sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3]) != 0;
+  const int kb = sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3];
+  unsafe = kb != 0;
+  timed_out = (kb & 2) != 0;
+  if (timed_out && ktid == 0 && p.status) atomicOr(p.status, kStatusWaitTimeout);
   if (ktid == 0) {
     cx.mask = int(mask);
     cx.unsafe = unsafe ? 1 : 0;
@@ -676,8 +671,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(BwdArgs p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+__global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p, const __grid_constant__ InputMaps tm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   BwdSmem2<T>& sm = *reinterpret_cast<BwdSmem2<T>*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
@@ -736,55 +731,65 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(BwdArgs p) {
     // prologue: stage the last chunk, its entering state and reset flags
     float4 s0rows[8];
     unsigned mask_next;
+    unsigned phase = 0;        // barrier phase of the next staging to wait for
+    bool pending = true;       // a staging was issued and not yet waited for
+    bool timed_out = false;
     {
+      if (ktid == 0) mbar_init(&sm.in_bar, 1);
+      named_bar(1, 128);
       const int64_t c = nc - 1;
       const int64_t t0 = c * kChunk;
-      stage7<T>(p, sm.in, b, h, t0, int(p.T - t0), ktid);
+      stage7<T>(p, tm, sm, b, h, t0, ktid);
       load_entry_rows(p, unit, nc, c, ktid, s0rows);
       mask_next = reset_bits_of(p, b, t0, int(p.T - t0), lane);
-      cp_async_wait_all();
     }
     cta_sync();
     for (int64_t it = 0; it <= nc; ++it) {
       const int64_t c = nc - 1 - it;   // chunk whose context is built now
-      if (c >= 0) {
+      if (c >= 0 && pending && !timed_out) {   // (an unsafe chunk stages nothing more: the unit stops)
         BCtx& cx = sm.ctx[c & 1];
         const unsigned mask = mask_next;
         bool unsafe = false;
-        build_context<T>(p, sm, cx, mask, s0rows, ktid, unsafe);
+        build_context<T>(p, sm, cx, mask, s0rows, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, unsafe,
+                         timed_out);
+        if (!timed_out) {
+          pending = false;
+          ++phase;
+        }
         // the staged inputs and entering state are consumed: prefetch the previous chunk
-        if (c > 0) {
+        if (c > 0 && !unsafe) {
           const int64_t tp = (c - 1) * kChunk;
-          stage7<T>(p, sm.in, b, h, tp, kChunk, ktid);
+          stage7<T>(p, tm, sm, b, h, tp, ktid);
+          pending = true;
           load_entry_rows(p, unit, nc, c - 1, ktid, s0rows);
           mask_next = reset_bits_of(p, b, tp, kChunk, lane);
         }
         if (!unsafe) finish_context<T>(sm, cx, mask, ktid);
-        cp_async_wait_all();
       }
       cta_sync();
       if (sm.stop) break;
     }
-    cp_async_wait_all();
+    // copies issued but never waited for (the unit stopped early) must land before the CTA exits
+    if (pending) mbar_wait_bounded(&sm.in_bar, phase & 1u, timed_out ? kWaitLimitNs / 100 : kWaitLimitNs);
   }
 }
 
 template <typename T>
-cudaError_t launch(const BwdArgs& p, cudaStream_t stream) {
+cudaError_t launch(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
   const size_t smem = sizeof(BwdSmem2<T>);
   cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  chunk_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p);
+  chunk_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_bwd(const BwdArgs& p, int dtype, cudaStream_t stream) {
+cudaError_t launch_chunk_bwd(const BwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream) {
   switch (dtype) {
-    case 0: return launch<float>(p, stream);
-    case 1: return launch<__nv_bfloat16>(p, stream);
-    case 2: return launch<__half>(p, stream);
+    case 0: return launch<float>(p, tm, stream);
+    case 1: return launch<__nv_bfloat16>(p, tm, stream);
+    case 2: return launch<__half>(p, tm, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -47,7 +47,7 @@ namespace {
 
 constexpr int kThreads = 256;
 constexpr int kIn = 6;       // staged inputs: r, w, k, v, a, b
-constexpr int kStrIn = 72;   // staged input row stride (elements)
+constexpr int kStrY = 72;    // row stride (elements) of the y staging tile
 constexpr int S68 = 68, S72 = 72, S20 = 20, S24 = 24;
 using bf16 = __nv_bfloat16;
 
@@ -69,15 +69,16 @@ struct __align__(16) Ctx {
 };
 
 template <typename T>
-struct __align__(16) FwdSmem3 {
+struct __align__(128) FwdSmem3 {
   Ctx ctx[2];
   float GA[32][S68];        // rows 0..15 at_t, 16..31 rt_t   [t][j]
   float GB[32][S68];        // rows 0..15 bh_t, 16..31 kh_t   [tau][j]
   __align__(16) float LabT[kChunk][S20];
   float W[kChunk][S72], Q[kChunk][S72];      // [t][j]
   float X[kChunk][S20], Z[kChunk][S20], M[kChunk][S20];
-  T in[kIn][kChunk][kStrIn];                 // staged inputs of the chunk being built
-  __align__(16) uint16_t Ys[kChunk][kStrIn]; // y of the last chunk [t][i] (16-bit outputs), written next iteration
+  __align__(128) T in[kIn][kChunk][kN];      // staged inputs of the chunk being built (TMA boxes)
+  __align__(16) uint16_t Ys[kChunk][kStrY]; // y of the last chunk [t][i] (16-bit outputs), written next iteration
+  unsigned long long in_bar;                 // completion of the bulk copies into `in` (one phase per chunk)
   int kbad[4];
 };
 
@@ -115,38 +116,33 @@ __device__ __forceinline__ void mask_nat(uint32_t (&a)[4], int s, int c4, unsign
   if (!k1) { a[2] = 0u; a[3] = 0u; }
 }
 
+// Stage the six inputs of chunk tokens t0..t0+15 into sm.in: one TMA box per input, issued by one
+// thread; rows past T arrive as zeros (K1 reads w there as 1, which leaves the state unchanged).
+// The copies complete phase c of sm.in_bar for chunk c.
 template <typename T>
-__device__ __forceinline__ void stage_chunk(const FwdArgs& p, T (*dst)[kChunk][kStrIn], int64_t b, int64_t h,
-                                            int64_t t0, int len, int ktid) {
-  constexpr int n = Vec16<T>::n;
-  constexpr int VPT = kN / n;
-  const T* src[kIn] = {static_cast<const T*>(p.r), static_cast<const T*>(p.w), static_cast<const T*>(p.k),
-                       static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b)};
+__device__ __forceinline__ void stage_chunk(const FwdArgs& p, const InputMaps& tm, FwdSmem3<T>& sm, int64_t b,
+                                            int64_t h, int64_t t0, int ktid) {
+  if (ktid == 0) {
+    mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + p.extra_tx);
 #pragma unroll
-  for (int m = 0; m < kIn; ++m) {
-    for (int idx = ktid; idx < kChunk * VPT; idx += 128) {
-      const int tt = idx / VPT, vec = idx - (idx / VPT) * VPT;
-      T* s = &dst[m][tt][vec * n];
-      if (tt < len) {
-        cp_async16(s, src[m] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * n);
-      } else {   // padding token: w = 1, everything else 0 -> leaves the state unchanged
-        const T fill = Elt<T>::from_f32(m == 1 ? 1.f : 0.f);
-#pragma unroll
-        for (int e = 0; e < n; ++e) s[e] = fill;
-      }
-    }
+    for (int m = 0; m < kIn; ++m) tma_load_4d(&sm.in[m][0][0], &tm.m[m], 0, int(h), int(t0), int(b), &sm.in_bar);
   }
-  cp_async_commit();
 }
 
 // ------------------------------------------------------------------ context warps
+// `degraded` (CTA-uniform, sticky): a wait for staged inputs ran out; from then on nothing more is
+// staged and every chunk takes the token path, which reads its inputs from global memory.
 template <typename T>
-__device__ __forceinline__ void build_context(const FwdArgs& p, FwdSmem3<T>& sm, Ctx& cx, unsigned mask, int64_t b,
-                                              int64_t h, int64_t c, int64_t nc, int ktid) {
+__device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps& tm, FwdSmem3<T>& sm, Ctx& cx,
+                                              unsigned mask, int64_t b, int64_t h, int64_t c, int64_t nc, int ktid,
+                                              bool& degraded) {
   const int kw = ktid >> 5, lane = ktid & 31;
   const int g = lane >> 2, c4 = lane & 3;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
-  const T (*X)[kChunk][kStrIn] = sm.in;
+  const T (*X)[kChunk][kN] = sm.in;
+  const int len = int(min64(kChunk, p.T - c * kChunk));
+
+  const bool timed_out = !degraded && !mbar_wait_bounded(&sm.in_bar, unsigned(c & 1), kWaitLimitNs);
 
   // ---- K1: decay products and decay-scaled operands.  Thread = (token quarter kw; columns lane
   // and lane + 32, as one packed fp32 pair); the transposed copies go out as one float4 per column.
@@ -154,14 +150,15 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, FwdSmem3<T>& sm,
   {
     const int tq = 4 * kw, ja = lane, jb = lane + 32;
     auto ld2 = [&](int m, int t) { return make_float2(Elt<T>::to_f32(X[m][t][ja]), Elt<T>::to_f32(X[m][t][jb])); };
+    auto ldw = [&](int t) { return t < len ? ld2(1, t) : make_float2(1.f, 1.f); };   // padding: w = 1
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
-    for (int t = 0; t < tq; ++t) lam = mul2(lam, ld2(1, t));
+    for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
     float at[2][4], bh[2][4], kh[2][4], vv[2][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = tq + u;
       const float2 lp = lam;
-      lam = mul2(lam, ld2(1, t));
+      lam = mul2(lam, ldw(t));
       bad |= !(lam.x >= 0x1p-40f && lam.x <= 0x1p40f) || !(lam.y >= 0x1p-40f && lam.y <= 0x1p40f);
       const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
       const float2 a2 = mul2(ld2(4, t), lp), r2 = mul2(ld2(0, t), lam);
@@ -194,19 +191,24 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, FwdSmem3<T>& sm,
       cx.lam15[jb] = lam.y;
     }
   }
-  const unsigned any_bad = __ballot_sync(0xffffffffu, bad);
-  if (lane == 0) sm.kbad[kw] = any_bad ? 1 : 0;
+  const unsigned any_bad = __ballot_sync(0xffffffffu, bad), any_to = __ballot_sync(0xffffffffu, timed_out);
+  if (lane == 0) sm.kbad[kw] = (any_bad ? 1 : 0) | (any_to ? 2 : 0);
   named_bar(1, 128);
-  const bool unsafe = (sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3]) != 0;
+  const int kb = sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3];
+  if ((kb & 2) && !degraded) {
+    degraded = true;
+    if (ktid == 0 && p.status) atomicOr(p.status, kStatusWaitTimeout);
+  }
+  const bool unsafe = kb != 0 || degraded;
   if (ktid == 0) {
     cx.mask = int(mask);
     cx.unsafe = unsafe ? 1 : 0;
   }
 
   // the staged inputs are consumed: fetch the next chunk while the rest is built
-  if (c + 1 < nc) {
+  if (c + 1 < nc && !degraded) {
     const int64_t t1 = (c + 1) * kChunk;
-    stage_chunk<T>(p, sm.in, b, h, t1, int(min64(kChunk, p.T - t1)), ktid);
+    stage_chunk<T>(p, tm, sm, b, h, t1, ktid);
   }
   if (unsafe) return;
 
@@ -529,8 +531,8 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned ma
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+__global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p, const __grid_constant__ InputMaps tm) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
   FwdSmem3<T>& sm = *reinterpret_cast<FwdSmem3<T>*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
@@ -597,12 +599,15 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
   } else {
     // prologue: stage chunk 0 and fetch its reset flags
     unsigned reset_bits;
+    bool degraded = false;
+    unsigned stuck = 0;   // parity of the phase whose wait ran out
     {
+      if (ktid == 0) mbar_init(&sm.in_bar, 1);
+      named_bar(1, 128);
       const int len0 = int(min64(kChunk, p.T));
-      stage_chunk<T>(p, sm.in, b, h, 0, len0, ktid);
+      stage_chunk<T>(p, tm, sm, b, h, 0, ktid);
       const bool f = p.reset && lane < len0 && p.reset[b * p.T + lane] != 0;
       reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
-      cp_async_wait_all();
     }
     cta_sync();
     for (int64_t it = 0; it <= nc; ++it) {
@@ -615,30 +620,33 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(FwdArgs p) {
           const bool f = p.reset && lane < len1 && p.reset[b * p.T + t1 + lane] != 0;
           reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
         }
-        build_context<T>(p, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid);
-        cp_async_wait_all();
+        const bool was_degraded = degraded;
+        build_context<T>(p, tm, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid, degraded);
+        if (degraded && !was_degraded) stuck = unsigned(c & 1);
       }
       cta_sync();
     }
+    // a wait that ran out may have left copies in flight: give them a bounded chance to land
+    if (degraded) mbar_wait_bounded(&sm.in_bar, stuck, kWaitLimitNs / 100);
   }
 }
 
 template <typename T>
-cudaError_t launch(const FwdArgs& p, cudaStream_t stream) {
+cudaError_t launch(const FwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
   const size_t smem = sizeof(FwdSmem3<T>);
   cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  chunk_fwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p);
+  chunk_fwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-cudaError_t launch_chunk_fwd(const FwdArgs& p, int dtype, cudaStream_t stream) {
+cudaError_t launch_chunk_fwd(const FwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream) {
   switch (dtype) {
-    case 0: return launch<float>(p, stream);
-    case 1: return launch<__nv_bfloat16>(p, stream);
-    case 2: return launch<__half>(p, stream);
+    case 0: return launch<float>(p, tm, stream);
+    case 1: return launch<__nv_bfloat16>(p, tm, stream);
+    case 2: return launch<__half>(p, tm, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -1,6 +1,8 @@
 // Internal launch interface between the C-ABI layer (wkv7_api.cu) and the kernels.
 #pragma once
 
+#include <cuda.h>
+
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -14,7 +16,15 @@ struct FwdArgs {
   void* y;                // [B,T,H,64]
   float* s_out;           // [B,H,64,64] or null
   float* ckpt;            // [B,H,ceil(T/16),64,64] or null
+  int* status;            // device status word: bits of wkv7 device errors (bounded waits that ran out)
+  unsigned extra_tx;      // test hook: bytes a staging expects beyond what it copies (0 in normal use)
 };
+
+// Bits of the device status word.
+constexpr int kStatusWaitTimeout = 1;
+
+// Wall-clock limit of one bounded wait on a staging barrier (the copies it waits for take microseconds).
+constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
 
 struct BwdArgs {
   int64_t B, T, H;
@@ -27,6 +37,8 @@ struct BwdArgs {
   void *dr, *dw, *dk, *dv, *da, *db;
   float* ds0;
   int* unit_flags;   // [B*H] in the workspace tail: the chunked backward marks units it could not handle
+  int* status;       // device status word (see FwdArgs)
+  unsigned extra_tx; // test hook (see FwdArgs)
 };
 
 struct StepArgs {
@@ -42,7 +54,17 @@ cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 // only_flagged: run only the (b,h) units whose unit_flags entry is non-zero (others exit at once).
 cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
-cudaError_t launch_chunk_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
-cudaError_t launch_chunk_bwd(const BwdArgs& p, int dtype, cudaStream_t stream);
+// Device address of this device's status word (looked up once per device).
+cudaError_t device_status_ptr(int** out);
+
+// Tensor maps of the token inputs for the chunked kernels' TMA staging.  Each [B,T,H,64] input is
+// viewed as the 4-D tensor {64, H, T, B} (innermost first) and one box is {64, 1, 16, 1}: the 16
+// tokens of a chunk for one head, rows past T filled with zeros.  Order r, w, k, v, a, b, dy.
+struct InputMaps {
+  CUtensorMap m[7];
+};
+
+cudaError_t launch_chunk_fwd(const FwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream);
+cudaError_t launch_chunk_bwd(const BwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream);
 
 }  // namespace wkv7

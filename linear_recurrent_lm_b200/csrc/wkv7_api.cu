@@ -1,8 +1,12 @@
 // C ABI of libwkv7 (declared in include/wkv7.h): argument validation and
 // dispatch to the sm_100a kernels.  Nothing here allocates memory or keeps
 // state between calls; every kernel runs on the caller's stream.
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <mutex>
 
 #include "kernels.h"
 #include "wkv7.h"
@@ -23,7 +27,8 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
 // Common descriptor checks.  On success fills the element counts.
 wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
   if (!d) return WKV7_ERR_NULL;
-  if (d->N != 64 || d->flags != 0u) return WKV7_ERR_UNSUPPORTED;
+  if (d->N != 64 || (d->flags & ~WKV7_FLAG_TEST_WAIT_TIMEOUT) != 0u) return WKV7_ERR_UNSUPPORTED;
+  if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
   if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
   if (d->algo != WKV7_ALGO_AUTO && d->algo != WKV7_ALGO_SCAN && d->algo != WKV7_ALGO_CHUNKED)
     return WKV7_ERR_UNSUPPORTED;
@@ -51,6 +56,48 @@ wkv7_status_t check_ptrs(bool need, std::initializer_list<const void*> ptrs) {
 }
 
 wkv7_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA; }
+
+// cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link to libcuda).
+PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
+  static std::once_flag once;
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(f);
+  });
+  return fn;
+}
+
+// Tensor maps of up to seven [B,T,H,64] inputs as {64, H, T, B} with a {64, 1, 16, 1} box (the
+// chunked kernels' staging).  Unused slots stay zero.
+wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const void*> ptrs, wkv7::InputMaps* tm) {
+  *tm = wkv7::InputMaps{};
+  if (d->T > INT32_MAX || d->H > INT32_MAX || d->B > INT32_MAX) return WKV7_ERR_SHAPE;   // 32-bit box coordinates
+  PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
+  if (!enc) return WKV7_ERR_CUDA;
+  const cuuint64_t es = d->dtype == WKV7_F32 ? 4 : 2;
+  const CUtensorMapDataType dt = d->dtype == WKV7_F32    ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32
+                                 : d->dtype == WKV7_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                         : CU_TENSOR_MAP_DATA_TYPE_FLOAT16;
+  const cuuint64_t dims[4] = {64, cuuint64_t(d->H), cuuint64_t(d->T), cuuint64_t(d->B)};
+  const cuuint64_t strides[3] = {64 * es, cuuint64_t(d->H) * 64 * es, cuuint64_t(d->T) * cuuint64_t(d->H) * 64 * es};
+  const cuuint32_t box[4] = {64, 1, 16, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  int i = 0;
+  for (const void* ptr : ptrs) {
+    if (enc(&tm->m[i++], dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return WKV7_ERR_CUDA;
+  }
+  return WKV7_OK;
+}
+
+// Bytes a staging barrier expects beyond its copies: the timeout test hook (see wkv7.h).
+unsigned test_extra_tx(const wkv7_desc_t* d) { return (d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) ? 16u : 0u; }
 
 bool use_chunked(const wkv7_desc_t* d) {
   if (d->algo == WKV7_ALGO_CHUNKED) return true;
@@ -109,10 +156,16 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   st = check_ptrs(false, {s0, s_out, workspace});
   if (st != WKV7_OK) return st;
   if (units == 0) return WKV7_OK;
-  wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace)};
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
+                  status, test_extra_tx(d)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_fwd(p, d->dtype, s));
-  return from_cuda(wkv7::launch_chunk_fwd(p, d->dtype, s));
+  wkv7::InputMaps tm;
+  st = encode_inputs(d, {r, w, k, v, a, b}, &tm);
+  if (st != WKV7_OK) return st;
+  return from_cuda(wkv7::launch_chunk_fwd(p, tm, d->dtype, s));
 }
 
 wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
@@ -131,12 +184,17 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   int* flags = d->T > 0 ? reinterpret_cast<int*>(static_cast<char*>(const_cast<void*>(workspace)) +
                                                  checkpoint_bytes(d, units))
                         : nullptr;
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
-                  dr, dw, dk, dv, da, db, ds0, flags};
+                  dr, dw, dk, dv, da, db, ds0, flags, status, test_extra_tx(d)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, false, s));
   // Chunked pass, then the exact scan for the units it marked (decays too small for 1/L scaling).
-  cudaError_t e = wkv7::launch_chunk_bwd(p, d->dtype, s);
+  wkv7::InputMaps tm;
+  st = encode_inputs(d, {r, w, k, v, a, b, dy}, &tm);
+  if (st != WKV7_OK) return st;
+  cudaError_t e = wkv7::launch_chunk_bwd(p, tm, d->dtype, s);
   if (e != cudaSuccess) return WKV7_ERR_CUDA;
   return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, true, s));
 }

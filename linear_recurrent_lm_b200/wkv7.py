@@ -9,6 +9,7 @@ stream.  The same entry points as the C ABI:
   -> dict(dr, dw, dk, dv, da, db, ds0)
 * ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
 * ``workspace_bytes(B, T, H, dtype)``
+* ``device_status(clear=True)`` -> OK or ERR_TIMEOUT (synchronises the device)
 
 Tensors are [B,T,H,64] (token inputs), [B,H,64,64] fp32 (states), [B,T] uint8
 (reset), [B] uint8 (active), all on one CUDA device and contiguous.  If the
@@ -28,6 +29,7 @@ LIB_PATH = os.path.join(_HERE, "libwkv7.so")
 (OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT,
  ERR_SCRATCH_LIMIT) = range(10)
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
+FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2}
 N_HEAD = 64
@@ -71,6 +73,8 @@ def lib() -> ctypes.CDLL:
         L.wkv7_step.argtypes = [dp] + [vp] * 10
         L.wkv7_train_step_noalloc.restype = ctypes.c_int
         L.wkv7_train_step_noalloc.argtypes = [dp] + [vp] * 20
+        L.wkv7_get_device_status.restype = ctypes.c_int
+        L.wkv7_get_device_status.argtypes = [ctypes.c_int]
         _lib = L
     return _lib
 
@@ -85,6 +89,11 @@ def make_desc(B: int, T: int, H: int, dtype, algo: str = "auto", N: int = N_HEAD
 
 def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16) -> int:
     return int(lib().wkv7_workspace_bytes(ctypes.byref(make_desc(B, T, H, dtype))))
+
+
+def device_status(clear: bool = True) -> int:
+    """The device status word of the current device (synchronises it): OK or ERR_TIMEOUT."""
+    return int(lib().wkv7_get_device_status(1 if clear else 0))
 
 
 def _ptr(x: Optional[torch.Tensor]):
@@ -108,7 +117,7 @@ def _token_shape(x: torch.Tensor):
 
 
 def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, workspace=None,
-            need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None):
+            need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None, flags: int = 0):
     """WKV-7 forward over [B,T,H,64] inputs.  Returns (y, s_out, workspace)."""
     B, T, H = _token_shape(r)
     dev = r.device
@@ -118,7 +127,7 @@ def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, worksp
         s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=dev, dtype=torch.float32)
     if workspace is None and need_workspace:
         workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype), 16), device=dev, dtype=torch.uint8)
-    d = make_desc(B, T, H, r.dtype, algo)
+    d = make_desc(B, T, H, r.dtype, algo, flags=flags)
     st = lib().wkv7_forward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, workspace)),
                             _stream(stream))
     _check(st, "wkv7_forward")
@@ -126,7 +135,7 @@ def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, worksp
 
 
 def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, grads=None,
-             want_ds0: bool = True, algo: str = "auto", stream=None) -> Dict[str, torch.Tensor]:
+             want_ds0: bool = True, algo: str = "auto", stream=None, flags: int = 0) -> Dict[str, torch.Tensor]:
     """WKV-7 backward from the checkpoints written by ``forward``."""
     B, T, H = _token_shape(r)
     g = dict(grads) if grads is not None else {}
@@ -135,7 +144,7 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
             g[n] = torch.empty_like(r)
     if g.get("ds0") is None and want_ds0:
         g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
-    d = make_desc(B, T, H, r.dtype, algo)
+    d = make_desc(B, T, H, r.dtype, algo, flags=flags)
     st = lib().wkv7_backward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, dy, dsT, workspace)),
                              *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
                              _stream(stream))

@@ -73,6 +73,10 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 1
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 17, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT)   # the test hook needs T <= 16
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 2)
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = 7
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.dtype = 9
@@ -114,3 +118,4 @@ def test_no_cpu_fallback_without_gpu(L):
         pytest.skip("host has a GPU")
     d = L.make_desc(1, 16, 1, torch.bfloat16)
     assert call_fwd(L, d) == L.ERR_CUDA
+    assert L.device_status() == L.ERR_CUDA      # the status word cannot be read without a device
