@@ -42,6 +42,9 @@ BYTES_PREFILL = 768 + 128
 BYTES_DECODE = 64 * 64 * 4 * 2 + 768 + 128
 
 
+NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal (context: the roofline uses the measured copy bandwidth)
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -362,6 +365,7 @@ def main():
                         "frac": (BYTES_FWD_TRAIN + BYTES_BWD) * units / (ms_per_step / 1e3) / 1e9 / peak},
             "roofline": {"bound": "hbm", "kernel": kname, "achieved": dominant[2], "peak": peak, "unit": "GB/s",
                          "frac": dominant[2] / peak, "peak_kind": peak_kind,
+                         "frac_of_nominal_8000": dominant[2] / NOMINAL_HBM_GBS,
                          "bytes_per_launch": dominant[3] * units,
                          "traffic": traffic},
             "cpu_baseline": cpu,

@@ -32,8 +32,8 @@
 // scan backward then recomputes exactly those units.
 //
 // Work split (one CTA of 8 warps per (b,h)), chunks in reverse, pipelined:
-//   warps 4-7 ("context") for chunk c-1: stage its inputs (cp.async) and
-//     its checkpoint, build the decay-scaled operands, the masked Gram, T,
+//   warps 4-7 ("context") for chunk c-1: stage its inputs (one TMA box per
+//     input on an mbarrier, bounded waits) and its checkpoint, build the decay-scaled operands, the masked Gram, T,
 //     W, X and the recomputed SA = W S0^T + X V into one half of a double
 //     buffer;
 //   warps 0-3 ("main") for chunk c: warp w owns rows 16w..16w+15 of dS as

@@ -28,7 +28,8 @@
 // 1/L scaling and is run token by token instead.
 //
 // Work split (one CTA of 8 warps per (b,h)), pipelined over chunks:
-//   warps 4-7 ("context") for chunk c+1: stage the inputs (cp.async), build
+//   warps 4-7 ("context") for chunk c+1: stage the inputs (one TMA box per
+//     input on an mbarrier, bounded waits), build
 //     the decay-scaled operands, the masked Gram of [At; Rt] and [Bh; Kh] and
 //     T into one half of a double-buffered context;
 //   warps 0-3 ("state") for chunk c: warp w owns rows 16w..16w+15 of S as
