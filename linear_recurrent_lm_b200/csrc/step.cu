@@ -3,80 +3,80 @@
 // The rwkv-metal page runs one token as plain array ops ("wkv7_step(...,
 // h_in)") and keeps "exact right-padding for ragged batches".  Here one
 // launch steps every (b,h) state: it is a pure stream over the 16 KiB state
-// (read once, written once) and therefore HBM-bound.  One CTA per (b,h), 256
-// threads; thread t owns row t/4 and the 16 columns 16*(t%4)..+15, held as
-// four float4 -- each warp reads and writes 2 KiB of contiguous state with
-// 16-byte accesses.  The two row dot products (sa and y) reduce over the 4
-// lanes of a row with two xor-shuffles.  Rows of the batch with active[b]==0
-// exit before touching the state, which therefore stays bitwise unchanged,
-// and write y = 0.
+// (read once, written once) and therefore HBM-bound.  One CTA per (b,h), 512
+// threads; thread t owns row t/8 and the 8 columns 8*(t%8)..+7, held as two
+// float4 -- each warp reads and writes 1 KiB of contiguous state with 16-byte
+// accesses, and few registers per thread keep many CTAs (and their loads) in
+// flight per SM.  The two row dot products (sa and y) reduce over the 8
+// lanes of a row with three xor-shuffles.  A row of the batch with active[b]==0
+// never writes its state, which therefore stays bitwise unchanged, and writes
+// y = 0; its flag is loaded together with the state and the inputs, so no
+// load waits for another.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace wkv7 {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 512;
 
+// Eight consecutive elements of T (16-byte aligned) as fp32.
 template <typename T>
-__device__ __forceinline__ void load16(const T* g, float* out) {
+__device__ __forceinline__ void load8(const T* g, float* out) {
   constexpr int n = Vec16<T>::n;
 #pragma unroll
-  for (int u = 0; u < 16 / n; ++u) {
+  for (int u = 0; u < 8 / n; ++u) {
     const uint4 raw = __ldg(reinterpret_cast<const uint4*>(g + u * n));
     unpack16<T>(raw, out + u * n);
   }
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads) step_kernel(StepArgs p) {
+__global__ void __launch_bounds__(kThreads, 3) step_kernel(StepArgs p) {
   const int64_t unit = blockIdx.x;
   const int64_t b = unit / p.H;
   const int t = threadIdx.x;
-  const int i = t >> 2, q = t & 3;
+  const int i = t >> 3, q = t & 7;   // row i, columns 8q..8q+7
   T* y = static_cast<T*>(p.y) + unit * kN;
-  if (p.active && !p.active[b]) {
-    if (q == 0) y[i] = Elt<T>::from_f32(0.f);
-    return;
-  }
-  float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 16);
-  float S[16];
-#pragma unroll
-  for (int u = 0; u < 4; ++u) {
-    const float4 s4 = row[u];
-    S[4 * u] = s4.x; S[4 * u + 1] = s4.y; S[4 * u + 2] = s4.z; S[4 * u + 3] = s4.w;
-  }
-  const int64_t o = unit * kN + q * 16;
-  float wv[16], kv[16], av[16], bv[16], rv[16];
-  load16<T>(static_cast<const T*>(p.a) + o, av);
-  load16<T>(static_cast<const T*>(p.w) + o, wv);
-  load16<T>(static_cast<const T*>(p.b) + o, bv);
-  load16<T>(static_cast<const T*>(p.k) + o, kv);
-  load16<T>(static_cast<const T*>(p.r) + o, rv);
+  const bool act = !p.active || p.active[b] != 0;
+  float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 8);
+  const float4 s_lo = row[0], s_hi = row[1];
+  float S[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
+  const int64_t o = unit * kN + q * 8;
+  float wv[8], kv[8], av[8], bv[8], rv[8];
+  load8<T>(static_cast<const T*>(p.a) + o, av);
+  load8<T>(static_cast<const T*>(p.w) + o, wv);
+  load8<T>(static_cast<const T*>(p.b) + o, bv);
+  load8<T>(static_cast<const T*>(p.k) + o, kv);
+  load8<T>(static_cast<const T*>(p.r) + o, rv);
   const float vi = Elt<T>::to_f32(static_cast<const T*>(p.v)[unit * kN + i]);
 
   float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 16; j += 2) {
+  for (int j = 0; j < 8; j += 2) {
     s0 = fmaf(S[j], av[j], s0);
     s1 = fmaf(S[j + 1], av[j + 1], s1);
   }
   float sa = s0 + s1;
   sa += __shfl_xor_sync(0xffffffffu, sa, 1);
   sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+  sa += __shfl_xor_sync(0xffffffffu, sa, 4);
 
   float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 16; ++j) {
+  for (int j = 0; j < 8; ++j) {
     S[j] = fmaf(S[j], wv[j], fmaf(sa, bv[j], vi * kv[j]));
     if (j & 1) y1 = fmaf(S[j], rv[j], y1); else y0 = fmaf(S[j], rv[j], y0);
   }
-#pragma unroll
-  for (int u = 0; u < 4; ++u) row[u] = make_float4(S[4 * u], S[4 * u + 1], S[4 * u + 2], S[4 * u + 3]);
+  if (act) {
+    row[0] = make_float4(S[0], S[1], S[2], S[3]);
+    row[1] = make_float4(S[4], S[5], S[6], S[7]);
+  }
   float yy = y0 + y1;
   yy += __shfl_xor_sync(0xffffffffu, yy, 1);
   yy += __shfl_xor_sync(0xffffffffu, yy, 2);
-  if (q == 0) y[i] = Elt<T>::from_f32(yy);
+  yy += __shfl_xor_sync(0xffffffffu, yy, 4);
+  if (q == 0) y[i] = Elt<T>::from_f32(act ? yy : 0.f);
 }
 
 template <typename T>
