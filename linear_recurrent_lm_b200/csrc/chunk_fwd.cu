@@ -42,6 +42,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.cuh"
+#include "tc05.cuh"
 
 namespace wkv7 {
 namespace {
@@ -49,16 +50,17 @@ namespace {
 constexpr int kThreads = 256;
 constexpr int kIn = 6;       // staged inputs: r, w, k, v, a, b
 constexpr int kStrY = 72;    // row stride (elements) of the y staging tile
-constexpr int S68 = 68, S72 = 72, S20 = 20, S24 = 24;
+constexpr int S68 = 68, S20 = 20;
 using bf16 = __nv_bfloat16;
 
 // Produced by the context warps for one chunk, consumed by the state warps one iteration later.
-struct __align__(16) Ctx {
+struct __align__(128) Ctx {
   float Rt[kChunk][S68];    // m0 . rt  [t][j]   (fp32, initial value of Q)
   float AtT[kN][S20];       // at       [j][tau]
-  float BhT[kN][S24];       // bh       [j][tau]
-  float KhT[kN][S20];       // kh       [j][tau]
-  float VT[kN][S20];        // v        [i][tau]
+  // tcgen05 operands, K-major canonical layout (cidx): rows j (or i), K = tau
+  __align__(128) float VTc[kN * kChunk];    // v         (A of both state products)
+  __align__(128) float BhTc[kN * kChunk];   // ls . bh   (B of S_16)
+  __align__(128) float KhTc[kN * kChunk];   // ls . kh   (B of S_16)
   float Tm[kChunk][S20];    // T        [t][tau]
   float TT[kChunk][S20];    // T^T      [tau][t]
   float LakT[kChunk][S20];  // Lak^T    [tau][t]
@@ -75,11 +77,14 @@ struct __align__(128) FwdSmem3 {
   float GA[32][S68];        // rows 0..15 at_t, 16..31 rt_t   [t][j]
   float GB[32][S68];        // rows 0..15 bh_t, 16..31 kh_t   [tau][j]
   __align__(16) float LabT[kChunk][S20];
-  float W[kChunk][S72], Q[kChunk][S72];      // [t][j]
-  float X[kChunk][S20], Z[kChunk][S20], M[kChunk][S20];
+  __align__(128) float B1[2 * kChunk * kN];      // [W; Q]: rows t (W) and 16 + t (Q), K = j (cidx, K 64)
+  __align__(128) float B1v[2 * kChunk * kChunk]; // [X; Z]: rows t and 16 + t, K = tau (cidx, K 16)
+  float M[kChunk][S20];
   __align__(128) T in[kIn][kChunk][kN];      // staged inputs of the chunk being built (TMA boxes)
   __align__(16) uint16_t Ys[kChunk][kStrY]; // y of the last chunk [t][i] (16-bit outputs), written next iteration
   unsigned long long in_bar;                 // completion of the bulk copies into `in` (one phase per chunk)
+  unsigned long long d1_bar, mma_bar;        // completion of a chunk's D1 MMAs / of all its MMAs (one phase per chunk)
+  uint32_t tmem_base;                        // TMEM: S0 (cols 0-63), D1 (64-95), D3 (128-191)
   int kbad[4];
 };
 
@@ -87,6 +92,15 @@ __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
 __device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 0;\n" ::: "memory"); }
+
+// Float index of element (r, k) of a K-major canonical tcgen05 operand with K = kdim (no swizzle:
+// 8-row x 16-byte core matrices, K-adjacent ones 128 bytes apart, row groups kdim/4 * 128 apart).
+__device__ __forceinline__ int cidx(int r, int k, int kdim) {
+  return (r >> 3) * (kdim * 8) + (k >> 2) * 32 + (r & 7) * 4 + (k & 3);
+}
+
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kTmS0 = 0, kTmD1 = 64, kTmD3 = 128;   // TMEM column offsets
 
 // Store four 8x8 b16 matrices from accumulator-fragment registers, transposed.
 __device__ __forceinline__ void stsm_x4_t(void* row_ptr, uint32_t r0, uint32_t r1, uint32_t r2, uint32_t r3) {
@@ -155,6 +169,7 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
     for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
     float at[2][4], bh[2][4], kh[2][4], vv[2][4];
+    const unsigned ls_bits = last_segment_bits(mask);   // S_16 sees only the chunk's last segment
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = tq + u;
@@ -179,13 +194,16 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
       cx.Rt[t][ja] = t < fr ? r2.x : 0.f;
       cx.Rt[t][jb] = t < fr ? r2.y : 0.f;
     }
+    const float l0 = (ls_bits >> tq) & 1u ? 1.f : 0.f, l1 = (ls_bits >> (tq + 1)) & 1u ? 1.f : 0.f;
+    const float l2 = (ls_bits >> (tq + 2)) & 1u ? 1.f : 0.f, l3 = (ls_bits >> (tq + 3)) & 1u ? 1.f : 0.f;
 #pragma unroll
     for (int q = 0; q < 2; ++q) {
       const int j = q ? jb : ja;
+      const int ci = cidx(j, tq, kChunk);   // four consecutive tau: one float4
       *reinterpret_cast<float4*>(&cx.AtT[j][tq]) = make_float4(at[q][0], at[q][1], at[q][2], at[q][3]);
-      *reinterpret_cast<float4*>(&cx.BhT[j][tq]) = make_float4(bh[q][0], bh[q][1], bh[q][2], bh[q][3]);
-      *reinterpret_cast<float4*>(&cx.KhT[j][tq]) = make_float4(kh[q][0], kh[q][1], kh[q][2], kh[q][3]);
-      *reinterpret_cast<float4*>(&cx.VT[j][tq]) = make_float4(vv[q][0], vv[q][1], vv[q][2], vv[q][3]);
+      *reinterpret_cast<float4*>(&cx.BhTc[ci]) = make_float4(l0 * bh[q][0], l1 * bh[q][1], l2 * bh[q][2], l3 * bh[q][3]);
+      *reinterpret_cast<float4*>(&cx.KhTc[ci]) = make_float4(l0 * kh[q][0], l1 * kh[q][1], l2 * kh[q][2], l3 * kh[q][3]);
+      *reinterpret_cast<float4*>(&cx.VTc[ci]) = make_float4(vv[q][0], vv[q][1], vv[q][2], vv[q][3]);
     }
     if (kw == 3) {
       cx.lam15[ja] = lam.x;
@@ -271,15 +289,34 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
 }
 
 // ------------------------------------------------------------------ state warps
+// One chunk of the state warps.  Steps a/b (mma.sync, 16x16 blocks) form W, Q, X, Z in the
+// tcgen05 operand layout; the state products then run as one batch of tcgen05 MMAs issued by one
+// thread (M = 64 rows i, accumulators in TMEM):
+//   D1 = S0 [W; Q]^T + V^T [X; Z]^T   (columns 0-15: SA^T, 16-31: Y^T),  S0 from TMEM (tf32)
+//   D3 = SA^T ls.Bh + V^T ls.Kh       (SA^T read back from D1 in TMEM as the A operand)
+// and S_16 = keep.S0 diag(L_15) + D3 diag(L_15) stays in the fp32 registers.  `mma_phase` counts
+// the batches issued so far (the parity of the mbarrier phase to wait for).
 template <typename T>
 __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, const Ctx& cx, float (&acc)[8][4],
-                                            int64_t b, int64_t h, int64_t t0, int len, int warp, int lane) {
+                                            int64_t b, int64_t h, int64_t t0, int len, int warp, int lane,
+                                            uint32_t tmem, unsigned& mma_phase) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
   const int j0 = 16 * warp;
   const unsigned mask = unsigned(cx.mask);
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
   const unsigned m0bits = (1u << fr) - 1u;   // tokens that S0 reaches
+  const uint32_t tlane = uint32_t(32 * warp) << 16;   // this warp's TMEM lanes (rows 16w..16w+15)
+
+  // ---- S0 in tf32 into TMEM (A operand of D1)
+  {
+    float s0t[8][4];
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) s0t[nt][e] = tf32f(acc[nt][e]);
+    tc::st_16x256b_x8(tmem + tlane + kTmS0, s0t);
+  }
 
   // ---- step a: W = T diag(m0) At (columns j0..j0+15), M = Mrb T (warp 0), X = T Lak (warp 1)
   uint32_t bat[2][4];   // At^T fragments of this warp's columns: [n-tile][k-step pair]
@@ -302,7 +339,7 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
-          *reinterpret_cast<float2*>(&sm.X[g + 8 * hh][8 * nt + 2 * c4]) =
+          *reinterpret_cast<float2*>(&sm.B1v[cidx(g + 8 * hh, 8 * nt + 2 * c4, kChunk)]) =
               make_float2(tf32f(xx[nt][2 * hh]), tf32f(xx[nt][2 * hh + 1]));
     }
     mask_nat(at[0], 0, c4, m0bits);
@@ -317,7 +354,7 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float2*>(&sm.W[g + 8 * hh][j0 + 8 * nt + 2 * c4]) =
+        *reinterpret_cast<float2*>(&sm.B1[cidx(g + 8 * hh, j0 + 8 * nt + 2 * c4, kN)]) =
             make_float2(tf32f(ww[nt][2 * hh]), tf32f(ww[nt][2 * hh + 1]));
     if (warp == 0) {   // M = Mrb T
       uint32_t am[2][4];
@@ -367,7 +404,7 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
       for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh)
-          *reinterpret_cast<float2*>(&sm.Z[g + 8 * hh][8 * nt + 2 * c4]) =
+          *reinterpret_cast<float2*>(&sm.B1v[cidx(kChunk + g + 8 * hh, 8 * nt + 2 * c4, kChunk)]) =
               make_float2(tf32f(zz[nt][2 * hh]), tf32f(zz[nt][2 * hh + 1]));
     }
     mask_nat(am[0], 0, c4, m0bits);
@@ -390,37 +427,47 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float2*>(&sm.Q[g + 8 * hh][j0 + 8 * nt + 2 * c4]) =
+        *reinterpret_cast<float2*>(&sm.B1[cidx(kChunk + g + 8 * hh, j0 + 8 * nt + 2 * c4, kN)]) =
             make_float2(tf32f(qq[nt][2 * hh]), tf32f(qq[nt][2 * hh + 1]));
   }
+  // operands visible to the tensor core, S0 in TMEM, then one thread issues the batch
+  tc::fence_smem_to_async();
+  tc::wait_st();
+  tc::fence_before_sync();
   named_bar(2, 128);
+  if (warp == 0 && lane == 0) {
+    tc::fence_after_sync();
+    constexpr uint32_t id32 = tc::idesc_tf32(64, 32), id64 = tc::idesc_tf32(64, 64);
+#pragma unroll
+    for (int s = 0; s < kN / 8; ++s)   // S0 [W; Q]^T over j, 8 per MMA
+      tc::mma_ts(tmem + kTmD1, tmem + kTmS0 + 8 * s, tc::smem_desc(&sm.B1[64 * s], 8 * kN * 4), id32, s > 0);
+#pragma unroll
+    for (int s = 0; s < 2; ++s)        // + V^T [X; Z]^T over tau
+      tc::mma_ss(tmem + kTmD1, tc::smem_desc(&cx.VTc[64 * s], 8 * kChunk * 4),
+                 tc::smem_desc(&sm.B1v[64 * s], 8 * kChunk * 4), id32, true);
+    // D3 reads D1 through the A-operand path: issue it only once D1 is complete
+    tc::commit(&sm.d1_bar);
+    if (!mbar_wait_bounded(&sm.d1_bar, mma_phase & 1u, kWaitLimitNs) && p.status) atomicOr(p.status, kStatusWaitTimeout);
+    tc::fence_after_sync();
+#pragma unroll
+    for (int s = 0; s < 2; ++s)        // D3 = SA^T ls.Bh (SA^T = D1 columns 0-15) ...
+      tc::mma_ts(tmem + kTmD3, tmem + kTmD1 + 8 * s, tc::smem_desc(&cx.BhTc[64 * s], 8 * kChunk * 4), id64, s > 0);
+#pragma unroll
+    for (int s = 0; s < 2; ++s)        // ... + V^T ls.Kh
+      tc::mma_ss(tmem + kTmD3, tc::smem_desc(&cx.VTc[64 * s], 8 * kChunk * 4),
+                 tc::smem_desc(&cx.KhTc[64 * s], 8 * kChunk * 4), id64, true);
+    tc::commit(&sm.mma_bar);
+  }
+  if (!mbar_wait_bounded(&sm.mma_bar, mma_phase & 1u, kWaitLimitNs) && threadIdx.x == 0 && p.status)
+    atomicOr(p.status, kStatusWaitTimeout);
+  ++mma_phase;
+  tc::fence_after_sync();
 
-  // ---- S1: SA^T, Y^T (rows i, columns t) = S0 [W^T | Q^T] + V^T [X^T | Z^T]
-  float sa[2][4] = {}, yy[2][4] = {};
-#pragma unroll
-  for (int ks = 0; ks < 8; ++ks) {
-    uint32_t a[4] = {to_tf32(acc[ks][0]), to_tf32(acc[ks][2]), to_tf32(acc[ks][1]), to_tf32(acc[ks][3])};
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      const uint2 wb = *reinterpret_cast<const uint2*>(&sm.W[8 * nt + g][8 * ks + 2 * c4]);
-      const uint2 qb = *reinterpret_cast<const uint2*>(&sm.Q[8 * nt + g][8 * ks + 2 * c4]);
-      mma1688(sa[nt], a, wb.x, wb.y);
-      mma1688(yy[nt], a, qb.x, qb.y);
-    }
-  }
-  uint32_t av[2][4];
-#pragma unroll
-  for (int s = 0; s < 2; ++s) ldsm_x4(av[s], a32_addr(&cx.VT[0][0], S20, row0, 8 * s, lane));
-#pragma unroll
-  for (int nt = 0; nt < 2; ++nt) {
-    uint32_t xb[4], zb[4];
-    ldsm_x4(xb, b32_2k_addr(&sm.X[0][0], S20, 8 * nt, 0, lane));
-    ldsm_x4(zb, b32_2k_addr(&sm.Z[0][0], S20, 8 * nt, 0, lane));
-    mma1688(sa[nt], av[0], xb[0], xb[1]);
-    mma1688(sa[nt], av[1], xb[2], xb[3]);
-    mma1688(yy[nt], av[0], zb[0], zb[1]);
-    mma1688(yy[nt], av[1], zb[2], zb[3]);
-  }
+  float yy[2][4], d[8][4];
+  tc::ld_16x256b_x2(tmem + tlane + kTmD1 + kChunk, yy);   // Y^T: D1 columns 16-31
+  tc::ld_16x256b_x8(tmem + tlane + kTmD3, d);
+  tc::wait_ld();
+
   if constexpr (sizeof(T) == 2) {   // Y^T fragments -> Ys[t][i]; written out after the next CTA barrier
     const int m = lane >> 3;
     stsm_x4_t(&sm.Ys[8 * (m >> 1) + (lane & 7)][row0 + 8 * (m & 1)], pack16<T>(yy[0][0], yy[0][1]),
@@ -436,41 +483,18 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
       }
   }
 
-  // ---- S3: S_16 = keep.S0 diag(L_15) + (SA^T Bh + V^T Kh) diag(L_15), last segment only
-  const unsigned seg_last = __popc(mask & 0xfffeu);
-  unsigned last_bits = 0u;
-#pragma unroll
-  for (int t = 0; t < kChunk; ++t) last_bits |= (unsigned(__popc(mask & ((2u << t) - 2u))) == seg_last ? 1u : 0u) << t;
+  // ---- S_16 = keep.S0 diag(L_15) + D3 diag(L_15)
   const float keep = mask == 0u ? 1.f : 0.f;
-  uint32_t asa[2][4];
-#pragma unroll
-  for (int s = 0; s < 2; ++s) {
-    const int k0 = 8 * s + 2 * c4;   // permuted k: a0,a1 <-> k0, a2,a3 <-> k0 + 1
-    const bool e0 = (last_bits >> k0) & 1u, e1 = (last_bits >> (k0 + 1)) & 1u;
-    asa[s][0] = e0 ? to_tf32(sa[s][0]) : 0u;
-    asa[s][1] = e0 ? to_tf32(sa[s][2]) : 0u;
-    asa[s][2] = e1 ? to_tf32(sa[s][1]) : 0u;
-    asa[s][3] = e1 ? to_tf32(sa[s][3]) : 0u;
-    mask_nat(av[s], s, c4, last_bits);
-  }
 #pragma unroll
   for (int jt = 0; jt < 8; ++jt) {
-    float d[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-    for (int s = 0; s < 2; ++s) {
-      const uint2 bb = *reinterpret_cast<const uint2*>(&cx.BhT[8 * jt + g][8 * s + 2 * c4]);
-      mma1688(d, asa[s], bb.x, bb.y);
-    }
-    uint32_t kb[4];
-    ldsm_x4(kb, b32_2k_addr(&cx.KhT[0][0], S20, 8 * jt, 0, lane));
-    mma1688(d, av[0], kb[0], kb[1]);
-    mma1688(d, av[1], kb[2], kb[3]);
     const float2 l2 = *reinterpret_cast<const float2*>(&cx.lam15[8 * jt + 2 * c4]);
-    acc[jt][0] = fmaf(keep * acc[jt][0], l2.x, d[0] * l2.x);
-    acc[jt][1] = fmaf(keep * acc[jt][1], l2.y, d[1] * l2.y);
-    acc[jt][2] = fmaf(keep * acc[jt][2], l2.x, d[2] * l2.x);
-    acc[jt][3] = fmaf(keep * acc[jt][3], l2.y, d[3] * l2.y);
+    acc[jt][0] = fmaf(keep * acc[jt][0], l2.x, d[jt][0] * l2.x);
+    acc[jt][1] = fmaf(keep * acc[jt][1], l2.y, d[jt][1] * l2.y);
+    acc[jt][2] = fmaf(keep * acc[jt][2], l2.x, d[jt][2] * l2.x);
+    acc[jt][3] = fmaf(keep * acc[jt][3], l2.y, d[jt][3] * l2.y);
   }
+  // the next batch overwrites D1/D3 and S0: every warp's loads are done before it is issued
+  tc::fence_before_sync();
 }
 
 // Token-by-token update of one chunk on the state fragments (decay out of range), inputs read from global.
@@ -559,7 +583,19 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         acc[nt][2 * hh] = v2.x;
         acc[nt][2 * hh + 1] = v2.y;
       }
-    cta_sync();   // chunk 0 staged
+    if (warp == 0) {   // 256 TMEM columns: two CTAs per SM fill the 512 exactly
+      tc::alloc(&sm.tmem_base, kTmemCols);
+      tc::relinquish();
+    }
+    if (tid == 0) {
+      mbar_init(&sm.d1_bar, 1);
+      mbar_init(&sm.mma_bar, 1);
+    }
+    tc::fence_before_sync();
+    cta_sync();   // chunk 0 staged; TMEM allocated
+    tc::fence_after_sync();
+    const uint32_t tmem = sm.tmem_base;
+    unsigned mma_phase = 0;
     // y of the previous chunk (16-bit outputs): this thread's 16-byte piece of token row tid/8
     T* ydst = nullptr;
     const int ytt = tid >> 3, ypart = tid & 7;
@@ -574,7 +610,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         const int64_t t0 = c * kChunk;
         const int len = int(min64(kChunk, p.T - t0));
         if (!cx.unsafe) {
-          state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane);
+          state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane, tmem, mma_phase);
           if (sizeof(T) == 2 && ytt < len) ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
         } else {
           state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
@@ -589,6 +625,10 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
       cta_sync();   // context of chunk it handed over; Ys complete
     }
     if (ydst) *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+    // every batch was waited for and every TMEM load is complete: release TMEM
+    named_bar(2, 128);
+    tc::fence_after_sync();
+    if (warp == 0) tc::dealloc(tmem, kTmemCols);
     if (p.s_out) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
@@ -624,6 +664,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         const bool was_degraded = degraded;
         build_context<T>(p, tm, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid, degraded);
         if (degraded && !was_degraded) stuck = unsigned(c & 1);
+        tc::fence_smem_to_async();   // the tcgen05 operands of the context, for the tensor core
       }
       cta_sync();
     }
