@@ -61,8 +61,7 @@ struct __align__(128) Ctx {
   __align__(128) float VTc[kN * kChunk];    // v         (A of both state products)
   __align__(128) float BhTc[kN * kChunk];   // ls . bh   (B of S_16)
   __align__(128) float KhTc[kN * kChunk];   // ls . kh   (B of S_16)
-  float Tm[kChunk][S20];    // T        [t][tau]
-  float TT[kChunk][S20];    // T^T      [tau][t]
+  float LabT[kChunk][S20];  // Lab^T    [tau][t] (fp32, for T)
   float LakT[kChunk][S20];  // Lak^T    [tau][t]
   float Mrb[kChunk][S20];   // Mrb      [t][tau]
   float Mrk[kChunk][S20];   // Mrk      [t][tau] (fp32, initial value of Z)
@@ -76,7 +75,8 @@ struct __align__(128) FwdSmem3 {
   Ctx ctx[2];
   float GA[32][S68];        // rows 0..15 at_t, 16..31 rt_t   [t][j]
   float GB[32][S68];        // rows 0..15 bh_t, 16..31 kh_t   [tau][j]
-  __align__(16) float LabT[kChunk][S20];
+  __align__(16) float Tm[kChunk][S20];      // T   [t][tau]  (state warps)
+  __align__(16) float TT[kChunk][S20];      // T^T [tau][t]
   __align__(128) float B1[2 * kChunk * kN];      // [W; Q]: rows t (W) and 16 + t (Q), K = j (cidx, K 64)
   __align__(128) float B1v[2 * kChunk * kChunk]; // [X; Z]: rows t and 16 + t, K = tau (cidx, K 16)
   float M[kChunk][S20];
@@ -253,38 +253,11 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
         bool ok = strict ? (tau < t) : (tau <= t);
         ok = ok && ((mask & ((2u << t) - (2u << tau))) == 0u);   // no reset in (tau, t]
         const float v = ok ? gr[nt][e] : 0.f;
-        if (kw == 0) sm.LabT[tau][t] = v;
+        if (kw == 0) cx.LabT[tau][t] = v;
         else if (kw == 1) cx.LakT[tau][t] = tf32f(v);
         else if (kw == 2) cx.Mrb[t][tau] = tf32f(v);
         else cx.Mrk[t][tau] = v;
       }
-  }
-  named_bar(1, 128);
-
-  // ---- K3: T = (I - Lab)^-1 by forward substitution, one column per lane (warp kw == 0)
-  if (kw == 0 && lane < kChunk) {
-    const int cc = lane;
-    float u[kChunk];
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
-#pragma unroll
-    for (int tau = 0; tau < kChunk - 1; ++tau) {
-      const float4* lrow = reinterpret_cast<const float4*>(&sm.LabT[tau][0]);
-      float lv[kChunk];
-#pragma unroll
-      for (int q = (tau + 1) / 4; q < 4; ++q) {
-        const float4 f = lrow[q];
-        lv[4 * q] = f.x; lv[4 * q + 1] = f.y; lv[4 * q + 2] = f.z; lv[4 * q + 3] = f.w;
-      }
-#pragma unroll
-      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
-    }
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float v = tf32f(u[t]);
-      cx.Tm[t][cc] = v;
-      cx.TT[cc][t] = v;
-    }
   }
 }
 
@@ -318,6 +291,33 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     tc::st_16x256b_x8(tmem + tlane + kTmS0, s0t);
   }
 
+  // ---- T = (I - Lab)^-1 by forward substitution, one column per lane (warp 0, lanes 0-15)
+  if (warp == 0 && lane < kChunk) {
+    const int cc = lane;
+    float u[kChunk];
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
+#pragma unroll
+    for (int tau = 0; tau < kChunk - 1; ++tau) {
+      const float4* lrow = reinterpret_cast<const float4*>(&cx.LabT[tau][0]);
+      float lv[kChunk];
+#pragma unroll
+      for (int q = (tau + 1) / 4; q < 4; ++q) {
+        const float4 f = lrow[q];
+        lv[4 * q] = f.x; lv[4 * q + 1] = f.y; lv[4 * q + 2] = f.z; lv[4 * q + 3] = f.w;
+      }
+#pragma unroll
+      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
+    }
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) {
+      const float v = tf32f(u[t]);
+      sm.Tm[t][cc] = v;
+      sm.TT[cc][t] = v;
+    }
+  }
+  named_bar(2, 128);
+
   // ---- step a: W = T diag(m0) At (columns j0..j0+15), M = Mrb T (warp 0), X = T Lak (warp 1)
   uint32_t bat[2][4];   // At^T fragments of this warp's columns: [n-tile][k-step pair]
 #pragma unroll
@@ -325,7 +325,7 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
   {
     uint32_t at[2][4];
 #pragma unroll
-    for (int s = 0; s < 2; ++s) ldsm_x4(at[s], a32_addr(&cx.Tm[0][0], S20, 0, 8 * s, lane));
+    for (int s = 0; s < 2; ++s) ldsm_x4(at[s], a32_addr(&sm.Tm[0][0], S20, 0, 8 * s, lane));
     if (warp == 1) {   // X = T Lak (unmasked T)
       float xx[2][4] = {};
 #pragma unroll
@@ -364,7 +364,7 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
 #pragma unroll
       for (int nt = 0; nt < 2; ++nt) {
         uint32_t bt[4];
-        ldsm_x4(bt, b32_2k_addr(&cx.TT[0][0], S20, 8 * nt, 0, lane));
+        ldsm_x4(bt, b32_2k_addr(&sm.TT[0][0], S20, 8 * nt, 0, lane));
         mma1688(mm[nt], am[0], bt[0], bt[1]);
         mma1688(mm[nt], am[1], bt[2], bt[3]);
       }
