@@ -639,33 +639,27 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, co
     }
   }
 
-  // ---- M11: dw = (reverse cumulative sum of d log L) / w.  Thread = (column pair, token half);
-  // the lower half adds the upper half's rows itself instead of waiting for it.
+  // ---- M11: dw = (reverse cumulative sum of d log L) / w.  Thread = (column pair, token quarter
+  // q = warp): each thread first adds the rows of the later quarters itself, then walks its four.
   {
-    const int j = 2 * (tid & 31), th = tid >> 5;   // warps 0 and 1: token halves 0..7 and 8..15
-    if (th < 2) {
-      const int tlo = th ? 8 : 0;
-      float2 cum = *reinterpret_cast<const float2*>(&sm.e3[j]);
-      if (keep) {
-        const float2 d01 = add2(*reinterpret_cast<const float2*>(&sm.dlam[0][j]), *reinterpret_cast<const float2*>(&sm.dlam[1][j]));
-        const float2 d23 = add2(*reinterpret_cast<const float2*>(&sm.dlam[2][j]), *reinterpret_cast<const float2*>(&sm.dlam[3][j]));
-        cum = fma2(*reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]), add2(d01, d23), cum);
-      }
-      if (!th) {
+    const int j = 2 * lane, q = warp, thi = 4 * q + 3;
+    float2 cum = *reinterpret_cast<const float2*>(&sm.e3[j]);
+    if (keep) {
+      const float2 d01 = add2(*reinterpret_cast<const float2*>(&sm.dlam[0][j]), *reinterpret_cast<const float2*>(&sm.dlam[1][j]));
+      const float2 d23 = add2(*reinterpret_cast<const float2*>(&sm.dlam[2][j]), *reinterpret_cast<const float2*>(&sm.dlam[3][j]));
+      cum = fma2(*reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]), add2(d01, d23), cum);
+    }
+    for (int t = kChunk - 1; t > thi; --t) cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
+    T* gdw = static_cast<T*>(p.dw) + tok_off(b, t0, h, p.T, p.H) + j;
+    const int64_t rs = p.H * kN;
+    float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[thi][j]);
 #pragma unroll
-        for (int t = 8; t < kChunk; ++t) cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
-      }
-      T* gdw = static_cast<T*>(p.dw) + tok_off(b, t0, h, p.T, p.H) + j;
-      const int64_t rs = p.H * kN;
-      float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[tlo + 7][j]);
-#pragma unroll
-      for (int u = 7; u >= 0; --u) {
-        const int t = tlo + u;
-        cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
-        const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
-        if (t < len) store2(gdw + t * rs, mul2(cum, mul2(Lp, make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y)))));
-        Lt = Lp;
-      }
+    for (int u = 3; u >= 0; --u) {
+      const int t = 4 * q + u;
+      cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
+      const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
+      if (t < len) store2(gdw + t * rs, mul2(cum, mul2(Lp, make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y)))));
+      Lt = Lp;
     }
   }
 }
