@@ -42,6 +42,26 @@ BYTES_PREFILL = 768 + 128
 BYTES_DECODE = 64 * 64 * 4 * 2 + 768 + 128
 
 
+def rank_seed(rank: int) -> int:
+    """Seed of a rank's synthetic batch: every rank draws a different batch of the same workload."""
+    return 1000 + WORKLOAD + rank
+
+
+def rank_max(values, device, world: int):
+    """Element-wise max over ranks of per-rank timings (ms); the identity on one rank."""
+    import torch
+    t = torch.tensor([float(v) for v in values], device=device, dtype=torch.float64)
+    if world > 1:
+        import torch.distributed as dist
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return [float(v) for v in t.tolist()]
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput under weak scaling: all ranks' tokens over the slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
 NOMINAL_HBM_GBS = 8000.0   # B200 HBM3e nominal (context: the roofline uses the measured copy bandwidth)
 
 
@@ -242,7 +262,7 @@ def main():
     from linear_recurrent_lm_b200 import wkv7
 
     dev = torch.device("cuda", local)
-    wl = I.make_workload(WORKLOAD, seed=1000 + WORKLOAD + rank)
+    wl = I.make_workload(WORKLOAD, seed=rank_seed(rank))
     B, T, H = wl.B, wl.T, wl.H
 
     def d(x):
@@ -293,13 +313,10 @@ def main():
     total_ms = start.elapsed_time(end)
     fwd_ms = [e[0].elapsed_time(e[1]) for e in evs]
     bwd_ms = [e[1].elapsed_time(e[2]) for e in evs]
-    t = torch.tensor([total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    total_ms, fwd_avg, bwd_avg = (float(v) for v in t.tolist())
+    total_ms, fwd_avg, bwd_avg = rank_max([total_ms, statistics.mean(fwd_ms), statistics.mean(bwd_ms)], dev, world)
     ms_per_step = total_ms / args.steps
     tokens_step = B * T * world
-    value = tokens_step / (ms_per_step / 1e3)
+    value = job_tokens_per_s(B * T, world, ms_per_step)
 
     # ---- e2e: through the public API with host buffers, copies inside the timed region
     host_in = [x.cpu().pin_memory() for x in xs] + [dy.cpu().pin_memory(), reset.cpu().pin_memory()]
@@ -328,11 +345,8 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    te = torch.tensor([e0.elapsed_time(e1)], device=dev, dtype=torch.float64)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item()) / args.e2e_steps
-    e2e_value = tokens_step / (e2e_ms / 1e3)
+    e2e_ms = rank_max([e0.elapsed_time(e1)], dev, world)[0] / args.e2e_steps
+    e2e_value = job_tokens_per_s(B * T, world, e2e_ms)
 
     secondary = {}
     if rank == 0 and not args.no_secondary:
