@@ -21,21 +21,25 @@
 // reset (At and Rt rows masked, i.e. columns of T and M), only the last
 // segment feeds S_16, and S0 drops out of S_16 if the chunk holds any reset.
 //
-// Precision: all products are tf32 mma.sync (m16n8k8) with fp32 accumulation;
-// operands are rounded to tf32 (nearest).  An emulation of exactly these
-// roundings against the fp64 oracle stays ~6x inside the bf16 tolerance.  A
-// chunk whose decay product leaves [2^-40, 2^40] (e.g. w = 0) cannot use the
-// 1/L scaling and is run token by token instead.
+// Precision: every product is tf32 with fp32 accumulation; operands are
+// rounded to tf32 (nearest) except SA^T, which the state product reads back
+// from tensor memory as tf32.  An emulation of the rounded operands against
+// the fp64 oracle stays ~6x inside the bf16 tolerance.  A chunk whose decay
+// product leaves [2^-40, 2^40] (e.g. w = 0) cannot use the 1/L scaling and is
+// run token by token instead.
 //
 // Work split (one CTA of 8 warps per (b,h)), pipelined over chunks:
 //   warps 4-7 ("context") for chunk c+1: stage the inputs (one TMA box per
-//     input on an mbarrier, bounded waits), build
-//     the decay-scaled operands, the masked Gram of [At; Rt] and [Bh; Kh] and
-//     T into one half of a double-buffered context;
+//     input on an mbarrier, bounded waits), build the decay-scaled operands
+//     (for the state products in the tcgen05 operand layout, Bh and Kh masked
+//     to the last segment) and the masked Gram of [At; Rt] and [Bh; Kh]
+//     (mma.sync) into one half of a double-buffered context;
 //   warps 0-3 ("state") for chunk c: warp w owns rows 16w..16w+15 of S as
-//     accumulator fragments for the whole sequence; they form W, X, M, Q, Z
-//     from the context, then the two state products, write y and the
-//     chunk-end checkpoint.
+//     fp32 accumulator fragments for the whole sequence; they solve for T,
+//     form W, X, M, Q, Z (mma.sync, 16x16 blocks), then one thread issues the
+//     two state products as tcgen05 MMAs (M = 64, accumulators in TMEM; see
+//     state_chunk), and the warps write y, update S and write the chunk-end
+//     checkpoint.
 // One CTA barrier per chunk hands the context over.
 #include <type_traits>
 

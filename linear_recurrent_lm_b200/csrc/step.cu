@@ -9,9 +9,8 @@
 // accesses, and few registers per thread keep many CTAs (and their loads) in
 // flight per SM.  The two row dot products (sa and y) reduce over the 8
 // lanes of a row with three xor-shuffles.  A row of the batch with active[b]==0
-// never writes its state, which therefore stays bitwise unchanged, and writes
-// y = 0; its flag is loaded together with the state and the inputs, so no
-// load waits for another.
+// returns before touching its state, which therefore stays bitwise unchanged
+// (and costs no bandwidth in a ragged batch), and writes y = 0.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -38,7 +37,10 @@ __global__ void __launch_bounds__(kThreads, 3) step_kernel(StepArgs p) {
   const int t = threadIdx.x;
   const int i = t >> 3, q = t & 7;   // row i, columns 8q..8q+7
   T* y = static_cast<T*>(p.y) + unit * kN;
-  const bool act = !p.active || p.active[b] != 0;
+  if (p.active && !p.active[b]) {   // padded row: its state is not even read
+    if (q == 0) y[i] = Elt<T>::from_f32(0.f);
+    return;
+  }
   float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 8);
   const float4 s_lo = row[0], s_hi = row[1];
   float S[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
@@ -68,15 +70,13 @@ __global__ void __launch_bounds__(kThreads, 3) step_kernel(StepArgs p) {
     S[j] = fmaf(S[j], wv[j], fmaf(sa, bv[j], vi * kv[j]));
     if (j & 1) y1 = fmaf(S[j], rv[j], y1); else y0 = fmaf(S[j], rv[j], y0);
   }
-  if (act) {
-    row[0] = make_float4(S[0], S[1], S[2], S[3]);
-    row[1] = make_float4(S[4], S[5], S[6], S[7]);
-  }
+  row[0] = make_float4(S[0], S[1], S[2], S[3]);
+  row[1] = make_float4(S[4], S[5], S[6], S[7]);
   float yy = y0 + y1;
   yy += __shfl_xor_sync(0xffffffffu, yy, 1);
   yy += __shfl_xor_sync(0xffffffffu, yy, 2);
   yy += __shfl_xor_sync(0xffffffffu, yy, 4);
-  if (q == 0) y[i] = Elt<T>::from_f32(act ? yy : 0.f);
+  if (q == 0) y[i] = Elt<T>::from_f32(yy);
 }
 
 template <typename T>
