@@ -153,9 +153,10 @@ __device__ __forceinline__ void load_entry_rows(const BwdArgs& p, int64_t unit, 
   }
 }
 
-__device__ __forceinline__ unsigned reset_bits_of(const BwdArgs& p, int64_t b, int64_t t0, int len, int lane) {
-  const bool f = p.reset && lane < len && p.reset[b * p.T + t0 + lane] != 0;
-  return __ballot_sync(0xffffffffu, f) & 0xffffu;
+// Reset flag of token 16c + lane of batch row b (false past T, for c < 0 or without flags).
+__device__ __forceinline__ bool reset_flag(const BwdArgs& p, int64_t b, int64_t c, int lane) {
+  const int64_t t = c * kChunk + lane;
+  return p.reset && c >= 0 && lane < kChunk && t < p.T && p.reset[b * p.T + t] != 0;
 }
 
 // ------------------------------------------------------------------ context warps
@@ -281,15 +282,19 @@ __device__ __forceinline__ void finish_context(BwdSmem2<T>& sm, BCtx& cx, unsign
 #pragma unroll
       for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
     }
+    // rows of Lab^T are loaded one step ahead, so each step waits only on its FMAs
+    float4 nxt[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&sm.LabT[0][0])[q];
 #pragma unroll
     for (int tau = 0; tau < kChunk - 1; ++tau) {
-      const float4* lrow = reinterpret_cast<const float4*>(&sm.LabT[tau][0]);
-      float lv[kChunk];
+      const float4 cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+      if (tau + 1 < kChunk - 1) {
 #pragma unroll
-      for (int q = (tau + 1) / 4; q < 4; ++q) {
-        const float4 f = lrow[q];
-        lv[4 * q] = f.x; lv[4 * q + 1] = f.y; lv[4 * q + 2] = f.z; lv[4 * q + 3] = f.w;
+        for (int q = (tau + 2) / 4; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&sm.LabT[tau + 1][0])[q];
       }
+      const float lv[kChunk] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w,
+                                cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
 #pragma unroll
       for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
     }
@@ -735,8 +740,10 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p,
       const int64_t t0 = c * kChunk;
       stage7<T>(p, tm, sm, b, h, t0, ktid);
       load_entry_rows(p, unit, nc, c, ktid, s0rows);
-      mask_next = reset_bits_of(p, b, t0, int(p.T - t0), lane);
+      mask_next = __ballot_sync(0xffffffffu, reset_flag(p, b, c, lane)) & 0xffffu;
     }
+    // the flag of the chunk staged next is loaded one iteration before its ballot, off the critical path
+    bool f_prev = reset_flag(p, b, nc - 2, lane);
     cta_sync();
     for (int64_t it = 0; it <= nc; ++it) {
       const int64_t c = nc - 1 - it;   // chunk whose context is built now
@@ -756,7 +763,8 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p,
           stage7<T>(p, tm, sm, b, h, tp, ktid);
           pending = true;
           load_entry_rows(p, unit, nc, c - 1, ktid, s0rows);
-          mask_next = reset_bits_of(p, b, tp, kChunk, lane);
+          mask_next = __ballot_sync(0xffffffffu, f_prev) & 0xffffu;   // chunk c-1
+          f_prev = reset_flag(p, b, c - 2, lane);
         }
         if (!unsafe) finish_context<T>(sm, cx, mask, ktid);
       }

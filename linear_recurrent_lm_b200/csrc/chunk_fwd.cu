@@ -301,15 +301,19 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     float u[kChunk];
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
+    // rows of Lab^T are loaded one step ahead, so each step waits only on its FMAs
+    float4 nxt[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&cx.LabT[0][0])[q];
 #pragma unroll
     for (int tau = 0; tau < kChunk - 1; ++tau) {
-      const float4* lrow = reinterpret_cast<const float4*>(&cx.LabT[tau][0]);
-      float lv[kChunk];
+      const float4 cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
+      if (tau + 1 < kChunk - 1) {
 #pragma unroll
-      for (int q = (tau + 1) / 4; q < 4; ++q) {
-        const float4 f = lrow[q];
-        lv[4 * q] = f.x; lv[4 * q + 1] = f.y; lv[4 * q + 2] = f.z; lv[4 * q + 3] = f.w;
+        for (int q = (tau + 2) / 4; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&cx.LabT[tau + 1][0])[q];
       }
+      const float lv[kChunk] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w,
+                                cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
 #pragma unroll
       for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
     }
@@ -449,17 +453,17 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
     for (int s = 0; s < 2; ++s)        // + V^T [X; Z]^T over tau
       tc::mma_ss(tmem + kTmD1, tc::smem_desc(&cx.VTc[64 * s], 8 * kChunk * 4),
                  tc::smem_desc(&sm.B1v[64 * s], 8 * kChunk * 4), id32, true);
+#pragma unroll
+    for (int s = 0; s < 2; ++s)        // D3 = V^T ls.Kh (independent of D1) ...
+      tc::mma_ss(tmem + kTmD3, tc::smem_desc(&cx.VTc[64 * s], 8 * kChunk * 4),
+                 tc::smem_desc(&cx.KhTc[64 * s], 8 * kChunk * 4), id64, s > 0);
     // D3 reads D1 through the A-operand path: issue it only once D1 is complete
     tc::commit(&sm.d1_bar);
     if (!mbar_wait_bounded(&sm.d1_bar, mma_phase & 1u, kWaitLimitNs) && p.status) atomicOr(p.status, kStatusWaitTimeout);
     tc::fence_after_sync();
 #pragma unroll
-    for (int s = 0; s < 2; ++s)        // D3 = SA^T ls.Bh (SA^T = D1 columns 0-15) ...
-      tc::mma_ts(tmem + kTmD3, tmem + kTmD1 + 8 * s, tc::smem_desc(&cx.BhTc[64 * s], 8 * kChunk * 4), id64, s > 0);
-#pragma unroll
-    for (int s = 0; s < 2; ++s)        // ... + V^T ls.Kh
-      tc::mma_ss(tmem + kTmD3, tc::smem_desc(&cx.VTc[64 * s], 8 * kChunk * 4),
-                 tc::smem_desc(&cx.KhTc[64 * s], 8 * kChunk * 4), id64, true);
+    for (int s = 0; s < 2; ++s)        // ... + SA^T ls.Bh (SA^T = D1 columns 0-15)
+      tc::mma_ts(tmem + kTmD3, tmem + kTmD1 + 8 * s, tc::smem_desc(&cx.BhTc[64 * s], 8 * kChunk * 4), id64, true);
     tc::commit(&sm.mma_bar);
   }
   if (!mbar_wait_bounded(&sm.mma_bar, mma_phase & 1u, kWaitLimitNs) && threadIdx.x == 0 && p.status)
