@@ -107,6 +107,34 @@ def test_small_decay_segments(W, algo):
         assert c >= COS, (n, c)
 
 
+def test_flagged_and_chunked_heads_in_one_batch(W):
+    """bf16 batch where some (b, h) heads hold a decay the 1/L scaling cannot take (w = 0 or
+    w < 1/16 inside a chunk) and the rest do not: the chunked pass marks exactly those heads, the
+    exact scan redoes them, and every head's gradients and dS0 must match the oracle."""
+    rng = np.random.default_rng(17)
+    B, T, H = 2, 200, 3
+    d = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    w = I.to_f64(d["w"])
+    w[0, 70:72, 1] = 0.0            # head (0, 1): w = 0 in chunk 4
+    w[1, 150, 2, :8] = 0.03         # head (1, 2): w < 1/16 in chunk 9
+    d["w"] = I.to_storage(w, "bf16")
+    dy = I.to_storage(rng.standard_normal((B, T, H, 64)), "bf16")
+    reset = np.zeros((B, T), np.uint8)
+    reset[0, 120] = 1
+    s0 = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    dsT = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    _, _, g = fwd_bwd(W, d, dy, s0=s0, reset=reset, dsT=dsT)
+    go, _ = oracle.backward(*inputs_f64(d), I.to_f64(dy), s0=s0.astype(np.float64), reset=reset,
+                            dsT=dsT.astype(np.float64))
+    for b in range(B):
+        for h in range(H):
+            for n in GRADS:
+                c = cosine(f64(g[n])[b, :, h], go[n][b, :, h])
+                assert c >= COS, (b, h, n, c)
+            c = cosine(f64(g["ds0"])[b, h], go["ds0"][b, h])
+            assert c >= COS, (b, h, "ds0", c)
+
+
 def test_backward_chaining(W):
     """dS0 of the second half fed as dS_T of the first equals one backward over the whole row."""
     import torch

@@ -140,6 +140,27 @@ def test_zero_decay_and_identity_tokens(W, algo):
 
 
 @pytest.mark.parametrize("algo", ALGOS)
+def test_scattered_token_path_chunks_between_tensor_core_chunks(W, algo):
+    """Chunks the chunked path must run token by token (w = 0 somewhere inside) scattered
+    between ordinary ones, with resets and an entering state: the chunked kernel alternates its
+    two paths many times within one sequence and must stay on the oracle throughout."""
+    rng = np.random.default_rng(13)
+    B, T, H = 2, 300, 3
+    d = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    w = I.to_f64(d["w"])
+    w[0, [5, 100, 101, 250]] = 0.0
+    w[1, [33, 34, 160, 299]] = 0.0
+    d["w"] = I.to_storage(w, "bf16")
+    reset = np.zeros((B, T), np.uint8)
+    reset[0, [50, 180]] = 1
+    reset[1, [0, 161, 200]] = 1
+    s0 = rng.standard_normal((B, H, 64, 64)).astype(np.float32)
+    y, s, _ = run_fwd(W, d, s0=s0, reset=reset, algo=algo)
+    yo, so, _ = oracle.forward(*inputs_f64(d), s0=s0.astype(np.float64), reset=reset)
+    check_fwd(y, s, yo, so, "bf16")
+
+
+@pytest.mark.parametrize("algo", ALGOS)
 def test_zero_tokens_and_single_unit(W, algo):
     import torch
     rng = np.random.default_rng(11)
