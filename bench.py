@@ -237,7 +237,7 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--algo", default="auto", choices=["auto", "scan", "chunked"])
-    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--only", choices=["fwd", "bwd", "prefill", "step"],
@@ -318,32 +318,54 @@ def main():
     tokens_step = B * T * world
     value = job_tokens_per_s(B * T, world, ms_per_step)
 
-    # ---- e2e: through the public API with host buffers, copies inside the timed region
+    # ---- e2e: through the public API with host buffers, copies inside the timed region.  Every step
+    # copies its inputs from pinned host memory and all of its outputs (y and the six gradients) back;
+    # the steps are pipelined two deep on three streams, as a training loop would run them: the H2D
+    # copy of step k+1 and the D2H copy of step k-1 overlap the kernels of step k.
     host_in = [x.cpu().pin_memory() for x in xs] + [dy.cpu().pin_memory(), reset.cpu().pin_memory()]
     host_out = [torch.empty(xs[0].shape, dtype=xs[0].dtype, pin_memory=True) for _ in range(7)]
-    dev_in = [torch.empty_like(x) for x in xs] + [torch.empty_like(dy), torch.empty_like(reset)]
+    dev_in = [[torch.empty_like(x) for x in host_in] for _ in range(2)]
+    dev_out = [[torch.empty_like(xs[0]) for _ in range(7)] for _ in range(2)]
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = sum(x.numel() * x.element_size() for x in host_out)
+    s_h2d, s_d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+    ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "comp", "out")}
+    gnames = ("dr", "dw", "dk", "dv", "da", "db")
 
-    def e2e_step():
-        for hsrc, dd in zip(host_in, dev_in):
-            dd.copy_(hsrc, non_blocking=True)
-        wkv7.forward(*dev_in[:6], reset=dev_in[7], y=y, s_out=s_out, workspace=ws, algo=args.algo)
-        wkv7.backward(*dev_in[:6], dev_in[6], ws, reset=dev_in[7], grads=grads, want_ds0=False, algo=args.algo)
-        outs = [y] + [grads[n] for n in ("dr", "dw", "dk", "dv", "da", "db")]
-        for o, hdst in zip(outs, host_out):
-            hdst.copy_(o, non_blocking=True)
+    def e2e_pipeline(n_steps, e_start=None, e_end=None):
+        for k in range(n_steps):
+            st = k % 2
+            with torch.cuda.stream(s_h2d):
+                if k == 0 and e_start is not None:
+                    e_start.record(s_h2d)
+                if k >= 2:
+                    s_h2d.wait_event(ev["comp"][st])          # step k-2 no longer reads this input set
+                for hsrc, dd in zip(host_in, dev_in[st]):
+                    dd.copy_(hsrc, non_blocking=True)
+                ev["in"][st].record(s_h2d)
+            stream.wait_event(ev["in"][st])
+            if k >= 2:
+                stream.wait_event(ev["out"][st])              # step k-2's outputs have been copied out
+            xin, outs = dev_in[st], dev_out[st]
+            wkv7.forward(*xin[:6], reset=xin[7], y=outs[0], s_out=s_out, workspace=ws, algo=args.algo)
+            wkv7.backward(*xin[:6], xin[6], ws, reset=xin[7], grads=dict(zip(gnames, outs[1:])), want_ds0=False,
+                          algo=args.algo)
+            ev["comp"][st].record(stream)
+            with torch.cuda.stream(s_d2h):
+                s_d2h.wait_event(ev["comp"][st])
+                for o, hdst in zip(outs, host_out):
+                    hdst.copy_(o, non_blocking=True)
+                ev["out"][st].record(s_d2h)
+                if k == n_steps - 1 and e_end is not None:
+                    e_end.record(s_d2h)
 
-    e2e_step()
+    e2e_pipeline(2)
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
     e0 = torch.cuda.Event(enable_timing=True)
     e1 = torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(args.e2e_steps):
-        e2e_step()
-    e1.record(stream)
+    e2e_pipeline(args.e2e_steps, e0, e1)
     torch.cuda.synchronize()
     e2e_ms = rank_max([e0.elapsed_time(e1)], dev, world)[0] / args.e2e_steps
     e2e_value = job_tokens_per_s(B * T, world, e2e_ms)
@@ -383,8 +405,12 @@ def main():
                          "bytes_per_launch": dominant[3] * units,
                          "traffic": traffic},
             "cpu_baseline": cpu,
-            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-            "gpu_launches": 2 * args.steps,
+            "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": e2e_ms, "steps": args.e2e_steps,
+                    "pipelining": "two deep: H2D of step k+1 and D2H of step k-1 overlap step k (pinned host buffers)"},
+            # per step: the forward kernel, the chunked backward and its exact re-run of flagged heads
+            # (which returns at once when none is flagged); the scan algorithm launches one kernel each way
+            "gpu_launches": (3 if args.algo != "scan" else 2) * args.steps,
             "clocks": clk.summary(),
             "secondary": secondary,
         }
