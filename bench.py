@@ -324,7 +324,7 @@ def main():
     # copy of step k+1 and the D2H copy of step k-1 overlap the kernels of step k.
     host_in = [x.cpu().pin_memory() for x in xs] + [dy.cpu().pin_memory(), reset.cpu().pin_memory()]
     host_out = [torch.empty(xs[0].shape, dtype=xs[0].dtype, pin_memory=True) for _ in range(7)]
-    dev_in = [[torch.empty_like(x) for x in host_in] for _ in range(2)]
+    dev_in = [[torch.empty_like(x, device=dev) for x in host_in] for _ in range(2)]
     dev_out = [[torch.empty_like(xs[0]) for _ in range(7)] for _ in range(2)]
     h2d = sum(x.numel() * x.element_size() for x in host_in)
     d2h = sum(x.numel() * x.element_size() for x in host_out)

@@ -97,7 +97,14 @@ def device_status(clear: bool = True) -> int:
 
 
 def _ptr(x: Optional[torch.Tensor]):
-    return None if x is None else ctypes.c_void_p(x.data_ptr())
+    """Device address of a contiguous CUDA tensor (the C ABI takes device pointers only)."""
+    if x is None:
+        return None
+    if not x.is_cuda:
+        raise ValueError(f"WKV-7 tensors must be on a CUDA device, got a {x.device} tensor of shape {tuple(x.shape)}")
+    if not x.is_contiguous():
+        raise ValueError(f"WKV-7 tensors must be contiguous, got strides {x.stride()} for shape {tuple(x.shape)}")
+    return ctypes.c_void_p(x.data_ptr())
 
 
 def _stream(stream) -> ctypes.c_void_p:

@@ -119,3 +119,15 @@ def test_no_cpu_fallback_without_gpu(L):
     d = L.make_desc(1, 16, 1, torch.bfloat16)
     assert call_fwd(L, d) == L.ERR_CUDA
     assert L.device_status() == L.ERR_CUDA      # the status word cannot be read without a device
+
+
+def test_binding_rejects_host_and_strided_tensors_before_any_call(L):
+    """The binding passes device pointers only: a host tensor (or a strided view) is refused in Python,
+    so a host address can never reach a kernel."""
+    import torch
+    x = torch.zeros(1, 16, 1, 64, dtype=torch.bfloat16)
+    with pytest.raises(ValueError, match="CUDA"):
+        L.forward(x, x, x, x, x, x)
+    with pytest.raises(ValueError, match="CUDA"):
+        L._ptr(torch.zeros(4))
+
