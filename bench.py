@@ -191,6 +191,54 @@ def cpu_oracle_sample(wl, budget_s: float = 10.0):
             "sample": f"{n} of {wl.B * wl.H} (b,h) units x T={wl.T}, fwd+bwd, fp64 C oracle, {t:.1f} s"}
 
 
+def oracle_table(cores: int):
+    """The fp64 C oracle on every workload: forward and forward+backward of workloads 1-3 and
+    the 128 ragged decode steps of workload 4, with all host cores and with one, each on a
+    bounded sample of whole (b, h) units (tokens/s scaled to the workload's H heads)."""
+    import oracle
+    out = {}
+
+    def time_units(wl, units, threads, bwd, prior=False):
+        src = wl.inputs
+        t0 = time.perf_counter()
+        by_b = {}
+        for b, h in units:
+            by_b.setdefault(b, []).append(h)
+        for b, hs in by_b.items():
+            part = [I.to_f64(src[n][b:b + 1, :, hs]) for n in I.NAMES]
+            reset = wl.reset[b:b + 1] if wl.reset is not None else None
+            s0 = None
+            if prior:
+                _, s0, _ = oracle.forward(*(I.to_f64(wl.prior[n][b:b + 1, :, hs]) for n in I.NAMES), nthreads=threads)
+            oracle.forward(*part, s0=s0, reset=reset, nthreads=threads)
+            if bwd:
+                oracle.backward(*part, I.to_f64(wl.dy[b:b + 1, :, hs]), s0=s0, reset=reset, nthreads=threads)
+        dt = time.perf_counter() - t0
+        return len(units) * wl.T / wl.H / dt
+
+    for idx, name in ((1, "c1_B2_T512_H12"), (2, "c2_prefill_B1_T1024_H32"), (3, "c3_packed_B8_T4096_H32")):
+        wl = I.make_workload(idx)
+        units = [(b, h) for b in range(wl.B) for h in range(wl.H)]
+        for threads, n_units in ((cores, min(len(units), 2 * cores if idx == 3 else len(units))), (1, min(len(units), 2))):
+            key = f"{name}_{'all_cores' if threads == cores else '1_core'}"
+            entry = {"fwd_tokens_per_s": time_units(wl, units[:n_units], threads, False, prior=idx == 2),
+                     "units": n_units}
+            if idx != 2:
+                entry["fwd_bwd_tokens_per_s"] = time_units(wl, units[:n_units], threads, True)
+            out[key] = entry
+    wl = I.make_workload(4)
+    rows = list(range(min(wl.B, 16)))
+    st = wl.state0[rows].astype(np.float64)
+    t0 = time.perf_counter()
+    active_tok = 0
+    for s in range(len(wl.steps)):
+        act = wl.active(s)[rows]
+        active_tok += int(act.sum())
+        _, st = oracle.step(*(I.to_f64(wl.steps[s][n][rows]) for n in I.NAMES), st, act)
+    out["c4_decode_128_steps_1_core"] = {"tokens_per_s": active_tok / (time.perf_counter() - t0), "rows": len(rows)}
+    return out
+
+
 def run_reference(args):
     """The oracle as the reference arm: same workload/metric, bounded sample per step."""
     rank = int(os.environ.get("RANK", "0"))
@@ -227,6 +275,7 @@ def run_reference(args):
         "config": {"workload": wl.name, "B": wl.B, "T": wl.T, "H": wl.H, "N": wl.N},
         "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "oracle_table": oracle_table(cores),
     }))
 
 
