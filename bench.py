@@ -422,6 +422,26 @@ def main():
     secondary = {}
     if rank == 0 and not args.no_secondary:
         secondary = measure_secondary(wkv7, dev, args.algo)
+        if args.algo != "scan":   # the token-order scan kernels on the same batch, for comparison
+            ev3 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            f_ms, b_ms = [], []
+            for rep in range(4):
+                ev3[0].record(stream)
+                wkv7.forward(*xs, reset=reset, y=y, s_out=s_out, workspace=ws, algo="scan")
+                ev3[1].record(stream)
+                wkv7.backward(*xs, dy, ws, reset=reset, grads=grads, want_ds0=False, algo="scan")
+                ev3[2].record(stream)
+                torch.cuda.synchronize()
+                if rep:
+                    f_ms.append(ev3[0].elapsed_time(ev3[1]))
+                    b_ms.append(ev3[1].elapsed_time(ev3[2]))
+            fm, bm = statistics.median(f_ms), statistics.median(b_ms)
+            units_s = B * T * H
+            peak_s, _ = measured_peaks()
+            secondary[f"scan_{wl.name}"] = {
+                "fwd_ms": fm, "bwd_ms": bm, "fwd_bwd_tokens_per_s": B * T / ((fm + bm) / 1e3),
+                "fwd_frac": BYTES_FWD_TRAIN * units_s / (fm / 1e3) / 1e9 / peak_s,
+                "bwd_frac": BYTES_BWD * units_s / (bm / 1e3) / 1e9 / peak_s}
 
     if world > 1:
         dist.barrier()
