@@ -276,7 +276,7 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
 template <typename T>
 __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, const Ctx& cx, float (&acc)[8][4],
                                             int64_t b, int64_t h, int64_t t0, int len, int warp, int lane,
-                                            uint32_t tmem, unsigned& mma_phase) {
+                                            uint32_t tmem, unsigned& mma_phase, float* ck_prev) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
   const int j0 = 16 * warp;
@@ -466,6 +466,13 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
       tc::mma_ts(tmem + kTmD3, tmem + kTmD1 + 8 * s, tc::smem_desc(&cx.BhTc[64 * s], 8 * kChunk * 4), id64, true);
     tc::commit(&sm.mma_bar);
   }
+  // while the tensor core works: the checkpoint of the state entering this chunk (the previous
+  // chunk's end state, still unchanged in the fragments), 512 contiguous bytes per warp and nt
+  if (ck_prev) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<float4*>(ck_prev + nt * 128) = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+  }
   if (!mbar_wait_bounded(&sm.mma_bar, mma_phase & 1u, kWaitLimitNs) && threadIdx.x == 0 && p.status)
     atomicOr(p.status, kStatusWaitTimeout);
   ++mma_phase;
@@ -503,6 +510,15 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
   }
   // the next batch overwrites D1/D3 and S0: every warp's loads are done before it is issued
   tc::fence_before_sync();
+}
+
+// The eight float4 of a checkpoint in the tiled order (ck == nullptr: none due).
+__device__ __forceinline__ void store_ck(float* ck, const float (&acc)[8][4]) {
+  if (ck) {
+#pragma unroll
+    for (int nt = 0; nt < 8; ++nt)
+      *reinterpret_cast<float4*>(ck + nt * 128) = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
+  }
 }
 
 // Token-by-token update of one chunk on the state fragments (decay out of range), inputs read from global.
@@ -607,6 +623,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
     // y of the previous chunk (16-bit outputs): this thread's 16-byte piece of token row tid/8
     T* ydst = nullptr;
     const int ytt = tid >> 3, ypart = tid & 7;
+    float* ck = nullptr;   // checkpoint slot of the state in the fragments (tiled order), if still due
     for (int64_t it = 0; it <= nc; ++it) {
       if (ydst) {
         *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
@@ -618,21 +635,19 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         const int64_t t0 = c * kChunk;
         const int len = int(min64(kChunk, p.T - t0));
         if (!cx.unsafe) {
-          state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane, tmem, mma_phase);
+          state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane, tmem, mma_phase, ck);
           if (sizeof(T) == 2 && ytt < len) ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
         } else {
+          store_ck(ck, acc);
           state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
         }
-        if (p.ckpt) {   // tiled checkpoint order: 512 contiguous bytes per warp and nt
-          float* base = p.ckpt + (unit * nc + c) * kN * kN + warp * 1024 + lane * 4;
-#pragma unroll
-          for (int nt = 0; nt < 8; ++nt)
-            *reinterpret_cast<float4*>(base + nt * 128) = make_float4(acc[nt][0], acc[nt][1], acc[nt][2], acc[nt][3]);
-        }
+        // this chunk's end state is checkpointed during the next chunk (or after the loop)
+        ck = p.ckpt ? p.ckpt + (unit * nc + c) * kN * kN + warp * 1024 + lane * 4 : nullptr;
       }
       cta_sync();   // context of chunk it handed over; Ys complete
     }
     if (ydst) *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+    store_ck(ck, acc);
     // every batch was waited for and every TMEM load is complete: release TMEM
     named_bar(2, 128);
     tc::fence_after_sync();
