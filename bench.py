@@ -75,24 +75,58 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+_KERNEL_HEADERS = ("common.cuh", "kernels.h", "mma.cuh", "tc05.cuh")
+
+
+def _strip_c_comments(text: str) -> str:
+    """C/CUDA source without comments, whitespace runs collapsed (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        if text.startswith("//", i):
+            j = text.find("\n", i)
+            i = n if j < 0 else j
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        elif text[i] == '"':
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        else:
+            out.append(text[i])
+            i += 1
+    return " ".join("".join(out).split())
+
+
+def kernel_code_sha256(source_file: str) -> str:
+    """Hash of a kernel's code: its .cu file and the shared headers, comments and layout ignored,
+    so that a profile stays attached to the kernel until the code itself changes."""
+    h = hashlib.sha256()
+    for rel in [source_file] + [f"linear_recurrent_lm_b200/csrc/{x}" for x in _KERNEL_HEADERS]:
+        with open(os.path.join(ROOT, rel)) as f:
+            h.update(_strip_c_comments(f.read()).encode())
+        h.update(b"\0")
+    return h.hexdigest()
+
+
 def kernel_traffic(kernel: str, workload: str):
-    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current code."""
     path = os.path.join(ROOT, "profiles", f"{kernel}_{workload}.md")
     if not os.path.exists(path):
         return None
     text = open(path).read()
-    m_src = re.search(r"source_sha256:\s*([0-9a-f]{64})", text)
+    m_code = re.search(r"code_sha256:\s*([0-9a-f]{64})", text)
     m_tr = re.search(r"traffic_bytes_per_launch:\s*([0-9.eE+]+)", text)
-    if not m_src or not m_tr:
-        return None
     src = re.search(r"source_file:\s*(\S+)", text)
-    if not src:
+    if not m_code or not m_tr or not src:
         return None
     try:
-        cur = hashlib.sha256(open(os.path.join(ROOT, src.group(1)), "rb").read()).hexdigest()
+        cur = kernel_code_sha256(src.group(1))
     except OSError:
         return None
-    return float(m_tr.group(1)) if cur == m_src.group(1) else None
+    return float(m_tr.group(1)) if cur == m_code.group(1) else None
 
 
 class Clocks:

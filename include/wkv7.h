@@ -1,11 +1,12 @@
 /*
  * wkv7.h -- C ABI of the B200 (sm_100a) WKV-7 library (libwkv7.so).
  *
- * WKV-7 is the recurrence at the core of RWKV-7 "Goose": the part of the
- * model that "doesn't map onto standard ops" and that the rwkv-metal page runs
- * as a hand-written kernel with a checkpointed backward ("The Metal WKV-7
- * kernel").  Per (batch b, head h) it keeps an fp32 N x N state S (row i =
- * value channel, column j = key channel) and, for each token t,
+ * WKV-7 is the recurrence at the core of RWKV-7 "Goose": the one part of the
+ * model that stock array operations cannot express efficiently, which the
+ * rwkv-metal page therefore runs as a hand-written kernel with a checkpointed
+ * backward (section "The Metal WKV-7 kernel").  Per (batch b, head h) it
+ * keeps an fp32 N x N state S (row i = value channel, column j = key channel)
+ * and, for each token t,
  *
  *     sa[i]   = sum_j S[i][j] * a_t[j]                 (S before the update)
  *     S[i][j] = S[i][j] * w_t[j] + sa[i] * b_t[j] + v_t[i] * k_t[j]
@@ -18,18 +19,18 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Head size N must be 64 (the HF model card page: "the kernel supports
- *   64-wide heads and FP32 WKV state"); anything else -> WKV7_ERR_UNSUPPORTED.
+ * - Head size N must be 64 (the HF model card page limits its kernel to heads
+ *   of 64 channels with an fp32 state); anything else -> WKV7_ERR_UNSUPPORTED.
  * - Activations r,w,k,v,a,b,y,dy and the gradients dr..db are [B,T,H,64],
  *   contiguous, row-major, all in the one dtype of the descriptor (f32, bf16
- *   or f16; "accepts BF16/FP16/FP32 activations", same page).  Outputs in a
+ *   or f16, the three activation types the same page lists).  Outputs in a
  *   16-bit dtype are rounded to nearest even.  w is the multiplicative decay
  *   (normally in (0,1]).
  * - States s0, s_out, dsT, ds0 and the decode state are fp32 [B,H,64,64],
  *   contiguous, S[i][j] at offset i*64+j.
  * - reset is [B,T] bytes: reset[b][t] != 0 zeroes the incoming state before
- *   token t (packed sequences: "Packed sequences are run with a state reset
- *   at each boundary", HF model card page).  At t = 0 it overrides s0.  No
+ *   token t (the HF model card page packs several documents into one row and
+ *   zeroes the state where each new one begins).  At t = 0 it overrides s0.  No
  *   gradient crosses a reset.
  * - Every pointer is a DEVICE pointer, 16-byte aligned (reset and active may
  *   have any alignment).  The caller allocates and owns every buffer; the
@@ -40,8 +41,8 @@
  *   the launch itself (cudaGetLastError); on any validation error nothing is
  *   launched and no output is touched.
  * - Any T >= 0 is accepted.  T need not be a multiple of 16 (the checkpoint
- *   interval): "pads independent sequences to its 16-token checkpoint
- *   interval" (HF model card page) -- here the padding is internal.
+ *   interval; the HF model card page pads separate sequences up to a multiple
+ *   of it) -- here the padding is internal.
  */
 #ifndef WKV7_H
 #define WKV7_H
@@ -71,8 +72,7 @@ typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
 /*
  * Algorithm.  SCAN: token-order scan on FP32 cores, state in registers.
  * CHUNKED: 16-token chunks with the intra-chunk products on tensor cores
- * (the chunk-parallel form the HF model card page mentions as its
- * "chunk-parallel path").  AUTO: CHUNKED for 16-bit inputs, SCAN for f32.
+ * (the chunk-parallel form that the HF model card page also mentions).  AUTO: CHUNKED for 16-bit inputs, SCAN for f32.
  * Both produce the same result up to floating-point rounding order.
  */
 typedef enum { WKV7_ALGO_AUTO = 0, WKV7_ALGO_SCAN = 1, WKV7_ALGO_CHUNKED = 2 } wkv7_algo_t;
@@ -118,9 +118,9 @@ const char* wkv7_status_string(wkv7_status_t status);
 /*
  * Bytes of workspace that wkv7_forward writes and wkv7_backward
  * reads: one fp32 64x64 state per (b, h) every 16 tokens, i.e.
- * B*H*ceil(T/16)*64*64*4 bytes (rwkv-metal page: "checkpointing the hidden
- * state every 16 tokens"; RWKV-MLX page, "Key Design Decisions" 2: "~12MB
- * extra memory" at B=2, T=512, 12 heads -- this formula gives 12.58 MB).
+ * B*H*ceil(T/16)*64*64*4 bytes (rwkv-metal page: the state is saved once per
+ * 16 tokens; RWKV-MLX page, "Key Design Decisions" 2, puts the cost near 12 MB
+ * at B=2, T=512, 12 heads -- this formula gives 12.58 MB).
  * Checkpoint c holds the state after token min(16(c+1), T) - 1, its element
  * (i, j) at offset (i/16)*1024 + (j/8)*128 + (4*(i%8) + (j%8)/2)*4
  * + 2*((i/8)%2) + j%2 (the order of the kernels' mma accumulator fragments, so
@@ -132,9 +132,9 @@ const char* wkv7_status_string(wkv7_status_t status);
 size_t wkv7_workspace_bytes(const wkv7_desc_t* desc);
 
 /*
- * Forward pass over T tokens (rwkv-metal page, "The Metal WKV-7 kernel":
- * "handles the whole sequence in one forward dispatch ... checkpointing the
- * hidden state every 16 tokens"; entry points wkv7_train / wkv7_train_with_state).
+ * Forward pass over T tokens (rwkv-metal page, "The Metal WKV-7 kernel": the
+ * full sequence is processed by a single forward launch that saves the state
+ * once per 16 tokens; entry points wkv7_train / wkv7_train_with_state).
  *
  *   r,w,k,v,a,b  in   [B,T,H,64] desc->dtype
  *   s0           in   [B,H,64,64] fp32 initial state, or NULL for zeros
@@ -149,8 +149,9 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* desc, const void* r, const void* w
                            const uint8_t* reset, void* y, float* s_out, void* workspace, void* stream);
 
 /*
- * Backward pass (rwkv-metal page: "one backward dispatch", reconstructing
- * each 16-token chunk from its checkpoint; "differentiable through h_in").
+ * Backward pass (rwkv-metal page: a single backward launch that rebuilds each
+ * 16-token chunk from its checkpoint, with gradients flowing into the initial
+ * state as well).
  * Inputs are those of the forward call that wrote `workspace` (same
  * descriptor, r..b, s0, reset), plus
  *
@@ -169,8 +170,9 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* desc, const void* r, const void* 
                             void* db, float* ds0, void* stream);
 
 /*
- * One decode token for B*H resident states, in place (rwkv-metal page:
- * "wkv7_step(..., h_in) one token"; "exact right-padding for ragged batches").
+ * One decode token for B*H resident states, in place (rwkv-metal page: a
+ * one-token step on a carried state, with ragged batches padded on the right
+ * without changing the padded rows' results).
  *
  *   desc         B, H, N=64, dtype; T must be 1; algo is ignored
  *   r..b         in      [B,H,64] desc->dtype (one token per row)

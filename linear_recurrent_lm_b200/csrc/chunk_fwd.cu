@@ -1,6 +1,6 @@
 // WKV-7 forward in 16-token chunks with the intra-chunk products on tensor
-// cores (algo CHUNKED) -- the "chunk-parallel path" of the HF model card page,
-// derived here from the recurrence.
+// cores (algo CHUNKED) -- the chunk-parallel form that the HF model card page
+// mentions, derived here from the recurrence.
 //
 // Inside a chunk of tokens t = 0..15 with entering state S0, let
 // L_t = prod_{s<=t} w_s (per key channel j) and write the state relative to

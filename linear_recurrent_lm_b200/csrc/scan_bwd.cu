@@ -7,9 +7,10 @@
 //   db = D^T sa;  dw = diag(D^T P_t);  da = P_t^T dsa;  D = D diag(w) + dsa a^T
 // and D = 0 after a token whose reset flag is set.
 //
-// Checkpointed as on the rwkv-metal page ("The Metal WKV-7 kernel": the
-// backward "reconstructs each chunk stably" from a state saved every 16
-// tokens, avoiding "the (1/decay)^T blow-up of full reconstruction"):
+// Checkpointed as on the rwkv-metal page ("The Metal WKV-7 kernel"): the
+// backward rebuilds each chunk from the state saved at its start, every 16
+// tokens, instead of running the whole sequence backwards through 1/w, which
+// would grow like (1/decay)^T:
 // chunks are visited in reverse.  Inside a chunk each reset-free segment is
 //   A) recomputed forward from its entering state (the previous checkpoint,
 //      s0, or zero after a reset), keeping sa_t for every token in shared

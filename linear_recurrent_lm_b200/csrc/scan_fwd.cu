@@ -6,9 +6,8 @@
 // 16-token slab of r,w,k,v,a,b is copied to shared memory with cp.async while
 // the previous slab is being consumed, widened once to fp32, and then read by
 // all threads as broadcasts.  After every 16 tokens (and after the last
-// token) the state is written to the checkpoint workspace, the
-// "checkpointing the hidden state every 16 tokens" of the rwkv-metal page
-// ("The Metal WKV-7 kernel").
+// token) the state is written to the checkpoint workspace: the 16-token
+// checkpoint interval of the rwkv-metal page ("The Metal WKV-7 kernel").
 #include "common.cuh"
 #include "kernels.h"
 

@@ -1,7 +1,8 @@
 // WKV-7 single-token decode step on B*H resident fp32 states, in place.
 //
-// The rwkv-metal page runs one token as plain array ops ("wkv7_step(...,
-// h_in)") and keeps "exact right-padding for ragged batches".  Here one
+// The rwkv-metal page steps one token on a carried state with plain array
+// operations and pads ragged batches on the right without changing the
+// results of the padded rows.  Here one
 // launch steps every (b,h) state: it is a pure stream over the 16 KiB state
 // (read once, written once) and therefore HBM-bound.  One CTA per (b,h), 512
 // threads; thread t owns row t/8 and the 8 columns 8*(t%8)..+7, held as two

@@ -16,7 +16,7 @@ and, for 16-bit storage, rounded once more to bf16/fp16 (RNE):
 * kk = kk_raw / ||kk_raw||_2 over the N channels of each (b,t,h)
 * a = -kk,  b = kk * sigmoid(z_iclr)
 
-This is the RWKV-7 "in-context learning rate" parametrisation: the decay is
+This is the RWKV-7 in-context-learning-rate parametrisation: the decay is
 data-dependent and kept inside (0,1), the removal key ``a`` is a unit vector
 and ``b`` scales it by a gate in (0,1) (RWKV-MLX page, "Architecture" and
 "Key Design Decisions"; rwkv-lab page, "GDN subset of RWKV-7", where the same

@@ -18,8 +18,8 @@
  *
  * i.e. S_t = S_{t-1} (diag(w_t) + a_t b_t^T) + v_t k_t^T and y_t = S_t r_t.
  * A reset flag at token t replaces the incoming state by zero before the
- * token is applied (packed sequences, HF model card page: "Packed sequences
- * are run with a state reset at each boundary").
+ * token is applied (packed sequences, HF model card page: the state is zeroed
+ * where each packed document begins).
  *
  * Layout: r,w,k,v,a,b,y,dy and the gradients are [B,T,H,N] row-major;
  * states are [B,H,N,N] row-major (S[i][j] at i*N+j); reset is [B,T] bytes.
@@ -276,8 +276,9 @@ int wkv7_oracle_backward(int64_t B, int64_t T, int64_t H, int64_t N, const doubl
 }
 
 /*
- * Single-token decode step on a resident state (rwkv-metal page, "wkv7_step";
- * "exact right-padding for ragged batches").  state is [B,H,N,N] in/out, the
+ * Single-token decode step on a resident state (rwkv-metal page: one token on
+ * a carried state; ragged batches padded on the right, the padded rows' results
+ * unchanged).  state is [B,H,N,N] in/out, the
  * token inputs and y are [B,H,N].  Rows with active[b] == 0 keep their state
  * untouched and get y = 0.  active may be NULL (all rows active).
  */
