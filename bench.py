@@ -75,7 +75,7 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
-_KERNEL_HEADERS = ("common.cuh", "kernels.h", "mma.cuh", "tc05.cuh")
+_KERNEL_HEADERS = ("common.cuh", "kernels.h", "mma.cuh", "tc05.cuh", "token_path.cuh")
 
 
 def _strip_c_comments(text: str) -> str:
@@ -319,13 +319,15 @@ def main():
     ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--algo", default="auto", choices=["auto", "scan", "chunked"])
+    ap.add_argument("--algo", default="auto", choices=["auto", "scan", "chunked", "chunked_fused", "chunked_split"])
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
     ap.add_argument("--only", choices=["fwd", "bwd", "prefill", "step"],
                     help="time one kernel alone (profiling entry point); prints its own JSON line")
     ap.add_argument("--B", type=int, default=None, help="batch override for --only")
+    ap.add_argument("--no-workspace", action="store_true",
+                    help="--only prefill: no workspace (the fused chunked form instead of the split one)")
     args = ap.parse_args()
     if args.impl == "reference":
         return run_reference(args)
@@ -541,21 +543,26 @@ def measure_secondary(wkv7, dev, algo):
     xs = [d(wl.inputs[n]) for n in I.NAMES]
     y = torch.empty_like(xs[0])
     s_out = torch.empty_like(s0)
-    times = []
-    for rep in range(25):
-        flush.fill_(float(rep))
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record()
-        wkv7.forward(*xs, s0=s0, y=y, s_out=s_out, need_workspace=False, algo=algo)
-        e1.record()
-        torch.cuda.synchronize()
-        if rep >= 5:
-            times.append(e0.elapsed_time(e1))
-    ms = statistics.median(times)
+    ws = torch.empty(wkv7.workspace_bytes(wl.B, wl.T, wl.H, xs[0].dtype), device=dev, dtype=torch.uint8)
     units = wl.B * wl.T * wl.H
-    gbs = BYTES_PREFILL * units / (ms / 1e3) / 1e9
-    out["prefill_B1_T1024_H32"] = {"tokens_per_s": wl.B * wl.T / (ms / 1e3), "ms": ms, "achieved_gbs": gbs,
-                                   "frac": gbs / peak, "l2": "flushed (512 MB write) before each rep"}
+    # With a workspace the 32 (b,h) units take the split chunked form (a chunk-parallel pass, then
+    # a short sequential one per unit); without one, the fused form (one CTA per unit).
+    for key, workspace in (("prefill_B1_T1024_H32", ws), ("prefill_B1_T1024_H32_no_workspace", None)):
+        times = []
+        for rep in range(25):
+            flush.fill_(float(rep))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            wkv7.forward(*xs, s0=s0, y=y, s_out=s_out, workspace=workspace, need_workspace=False, algo=algo)
+            e1.record()
+            torch.cuda.synchronize()
+            if rep >= 5:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        gbs = BYTES_PREFILL * units / (ms / 1e3) / 1e9
+        out[key] = {"tokens_per_s": wl.B * wl.T / (ms / 1e3), "ms": ms, "achieved_gbs": gbs,
+                    "frac": gbs / peak, "workspace": workspace is not None,
+                    "l2": "flushed (512 MB write) before each rep"}
 
     wl = I.make_workload(4)
     state = d(wl.state0)
@@ -603,11 +610,13 @@ def run_only(args):
     else:
         xs = [d(wl.inputs[n]) for n in I.NAMES]
         reset = d(wl.reset) if wl.reset is not None else None
-        y, s_out, ws = wkv7.forward(*xs, reset=reset, algo=args.algo, need_workspace=args.only != "prefill")
+        # prefill: with a workspace (the split chunked form for few units) unless --no-workspace
+        want_ws = args.only != "prefill" or not args.no_workspace
+        y, s_out, ws = wkv7.forward(*xs, reset=reset, algo=args.algo, need_workspace=want_ws)
         units = wl.B * wl.T * wl.H
         if args.only in ("fwd", "prefill"):
             fn = lambda: wkv7.forward(*xs, reset=reset, y=y, s_out=s_out, workspace=ws, algo=args.algo,
-                                      need_workspace=args.only == "fwd")
+                                      need_workspace=False)
             per = BYTES_FWD_TRAIN if args.only == "fwd" else BYTES_PREFILL
         else:
             dy = d(wl.dy)

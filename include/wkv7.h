@@ -72,10 +72,27 @@ typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
 /*
  * Algorithm.  SCAN: token-order scan on FP32 cores, state in registers.
  * CHUNKED: 16-token chunks with the intra-chunk products on tensor cores
- * (the chunk-parallel form that the HF model card page also mentions).  AUTO: CHUNKED for 16-bit inputs, SCAN for f32.
- * Both produce the same result up to floating-point rounding order.
+ * (the chunk-parallel form that the HF model card page also mentions), in
+ * one of two forms for the forward pass:
+ *   - fused: one CTA per (b,h) does everything chunk by chunk;
+ *   - split: first every chunk's state-independent products in parallel,
+ *     then one short sequential pass per (b,h).  It needs the workspace
+ *     (its first pass leaves its results in the checkpoint slots and in the
+ *     first 128 bytes of each row of y, which the second pass overwrites).
+ * CHUNKED picks split when a workspace is passed and B*H is at most the
+ * device's SM count, fused otherwise; CHUNKED_FUSED and CHUNKED_SPLIT force
+ * one (CHUNKED_SPLIT without a workspace: WKV7_ERR_WORKSPACE).  The
+ * backward has one chunked form, which all three select.  AUTO: CHUNKED for
+ * 16-bit inputs, SCAN for f32.  All produce the same result up to
+ * floating-point rounding order.
  */
-typedef enum { WKV7_ALGO_AUTO = 0, WKV7_ALGO_SCAN = 1, WKV7_ALGO_CHUNKED = 2 } wkv7_algo_t;
+typedef enum {
+  WKV7_ALGO_AUTO = 0,
+  WKV7_ALGO_SCAN = 1,
+  WKV7_ALGO_CHUNKED = 2,
+  WKV7_ALGO_CHUNKED_FUSED = 3,
+  WKV7_ALGO_CHUNKED_SPLIT = 4
+} wkv7_algo_t;
 
 typedef struct {
   int64_t B;      /* batch rows                                  */
@@ -142,7 +159,11 @@ size_t wkv7_workspace_bytes(const wkv7_desc_t* desc);
  *   y            out  [B,T,H,64] desc->dtype
  *   s_out        out  [B,H,64,64] fp32 final state, or NULL
  *   workspace    out  wkv7_workspace_bytes(desc) bytes of checkpoints for the
- *                     backward, or NULL (inference: no checkpoints written)
+ *                     backward, or NULL (inference: no checkpoints written).
+ *                     Passing one for inference as well lets a forward with
+ *                     B*H at most the SM count run the split chunked form,
+ *                     several times faster there.
+ * y must not overlap any input.
  */
 wkv7_status_t wkv7_forward(const wkv7_desc_t* desc, const void* r, const void* w, const void* k,
                            const void* v, const void* a, const void* b, const float* s0,

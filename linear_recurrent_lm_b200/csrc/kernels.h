@@ -65,6 +65,10 @@ struct InputMaps {
 };
 
 cudaError_t launch_chunk_fwd(const FwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream);
+// Split form of the chunked forward for few (b,h) units: a chunk-parallel pass, then one sequential
+// pass per unit.  Needs p.ckpt (the checkpoint slots carry the first pass's results) and uses the
+// first 128 bytes of every row of y of each full chunk as scratch before writing y there.
+cudaError_t launch_chunk_split_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_chunk_bwd(const BwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream);
 
 }  // namespace wkv7

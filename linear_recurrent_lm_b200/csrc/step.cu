@@ -2,16 +2,25 @@
 //
 // The rwkv-metal page steps one token on a carried state with plain array
 // operations and pads ragged batches on the right without changing the
-// results of the padded rows.  Here one
-// launch steps every (b,h) state: it is a pure stream over the 16 KiB state
-// (read once, written once) and therefore HBM-bound.  One CTA per (b,h), 512
-// threads; thread t owns row t/8 and the 8 columns 8*(t%8)..+7, held as two
-// float4 -- each warp reads and writes 1 KiB of contiguous state with 16-byte
-// accesses, and few registers per thread keep many CTAs (and their loads) in
-// flight per SM.  The two row dot products (sa and y) reduce over the 8
-// lanes of a row with three xor-shuffles.  A row of the batch with active[b]==0
-// returns before touching its state, which therefore stays bitwise unchanged
-// (and costs no bandwidth in a ragged batch), and writes y = 0.
+// results of the padded rows.  Here one launch steps every (b,h) state: it is
+// a pure stream over the 16 KiB state (read once, written once) and therefore
+// HBM-bound.
+//
+// A persistent grid of (SM count x resident CTAs per SM) CTAs of 512 threads
+// walks the B*H units with a grid stride.  Within a unit, thread t owns row
+// t/8 and the 8 columns 8*(t%8)..+7, held as two float4 -- each warp reads and
+// writes 1 KiB of contiguous state with 16-byte accesses, and few registers per
+// thread keep three CTAs (and their loads) in flight per SM.  The two row dot
+// products (sa and y) reduce over the 8 lanes of a row with three
+// xor-shuffles.  A unit whose batch row has active[b] == 0 is skipped without
+// touching its state, which therefore stays bitwise unchanged (and costs no
+// bandwidth in a ragged batch), and gets y = 0; skipping costs one loop
+// iteration instead of a CTA launch.
+//
+// Consecutive decode steps are launched with programmatic dependent launch:
+// the next step's CTAs take the SM slots of this step's finished CTAs and wait
+// (griddepcontrol.wait) until this grid has completed and its writes are
+// visible, so the launch latency of step n+1 overlaps the tail of step n.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -19,6 +28,8 @@ namespace wkv7 {
 namespace {
 
 constexpr int kThreads = 512;
+constexpr int kMinBlocks = 3;
+constexpr int kMaxDevices = 64;
 
 // Eight consecutive elements of T (16-byte aligned) as fp32.
 template <typename T>
@@ -32,57 +43,96 @@ __device__ __forceinline__ void load8(const T* g, float* out) {
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 3) step_kernel(StepArgs p) {
-  const int64_t unit = blockIdx.x;
-  const int64_t b = unit / p.H;
+__global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) {
+  // Everything this grid reads or writes may belong to the grid launched before it.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = threadIdx.x;
   const int i = t >> 3, q = t & 7;   // row i, columns 8q..8q+7
-  T* y = static_cast<T*>(p.y) + unit * kN;
-  if (p.active && !p.active[b]) {   // padded row: its state is not even read
-    if (q == 0) y[i] = Elt<T>::from_f32(0.f);
-    return;
-  }
-  float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 8);
-  const float4 s_lo = row[0], s_hi = row[1];
-  float S[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
-  const int64_t o = unit * kN + q * 8;
-  float wv[8], kv[8], av[8], bv[8], rv[8];
-  load8<T>(static_cast<const T*>(p.a) + o, av);
-  load8<T>(static_cast<const T*>(p.w) + o, wv);
-  load8<T>(static_cast<const T*>(p.b) + o, bv);
-  load8<T>(static_cast<const T*>(p.k) + o, kv);
-  load8<T>(static_cast<const T*>(p.r) + o, rv);
-  const float vi = Elt<T>::to_f32(static_cast<const T*>(p.v)[unit * kN + i]);
+  const int64_t units = p.B * p.H;
+  for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    T* y = static_cast<T*>(p.y) + unit * kN;
+    if (p.active && !p.active[unit / p.H]) {   // padded row: its state is not even read
+      if (q == 0) y[i] = Elt<T>::from_f32(0.f);
+      continue;
+    }
+    float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 8);
+    const float4 s_lo = row[0], s_hi = row[1];
+    float S[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
+    const int64_t o = unit * kN + q * 8;
+    float wv[8], kv[8], av[8], bv[8], rv[8];
+    load8<T>(static_cast<const T*>(p.a) + o, av);
+    load8<T>(static_cast<const T*>(p.w) + o, wv);
+    load8<T>(static_cast<const T*>(p.b) + o, bv);
+    load8<T>(static_cast<const T*>(p.k) + o, kv);
+    load8<T>(static_cast<const T*>(p.r) + o, rv);
+    const float vi = Elt<T>::to_f32(static_cast<const T*>(p.v)[unit * kN + i]);
 
-  float s0 = 0.f, s1 = 0.f;
+    float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; j += 2) {
-    s0 = fmaf(S[j], av[j], s0);
-    s1 = fmaf(S[j + 1], av[j + 1], s1);
-  }
-  float sa = s0 + s1;
-  sa += __shfl_xor_sync(0xffffffffu, sa, 1);
-  sa += __shfl_xor_sync(0xffffffffu, sa, 2);
-  sa += __shfl_xor_sync(0xffffffffu, sa, 4);
+    for (int j = 0; j < 8; j += 2) {
+      s0 = fmaf(S[j], av[j], s0);
+      s1 = fmaf(S[j + 1], av[j + 1], s1);
+    }
+    float sa = s0 + s1;
+    sa += __shfl_xor_sync(0xffffffffu, sa, 1);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 2);
+    sa += __shfl_xor_sync(0xffffffffu, sa, 4);
 
-  float y0 = 0.f, y1 = 0.f;
+    float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    S[j] = fmaf(S[j], wv[j], fmaf(sa, bv[j], vi * kv[j]));
-    if (j & 1) y1 = fmaf(S[j], rv[j], y1); else y0 = fmaf(S[j], rv[j], y0);
+    for (int j = 0; j < 8; ++j) {
+      S[j] = fmaf(S[j], wv[j], fmaf(sa, bv[j], vi * kv[j]));
+      if (j & 1) y1 = fmaf(S[j], rv[j], y1); else y0 = fmaf(S[j], rv[j], y0);
+    }
+    row[0] = make_float4(S[0], S[1], S[2], S[3]);
+    row[1] = make_float4(S[4], S[5], S[6], S[7]);
+    float yy = y0 + y1;
+    yy += __shfl_xor_sync(0xffffffffu, yy, 1);
+    yy += __shfl_xor_sync(0xffffffffu, yy, 2);
+    yy += __shfl_xor_sync(0xffffffffu, yy, 4);
+    if (q == 0) y[i] = Elt<T>::from_f32(yy);
   }
-  row[0] = make_float4(S[0], S[1], S[2], S[3]);
-  row[1] = make_float4(S[4], S[5], S[6], S[7]);
-  float yy = y0 + y1;
-  yy += __shfl_xor_sync(0xffffffffu, yy, 1);
-  yy += __shfl_xor_sync(0xffffffffu, yy, 2);
-  yy += __shfl_xor_sync(0xffffffffu, yy, 4);
-  if (q == 0) y[i] = Elt<T>::from_f32(yy);
+}
+
+// Resident grid size for this device and element type, looked up once.
+template <typename T>
+cudaError_t grid_size(int64_t units, unsigned* out) {
+  static int cached[kMaxDevices] = {};   // SMs x resident CTAs per SM; 0 = not looked up yet
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int slots = (dev >= 0 && dev < kMaxDevices) ? cached[dev] : 0;
+  if (slots == 0) {
+    int sms = 0, per_sm = 0;
+    e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e != cudaSuccess) return e;
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<T>, kThreads, 0);
+    if (e != cudaSuccess) return e;
+    slots = sms * (per_sm > 0 ? per_sm : 1);
+    if (dev >= 0 && dev < kMaxDevices) cached[dev] = slots;
+  }
+  *out = unsigned(units < int64_t(slots) ? units : int64_t(slots));
+  return cudaSuccess;
 }
 
 template <typename T>
 cudaError_t launch(const StepArgs& p, cudaStream_t stream) {
-  step_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), 0, stream>>>(p);
+  unsigned grid = 0;
+  cudaError_t e = grid_size<T>(p.B * p.H, &grid);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, step_kernel<T>, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

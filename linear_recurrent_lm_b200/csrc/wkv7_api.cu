@@ -30,8 +30,7 @@ wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elem
   if (d->N != 64 || (d->flags & ~WKV7_FLAG_TEST_WAIT_TIMEOUT) != 0u) return WKV7_ERR_UNSUPPORTED;
   if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
   if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
-  if (d->algo != WKV7_ALGO_AUTO && d->algo != WKV7_ALGO_SCAN && d->algo != WKV7_ALGO_CHUNKED)
-    return WKV7_ERR_UNSUPPORTED;
+  if (d->algo < WKV7_ALGO_AUTO || d->algo > WKV7_ALGO_CHUNKED_SPLIT) return WKV7_ERR_UNSUPPORTED;
   if (d->B < 0 || d->T < 0 || d->H < 0) return WKV7_ERR_SHAPE;
   int64_t bh, bth, e;
   if (!mul_ok(d->B, d->H, &bh) || bh > kMaxGrid) return WKV7_ERR_SHAPE;
@@ -100,9 +99,26 @@ wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const vo
 unsigned test_extra_tx(const wkv7_desc_t* d) { return (d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) ? 16u : 0u; }
 
 bool use_chunked(const wkv7_desc_t* d) {
-  if (d->algo == WKV7_ALGO_CHUNKED) return true;
   if (d->algo == WKV7_ALGO_SCAN) return false;
-  return d->dtype != WKV7_F32;
+  if (d->algo == WKV7_ALGO_AUTO) return d->dtype != WKV7_F32;
+  return true;
+}
+
+// Split form of the chunked forward: forced, or chosen for few units (at most one per SM) when a
+// workspace is there to carry its first pass.  The timeout test hook exercises the fused form only.
+wkv7_status_t use_split(const wkv7_desc_t* d, int64_t units, const void* workspace, bool* split) {
+  *split = false;
+  if (d->algo == WKV7_ALGO_CHUNKED_SPLIT) {
+    if (!workspace) return WKV7_ERR_WORKSPACE;
+    *split = d->flags == 0u;
+    return WKV7_OK;
+  }
+  if (d->algo == WKV7_ALGO_CHUNKED_FUSED || !workspace || d->flags != 0u) return WKV7_OK;
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return WKV7_ERR_CUDA;
+  *split = units <= int64_t(sms);
+  return WKV7_OK;
 }
 
 }  // namespace
@@ -162,6 +178,10 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
                   status, test_extra_tx(d)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_fwd(p, d->dtype, s));
+  bool split = false;
+  st = use_split(d, units, workspace, &split);
+  if (st != WKV7_OK) return st;
+  if (split) return from_cuda(wkv7::launch_chunk_split_fwd(p, d->dtype, s));
   wkv7::InputMaps tm;
   st = encode_inputs(d, {r, w, k, v, a, b}, &tm);
   if (st != WKV7_OK) return st;

@@ -31,7 +31,7 @@ LIB_PATH = os.path.join(_HERE, "libwkv7.so")
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
-ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2}
+ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2, "chunked_fused": 3, "chunked_split": 4}
 N_HEAD = 64
 CHUNK = 16
 

@@ -43,7 +43,7 @@ def check_grads(g, go, sl=slice(None)):
     return out
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked"))
+@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
 def test_config1_fwd_bwd(W, algo):
     """184M-model layer shape: B=2, T=512, H=12, bf16, checkpoint every 16 tokens."""
     wl = I.make_workload(1)
@@ -52,7 +52,7 @@ def test_config1_fwd_bwd(W, algo):
     check_grads(g, go)
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked"))
+@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
 def test_config3_full_size_sampled_units(W, algo):
     """B=8, T=4096, H=32 packed documents with resets, gradients of sampled units."""
     wl = I.make_workload(3)
@@ -66,7 +66,7 @@ def test_config3_full_size_sampled_units(W, algo):
             assert c >= COS, ((b, h), n, c)
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked"))
+@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
 @pytest.mark.parametrize("T", [1, 15, 17, 40, 100])
 def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
@@ -90,7 +90,7 @@ def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
     assert np.all(f64(g["ds0"])[1] == 0.0)
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked"))
+@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
 def test_small_decay_segments(W, algo):
     """Decays far below the generator's range (prod w < 2^-16 over a chunk) and w = 0."""
     rng = np.random.default_rng(7)

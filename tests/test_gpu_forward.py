@@ -17,7 +17,8 @@ TOL = {"f32": 1e-4, "bf16": 2e-2, "f16": 5e-3}
 # inputs on the exact-fp32 scan.  An emulation of the same roundings puts its error near 4e-3
 # of RMS; the explicit CHUNKED path on fp32 inputs is held to 1e-2.
 TOL_CHUNKED_F32 = 1e-2
-ALGOS = ("scan", "chunked")
+# "chunked" picks one of the two chunked forms by size; the tests force each of them.
+ALGOS = ("scan", "chunked_fused", "chunked_split")
 
 
 @pytest.fixture(scope="module")
@@ -35,7 +36,7 @@ def run_fwd(W, d, s0=None, reset=None, algo="auto"):
 
 
 def check_fwd(y, s, yo, so, dtype, algo="scan"):
-    tol = TOL_CHUNKED_F32 if (dtype == "f32" and algo == "chunked") else TOL[dtype]
+    tol = TOL_CHUNKED_F32 if (dtype == "f32" and algo.startswith("chunked")) else TOL[dtype]
     ey = err_rms_excess(f64(y), yo, dtype)
     es = err_rms(f64(s), so)
     assert ey <= tol, ("y", ey)
@@ -75,7 +76,8 @@ def test_config2_prefill_chained_equals_single(W, algo):
     import torch
     wl = I.make_workload(2)
     _, s_prior, _ = run_fwd(W, wl.prior, algo=algo)
-    y, s, _ = W.forward(*inputs_dev(wl.inputs), s0=s_prior, algo=algo, need_workspace=False)
+    # inference call: no checkpoints wanted, but the split form needs the workspace for its first pass
+    y, s, _ = W.forward(*inputs_dev(wl.inputs), s0=s_prior, algo=algo, need_workspace=algo == "chunked_split")
     full = {n: np.concatenate([wl.prior[n], wl.inputs[n]], axis=1) for n in I.NAMES}
     yf, sf, _ = run_fwd(W, full, algo=algo)
     # split at a multiple of 16: the same arithmetic in the same order
@@ -170,10 +172,53 @@ def test_zero_tokens_and_single_unit(W, algo):
     assert torch.equal(s.cpu(), torch.from_numpy(s0))
 
 
-def test_forward_is_deterministic(W):
+@pytest.mark.parametrize("algo", ("chunked_fused", "chunked_split"))
+def test_forward_is_deterministic(W, algo):
     import torch
     wl = I.make_workload(1)
-    a = run_fwd(W, wl.inputs)
-    b = run_fwd(W, wl.inputs)
+    a = run_fwd(W, wl.inputs, algo=algo)
+    b = run_fwd(W, wl.inputs, algo=algo)
     n_ck = 2 * 12 * 32 * 64 * 64 * 4          # the checkpoints; the workspace tail belongs to the backward
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1]) and torch.equal(a[2][:n_ck], b[2][:n_ck])
+
+
+def test_chunked_picks_split_for_few_units_with_a_workspace(W):
+    """CHUNKED runs the split form when a workspace is given and B*H fits in one CTA per SM (its
+    results then equal CHUNKED_SPLIT's bit for bit), the fused form otherwise; CHUNKED_SPLIT
+    without a workspace is refused before anything is launched."""
+    import torch
+    wl = I.make_workload(1)                                # 24 (b,h) units
+    xs = inputs_dev(wl.inputs)
+    ya, sa, wa = W.forward(*xs, algo="chunked")
+    yb, sb, wb = W.forward(*xs, algo="chunked_split")
+    assert torch.equal(ya, yb) and torch.equal(sa, sb)
+    yc, sc, _ = W.forward(*xs, algo="chunked", need_workspace=False)
+    yd, sd, _ = W.forward(*xs, algo="chunked_fused", need_workspace=False)
+    assert torch.equal(yc, yd) and torch.equal(sc, sd)
+    with pytest.raises(W.WKV7Error):
+        W.forward(*xs, algo="chunked_split", need_workspace=False)
+
+
+def test_split_form_reuses_buffers_across_calls(W):
+    """The split form leaves its first pass's results in the checkpoint slots and in y before
+    overwriting them: a second call into the same buffers with other inputs (decays that force
+    some chunks onto the token path this time) must not see anything of the first."""
+    import torch
+    rng = np.random.default_rng(21)
+    B, T, H = 2, 96, 3
+    d1 = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    d2 = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    w2 = I.to_f64(d2["w"])
+    w2[0, 20] = 0.0
+    w2[1, 70] = 0.0
+    d2["w"] = I.to_storage(w2, "bf16")
+    y, s, ws = W.forward(*inputs_dev(d1), algo="chunked_split")
+    y2, s2, ws2 = W.forward(*inputs_dev(d2), algo="chunked_split", y=y, s_out=s, workspace=ws)
+    assert y2.data_ptr() == y.data_ptr() and ws2.data_ptr() == ws.data_ptr()
+    yo, so, _ = oracle.forward(*inputs_f64(d2))
+    check_fwd(y2, s2, yo, so, "bf16")
+    ck = checkpoint_states(ws2, B, H, T // 16)
+    for c in (0, 1, 4, 5):
+        part = {n: d2[n][:, : 16 * (c + 1)] for n in I.NAMES}
+        _, sc, _ = oracle.forward(*inputs_f64(part))
+        assert err_rms(ck[:, :, c], sc) <= 2e-2

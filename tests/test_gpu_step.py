@@ -55,3 +55,29 @@ def test_step_equals_one_token_forward(W, dtype):
     assert err_rms_excess(f64(y_s), yo[:, 0], dtype) <= tol
     assert err_rms(f64(st), so) <= 1e-4
     assert err_rms(f64(st), f64(s_f)) <= 1e-5
+
+
+@pytest.mark.parametrize("B,H", [(3, 2), (64, 8)])
+def test_back_to_back_steps_see_each_others_state(W, B, H):
+    """Steps launched back to back with no host work between them: every step must read the
+    state its predecessor wrote (the launches overlap their predecessors' tails), whether the
+    batch needs fewer CTAs than the GPU holds or many units per CTA."""
+    import torch
+    rng = np.random.default_rng(11)
+    n_steps = 24
+    toks = [I.draw_inputs(rng, (B, 1, H, 64), "bf16") for _ in range(n_steps)]
+    acts = [(rng.random(B) < 0.8).astype(np.uint8) for _ in range(n_steps)]
+    s0 = (0.1 * rng.standard_normal((B, H, 64, 64))).astype(np.float32)
+    dev_in = [[to_dev(t[n][:, 0]) for n in I.NAMES] for t in toks]
+    dev_act = [to_dev(a) for a in acts]
+    ys = [torch.empty_like(dev_in[0][0]) for _ in range(n_steps)]
+    state = to_dev(s0)
+    torch.cuda.synchronize()
+    for s in range(n_steps):
+        W.step(*dev_in[s], state, dev_act[s], y=ys[s])
+    torch.cuda.synchronize()
+    st_o = s0.astype(np.float64)
+    for s in range(n_steps):
+        yo, st_o = oracle.step(*(I.to_f64(toks[s][n][:, 0], "bf16") for n in I.NAMES), st_o, acts[s])
+        assert err_rms_excess(f64(ys[s]), yo, "bf16") <= 2e-2
+    assert err_rms(f64(state), st_o) <= 2e-2
