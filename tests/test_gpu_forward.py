@@ -222,3 +222,18 @@ def test_split_form_reuses_buffers_across_calls(W):
         part = {n: d2[n][:, : 16 * (c + 1)] for n in I.NAMES}
         _, sc, _ = oracle.forward(*inputs_f64(part))
         assert err_rms(ck[:, :, c], sc) <= 2e-2
+
+
+@pytest.mark.parametrize("algo", ("chunked_fused", "chunked_split"))
+def test_chunked_forms_run_full_chunks_on_the_tensor_cores(W, algo):
+    """Both chunked forms fall back to the exact token path only for chunks that need it: on
+    ordinary decays their y differs from the fp32 scan by tf32 rounding (well above the ~1e-6 of
+    two fp32 token-order computations) while staying inside the bf16 bound."""
+    rng = np.random.default_rng(31)
+    d = I.draw_inputs(rng, (2, 256, 4, 64), "f32")
+    yc, sc, _ = run_fwd(W, d, algo=algo)
+    ys, ss, _ = run_fwd(W, d, algo="scan")
+    assert err_rms(f64(yc), f64(ys)) > 1e-5
+    assert err_rms(f64(sc), f64(ss)) > 1e-5
+    yo, so, _ = oracle.forward(*inputs_f64(d))
+    assert err_rms(f64(yc), yo) <= TOL_CHUNKED_F32 and err_rms(f64(sc), so) <= TOL_CHUNKED_F32
