@@ -65,7 +65,6 @@ __device__ __forceinline__ void mask_nat(uint32_t (&a)[4], int s, int c4, unsign
   if (!k1) { a[2] = 0u; a[3] = 0u; }
 }
 __device__ __forceinline__ uint32_t fu(float x) { return __float_as_uint(x); }
-
 // Reset bits of the chunk at t0 (every lane of the calling warp gets them).
 __device__ __forceinline__ unsigned chunk_mask(const FwdArgs& p, int64_t b, int64_t t0, int len, int lane) {
   const bool f = p.reset && lane < len && p.reset[b * p.T + t0 + lane] != 0;
@@ -406,36 +405,48 @@ struct __align__(16) ChainSmem {
   __align__(16) T Ys[kChunk][kStrY];   // y of the chunk [t][i]
 };
 
-// Issue the copies of chunk c's operands into `bf` (full chunks only; always one commit group).
+// Per-thread sources of phase 2's copies, fixed for the whole sequence: chunk c reads the same rows
+// c * 16 tokens further on, and its checkpoint slot c * 4096 floats further on.
 template <typename T>
-__device__ __forceinline__ void chain_stage(const FwdArgs& p, ChainBuf<T>& bf, int64_t unit, int64_t b, int64_t h,
-                                            int64_t c, int64_t nc, int64_t nfull, int tid) {
+struct StagePlan {
+  static constexpr int kPieces = kN * int(sizeof(T)) / 16;   // 16-byte pieces per row of v
+  static constexpr int kVPer = kChunk * kPieces / kThreads;   // pieces of v per thread per chunk
+  const float* slot0;        // checkpoint slot of chunk 0 of this unit
+  const T* yrow0;            // y row (token tid/8) of chunk 0
+  const T* vrow0[kVPer];     // v rows of this thread's pieces, chunk 0
+  int64_t chunk_elems;       // elements from a row to the same row of the next chunk
+};
+
+// Issue the copies of chunk c's operands into `bf` (full chunks only; always one commit group).  The
+// 16 KiB slot is contiguous: float 4i of it lands in W|Q (rows padded to 72) for i < 512, in
+// Bl^T|Kx^T (rows padded to 24) above.
+template <typename T>
+__device__ __forceinline__ void chain_stage(const StagePlan<T>& sp, ChainBuf<T>& bf, int64_t c, int64_t nfull,
+                                            int tid) {
   if (c < nfull) {
-    const float* slot = p.ckpt + (unit * nc + c) * (kN * kN);
-    const int64_t t0 = c * kChunk;
-    // W, Q: 16 rows x 16 pieces each
-    for (int idx = tid; idx < 2 * kChunk * 16; idx += kThreads) {
-      const int q = idx >> 8, rem = idx & 255, t = rem >> 4, piece = rem & 15;
-      float* dst = q ? &bf.Q[t][4 * piece] : &bf.W[t][4 * piece];
-      cp_async16(dst, slot + (q ? kOffQ : kOffW) + t * kN + 4 * piece);
+    const float* slot = sp.slot0 + c * (kN * kN);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const int i = tid + k * kThreads;
+      float* dst;
+      if (k < 4) {
+        const int q = i >> 8, t = (i >> 4) & 15, piece = i & 15;
+        dst = &bf.W[0][0] + q * (kChunk * S72) + t * S72 + 4 * piece;
+      } else {
+        const int q = (i >> 8) - 2, j = (i >> 2) & 63, piece = i & 3;
+        dst = &bf.BlT[0][0] + q * (kN * S24) + j * S24 + 4 * piece;
+      }
+      cp_async16(dst, slot + 4 * i);
     }
-    // Bl^T, Kx^T: 64 rows x 4 pieces each
-    for (int idx = tid; idx < 2 * kN * 4; idx += kThreads) {
-      const int q = idx >> 8, rem = idx & 255, j = rem >> 2, piece = rem & 3;
-      float* dst = q ? &bf.KxT[j][4 * piece] : &bf.BlT[j][4 * piece];
-      cp_async16(dst, slot + (q ? kOffKx : kOffBl) + j * kChunk + 4 * piece);
-    }
-    // Z and ext from the first 128 bytes of each y row; the v rows
-    {
-      const int t = tid >> 3, part = tid & 7;
-      const float* yrow = reinterpret_cast<const float*>(static_cast<const T*>(p.y) + tok_off(b, t0 + t, h, p.T, p.H));
-      cp_async16(part < 4 ? &bf.Z[t][4 * part] : &bf.ext[t][4 * (part - 4)], yrow + 4 * part);
-    }
-    constexpr int kPieces = kN * int(sizeof(T)) / 16;
-    for (int idx = tid; idx < kChunk * kPieces; idx += kThreads) {
-      const int t = idx / kPieces, piece = idx - t * kPieces;
-      cp_async16(&bf.v[t][piece * (16 / int(sizeof(T)))],
-                 static_cast<const T*>(p.v) + tok_off(b, t0 + t, h, p.T, p.H) + piece * (16 / int(sizeof(T))));
+    const int64_t off = c * sp.chunk_elems;
+    const int part = tid & 7;
+    const float* yrow = reinterpret_cast<const float*>(sp.yrow0 + off);
+    cp_async16(part < 4 ? &bf.Z[tid >> 3][4 * part] : &bf.ext[tid >> 3][4 * (part - 4)], yrow + 4 * part);
+#pragma unroll
+    for (int k = 0; k < StagePlan<T>::kVPer; ++k) {
+      const int idx = tid + k * kThreads;
+      const int t = idx / StagePlan<T>::kPieces, piece = idx - t * StagePlan<T>::kPieces;
+      cp_async16(&bf.v[t][piece * (16 / int(sizeof(T)))], sp.vrow0[k] + off + piece * (16 / int(sizeof(T))));
     }
   }
   cp_async_commit();
@@ -471,12 +482,22 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
       acc[nt][2 * hh + 1] = v2.y;
     }
 
+  StagePlan<T> sp;
+  sp.slot0 = p.ckpt + unit * nc * (kN * kN);
+  sp.chunk_elems = int64_t(kChunk) * p.H * kN;
+  sp.yrow0 = static_cast<const T*>(p.y) + tok_off(b, tid >> 3, h, p.T, p.H);
 #pragma unroll
-  for (int k = 0; k < kRing - 1; ++k) chain_stage<T>(p, sm.buf[k], unit, b, h, k, nc, nfull, tid);
+  for (int k = 0; k < StagePlan<T>::kVPer; ++k)
+    sp.vrow0[k] = static_cast<const T*>(p.v) + tok_off(b, (tid + k * kThreads) / StagePlan<T>::kPieces, h, p.T, p.H);
+  T* const ybase = static_cast<T*>(p.y) + tok_off(b, 0, h, p.T, p.H);   // token 0 of this (b,h)
+  const int64_t tok_stride = p.H * kN;
+
+#pragma unroll
+  for (int k = 0; k < kRing - 1; ++k) chain_stage<T>(sp, sm.buf[k], k, nfull, tid);
 
   for (int64_t c = 0; c < nc; ++c) {
     // the buffer of chunk c - 1 is free (barrier at the end of the last iteration): refill it
-    chain_stage<T>(p, sm.buf[(c + kRing - 1) % kRing], unit, b, h, c + kRing - 1, nc, nfull, tid);
+    chain_stage<T>(sp, sm.buf[(c + kRing - 1) % kRing], c + kRing - 1, nfull, tid);
     cp_async_wait_group<kRing - 1>();
     __syncthreads();
     const ChainBuf<T>& bf = sm.buf[c % kRing];
@@ -575,9 +596,10 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
     __syncthreads();   // Ys complete; every read of this chunk's operand slot is done
     {
       constexpr int kPieces = kN * int(sizeof(T)) / 16;
+#pragma unroll
       for (int idx = tid; idx < kChunk * kPieces; idx += kThreads) {
         const int t = idx / kPieces, piece = idx - t * kPieces;
-        *reinterpret_cast<uint4*>(static_cast<T*>(p.y) + tok_off(b, t0 + t, h, p.T, p.H) + piece * (16 / int(sizeof(T)))) =
+        *reinterpret_cast<uint4*>(ybase + (t0 + t) * tok_stride + piece * (16 / int(sizeof(T)))) =
             *reinterpret_cast<const uint4*>(&sm.Ys[t][piece * (16 / int(sizeof(T)))]);
       }
     }
