@@ -171,6 +171,7 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   if (st != WKV7_OK) return st;
   st = check_ptrs(false, {s0, s_out, workspace});
   if (st != WKV7_OK) return st;
+  if (d->algo == WKV7_ALGO_CHUNKED_SPLIT && te > 0 && !workspace) return WKV7_ERR_WORKSPACE;
   if (units == 0) return WKV7_OK;
   int* status = nullptr;
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;

@@ -79,6 +79,12 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = 7
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = -1
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    # the split chunked forward carries its first pass in the workspace: required even for inference
+    assert call_fwd(L, L.make_desc(1, 16, 1, torch.bfloat16, "chunked_split")) == L.ERR_WORKSPACE
+    assert call_fwd(L, L.make_desc(0, 16, 1, torch.bfloat16, "chunked_split"),
+                    r=None, w=None, k=None, v=None, a=None, b=None, y=None) == L.OK   # nothing to run
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.dtype = 9
     assert call_fwd(L, bad) == L.ERR_DTYPE
     assert call_fwd(L, L.make_desc(-1, 16, 1, torch.bfloat16)) == L.ERR_SHAPE
