@@ -21,6 +21,8 @@
 // the next step's CTAs take the SM slots of this step's finished CTAs and wait
 // (griddepcontrol.wait) until this grid has completed and its writes are
 // visible, so the launch latency of step n+1 overlaps the tail of step n.
+#include <atomic>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -95,14 +97,15 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) 
   }
 }
 
-// Resident grid size for this device and element type, looked up once.
+// Resident grid size for this device and element type, looked up once (concurrent first calls
+// may both look it up; they store the same value).
 template <typename T>
 cudaError_t grid_size(int64_t units, unsigned* out) {
-  static int cached[kMaxDevices] = {};   // SMs x resident CTAs per SM; 0 = not looked up yet
+  static std::atomic<int> cached[kMaxDevices];   // SMs x resident CTAs per SM; 0 = not looked up yet
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int slots = (dev >= 0 && dev < kMaxDevices) ? cached[dev] : 0;
+  int slots = (dev >= 0 && dev < kMaxDevices) ? cached[dev].load(std::memory_order_relaxed) : 0;
   if (slots == 0) {
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
@@ -110,7 +113,7 @@ cudaError_t grid_size(int64_t units, unsigned* out) {
     e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<T>, kThreads, 0);
     if (e != cudaSuccess) return e;
     slots = sms * (per_sm > 0 ? per_sm : 1);
-    if (dev >= 0 && dev < kMaxDevices) cached[dev] = slots;
+    if (dev >= 0 && dev < kMaxDevices) cached[dev].store(slots, std::memory_order_relaxed);
   }
   *out = unsigned(units < int64_t(slots) ? units : int64_t(slots));
   return cudaSuccess;
