@@ -64,7 +64,8 @@ typedef enum {
   WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, unknown flags, or T != 1 for a step     */
   WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
   WKV7_ERR_TIMEOUT = 8,     /* reserved for device-side bounded waits                          */
-  WKV7_ERR_SCRATCH_LIMIT = 9 /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
+  WKV7_ERR_SCRATCH_LIMIT = 9, /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
+  WKV7_ERR_NONFINITE = 10    /* WKV7_FLAG_CHECK_FINITE found a NaN or infinity in an output       */
 } wkv7_status_t;
 
 typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
@@ -101,7 +102,7 @@ typedef struct {
   int32_t N;      /* head size: must be 64                       */
   int32_t dtype;  /* wkv7_dtype_t of every activation/gradient   */
   int32_t algo;   /* wkv7_algo_t                                 */
-  uint32_t flags; /* 0, or WKV7_FLAG_TEST_WAIT_TIMEOUT (below)     */
+  uint32_t flags; /* 0, or the WKV7_FLAG_* bits below            */
 } wkv7_desc_t;
 
 /*
@@ -116,13 +117,25 @@ typedef struct {
 #define WKV7_FLAG_TEST_WAIT_TIMEOUT 0x80000000u
 
 /*
+ * desc->flags bit: after the call's kernels, scan its floating outputs on the
+ * same stream (forward: y and s_out; backward: dr..db and ds0; step: y and
+ * the updated state) and record any NaN or infinity in the device status
+ * word, which wkv7_get_device_status() then reports as WKV7_ERR_NONFINITE.
+ * The scan reads each output once more; the results themselves are
+ * unchanged.  It may be combined with WKV7_FLAG_TEST_WAIT_TIMEOUT.
+ */
+#define WKV7_FLAG_CHECK_FINITE 0x1u
+
+/*
  * Device status word (the device-side error channel of the boundary).
  * Kernels record errors they cannot return from an asynchronous launch --
- * today a bounded wait on staged inputs that ran out -- in one word per
- * device.  This call synchronises the current device, reads the word and,
- * if `clear` is non-zero, resets it.  Returns WKV7_OK, WKV7_ERR_TIMEOUT if a
- * wait ran out since the last clear, or WKV7_ERR_CUDA if synchronising or
- * reading failed (e.g. no device).
+ * a bounded wait that ran out, or a non-finite output found under
+ * WKV7_FLAG_CHECK_FINITE -- in one word per device.  This call synchronises
+ * the current device, reads the word and, if `clear` is non-zero, resets
+ * it.  Returns WKV7_OK, WKV7_ERR_TIMEOUT if a wait ran out since the last
+ * clear (this takes precedence), WKV7_ERR_NONFINITE if a checked output
+ * held a NaN or infinity, or WKV7_ERR_CUDA if synchronising or reading
+ * failed (e.g. no device).
  */
 wkv7_status_t wkv7_get_device_status(int clear);
 

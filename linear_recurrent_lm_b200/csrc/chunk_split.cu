@@ -20,7 +20,7 @@
 //
 // Phase 1 hands its results over in memory the call already owns: W, Q, Bl^T and Kx^T fill the
 // chunk's 16 KiB checkpoint slot exactly, and Z, L_15 and a completion marker go into the first
-// 128 bytes of each of the chunk's 16 rows of y.  Phase 2 reads both (cp.async, three chunks
+// 128 bytes of each of the chunk's 16 rows of y.  Phase 2 reads both (cp.async, two chunks
 // ahead) before it writes y and the chunk-end checkpoint over them.  A chunk whose decay product
 // leaves [2^-40, 2^40] gets no operands (phase 1 writes marker 0) and, like a ragged last chunk,
 // is run token by token in phase 2.

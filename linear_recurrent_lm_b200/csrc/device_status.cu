@@ -45,5 +45,6 @@ extern "C" wkv7_status_t wkv7_get_device_status(int clear) {
     const int zero = 0;
     if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
   }
-  return (v & wkv7::kStatusWaitTimeout) ? WKV7_ERR_TIMEOUT : WKV7_OK;
+  if (v & wkv7::kStatusWaitTimeout) return WKV7_ERR_TIMEOUT;
+  return (v & wkv7::kStatusNonFinite) ? WKV7_ERR_NONFINITE : WKV7_OK;
 }

@@ -22,6 +22,7 @@ struct FwdArgs {
 
 // Bits of the device status word.
 constexpr int kStatusWaitTimeout = 1;
+constexpr int kStatusNonFinite = 2;
 
 // Wall-clock limit of one bounded wait on a staging barrier (the copies it waits for take microseconds).
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
@@ -54,6 +55,9 @@ cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 // only_flagged: run only the (b,h) units whose unit_flags entry is non-zero (others exit at once).
 cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
+// Set kStatusNonFinite in *status if any of the n elements at x (dtype as above; 16-byte aligned)
+// is NaN or infinite.  x == nullptr or n == 0: nothing is launched.
+cudaError_t launch_finite_scan(const void* x, int64_t n, int dtype, int* status, cudaStream_t stream);
 // Device address of this device's status word (looked up once per device).
 cudaError_t device_status_ptr(int** out);
 

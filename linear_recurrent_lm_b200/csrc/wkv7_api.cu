@@ -6,6 +6,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <initializer_list>
 #include <mutex>
 
 #include "kernels.h"
@@ -27,7 +28,8 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
 // Common descriptor checks.  On success fills the element counts.
 wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
   if (!d) return WKV7_ERR_NULL;
-  if (d->N != 64 || (d->flags & ~WKV7_FLAG_TEST_WAIT_TIMEOUT) != 0u) return WKV7_ERR_UNSUPPORTED;
+  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE)) != 0u)
+    return WKV7_ERR_UNSUPPORTED;
   if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
   if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
   if (d->algo < WKV7_ALGO_AUTO || d->algo > WKV7_ALGO_CHUNKED_SPLIT) return WKV7_ERR_UNSUPPORTED;
@@ -55,6 +57,22 @@ wkv7_status_t check_ptrs(bool need, std::initializer_list<const void*> ptrs) {
 }
 
 wkv7_status_t from_cuda(cudaError_t e) { return e == cudaSuccess ? WKV7_OK : WKV7_ERR_CUDA; }
+
+// Under WKV7_FLAG_CHECK_FINITE: after a call's kernels succeeded, scan its outputs (pointer, element
+// count, dtype code) on the same stream.
+struct Output {
+  const void* ptr;
+  int64_t n;
+  int dtype;
+};
+wkv7_status_t check_outputs(const wkv7_desc_t* d, cudaError_t launched, std::initializer_list<Output> outs, int* status,
+                            cudaStream_t s) {
+  if (launched != cudaSuccess) return WKV7_ERR_CUDA;
+  if (!(d->flags & WKV7_FLAG_CHECK_FINITE)) return WKV7_OK;
+  for (const Output& o : outs)
+    if (wkv7::launch_finite_scan(o.ptr, o.n, o.dtype, status, s) != cudaSuccess) return WKV7_ERR_CUDA;
+  return WKV7_OK;
+}
 
 // cuTensorMapEncodeTiled from the driver, looked up once through the runtime (no link to libcuda).
 PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
@@ -110,10 +128,10 @@ wkv7_status_t use_split(const wkv7_desc_t* d, int64_t units, const void* workspa
   *split = false;
   if (d->algo == WKV7_ALGO_CHUNKED_SPLIT) {
     if (!workspace) return WKV7_ERR_WORKSPACE;
-    *split = d->flags == 0u;
+    *split = (d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) == 0u;
     return WKV7_OK;
   }
-  if (d->algo == WKV7_ALGO_CHUNKED_FUSED || !workspace || d->flags != 0u) return WKV7_OK;
+  if (d->algo == WKV7_ALGO_CHUNKED_FUSED || !workspace || (d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT)) return WKV7_OK;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return WKV7_ERR_CUDA;
@@ -139,6 +157,7 @@ const char* wkv7_status_string(wkv7_status_t s) {
     case WKV7_ERR_CUDA: return "CUDA launch failed";
     case WKV7_ERR_TIMEOUT: return "device-side wait timed out";
     case WKV7_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of wkv7_train_step_noalloc";
+    case WKV7_ERR_NONFINITE: return "an output checked under WKV7_FLAG_CHECK_FINITE holds a NaN or infinity";
   }
   return "unknown status";
 }
@@ -178,15 +197,16 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
                   status, test_extra_tx(d)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_fwd(p, d->dtype, s));
+  const std::initializer_list<Output> outs = {{y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}};
+  if (d->T == 0 || !use_chunked(d)) return check_outputs(d, wkv7::launch_scan_fwd(p, d->dtype, s), outs, status, s);
   bool split = false;
   st = use_split(d, units, workspace, &split);
   if (st != WKV7_OK) return st;
-  if (split) return from_cuda(wkv7::launch_chunk_split_fwd(p, d->dtype, s));
+  if (split) return check_outputs(d, wkv7::launch_chunk_split_fwd(p, d->dtype, s), outs, status, s);
   wkv7::InputMaps tm;
   st = encode_inputs(d, {r, w, k, v, a, b}, &tm);
   if (st != WKV7_OK) return st;
-  return from_cuda(wkv7::launch_chunk_fwd(p, tm, d->dtype, s));
+  return check_outputs(d, wkv7::launch_chunk_fwd(p, tm, d->dtype, s), outs, status, s);
 }
 
 wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
@@ -210,14 +230,18 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
                   dr, dw, dk, dv, da, db, ds0, flags, status, test_extra_tx(d)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (d->T == 0 || !use_chunked(d)) return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, false, s));
+  const std::initializer_list<Output> outs = {{dr, te, d->dtype}, {dw, te, d->dtype}, {dk, te, d->dtype},
+                                              {dv, te, d->dtype}, {da, te, d->dtype}, {db, te, d->dtype},
+                                              {ds0, units * 64 * 64, WKV7_F32}};
+  if (d->T == 0 || !use_chunked(d))
+    return check_outputs(d, wkv7::launch_scan_bwd(p, d->dtype, false, s), outs, status, s);
   // Chunked pass, then the exact scan for the units it marked (decays too small for 1/L scaling).
   wkv7::InputMaps tm;
   st = encode_inputs(d, {r, w, k, v, a, b, dy}, &tm);
   if (st != WKV7_OK) return st;
   cudaError_t e = wkv7::launch_chunk_bwd(p, tm, d->dtype, s);
   if (e != cudaSuccess) return WKV7_ERR_CUDA;
-  return from_cuda(wkv7::launch_scan_bwd(p, d->dtype, true, s));
+  return check_outputs(d, wkv7::launch_scan_bwd(p, d->dtype, true, s), outs, status, s);
 }
 
 wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
@@ -229,8 +253,12 @@ wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, cons
   st = check_ptrs(units > 0, {r, w, k, v, a, b, state, y});
   if (st != WKV7_OK) return st;
   if (units == 0) return WKV7_OK;
+  int* status = nullptr;
+  if ((d->flags & WKV7_FLAG_CHECK_FINITE) && wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y};
-  return from_cuda(wkv7::launch_step(p, d->dtype, static_cast<cudaStream_t>(stream)));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return check_outputs(d, wkv7::launch_step(p, d->dtype, s), {{y, units * 64, d->dtype}, {state, units * 64 * 64, WKV7_F32}},
+                       status, s);
 }
 
 }  // extern "C"

@@ -9,7 +9,7 @@ stream.  The same entry points as the C ABI:
   -> dict(dr, dw, dk, dv, da, db, ds0)
 * ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
 * ``workspace_bytes(B, T, H, dtype)``
-* ``device_status(clear=True)`` -> OK or ERR_TIMEOUT (synchronises the device)
+* ``device_status(clear=True)`` -> OK, ERR_TIMEOUT or ERR_NONFINITE (synchronises the device)
 
 Tensors are [B,T,H,64] (token inputs), [B,H,64,64] fp32 (states), [B,T] uint8
 (reset), [B] uint8 (active), all on one CUDA device and contiguous.  If the
@@ -27,9 +27,10 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libwkv7.so")
 
 (OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT,
- ERR_SCRATCH_LIMIT) = range(10)
+ ERR_SCRATCH_LIMIT, ERR_NONFINITE) = range(11)
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
+FLAG_CHECK_FINITE = 0x1                    # WKV7_FLAG_CHECK_FINITE: scan outputs for NaN / Inf
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2, "chunked_fused": 3, "chunked_split": 4}
 N_HEAD = 64
@@ -92,7 +93,7 @@ def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16) -> int:
 
 
 def device_status(clear: bool = True) -> int:
-    """The device status word of the current device (synchronises it): OK or ERR_TIMEOUT."""
+    """The device status word of the current device (synchronises it): OK, ERR_TIMEOUT or ERR_NONFINITE."""
     return int(lib().wkv7_get_device_status(1 if clear else 0))
 
 
@@ -159,14 +160,14 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
     return g
 
 
-def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None):
+def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None, flags: int = 0):
     """One decode token on ``state`` [B,H,64,64] (in place).  Inputs [B,H,64].  Returns y."""
     if r.dim() != 3 or r.shape[-1] != N_HEAD:
         raise ValueError(f"expected [B,H,{N_HEAD}], got {tuple(r.shape)}")
     B, H = int(r.shape[0]), int(r.shape[1])
     if y is None:
         y = torch.empty_like(r)
-    d = make_desc(B, 1, H, r.dtype)
+    d = make_desc(B, 1, H, r.dtype, flags=flags)
     st = lib().wkv7_step(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, state, active, y)), _stream(stream))
     _check(st, "wkv7_step")
     return y

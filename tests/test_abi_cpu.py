@@ -37,8 +37,8 @@ def test_exports_every_declared_symbol(L):
 def test_version_and_status_strings(L):
     lib = L.lib()
     assert lib.wkv7_version() >= 100
-    for s in range(9):
-        assert lib.wkv7_status_string(s)
+    strings = [lib.wkv7_status_string(s) for s in range(L.ERR_NONFINITE + 1)]
+    assert all(strings) and b"unknown status" not in strings and len(set(strings)) == len(strings)
     assert lib.wkv7_status_string(12345) == b"unknown status"
 
 
@@ -71,7 +71,7 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, None) == L.ERR_NULL
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.N = 32
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
-    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 1
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 2                 # no such flag bit
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 17, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT)   # the test hook needs T <= 16
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
@@ -124,6 +124,10 @@ def test_no_cpu_fallback_without_gpu(L):
         pytest.skip("host has a GPU")
     d = L.make_desc(1, 16, 1, torch.bfloat16)
     assert call_fwd(L, d) == L.ERR_CUDA
+    # the output check is a valid flag on its own and with the timeout hook (T <= 16)
+    assert call_fwd(L, L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_CHECK_FINITE)) == L.ERR_CUDA
+    both = L.FLAG_CHECK_FINITE | L.FLAG_TEST_WAIT_TIMEOUT
+    assert call_fwd(L, L.make_desc(1, 16, 1, torch.bfloat16, flags=both)) == L.ERR_CUDA
     assert L.device_status() == L.ERR_CUDA      # the status word cannot be read without a device
 
 

@@ -75,3 +75,45 @@ def test_backward_wait_timeout_is_reported_and_gradients_stay_correct(W):
     # the context is still usable
     _, _, ws = W.forward(*xs, s0=to_dev(s0))
     assert W.device_status() == W.OK
+
+
+@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
+def test_check_finite_flags_nonfinite_outputs_only(W, algo):
+    """WKV7_FLAG_CHECK_FINITE scans the outputs after the call: finite results leave the status
+    OK; an infinity in v (which reaches y and the state) is reported as NONFINITE, and the
+    results of the call are the same as without the flag."""
+    import torch
+    d, dy, s0 = _case(40)
+    xs = inputs_dev(d)
+    W.device_status(clear=True)
+    y0, s_0, _ = W.forward(*xs, s0=to_dev(s0), algo=algo)
+    y1, s_1, ws = W.forward(*xs, s0=to_dev(s0), algo=algo, flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status() == W.OK
+    assert torch.equal(y0, y1) and torch.equal(s_0, s_1)
+    g = W.backward(*xs, to_dev(dy), ws, s0=to_dev(s0), algo=algo, flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status() == W.OK
+    v = I.to_f64(d["v"])
+    v[0, 33, 1, 7] = np.inf
+    bad = dict(d, v=I.to_storage(v, "bf16"))
+    W.forward(*inputs_dev(bad), s0=to_dev(s0), algo=algo)            # unchecked: nothing recorded
+    assert W.device_status() == W.OK
+    W.forward(*inputs_dev(bad), s0=to_dev(s0), algo=algo, flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status(clear=False) == W.ERR_NONFINITE
+    assert W.device_status() == W.ERR_NONFINITE                       # cleared by this read
+    assert W.device_status() == W.OK
+    dyb = I.to_f64(dy)
+    dyb[0, 5, 0, 3] = np.nan
+    W.backward(*xs, to_dev(I.to_storage(dyb, "bf16")), ws, s0=to_dev(s0), algo=algo, flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status() == W.ERR_NONFINITE
+
+
+def test_check_finite_on_the_decode_step(W):
+    rng = np.random.default_rng(8)
+    d = I.draw_inputs(rng, (4, 1, 3, 64), "bf16")
+    state = (0.1 * rng.standard_normal((4, 3, 64, 64))).astype(np.float32)
+    W.device_status(clear=True)
+    W.step(*(to_dev(d[n][:, 0]) for n in I.NAMES), to_dev(state), flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status() == W.OK
+    state[2, 1, 10, 20] = np.inf
+    W.step(*(to_dev(d[n][:, 0]) for n in I.NAMES), to_dev(state), flags=W.FLAG_CHECK_FINITE)
+    assert W.device_status() == W.ERR_NONFINITE
