@@ -35,7 +35,9 @@
  * - Every pointer is a DEVICE pointer, 16-byte aligned (reset and active may
  *   have any alignment).  The caller allocates and owns every buffer; the
  *   library allocates nothing, keeps no per-call state and may be called from
- *   several host threads on different streams.
+ *   several host threads on different streams -- except
+ *   wkv7_train_step_noalloc, whose calls share one fixed scratch array of the
+ *   library and must not overlap (see there).
  * - `stream` is a cudaStream_t (NULL = the legacy default stream).  Calls are
  *   asynchronous on it.  The returned status covers argument validation and
  *   the launch itself (cudaGetLastError); on any validation error nothing is
@@ -57,11 +59,11 @@ extern "C" {
 typedef enum {
   WKV7_OK = 0,
   WKV7_ERR_NULL = 1,        /* a required pointer is NULL                                    */
-  WKV7_ERR_SHAPE = 2,       /* B, T or H negative, or the element count overflows int64       */
+  WKV7_ERR_SHAPE = 2,       /* B, T or H negative, or an element or workspace byte count overflows int64 */
   WKV7_ERR_DTYPE = 3,       /* dtype code is not a wkv7_dtype_t                               */
   WKV7_ERR_ALIGN = 4,       /* a tensor pointer is not 16-byte aligned                        */
   WKV7_ERR_WORKSPACE = 5,   /* backward without a checkpoint workspace                        */
-  WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo, unknown flags, or T != 1 for a step     */
+  WKV7_ERR_UNSUPPORTED = 6, /* N != 64, unknown algo or flags, CHUNKED* with f32, T != 1 for a step */
   WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
   WKV7_ERR_TIMEOUT = 8,     /* reserved for device-side bounded waits                          */
   WKV7_ERR_SCRATCH_LIMIT = 9, /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
@@ -84,8 +86,11 @@ typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
  * device's SM count, fused otherwise; CHUNKED_FUSED and CHUNKED_SPLIT force
  * one (CHUNKED_SPLIT without a workspace: WKV7_ERR_WORKSPACE).  The
  * backward has one chunked form, which all three select.  AUTO: CHUNKED for
- * 16-bit inputs, SCAN for f32.  All produce the same result up to
- * floating-point rounding order.
+ * 16-bit inputs, SCAN for f32.  The chunked kernels compute their products
+ * in tf32 (fp32 accumulation), which cannot hold f32 results to the 1e-4
+ * bound that f32 inputs ask for: any CHUNKED* algo with f32 inputs is
+ * refused (WKV7_ERR_UNSUPPORTED).  All produce the same result up to
+ * floating-point rounding.
  */
 typedef enum {
   WKV7_ALGO_AUTO = 0,
@@ -236,10 +241,12 @@ wkv7_status_t wkv7_step(const wkv7_desc_t* desc, const void* r, const void* w, c
  * WKV7_ERR_SCRATCH_LIMIT before anything is launched (32 MiB holds, e.g.,
  * B=2, T=512, H=12, or B*H*ceil(T/16) <= 2047 checkpoints).
  *
- * The first call on a device looks up the array's device address for that
- * device; make that first call before any stream capture.  All calls share
- * the array and it keeps the last call's contents (nothing in it needs to
- * start at zero), so calls that overlap on the GPU -- on different streams
+ * Every call looks up the array's device address on the calling device
+ * (the runtime's symbol lookup; nothing is cached, so a cudaDeviceReset in
+ * between is harmless).  The first call on a device also loads the library's
+ * module there; make that first call before any stream capture.  All calls
+ * share the array and it keeps the last call's contents (nothing in it needs
+ * to start at zero), so calls that overlap on the GPU -- on different streams
  * or different host threads -- race on it and must be serialised by the
  * caller.
  */

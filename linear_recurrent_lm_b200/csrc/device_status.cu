@@ -2,8 +2,6 @@
 // that ran out); wkv7_get_device_status() reads it after synchronising.  One word per device.
 #include <cuda_runtime.h>
 
-#include <mutex>
-
 #include "kernels.h"
 #include "wkv7.h"
 
@@ -11,28 +9,17 @@ namespace {
 
 static __device__ int g_device_status;
 
-constexpr int kMaxDevices = 256;
-std::mutex g_lock;
-int* g_status_ptr[kMaxDevices] = {};
-
 }  // namespace
 
 namespace wkv7 {
 
+// Looked up on every call, never cached: after a cudaDeviceReset the module is loaded again and the
+// word may sit at another address.  (Host code sees g_device_status only as a host-side stand-in.)
 cudaError_t device_status_ptr(int** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> guard(g_lock);
-  if (!g_status_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_device_status);
-    if (e != cudaSuccess) return e;
-    g_status_ptr[dev] = static_cast<int*>(p);
-  }
-  *out = g_status_ptr[dev];
-  return cudaSuccess;
+  void* p = nullptr;
+  const cudaError_t e = cudaGetSymbolAddress(&p, g_device_status);
+  *out = static_cast<int*>(p);
+  return e;
 }
 
 }  // namespace wkv7

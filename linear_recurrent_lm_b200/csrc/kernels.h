@@ -6,6 +6,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "wkv7.h"
+
 namespace wkv7 {
 
 struct FwdArgs {
@@ -49,6 +51,9 @@ struct StepArgs {
   const uint8_t* active;
   void* y;
 };
+
+// Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).
+wkv7_status_t validate_desc(const wkv7_desc_t* d);
 
 // dtype: 0 = f32, 1 = bf16, 2 = f16.  Each returns the launch status.
 cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);

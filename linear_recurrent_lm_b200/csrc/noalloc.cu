@@ -10,17 +10,16 @@
 //
 // The array is a file-scope __device__ object: every GPU that loads the
 // library holds its WKV7_NOALLOC_SCRATCH_BYTES until the process exits.  Its
-// device address is looked up once per device (cudaGetSymbolAddress, with
-// that device current) by the first call made on that device, so the first
-// call on each device should come before any stream capture.  Every call
-// shares the one array and it keeps the previous call's contents; nothing in
-// it needs to start at zero (the forward writes every checkpoint and the
-// backward writes every mark before reading them), but two calls that
-// overlap on the GPU race on it.
+// device address is looked up on every call (cudaGetSymbolAddress, with the
+// calling device current), never cached: after a cudaDeviceReset the module
+// is loaded again and the array may sit elsewhere.  Only the first call on a
+// device loads the module, so that first call should come before any stream
+// capture.  Every call shares the one array and it keeps the previous call's
+// contents; nothing in it needs to start at zero (the forward writes every
+// checkpoint and the backward writes every mark before reading them), but
+// two calls that overlap on the GPU race on it.
 #include <cuda_runtime.h>
 #include <stdint.h>
-
-#include <mutex>
 
 #include "kernels.h"
 #include "wkv7.h"
@@ -29,25 +28,11 @@ namespace {
 
 static __device__ __align__(256) unsigned char g_noalloc_scratch[WKV7_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 256;
-std::mutex g_setup_lock;
-void* g_scratch_ptr[kMaxDevices] = {};
-
-// Device address of the scratch array on the current device (set up once per device).
+// Device address of the scratch array on the current device.  Host code sees g_noalloc_scratch only
+// as a host-side stand-in, so the address comes from the runtime, looked up afresh on every call.
 cudaError_t scratch_for_current_device(void** out) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
-  std::lock_guard<std::mutex> guard(g_setup_lock);
-  if (!g_scratch_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return e;
-    g_scratch_ptr[dev] = p;
-  }
-  *out = g_scratch_ptr[dev];
-  return cudaSuccess;
+  *out = nullptr;
+  return cudaGetSymbolAddress(out, g_noalloc_scratch);
 }
 
 }  // namespace
@@ -57,12 +42,10 @@ extern "C" wkv7_status_t wkv7_train_step_noalloc(const wkv7_desc_t* d, const voi
                                                  const uint8_t* reset, void* y, float* s_out, const void* dy,
                                                  const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
                                                  void* db, float* ds0, void* stream) {
-  if (!d) return WKV7_ERR_NULL;
+  const wkv7_status_t valid = wkv7::validate_desc(d);
+  if (valid != WKV7_OK) return valid;
   const size_t need = wkv7_workspace_bytes(d);
-  if (need == 0 && d->T != 0) {
-    // invalid descriptor: let the regular entry point report which check failed
-    return wkv7_forward(d, r, w, k, v, a, b, s0, reset, y, s_out, nullptr, stream);
-  }
+  if (need == 0 && d->T != 0) return WKV7_ERR_SHAPE;   // (an accepted descriptor always has a size)
   if (need > size_t(WKV7_NOALLOC_SCRATCH_BYTES)) return WKV7_ERR_SCRATCH_LIMIT;
   void* scratch = nullptr;
   if (d->T > 0) {

@@ -39,9 +39,21 @@ wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elem
   if (!mul_ok(bh, d->T, &bth) || !mul_ok(bth, 64 * 4, &e)) return WKV7_ERR_SHAPE;   // byte count fits
   int64_t st;
   if (!mul_ok(bh, 64 * 64 * 4, &st)) return WKV7_ERR_SHAPE;
+  // the checkpoint workspace (one 16 KiB state per head per 16 tokens, then one int per head) must
+  // have a byte count too, so that wkv7_workspace_bytes is non-zero for every accepted T > 0
+  int64_t ck;
+  if (!mul_ok(bh, (d->T + 15) / 16, &ck) || !mul_ok(ck, 64 * 64 * 4, &ck) || ck > INT64_MAX - (bh * 4 + 15))
+    return WKV7_ERR_SHAPE;
   *units = bh;
   *tok_elems = bth * 64;
   return WKV7_OK;
+}
+
+// The chunked kernels compute their products in tf32 (11 significant bits): on f32 inputs they
+// cannot hold the 1e-4 bound that f32 results must meet, so only the exact scan takes f32.  (A
+// decode step has no algorithm choice and is not affected.)
+wkv7_status_t check_algo_dtype(const wkv7_desc_t* d) {
+  return (d->dtype == WKV7_F32 && d->algo >= WKV7_ALGO_CHUNKED) ? WKV7_ERR_UNSUPPORTED : WKV7_OK;
 }
 
 // Every listed pointer must be non-null (when `need`) and 16-byte aligned (when non-null).
@@ -141,6 +153,14 @@ wkv7_status_t use_split(const wkv7_desc_t* d, int64_t units, const void* workspa
 
 }  // namespace
 
+namespace wkv7 {
+wkv7_status_t validate_desc(const wkv7_desc_t* d) {
+  int64_t units = 0, te = 0;
+  const wkv7_status_t st = check_desc(d, &units, &te);
+  return st != WKV7_OK ? st : check_algo_dtype(d);
+}
+}  // namespace wkv7
+
 extern "C" {
 
 int wkv7_version(void) { return 100; }
@@ -186,6 +206,8 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   int64_t units = 0, te = 0;
   wkv7_status_t st = check_desc(d, &units, &te);
   if (st != WKV7_OK) return st;
+  st = check_algo_dtype(d);
+  if (st != WKV7_OK) return st;
   st = check_ptrs(te > 0, {r, w, k, v, a, b, y});
   if (st != WKV7_OK) return st;
   st = check_ptrs(false, {s0, s_out, workspace});
@@ -215,6 +237,8 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
                             void* da, void* db, float* ds0, void* stream) {
   int64_t units = 0, te = 0;
   wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_algo_dtype(d);
   if (st != WKV7_OK) return st;
   st = check_ptrs(te > 0, {r, w, k, v, a, b, dy, dr, dw, dk, dv, da, db});
   if (st != WKV7_OK) return st;

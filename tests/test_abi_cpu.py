@@ -77,6 +77,8 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 2)
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+    for algo in ("chunked", "chunked_fused", "chunked_split"):      # tf32 products cannot meet the f32 bound
+        assert call_fwd(L, L.make_desc(1, 16, 1, torch.float32, algo), ws=FAKE) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = 7
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.algo = -1
@@ -99,6 +101,24 @@ def test_forward_validation_codes(L):
     # empty problems launch nothing and succeed
     assert call_fwd(L, L.make_desc(0, 16, 4, torch.bfloat16), r=None, w=None, k=None, v=None, a=None, b=None, y=None) == L.OK
     assert call_fwd(L, L.make_desc(3, 16, 0, torch.bfloat16), r=None, w=None, k=None, v=None, a=None, b=None, y=None) == L.OK
+
+
+def test_workspace_byte_count_overflow_is_a_shape_error(L):
+    """A descriptor whose token tensors fit in int64 bytes but whose checkpoint workspace does not
+    (B*H*ceil(T/16)*16 KiB, four times the bytes of one bf16 input) is refused everywhere: the
+    workspace size would be 0, and without its scratch the no-allocation entry point must not run
+    the forward and skip the backward."""
+    import torch
+    d = L.make_desc(1, 1 << 54, 1, torch.bfloat16)       # 2^54 tokens: 2^62 bytes of f32 activations
+    assert L.workspace_bytes(1, 1 << 54, 1) == 0
+    assert call_fwd(L, d) == L.ERR_SHAPE
+    lib = L.lib()
+    vp = lambda x: None if x is None else ctypes.c_void_p(x)
+    st = lib.wkv7_train_step_noalloc(ctypes.byref(d), *map(vp, [FAKE] * 6), None, None, vp(FAKE), None, vp(FAKE),
+                                     None, *map(vp, [FAKE] * 6), None, None)
+    assert st == L.ERR_SHAPE
+    # one step below the limit is still a valid shape with a non-zero workspace
+    assert L.workspace_bytes(1, 1 << 48, 1) == (1 << 44) * 16384 + 16
 
 
 def test_backward_and_step_validation_codes(L):

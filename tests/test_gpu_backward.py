@@ -66,8 +66,8 @@ def test_config3_full_size_sampled_units(W, algo):
             assert c >= COS, ((b, h), n, c)
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
-@pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
+@pytest.mark.parametrize("algo,dtype", [(a, dt) for a in ("scan", "chunked_fused", "chunked_split")
+                                         for dt in ("f32", "bf16", "f16") if not (dt == "f32" and a != "scan")])
 @pytest.mark.parametrize("T", [1, 15, 17, 40, 100])
 def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
     rng = np.random.default_rng(100 + T)
@@ -94,14 +94,15 @@ def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
 def test_small_decay_segments(W, algo):
     """Decays far below the generator's range (prod w < 2^-16 over a chunk) and w = 0."""
     rng = np.random.default_rng(7)
-    d = I.draw_inputs(rng, (1, 64, 2, 64), "f32")
-    w = d["w"].astype(np.float64)
+    dt = "f32" if algo == "scan" else "bf16"
+    d = I.draw_inputs(rng, (1, 64, 2, 64), dt)
+    w = I.to_f64(d["w"])
     w[:, 10:26] *= 0.2
     w[:, 40:42] = 0.0
-    d["w"] = w.astype(np.float32)
-    dy = rng.standard_normal((1, 64, 2, 64)).astype(np.float32)
+    d["w"] = I.to_storage(w, dt)
+    dy = I.to_storage(rng.standard_normal((1, 64, 2, 64)), dt)
     _, _, g = fwd_bwd(W, d, dy, algo=algo)
-    go, _ = oracle.backward(*inputs_f64(d), dy.astype(np.float64))
+    go, _ = oracle.backward(*inputs_f64(d), I.to_f64(dy))
     for n in GRADS + ("ds0",):
         c = cosine(f64(g[n]), go[n])
         assert c >= COS, (n, c)
