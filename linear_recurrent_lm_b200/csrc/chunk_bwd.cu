@@ -1,90 +1,199 @@
-// WKV-7 backward in 16-token chunks on tensor cores (algo CHUNKED).
+// WKV-7 backward in 16-token chunks on the fifth-generation tensor cores (algo CHUNKED).
 //
-// Exact reverse mode of the chunk formulas of the forward (see chunk_fwd.cu):
-// inside a chunk with entering state S0, decay products L_t = prod_{s<=t} w_s
-// and At = a L_{t-1}, Rt = r L_t, Bh = b / L_t, Kh = k / L_t,
-//   SA = m0.At S0^T + Lab SA + Lak V,    Y = m0.Rt S0^T + Mrb SA + Mrk V,
-//   S16 = keep.S0 diag(L_15) + (SA^T ls.Bh + V^T ls.Kh) diag(L_15)
-// where Lab = At Bh^T, Lak = At Kh^T (strictly lower), Mrb = Rt Bh^T,
-// Mrk = Rt Kh^T (lower), all masked to token pairs with no reset between them;
-// m0 marks tokens before the chunk's first reset, ls the tokens of its last
-// segment, keep = "no reset in the chunk".  Given dY and dS16 (the gradient
-// carried from the next chunk), with dSl = dS16 diag(L_15):
-//   dSA  = Mrb^T dY + ls.Bh dSl^T,   dU = (I - Lab)^-T dSA,
-//   dV   = Mrk^T dY + ls.Kh dSl^T + Lak^T dU,
-//   dMrb = dY SA^T, dMrk = dY V^T, dLab = dU SA^T, dLak = dU V^T   (masked),
-//   dAt  = dLab Bh + dLak Kh + m0.dU S0,   dRt = dMrb Bh + dMrk Kh + m0.dY S0,
-//   dBh  = dLab^T At + dMrb^T Rt + ls.L_15.(SA dS16),
-//   dKh  = dLak^T At + dMrk^T Rt + ls.L_15.(V dS16),
-//   dS0  = keep.dSl + (m0.dY)^T Rt + (m0.dU)^T At
-// and, through the decay, with d log L_t = dr r + da_{t+1} a_{t+1} - db b - dk k
-// (plus, at t = 15, keep.L_15 sum_i dS16 o S0 and the last segment's
-// dBb o Bb + dKb o Kb), d log w_s = sum_{t >= s} d log L_t and dw = d log w / w.
-// The pages print no backward; this is derived from the chunk forward, which
-// itself is the recurrence regrouped (RWKV-MLX page, "Key Design Decisions" 2:
-// state checkpoints every 16 tokens; rwkv-metal page: the backward recomputes
-// each chunk from its checkpoint).
+// Exact reverse mode of the chunk formulas of the forward (see chunk_fwd.cu): inside a chunk with
+// entering state S0 and decay products L_t = prod_{s<=t} w_s, At = a L_{t-1}, Rt = r L_t,
+// Bh = b / L_t, Kh = k / L_t, the masked Gram blocks Lab = At Bh^T, Lak = At Kh^T (strictly lower),
+// Mrb = Rt Bh^T, Mrk = Rt Kh^T (lower), T = (I - Lab)^-1, W = T m0.At, X = T Lak and
+//   SA = W S0^T + X V,   S16 = keep.S0 diag(L_15) + (SA^T Bl + V^T Kl) diag(L_15)
+// (m0: tokens before the chunk's first reset, ls: tokens of its last segment, Bl = ls.Bh,
+// Kl = ls.Kh, keep: no reset in the chunk).  Given dY and the gradient dS16 carried from the next
+// chunk, with dSl = dS16 diag(L_15):
+//   dSA = Mrb^T dY + Bl dSl^T,   dU = T^T dSA,   dV = Mrk^T dY + Kl dSl^T + Lak^T dU,
+//   dS0 = keep.dSl + (m0.dY)^T Rt + (m0.dU)^T At,
+//   dMrb = dY SA^T, dMrk = dY V^T, dLab = dU SA^T, dLak = dU V^T   (masked like their blocks),
+//   dAt = dLab Bh + dLak Kh + m0.dU S0,   dRt = dMrb Bh + dMrk Kh + m0.dY S0,
+//   dBh = dLab^T At + dMrb^T Rt + ls.(SA dSl),   dKh = dLak^T At + dMrk^T Rt + ls.(V dSl),
+// and through the decays d log L_t = dRt.Rt + dAt_{t+1}.At_{t+1} - dBh.Bh - dKh.Kh, plus at t = 15
+// the L_15 terms keep.sum_i dSl o S0 + sum_tau ls.((SA dSl) o Bh + (V dSl) o Kh);
+// d log w_s = sum_{t >= s} d log L_t and dw = d log w / w.  The pages print no backward; this is
+// derived from the chunk forward, itself the recurrence regrouped (RWKV-MLX page, "Key Design
+// Decisions" 2: state checkpoints every 16 tokens; rwkv-metal page: the backward rebuilds each
+// chunk from its checkpoint).
 //
-// Gradients need cosine >= 0.999, so every product here is a single bf16
-// mma.sync (m16n8k16) with fp32 accumulation.  A chunk with a decay outside
-// the range the 1/L scaling tolerates (some w < 1/16, or L_15 outside
-// [2^-40, 2^40]) makes the CTA stop and mark its unit in `unit_flags`; the
+// Everything runs transposed so that the tensor core's 64-row side is a state dimension: the
+// carried gradient is dS^T (TMEM rows = key channel j), G1 = dSl [Bh|Kh]^T and G2 = dY^T [Mrb|Mrk]
+// have rows = value channel i (dSA^T = ls o G1b + G2b, dU^T = dSA^T T, dV^T = ls o G1k + G2k +
+// dU^T Lak follow on the FP32 cores, one thread per i), and the key-space gradients dAt^T, dRt^T,
+// dBh^T, dKh^T have rows = j, so that one thread owns one key channel over all 16 tokens of the
+// chunk and keeps the reverse sum for dw in its registers.
+//
+// Precision: the tensor-core products take bf16 operands split in two, x = hi + lo with
+// hi = bf16(x), lo = bf16(x - hi), and accumulate hi.hi + hi.lo + lo.hi in fp32 (lo.lo, about
+// 2^-16 of the product, is dropped); the inputs v and dy are exact in bf16 when they arrive in
+// bf16 and then skip their lo half.  The carried dS^T, the decay scalings, the small 16x16 solves
+// and the per-token outputs are fp32.  A chunk whose decays the 1/L scaling cannot take (some
+// w < 1/16, or L_15 outside [2^-40, 2^40]) stops the CTA and marks its unit in `unit_flags`; the
 // scan backward then recomputes exactly those units.
 //
-// Work split (one CTA of 8 warps per (b,h)), chunks in reverse, pipelined:
-//   warps 4-7 ("context") for chunk c-1: stage its inputs (one TMA box per
-//     input on an mbarrier, bounded waits) and its checkpoint, build the decay-scaled operands, the masked Gram, T,
-//     W, X and the recomputed SA = W S0^T + X V into one half of a double
-//     buffer;
-//   warps 0-3 ("main") for chunk c: warp w owns rows 16w..16w+15 of dS as
-//     accumulator fragments (the only quantity carried from chunk to chunk)
-//     and columns 16w..16w+15 of the key-space gradients; they run the
-//     dS chain, the gradient products and the per-token outputs.
+// Shared-memory operands are "core arrays": a P x Q matrix of bf16 stored as 8-row x 8-column
+// (16-byte) core matrices, element (p, q) at (p/8)(8Q) + (q/8)64 + (p%8)8 + q%8.  The tensor core
+// reads one either K-major (rows = M or N, columns = K: LBO 128 bytes, SBO 16Q bytes, 256 bytes
+// per K step of 16) or MN-major (columns = M or N, rows = K: LBO 16Q bytes, SBO 128 bytes, 32Q
+// bytes per K step), so each matrix is stored once whichever way round a product needs it.
+// Products with fewer than 64 useful rows read 64 anyway; the extra rows come from the arrays
+// that follow (always inside the CTA's shared memory) and their results are never read.
+//
+// Work split: one CTA of 8 warps per (b,h) (about 200 KB of shared memory and 512 TMEM columns,
+// so one CTA per SM), chunks in reverse, pipelined:
+//   warps 4-7 ("context") for chunk c-1: stage its inputs (one TMA box per input) and its
+//     checkpoint (one bulk copy) on an mbarrier with bounded waits, build the decay-scaled
+//     operands, the masked Gram (tcgen05), T by substitution, W, X, and SA^T = S0 W^T + V^T X^T
+//     (tcgen05) into one half of a double buffer;
+//   warps 0-3 ("main") for chunk c: scale the carried dS^T, then one thread issues the products
+//     in three batches (chain: G1, G2, Rt^T m0.dY; then At^T m0.dU, the gradient Gram and the S0
+//     and dSl parts of the key-space products; then their Gram parts), while the warps write dv
+//     and, per key channel, da, dr, db, dk and dw.
 // One CTA barrier per chunk hands the context over.
 #include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.cuh"
+#include "tc05.cuh"
 
 namespace wkv7 {
 namespace {
 
 constexpr int kThreads = 256;
-constexpr int kStr = 72;
-constexpr int kStrS = 24;
-constexpr int kStrG = 40;
 constexpr int kIn = 7;   // r, w, k, v, a, b, dy
+constexpr int S20 = 20;
 using bf16 = __nv_bfloat16;
 
-struct __align__(16) BCtx {
-  bf16 GA[32][kStr];      // rows 0..15 at, 16..31 rt   [t][j]
-  bf16 GB[32][kStr];      // rows 0..15 bh, 16..31 kh   [tau][j]
-  bf16 S0b[kN][kStr];     // entering state             [i][j]
-  bf16 SAb[kChunk][kStr]; // recomputed SA              [tau][i]
-  bf16 Vb[kChunk][kStr];  // v                          [tau][i]
-  bf16 DYb[kChunk][kStr]; // dy                         [t][i]
-  bf16 Tb[kChunk][kStrS], Mrbb[kChunk][kStrS], Mrkb[kChunk][kStrS], Lakb[kChunk][kStrS];   // [t][tau]
-  float lam[kChunk][kN + 4];   // L_t [t][j]
-  int mask, unsafe;
-  unsigned ls_bits;            // tokens of the chunk's last segment
+// TMEM columns (512 allocated: one CTA per SM).  Every accumulator has M = 64 rows.
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColGram = 0;    // context: [At; Rt] [Bh; Kh]^T  (32; rows t)
+constexpr uint32_t kColSA = 32;     // context: SA^T                  (16; rows i)
+constexpr uint32_t kColDS = 64;     // main: dS^T                     (64; rows j)
+constexpr uint32_t kColG1 = 128;    // main: dSl [Bh|Kh]^T            (32; rows i)
+constexpr uint32_t kColG2 = 160;    // main: dY^T [Mrb|Mrk]           (32; rows i)
+constexpr uint32_t kColGG = 192;    // main: [dY; dU] [SA^T | v^T]     (32; rows t and 16 + t)
+constexpr uint32_t kColE = 256;     // main: dAt^T | dRt^T | dBg^T | dKg^T | (SA dSl)^T | (V dSl)^T  (96; rows j)
+
+// bf16 index of element (p, q) of a core array with Q columns.
+__device__ __forceinline__ int cb(int p, int q, int Q) { return (p >> 3) * (Q * 8) + (q >> 3) * 64 + (p & 7) * 8 + (q & 7); }
+
+// A matrix split in two bf16 core arrays (hi, then lo).
+template <int P, int Q>
+struct Split {
+  bf16 hi[P * Q];
+  bf16 lo[P * Q];
+};
+
+// Split 8 fp32 values into one 16-byte row of hi and one of lo at element index e.
+template <int P, int Q>
+__device__ __forceinline__ void put8(Split<P, Q>& m, int e, const float (&x)[8]) {
+  uint32_t h[4], l[4];
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const __nv_bfloat162 hh = __floats2bfloat162_rn(x[2 * u], x[2 * u + 1]);
+    const float2 hf = __bfloat1622float2(hh);
+    const __nv_bfloat162 ll = __floats2bfloat162_rn(x[2 * u] - hf.x, x[2 * u + 1] - hf.y);
+    h[u] = *reinterpret_cast<const uint32_t*>(&hh);
+    l[u] = *reinterpret_cast<const uint32_t*>(&ll);
+  }
+  *reinterpret_cast<uint4*>(&m.hi[e]) = make_uint4(h[0], h[1], h[2], h[3]);
+  *reinterpret_cast<uint4*>(&m.lo[e]) = make_uint4(l[0], l[1], l[2], l[3]);
+}
+// The 8 values (hi + lo) of one 16-byte row at element index e.
+template <int P, int Q>
+__device__ __forceinline__ void get8(const Split<P, Q>& m, int e, float (&x)[8]) {
+  const uint4 h = *reinterpret_cast<const uint4*>(&m.hi[e]), l = *reinterpret_cast<const uint4*>(&m.lo[e]);
+  const uint32_t hw[4] = {h.x, h.y, h.z, h.w}, lw[4] = {l.x, l.y, l.z, l.w};
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const float2 a = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&hw[u]));
+    const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[u]));
+    x[2 * u] = a.x + c.x;
+    x[2 * u + 1] = a.y + c.y;
+  }
+}
+
+// One operand of a product: a split core array with Q columns, read K-major (rows = M/N, columns
+// = K) or MN-major (columns = M/N, rows = K).  The layout is a compile-time constant; only the
+// shared-memory addresses of the hi and lo arrays (already offset to the first row used) are not.
+template <int Q, bool MN>
+struct Op {
+  uint32_t hi, lo;   // shared-memory byte addresses; lo == 0: the values are exact in bf16
+  // Descriptor of K step ks: the 16-byte start-address field advances by a constant per step.
+  __device__ __forceinline__ uint64_t desc(uint32_t base, int ks) const {
+    constexpr uint32_t kLbo = MN ? uint32_t(Q) * 16 : 128u, kSbo = MN ? 128u : uint32_t(Q) * 16;
+    constexpr uint32_t kStep = MN ? uint32_t(Q) * 32 : 256u;   // bytes per K step of 16
+    const uint32_t lo32 = (((base + uint32_t(ks) * kStep) >> 4) & 0x3FFFu) | ((kLbo >> 4) << 16);
+    constexpr uint32_t hi32 = (kSbo >> 4) | (1u << 14);          // SBO, descriptor version 1 (bit 46)
+    return (uint64_t(hi32) << 32) | lo32;
+  }
+};
+// The operand starting at row row0 and column col0 (both multiples of 8) of a split core array.
+template <int Q, bool MN, int P>
+__device__ __forceinline__ Op<Q, MN> op(const Split<P, Q>& m, bool exact = false, int row0 = 0, int col0 = 0) {
+  const int e = cb(row0, col0, Q);
+  return Op<Q, MN>{tc::smem_u32addr(m.hi + e), exact ? 0u : tc::smem_u32addr(m.lo + e)};
+}
+// Store one value as its hi and lo halves at element index e (a single element of a core row).
+template <int P, int Q>
+__device__ __forceinline__ void put1(Split<P, Q>& m, int e, float x) {
+  const bf16 h = __float2bfloat16_rn(x);
+  m.hi[e] = h;
+  m.lo[e] = __float2bfloat16_rn(x - __bfloat162float(h));
+}
+// D (+)= A B over NKS K steps of 16 (M = 64): hi.hi + hi.lo + lo.hi.  Issued by one thread.
+template <int N, int NKS, int QA, bool MA, int QB, bool MB>
+__device__ __forceinline__ void mma3(uint32_t d, const Op<QA, MA>& a, const Op<QB, MB>& b, bool accumulate) {
+  constexpr uint32_t id = tc::idesc_bf16(64, N, MA ? 1 : 0, MB ? 1 : 0);
+#pragma unroll
+  for (int ks = 0; ks < NKS; ++ks) {
+    const uint64_t ah = a.desc(a.hi, ks), bh = b.desc(b.hi, ks);
+    tc::mma_bf16(d, ah, bh, id, accumulate || ks > 0);
+    if (b.lo) tc::mma_bf16(d, ah, b.desc(b.lo, ks), id, true);
+    if (a.lo) tc::mma_bf16(d, a.desc(a.lo, ks), bh, id, true);
+  }
+}
+
+// Produced by the context warps for one chunk, read by the main warps one iteration later.  The
+// order of the arrays matters: 64-row reads of AR and DY run on into the arrays after them.
+template <typename T>
+struct __align__(128) Ctx {
+  Split<32, 64> AR;      // rows 0-15 At [t][j], rows 16-31 Rt [t][j]
+  Split<32, 64> BK;      // rows 0-15 Bh [tau][j], rows 16-31 Kh [tau][j]
+  Split<32, 64> DYU;     // rows 0-15 dy [t][i]; rows 16-31 dU [t][i], written by the main warps
+  Split<64, 32> DUY;     // [i][m0.dU^T (t) | m0.dy^T (t)]: the dU half is written by the main warps
+  Split<64, 32> SV;      // [i][SA^T (tau) | v^T (tau)]
+  Split<64, 64> S0T;     // S0^T [j][i]
+  Split<16, 32> MM;      // [t][Mrb[t][0..15] | Mrk[t][0..15]]
+  __align__(16) float Tp[kChunk][kChunk];     // T [t][tau]
+  __align__(16) float LakP[kChunk][kChunk];   // Lak [t][tau]
+  __align__(16) float lam[kChunk][kN];        // L_t [t][j]
+  __align__(16) float lamT[kN][kChunk + 4];   // L_t [j][t] (rows padded against bank conflicts)
+  __align__(16) T rabkT[4][kN][kChunk + 8];   // r, a, b, k of the chunk [j][t]
+  int mask;                     // reset bits of the chunk
+  int unsafe;                   // decay out of range (or staging timed out): the unit is re-run exactly
 };
 
 template <typename T>
-struct __align__(128) BwdSmem2 {
-  BCtx ctx[2];
-  __align__(128) T in[kIn][kChunk][kN];   // staged inputs of the chunk being built (TMA boxes)
-  __align__(16) float LabT[kChunk][20];
-  __align__(16) float LakT[kChunk][20];
-  bf16 Wb[kChunk][kStr], Xb[kChunk][kStrS];
-  bf16 DUb[kChunk][kStr];     // dU   [tau][i]
-  bf16 dSb[kN][kStr];         // dS16 [i][j]
-  bf16 dG[32][kStrG];         // [dMrb dMrk; dLab dLak]
-  bf16 dVs[kChunk][kStr];     // dv staging [tau][i]
-  __align__(16) float DL[kChunk][kN + 4];   // d log L_t without the chunk-end term
-  __align__(16) float e3[kN];
-  __align__(16) float dlam[4][kN];
-  unsigned long long in_bar;   // completion of the bulk copies into `in` (one phase per staged chunk)
+struct __align__(128) BwdSmem {
+  Ctx<T> ctx[2];
+  Split<64, 64> dSlT;    // dSl^T [j][i]                                        (main)
+  Split<32, 32> G4;      // rows t: [dLab[t] | dLak[t]], rows 16 + t: [dMrb[t] | dMrk[t]]   (main)
+  Split<16, 64> WC;      // W [tau][j]                         (context)
+  Split<16, 16> XC;      // X [tau][t]                         (context)
+  __align__(16) float Atf[kChunk][kN];      // At [t][j] in fp32     (context)
+  __align__(16) float LabT[kChunk][S20];    // Lab^T [tau][t]   (context)
+  __align__(128) float ck[kN * kN];         // checkpoint entering the chunk being built (tiled order)
+  __align__(128) T stg[kIn][kChunk][kN];    // staged inputs of the chunk being built (TMA boxes)
+  unsigned long long in_bar;                // staged inputs and checkpoint landed (one phase per staged chunk)
+  unsigned long long gram_bar, sa_bar;      // context MMAs complete (one phase per chunk each)
+  unsigned long long u_bar, chain_bar, gg_bar, e_bar;   // main MMAs complete (one phase per chunk each)
+  uint32_t tmem_base;
   int kbad[4];
   int stop;
 };
@@ -100,57 +209,15 @@ __device__ __forceinline__ float rcp_approx(float x) {
   return r;
 }
 
-__device__ __forceinline__ void frag_to_a(const float (&lo)[4], const float (&hi)[4], uint32_t (&a)[4]) {
-  a[0] = pack_bf16(lo[0], lo[1]);
-  a[1] = pack_bf16(lo[2], lo[3]);
-  a[2] = pack_bf16(hi[0], hi[1]);
-  a[3] = pack_bf16(hi[2], hi[3]);
+// Bounded wait on an MMA-completion barrier; a wait that runs out is recorded in the status word.
+__device__ __forceinline__ void mma_wait(const BwdArgs& p, unsigned long long* bar, unsigned parity) {
+  if (!mbar_wait_bounded(bar, parity, kWaitLimitNs) && p.status) atomicOr(p.status, kStatusWaitTimeout);
+  tc::fence_after_sync();
 }
 
-// Keep only the bf16 halves of an m16n8k16 A fragment whose k index is set in `bits`.
-__device__ __forceinline__ void mask_k16(uint32_t (&a)[4], int c4, unsigned bits) {
-  const int k0 = 2 * c4, k1 = 8 + 2 * c4;
-  const uint32_t m0 = ((bits >> k0) & 1u ? 0x0000ffffu : 0u) | ((bits >> (k0 + 1)) & 1u ? 0xffff0000u : 0u);
-  const uint32_t m1 = ((bits >> k1) & 1u ? 0x0000ffffu : 0u) | ((bits >> (k1 + 1)) & 1u ? 0xffff0000u : 0u);
-  a[0] &= m0;
-  a[1] &= m0;
-  a[2] &= m1;
-  a[3] &= m1;
-}
-
-// Stage the seven inputs (r, w, k, v, a, b, dy) of chunk tokens t0..t0+15 into sm.in: one TMA box
-// per input, issued by one thread; rows past T arrive as zeros (K1 reads w there as 1).
-template <typename T>
-__device__ __forceinline__ void stage7(const BwdArgs& p, const InputMaps& tm, BwdSmem2<T>& sm, int64_t b, int64_t h,
-                                       int64_t t0, int ktid) {
-  if (ktid == 0) {
-    mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + p.extra_tx);
-#pragma unroll
-    for (int m = 0; m < kIn; ++m) tma_load_4d(&sm.in[m][0][0], &tm.m[m], 0, int(h), int(t0), int(b), &sm.in_bar);
-  }
-}
-
-// State entering chunk c (checkpoint c-1, s0 or zero) as accumulator fragments: context thread
-// (warp kw, lane 4g + c4) holds s[nt] = S[16kw + g][8nt + 2c4 + {0,1}], S[16kw + g + 8][same].
-__device__ __forceinline__ void load_entry_rows(const BwdArgs& p, int64_t unit, int64_t nc, int64_t c, int ktid,
-                                                float4 (&s)[8]) {
-  if (c > 0) {   // tiled checkpoint order: one contiguous 512-byte row of float4 per warp and nt
-    const float* src = p.ckpt + (unit * nc + (c - 1)) * kN * kN + (ktid >> 5) * 1024 + (ktid & 31) * 4;
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) s[nt] = *reinterpret_cast<const float4*>(src + nt * 128);
-  } else if (p.s0) {
-    const int lane = ktid & 31;
-    const float* src = p.s0 + unit * kN * kN + (16 * (ktid >> 5) + (lane >> 2)) * kN + 2 * (lane & 3);
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const float2 lo = *reinterpret_cast<const float2*>(src + 8 * nt);
-      const float2 hi = *reinterpret_cast<const float2*>(src + 8 * kN + 8 * nt);
-      s[nt] = make_float4(lo.x, lo.y, hi.x, hi.y);
-    }
-  } else {
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) s[nt] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
+// Causal and same-segment mask of one (t, tau) pair of the chunk.
+__device__ __forceinline__ bool pair_ok(unsigned mask, int t, int tau, bool strict) {
+  return (strict ? tau < t : tau <= t) && (mask & ((2u << t) - (2u << tau))) == 0u;
 }
 
 // Reset flag of token 16c + lane of batch row b (false past T, for c < 0 or without flags).
@@ -159,556 +226,571 @@ __device__ __forceinline__ bool reset_flag(const BwdArgs& p, int64_t b, int64_t 
   return p.reset && c >= 0 && lane < kChunk && t < p.T && p.reset[b * p.T + t] != 0;
 }
 
-// ------------------------------------------------------------------ context warps
-// A wait for staged inputs that runs out marks the chunk unsafe (the unit is then recomputed by the
-// exact scan, which reads global memory) and sets `timed_out`, after which nothing more is staged.
+// Stage chunk c: the seven inputs of its tokens (one TMA box each; rows past T arrive as zeros, K1
+// reads w there as 1) and, for c > 0, the checkpoint entering it (one bulk copy), issued by one
+// thread on in_bar.
 template <typename T>
-__device__ __forceinline__ void build_context(const BwdArgs& p, BwdSmem2<T>& sm, BCtx& cx, unsigned mask,
-                                              const float4 (&s0rows)[8], int ktid, int len, unsigned parity,
-                                              bool& unsafe, bool& timed_out) {
+__device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, int64_t unit, int64_t b,
+                                      int64_t h, int64_t c, int64_t nc, int ktid) {
+  if (ktid == 0) {
+    const unsigned ck_bytes = c > 0 ? unsigned(kN * kN * sizeof(float)) : 0u;
+    mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + ck_bytes + p.extra_tx);
+#pragma unroll
+    for (int m = 0; m < kIn; ++m)
+      tma_load_4d(&sm.stg[m][0][0], &tm.m[m], 0, int(h), int(c * kChunk), int(b), &sm.in_bar);
+    if (c > 0) bulk_g2s(sm.ck, p.ckpt + (unit * nc + (c - 1)) * kN * kN, ck_bytes, &sm.in_bar);
+  }
+}
+
+// ------------------------------------------------------------------ context warps
+// Decay products, decay-scaled operands, v, dy, S0^T, L_t and the raw r, a, b, k for the main
+// warps' per-token outputs.  A wait for the staged data that runs out marks the chunk unsafe (the
+// unit is then recomputed by the exact scan) and sets `timed_out`, after which nothing more is
+// staged.
+template <typename T>
+__device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
+                                                 int64_t unit, int64_t c, int ktid, int len, unsigned parity,
+                                                 uint32_t tmem, bool& unsafe, bool& timed_out) {
   const int kw = ktid >> 5, lane = ktid & 31;
   const bool to = !mbar_wait_bounded(&sm.in_bar, parity, kWaitLimitNs);
-  const T (*X)[kChunk][kN] = sm.in;
+  const T (*X)[kChunk][kN] = sm.stg;
+  const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
 
-  // ---- K1: decay products, scaled operands, v/dy copies, entering state in bf16.
-  // Thread = (column pair 2jp, 2jp+1; token quarter kw), two columns per packed fp32 op.
+  // ---- pass B: thread = (token t, 8 channels from j0); one 16-byte core row per array
   bool bad = false;
   {
-    const int j = 2 * lane, t0 = 4 * kw;
-    // L_{t0-1}: product of the earlier quarters' decays (warp-uniform trip count)
-    float2 lam = make_float2(1.f, 1.f);
-    auto ldw = [&](int t) { return t < len ? load2(&X[1][t][j]) : make_float2(1.f, 1.f); };   // padding: w = 1
-    for (int t = 0; t < t0; ++t) lam = mul2(lam, ldw(t));
-    float2 wmin = make_float2(1.f, 1.f), lmin = make_float2(1.f, 1.f), lmax = lmin;
+    const int t = (lane & 7) + 8 * (kw & 1), j0 = 8 * ((lane >> 3) + 4 * (kw >> 1));
+    // L_{t-1} and L_t: products of the staged decays (rows past T count as w = 1)
+    float L[8], Lp[8];
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const int t = t0 + u;
-      const float2 lp = lam, w2 = ldw(t);
-      lam = mul2(lam, w2);
-      wmin = make_float2(fminf(wmin.x, w2.x), fminf(wmin.y, w2.y));
-      lmin = make_float2(fminf(lmin.x, lam.x), fminf(lmin.y, lam.y));
-      lmax = make_float2(fmaxf(lmax.x, lam.x), fmaxf(lmax.y, lam.y));
-      const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
-      const float2 at = mul2(load2(&X[4][t][j]), lp), rt = mul2(load2(&X[0][t][j]), lam);
-      const float2 bh = mul2(load2(&X[5][t][j]), inv), kh = mul2(load2(&X[2][t][j]), inv);
-      *reinterpret_cast<float2*>(&cx.lam[t][j]) = lam;
-      *reinterpret_cast<uint32_t*>(&cx.GA[t][j]) = pack_bf16(at.x, at.y);
-      *reinterpret_cast<uint32_t*>(&cx.GA[16 + t][j]) = pack_bf16(rt.x, rt.y);
-      *reinterpret_cast<uint32_t*>(&cx.GB[t][j]) = pack_bf16(bh.x, bh.y);
-      *reinterpret_cast<uint32_t*>(&cx.GB[16 + t][j]) = pack_bf16(kh.x, kh.y);
-      if constexpr (std::is_same<T, bf16>::value) {
-        *reinterpret_cast<uint32_t*>(&cx.Vb[t][j]) = *reinterpret_cast<const uint32_t*>(&X[3][t][j]);
-        *reinterpret_cast<uint32_t*>(&cx.DYb[t][j]) = *reinterpret_cast<const uint32_t*>(&X[6][t][j]);
-      } else {
-        const float2 v2 = load2(&X[3][t][j]), d2 = load2(&X[6][t][j]);
-        *reinterpret_cast<uint32_t*>(&cx.Vb[t][j]) = pack_bf16(v2.x, v2.y);
-        *reinterpret_cast<uint32_t*>(&cx.DYb[t][j]) = pack_bf16(d2.x, d2.y);
-      }
+    for (int u = 0; u < 8; ++u) Lp[u] = 1.f;
+    for (int s2 = 0; s2 < t; ++s2) {
+      float w[8];
+      unpack16<T>(*reinterpret_cast<const uint4*>(&X[1][s2][j0]), w);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) Lp[u] *= s2 < len ? w[u] : 1.f;
     }
-    // every L_t of the chunk lies in exactly one quarter, so the CTA-wide ballot sees all of them
-    bad = !(fminf(wmin.x, wmin.y) >= 0.0625f && fminf(lmin.x, lmin.y) >= 0x1p-40f && fmaxf(lmax.x, lmax.y) <= 0x1p40f);
-    const int row = 16 * kw + (lane >> 2), col = 2 * (lane & 3);
+    {
+      float w[8];
+      unpack16<T>(*reinterpret_cast<const uint4*>(&X[1][t][j0]), w);
+      float wmin = 1.f, lmin = 1.f, lmax = 1.f;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      *reinterpret_cast<uint32_t*>(&cx.S0b[row][8 * nt + col]) = pack_bf16(s0rows[nt].x, s0rows[nt].y);
-      *reinterpret_cast<uint32_t*>(&cx.S0b[row + 8][8 * nt + col]) = pack_bf16(s0rows[nt].z, s0rows[nt].w);
+      for (int u = 0; u < 8; ++u) {
+        const float wu = t < len ? w[u] : 1.f;
+        L[u] = Lp[u] * wu;
+        wmin = fminf(wmin, wu);
+        lmin = fminf(lmin, L[u]);
+        lmax = fmaxf(lmax, L[u]);
+      }
+      bad = !(wmin >= 0.0625f && lmin >= 0x1p-40f && lmax <= 0x1p40f);
+    }
+    *reinterpret_cast<float4*>(&cx.lam[t][j0]) = make_float4(L[0], L[1], L[2], L[3]);
+    *reinterpret_cast<float4*>(&cx.lam[t][j0 + 4]) = make_float4(L[4], L[5], L[6], L[7]);
+    float in[kIn][8];
+#pragma unroll
+    for (int m = 0; m < kIn; ++m) unpack16<T>(*reinterpret_cast<const uint4*>(&X[m][t][j0]), in[m]);
+    float at[8], rt[8], bh[8], kh[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const float il = rcp_approx(L[u]);
+      at[u] = in[4][u] * Lp[u];
+      rt[u] = in[0][u] * L[u];
+      bh[u] = in[5][u] * il;
+      kh[u] = in[2][u] * il;
+    }
+    *reinterpret_cast<float4*>(&sm.Atf[t][j0]) = make_float4(at[0], at[1], at[2], at[3]);
+    *reinterpret_cast<float4*>(&sm.Atf[t][j0 + 4]) = make_float4(at[4], at[5], at[6], at[7]);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {   // transposed copies for the per-key-channel outputs (exact)
+      cx.lamT[j0 + u][t] = L[u];
+      cx.rabkT[0][j0 + u][t] = Elt<T>::from_f32(in[0][u]);
+      cx.rabkT[1][j0 + u][t] = Elt<T>::from_f32(in[4][u]);
+      cx.rabkT[2][j0 + u][t] = Elt<T>::from_f32(in[5][u]);
+      cx.rabkT[3][j0 + u][t] = Elt<T>::from_f32(in[2][u]);
+    }
+    put8(cx.AR, cb(t, j0, 64), at);
+    put8(cx.AR, cb(16 + t, j0, 64), rt);
+    put8(cx.BK, cb(t, j0, 64), bh);
+    put8(cx.BK, cb(16 + t, j0, 64), kh);
+    put8(cx.DYU, cb(t, j0, 64), in[6]);
+    const bool m0t = t < fr;
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {   // v^T and m0.dy^T: column t of rows j0..j0+7
+      put1(cx.SV, cb(j0 + u, 16 + t, 32), in[3][u]);
+      put1(cx.DUY, cb(j0 + u, 16 + t, 32), m0t ? in[6][u] : 0.f);
     }
   }
   const unsigned any_bad = __ballot_sync(0xffffffffu, bad), any_to = __ballot_sync(0xffffffffu, to);
   if (lane == 0) sm.kbad[kw] = (any_bad ? 1 : 0) | (any_to ? 2 : 0);
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
   named_bar(1, 128);
   const int kb = sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3];
   unsafe = kb != 0;
   timed_out = (kb & 2) != 0;
+  // ---- the Gram [At; Rt] [Bh; Kh]^T runs on the tensor core while S0^T is built (M = 64: rows
+  // 32-63 read the arrays that follow and are unused)
+  if (!unsafe && ktid == 0) {
+    tc::fence_after_sync();
+    mma3<32, 4>(tmem + kColGram, op<64, false>(cx.AR), op<64, false>(cx.BK), false);
+    tc::commit(&sm.gram_bar);
+  }
+  // ---- pass C: S0^T [j][i] from the checkpoint (tiled order), s0 or zero; thread = 4 x (j, 8 i)
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int idx = ktid + 128 * u;
+    const int j = (idx & 7) + 8 * (idx >> 6), i0 = 8 * ((idx >> 3) & 7);
+    float s[8];
+    if (c > 0) {   // rows i0..i0+7 of column j sit 16 floats apart in the tiled order
+      const float* src = sm.ck + ckpt_off(i0, j);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[e] = src[16 * e];
+    } else if (p.s0) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[e] = p.s0[(unit * kN + i0 + e) * kN + j];
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s[e] = 0.f;
+    }
+    put8(cx.S0T, cb(j, i0, 64), s);
+  }
+  tc::fence_smem_to_async();
+  named_bar(1, 128);
   if (timed_out && ktid == 0 && p.status) atomicOr(p.status, kStatusWaitTimeout);
   if (ktid == 0) {
     cx.mask = int(mask);
     cx.unsafe = unsafe ? 1 : 0;
-    cx.ls_bits = last_segment_bits(mask);
   }
 }
 
+// The rest of the context: Gram, T, W, X and SA^T (safe chunks only).
 template <typename T>
-__device__ __forceinline__ void finish_context(BwdSmem2<T>& sm, BCtx& cx, unsigned mask, int ktid) {
+__device__ __forceinline__ void context_products(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
+                                                 int ktid, uint32_t tmem, unsigned phase) {
+  constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
   const int kw = ktid >> 5, lane = ktid & 31;
-  const int g = lane >> 2, c4 = lane & 3;
+  const uint32_t tlane = uint32_t(32 * kw) << 16;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
 
-  // ---- K2: Gram block of this warp (single bf16), masked
-  {
-    const int m0 = (kw >> 1) * 16, n0 = (kw & 1) * 16;
-    float gr[2][4] = {};
+  // ---- the masked Gram (issued with the operands)
+  mma_wait(p, &sm.gram_bar, phase & 1u);
+  if (kw < 2) {   // warp 0: rows t of [Lab | Lak]; warp 1: rows t of [Mrb | Mrk] (lanes 0-15)
+    float g0[16], g1[16];
+    tc::ld_32x32b_x16(tmem + tlane + kColGram, g0);
+    tc::ld_32x32b_x16(tmem + tlane + kColGram + 16, g1);
+    tc::wait_ld();
+    const int t = lane;
+    if (t < kChunk) {
+      const bool strict = kw == 0;
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4], bb[4];
-      ldsm_x4(a, a_rowmajor_addr(&cx.GA[0][0], kStr, m0, 16 * ks, lane));
-      ldsm_x4(bb, b_nmajor_addr(&cx.GB[0][0], kStr, n0, 16 * ks, lane));
-      mma16816(gr[0], a, bb[0], bb[1]);
-      mma16816(gr[1], a, bb[2], bb[3]);
-    }
-    const bool strict = kw < 2;
-    const int st0 = seg_of(mask, g), st1 = seg_of(mask, g + 8);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = g + (e >> 1) * 8;
-        const int tau = 8 * nt + 2 * c4 + (e & 1);
-        const bool ok = (strict ? (tau < t) : (tau <= t)) && seg_of(mask, tau) == ((e >> 1) ? st1 : st0);
-        const float v = ok ? gr[nt][e] : 0.f;
-        if (kw == 0) sm.LabT[tau][t] = v;
-        else if (kw == 1) { sm.LakT[tau][t] = v; cx.Lakb[t][tau] = __float2bfloat16_rn(v); }
-        else if (kw == 2) cx.Mrbb[t][tau] = __float2bfloat16_rn(v);
-        else cx.Mrkb[t][tau] = __float2bfloat16_rn(v);
+      for (int tau = 0; tau < kChunk; ++tau) {
+        const bool ok = pair_ok(mask, t, tau, strict);
+        g0[tau] = ok ? g0[tau] : 0.f;
+        g1[tau] = ok ? g1[tau] : 0.f;
       }
+      if (kw == 0) {
+#pragma unroll
+        for (int tau = 0; tau < kChunk; ++tau) {
+          sm.LabT[tau][t] = g0[tau];
+          cx.LakP[t][tau] = g1[tau];
+        }
+      } else {   // [Mrb | Mrk] row t: four 16-byte core rows
+        float v[8];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[e] = q < 2 ? g0[8 * q + e] : g1[8 * (q - 2) + e];
+          put8(cx.MM, cb(t, 8 * q, 32), v);
+        }
+      }
+    }
   }
+  tc::fence_before_sync();
   named_bar(1, 128);
 
-  // ---- K3: T = (I - Lab)^-1, W = T diag(m0) At, X = T Lak by forward substitution (threads 0..95)
-  if (ktid < 96) {
+  // ---- T = (I - Lab)^-1 by forward substitution, one column per thread (threads 0-15)
+  if (ktid < kChunk) {
+    const int cc = ktid;
     float u[kChunk];
-    const int cc = ktid < 64 ? ktid : (ktid < 80 ? ktid - 64 : ktid - 80);
-    if (ktid < 64) {
 #pragma unroll
-      for (int t = 0; t < kChunk; ++t) u[t] = t < fr ? __bfloat162float(cx.GA[t][cc]) : 0.f;
-    } else if (ktid < 80) {
-      const float4* col = reinterpret_cast<const float4*>(&sm.LakT[cc][0]);
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const float4 f = col[q];
-        u[4 * q] = f.x; u[4 * q + 1] = f.y; u[4 * q + 2] = f.z; u[4 * q + 3] = f.w;
-      }
-    } else {
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
-    }
-    // rows of Lab^T are loaded one step ahead, so each step waits only on its FMAs
-    float4 nxt[4];
-#pragma unroll
-    for (int q = 0; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&sm.LabT[0][0])[q];
+    for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
 #pragma unroll
     for (int tau = 0; tau < kChunk - 1; ++tau) {
-      const float4 cur[4] = {nxt[0], nxt[1], nxt[2], nxt[3]};
-      if (tau + 1 < kChunk - 1) {
 #pragma unroll
-        for (int q = (tau + 2) / 4; q < 4; ++q) nxt[q] = reinterpret_cast<const float4*>(&sm.LabT[tau + 1][0])[q];
-      }
-      const float lv[kChunk] = {cur[0].x, cur[0].y, cur[0].z, cur[0].w, cur[1].x, cur[1].y, cur[1].z, cur[1].w,
-                                cur[2].x, cur[2].y, cur[2].z, cur[2].w, cur[3].x, cur[3].y, cur[3].z, cur[3].w};
-#pragma unroll
-      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(lv[t], u[tau], u[t]);
+      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(sm.LabT[tau][t], u[tau], u[t]);
     }
-    if (ktid < 64) {
 #pragma unroll
-      for (int t = 0; t < kChunk; ++t) sm.Wb[t][cc] = __float2bfloat16_rn(u[t]);
-    } else if (ktid < 80) {
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) sm.Xb[t][cc] = __float2bfloat16_rn(u[t]);
-    } else {
-#pragma unroll
-      for (int t = 0; t < kChunk; ++t) cx.Tb[t][cc] = __float2bfloat16_rn(u[t]);
-    }
+    for (int t = 0; t < kChunk; ++t) cx.Tp[t][cc] = u[t];
   }
   named_bar(1, 128);
 
-  // ---- K4: SA = W S0^T + X V for rows i = 16kw..16kw+15, stored [tau][i]
+  // ---- X = T Lak: thread -> (tau, two t); W = T m0.At: thread -> (tau, 8 j)
   {
-    const int i0 = 16 * kw;
-    float sa[2][4] = {};
+    const int tau = ktid >> 3;
+    if ((ktid & 7) < 2) {   // X row tau, columns 8 (ktid & 7) .. +7
+      const int t0 = 8 * (ktid & 7);
+      float x[8] = {};
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4], bs[4];
-      ldsm_x4(a, a_rowmajor_addr(&sm.Wb[0][0], kStr, 0, 16 * ks, lane));
-      ldsm_x4(bs, b_nmajor_addr(&cx.S0b[0][0], kStr, i0, 16 * ks, lane));
-      mma16816(sa[0], a, bs[0], bs[1]);
-      mma16816(sa[1], a, bs[2], bs[3]);
+      for (int s = 0; s < kChunk; ++s) {
+        const float tv = cx.Tp[tau][s];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = fmaf(tv, cx.LakP[s][t0 + e], x[e]);
+      }
+      put8(sm.XC, cb(tau, t0, 16), x);
     }
-    uint32_t ax[4], bv[4];
-    ldsm_x4(ax, a_rowmajor_addr(&sm.Xb[0][0], kStrS, 0, 0, lane));
-    ldsm_x4_t(bv, b_kmajor_addr(&cx.Vb[0][0], kStr, 0, i0, lane));
-    mma16816(sa[0], ax, bv[0], bv[1]);
-    mma16816(sa[1], ax, bv[2], bv[3]);
+    const int j0 = 8 * (ktid & 7);
+    float w[8] = {};
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<uint32_t*>(&cx.SAb[g + 8 * hh][i0 + 8 * nt + 2 * c4]) =
-            pack_bf16(sa[nt][2 * hh], sa[nt][2 * hh + 1]);
+    for (int t = 0; t < kChunk; ++t) {
+      const float tv = t < fr ? cx.Tp[tau][t] : 0.f;
+      const float4 a0 = *reinterpret_cast<const float4*>(&sm.Atf[t][j0]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&sm.Atf[t][j0 + 4]);
+      w[0] = fmaf(tv, a0.x, w[0]); w[1] = fmaf(tv, a0.y, w[1]); w[2] = fmaf(tv, a0.z, w[2]); w[3] = fmaf(tv, a0.w, w[3]);
+      w[4] = fmaf(tv, a1.x, w[4]); w[5] = fmaf(tv, a1.y, w[5]); w[6] = fmaf(tv, a1.z, w[6]); w[7] = fmaf(tv, a1.w, w[7]);
+    }
+    put8(sm.WC, cb(tau, j0, 64), w);
   }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  named_bar(1, 128);
+
+  // ---- SA^T = S0 W^T + V^T X^T  (A: S0^T and v read MN-major, rows i)
+  if (ktid == 0) {
+    tc::fence_after_sync();
+    mma3<16, 4>(tmem + kColSA, op<64, true>(cx.S0T), op<64, false>(sm.WC), false);
+    mma3<16, 1>(tmem + kColSA, op<32, false>(cx.SV, kExactIn, 0, 16), op<16, false>(sm.XC), true);   // v^T half of SV
+    tc::commit(&sm.sa_bar);
+  }
+  mma_wait(p, &sm.sa_bar, phase & 1u);
+  {
+    float sa[16];
+    tc::ld_32x32b_x16(tmem + tlane + kColSA, sa);
+    tc::wait_ld();
+    if (lane < 16) {
+      const int i = 16 * kw + lane;
+      float v[8];
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = sa[8 * q + e];
+        put8(cx.SV, cb(i, 8 * q, 32), v);
+      }
+    }
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
 }
 
 // ------------------------------------------------------------------ main warps
 template <typename T>
-__device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem2<T>& sm, const BCtx& cx, float (&dS)[8][4],
-                                           int64_t b, int64_t h, int64_t t0, int len, int warp, int lane) {
-  const int tid = threadIdx.x;
-  const int g = lane >> 2, c4 = lane & 3;
-  const int row0 = 16 * warp, j0 = 16 * warp;
+__device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, int64_t b, int64_t h,
+                                           int64_t t0, int len, int warp, int lane, uint32_t tmem, unsigned phase) {
+  constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
+  const uint32_t tlane = uint32_t(32 * warp) << 16;
   const unsigned mask = unsigned(cx.mask);
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
-  const unsigned m0bits = (1u << fr) - 1u;
+  const unsigned ls_bits = last_segment_bits(mask);
   const bool keep = mask == 0u;
-  const unsigned ls_bits = cx.ls_bits;
-  // staging of da, dr, db, dk [q][t][j] in bf16; reuses dSb, which is dead after M8
-  bf16 (*gst)[kChunk][kStr] = reinterpret_cast<bf16 (*)[kChunk][kStr]>(&sm.dSb[0][0]);
+  const int row = 16 * warp + (lane & 15);   // TMEM row of this thread (both halves of the warp)
+  const int half = lane >> 4;                // which half of a row's columns this thread holds
 
-  // ---- M1: [dSA^T | dV^T] = dSl [ls.Bh | ls.Kh]^T + dY^T [Mrb | Mrk]   (rows i of this warp)
-  float acc4[4][4] = {};
+  // ---- M1: dSl^T = L_15 dS^T (row j = row) into shared memory for the chain products.  This
+  // thread holds columns 16 half + (0..15) and 32 + 16 half + (0..15) of its row.
+  float d[32];
   {
-    const bool ls_lo = (ls_bits >> g) & 1u, ls_hi = (ls_bits >> (8 + g)) & 1u;
+    float x[16];
+    tc::ld_16x32bx2_x16(tmem + tlane + kColDS, x);
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      const float2 la = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][16 * ks + 2 * c4]);
-      const float2 lb = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][16 * ks + 8 + 2 * c4]);
-      const float2 p0 = mul2(make_float2(dS[2 * ks][0], dS[2 * ks][1]), la);
-      const float2 p1 = mul2(make_float2(dS[2 * ks][2], dS[2 * ks][3]), la);
-      const float2 p2 = mul2(make_float2(dS[2 * ks + 1][0], dS[2 * ks + 1][1]), lb);
-      const float2 p3 = mul2(make_float2(dS[2 * ks + 1][2], dS[2 * ks + 1][3]), lb);
-      uint32_t a[4] = {pack_bf16(p0.x, p0.y), pack_bf16(p1.x, p1.y), pack_bf16(p2.x, p2.y), pack_bf16(p3.x, p3.y)};
-      uint32_t bb[4], bk[4];
-      ldsm_x4(bb, b_nmajor_addr(&cx.GB[0][0], kStr, 0, 16 * ks, lane));
-      ldsm_x4(bk, b_nmajor_addr(&cx.GB[0][0], kStr, 16, 16 * ks, lane));
-      if (!ls_lo) { bb[0] = 0u; bb[1] = 0u; bk[0] = 0u; bk[1] = 0u; }
-      if (!ls_hi) { bb[2] = 0u; bb[3] = 0u; bk[2] = 0u; bk[3] = 0u; }
-      mma16816(acc4[0], a, bb[0], bb[1]);
-      mma16816(acc4[1], a, bb[2], bb[3]);
-      mma16816(acc4[2], a, bk[0], bk[1]);
-      mma16816(acc4[3], a, bk[2], bk[3]);
-    }
-    uint32_t ay[4], bm[4], bk[4];
-    ldsm_x4_t(ay, a_kmajor_addr(&cx.DYb[0][0], kStr, 0, row0, lane));
-    ldsm_x4_t(bm, b_kmajor_addr(&cx.Mrbb[0][0], kStrS, 0, 0, lane));
-    ldsm_x4_t(bk, b_kmajor_addr(&cx.Mrkb[0][0], kStrS, 0, 0, lane));
-    mma16816(acc4[0], ay, bm[0], bm[1]);
-    mma16816(acc4[1], ay, bm[2], bm[3]);
-    mma16816(acc4[2], ay, bk[0], bk[1]);
-    mma16816(acc4[3], ay, bk[2], bk[3]);
+    for (int e = 0; e < 16; ++e) d[e] = x[e];
+    tc::ld_16x32bx2_x16(tmem + tlane + kColDS + 32, x);
+#pragma unroll
+    for (int e = 0; e < 16; ++e) d[16 + e] = x[e];
   }
-  // ---- M2: dU^T = dSA^T T ; M3: dV^T += dU^T Lak
+  tc::wait_ld();
   {
-    uint32_t adsa[4], bt[4];
-    frag_to_a(acc4[0], acc4[1], adsa);
-    ldsm_x4_t(bt, b_kmajor_addr(&cx.Tb[0][0], kStrS, 0, 0, lane));
-    float du[2][4] = {};
-    mma16816(du[0], adsa, bt[0], bt[1]);
-    mma16816(du[1], adsa, bt[2], bt[3]);
+    const float l15 = cx.lam[kChunk - 1][row];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
+    for (int e = 0; e < 32; ++e) d[e] *= l15;
 #pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sm.DUb[8 * nt + 2 * c4 + (e & 1)][row0 + g + 8 * (e >> 1)] = __float2bfloat16_rn(du[nt][e]);
-    uint32_t adu[4], bl[4];
-    frag_to_a(du[0], du[1], adu);
-    ldsm_x4_t(bl, b_kmajor_addr(&cx.Lakb[0][0], kStrS, 0, 0, lane));
-    mma16816(acc4[2], adu, bl[0], bl[1]);
-    mma16816(acc4[3], adu, bl[2], bl[3]);
+    for (int q = 0; q < 4; ++q) {
+      float v[8];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e)
-        sm.dVs[8 * nt + 2 * c4 + (e & 1)][row0 + g + 8 * (e >> 1)] = __float2bfloat16_rn(acc4[2 + nt][e]);
+      for (int e = 0; e < 8; ++e) v[e] = d[8 * q + e];
+      put8(sm.dSlT, cb(row, 32 * (q >> 1) + 16 * half + 8 * (q & 1), 64), v);
+    }
   }
-  // ---- M4: dS16 in bf16 for the column products; partial sum_i S0 o dS16 over this warp's rows
-  {
-    float part[16];
-#pragma unroll
-    for (int nt = 0; nt < 8; ++nt) {
-      const int col = 8 * nt + 2 * c4;
-      float2 s_lo = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.S0b[row0 + g][col]));
-      float2 s_hi = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.S0b[row0 + g + 8][col]));
-      const float2 pr = fma2(s_lo, make_float2(dS[nt][0], dS[nt][1]), mul2(s_hi, make_float2(dS[nt][2], dS[nt][3])));
-      part[2 * nt] = pr.x;
-      part[2 * nt + 1] = pr.y;
-      *reinterpret_cast<uint32_t*>(&sm.dSb[row0 + g][col]) = pack_bf16(dS[nt][0], dS[nt][1]);
-      *reinterpret_cast<uint32_t*>(&sm.dSb[row0 + g + 8][col]) = pack_bf16(dS[nt][2], dS[nt][3]);
-    }
-#pragma unroll
-    for (int k = 0; k < 8; ++k) {
-      const bool up = lane & 16;
-      const float send = up ? part[k] : part[k + 8];
-      const float kv = up ? part[k + 8] : part[k];
-      part[k] = kv + __shfl_xor_sync(0xffffffffu, send, 16);
-    }
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const bool up = lane & 8;
-      const float send = up ? part[k] : part[k + 4];
-      const float kv = up ? part[k + 4] : part[k];
-      part[k] = kv + __shfl_xor_sync(0xffffffffu, send, 8);
-    }
-#pragma unroll
-    for (int k = 0; k < 2; ++k) {
-      const bool up = lane & 4;
-      const float send = up ? part[k] : part[k + 2];
-      const float kv = up ? part[k + 2] : part[k];
-      part[k] = kv + __shfl_xor_sync(0xffffffffu, send, 4);
-    }
-    const int idx = 8 * ((lane >> 4) & 1) + 4 * ((lane >> 3) & 1) + 2 * ((lane >> 2) & 1);
-    sm.dlam[warp][8 * (idx >> 1) + 2 * c4] = part[0];
-    sm.dlam[warp][8 * (idx >> 1) + 2 * c4 + 1] = part[1];
-  }
-  named_bar(2, 128);   // DUb, dVs, dSb, dlam complete
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  named_bar(2, 128);
 
-  // ---- M5: gradient entering the chunk: keep.dSl + (m0.dY)^T Rt + (m0.dU)^T At
+  // ---- M2: G1 = dSl [Bh|Kh]^T, G2 = dY^T [Mrb|Mrk]
+  if (threadIdx.x == 0) {
+    tc::fence_after_sync();
+    mma3<32, 4>(tmem + kColG1, op<64, true>(sm.dSlT), op<64, false>(cx.BK), false);
+    mma3<32, 1>(tmem + kColG2, op<64, true>(cx.DYU, kExactIn), op<32, true>(cx.MM), false);   // dy rows of DYU
+    tc::commit(&sm.u_bar);
+  }
+  // while the tensor core works: keep.dSl^T back into TMEM (the start of dS0^T) and the L_15 term
+  // keep.sum_i dSl o S0 of this key channel (each half of the row, then both halves added)
+  float dl15 = 0.f;
   {
     if (keep) {
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) {
-        const float2 l = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][8 * nt + 2 * c4]);
-        const float2 u0 = mul2(make_float2(dS[nt][0], dS[nt][1]), l);
-        const float2 u1 = mul2(make_float2(dS[nt][2], dS[nt][3]), l);
-        dS[nt][0] = u0.x; dS[nt][1] = u0.y; dS[nt][2] = u1.x; dS[nt][3] = u1.y;
-      }
-    } else {
+      for (int q = 0; q < 4; ++q) {
+        float s0[8];
+        get8(cx.S0T, cb(row, 32 * (q >> 1) + 16 * half + 8 * (q & 1), 64), s0);
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt) dS[nt][0] = dS[nt][1] = dS[nt][2] = dS[nt][3] = 0.f;
-    }
-    uint32_t ay[4], au[4];
-    ldsm_x4_t(ay, a_kmajor_addr(&cx.DYb[0][0], kStr, 0, row0, lane));
-    ldsm_x4_t(au, a_kmajor_addr(&sm.DUb[0][0], kStr, 0, row0, lane));
-    mask_k16(ay, c4, m0bits);
-    mask_k16(au, c4, m0bits);
-#pragma unroll
-    for (int np = 0; np < 4; ++np) {
-      uint32_t br[4], ba[4];
-      ldsm_x4_t(br, b_kmajor_addr(&cx.GA[0][0], kStr, 16, 16 * np, lane));
-      ldsm_x4_t(ba, b_kmajor_addr(&cx.GA[0][0], kStr, 0, 16 * np, lane));
-#pragma unroll
-      for (int u = 0; u < 2; ++u) {
-        mma16816(dS[2 * np + u], ay, br[2 * u], br[2 * u + 1]);
-        mma16816(dS[2 * np + u], au, ba[2 * u], ba[2 * u + 1]);
+        for (int e = 0; e < 8; ++e) dl15 = fmaf(d[8 * q + e], s0[e], dl15);
       }
     }
-  }
-  // ---- dv out (coalesced from the staging tile)
-  {
-    T* dv = static_cast<T*>(p.dv);
-    const int tt = tid >> 3, part = tid & 7;
-    if (tt < len) {
-      alignas(16) T vals[8];
+    dl15 += __shfl_xor_sync(0xffffffffu, dl15, 16);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) vals[u] = Elt<T>::from_f32(__bfloat162float(sm.dVs[tt][part * 8 + u]));
-      uint4* dst = reinterpret_cast<uint4*>(dv + tok_off(b, t0 + tt, h, p.T, p.H) + part * 8);
-      const uint4* sv = reinterpret_cast<const uint4*>(vals);
+    for (int h2 = 0; h2 < 2; ++h2) {
+      float x[16];
 #pragma unroll
-      for (int u = 0; u < int(sizeof(vals) / 16); ++u) dst[u] = sv[u];
+      for (int e = 0; e < 16; ++e) x[e] = keep ? d[16 * h2 + e] : 0.f;
+      tc::st_16x32bx2_x16(tmem + tlane + kColDS + 32 * h2, x);
     }
+    tc::wait_st();
   }
-  // ---- M7: gradient Gram block (warp = block): [dMrb dMrk; dLab dLak], masked
-  {
-    const bf16* Asrc = (warp >> 1) ? &sm.DUb[0][0] : &cx.DYb[0][0];
-    const bf16* Bsrc = (warp & 1) ? &cx.Vb[0][0] : &cx.SAb[0][0];
-    float gr[2][4] = {};
-#pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t a[4], bb[4];
-      ldsm_x4(a, a_rowmajor_addr(Asrc, kStr, 0, 16 * ks, lane));
-      ldsm_x4(bb, b_nmajor_addr(Bsrc, kStr, 0, 16 * ks, lane));
-      mma16816(gr[0], a, bb[0], bb[1]);
-      mma16816(gr[1], a, bb[2], bb[3]);
-    }
-    const bool strict = (warp >> 1) != 0;
-    const int st0 = seg_of(mask, g), st1 = seg_of(mask, g + 8);
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int t = g + (e >> 1) * 8;
-        const int tau = 8 * nt + 2 * c4 + (e & 1);
-        const bool ok = (strict ? (tau < t) : (tau <= t)) && seg_of(mask, tau) == ((e >> 1) ? st1 : st0);
-        sm.dG[(warp >> 1) * 16 + t][(warp & 1) * 16 + tau] = __float2bfloat16_rn(ok ? gr[nt][e] : 0.f);
-      }
-  }
-  // ---- M8: [dRt; dAt] from S0 and [dBb; dKb] from dS16, columns j0..j0+15
-  float xr[2][4] = {}, xa[2][4] = {}, xb[2][4] = {}, xk[2][4] = {};
-#pragma unroll
-  for (int ks = 0; ks < 4; ++ks) {
-    uint32_t ay[4], au[4], asa[4], av[4], bs[4], bd[4];
-    ldsm_x4(ay, a_rowmajor_addr(&cx.DYb[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(au, a_rowmajor_addr(&sm.DUb[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(asa, a_rowmajor_addr(&cx.SAb[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4(av, a_rowmajor_addr(&cx.Vb[0][0], kStr, 0, 16 * ks, lane));
-    ldsm_x4_t(bs, b_kmajor_addr(&cx.S0b[0][0], kStr, 16 * ks, j0, lane));
-    ldsm_x4_t(bd, b_kmajor_addr(&sm.dSb[0][0], kStr, 16 * ks, j0, lane));
-#pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      mma16816(xr[nt], ay, bs[2 * nt], bs[2 * nt + 1]);
-      mma16816(xa[nt], au, bs[2 * nt], bs[2 * nt + 1]);
-      mma16816(xb[nt], asa, bd[2 * nt], bd[2 * nt + 1]);
-      mma16816(xk[nt], av, bd[2 * nt], bd[2 * nt + 1]);
-    }
-  }
-  named_bar(2, 128);   // dG complete
+  mma_wait(p, &sm.u_bar, phase & 1u);
 
-  // ---- M9/M10: key-space gradients of columns j0..j0+15 and the per-token outputs
+  // ---- M3: dSA^T, dU^T = dSA^T T and dV^T per value channel i = row (FP32 cores); this thread holds
+  // tokens 8 half .. 8 half + 7 of its row; dv out, dU into shared memory
   {
-    float dA[2][4] = {}, dR[2][4] = {}, dB[2][4] = {}, dK[2][4] = {};
+    float g1b[8], g1k[8], g2b[8], g2k[8];
+    tc::ld_16x32bx2_x8(tmem + tlane + kColG1, g1b);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColG1 + 16, g1k);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColG2, g2b);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColG2 + 16, g2k);
+    tc::wait_ld();
+    const int i = row, tb = 8 * half;
+    float dsa[16], du[8], dv[8];
 #pragma unroll
-    for (int ks = 0; ks < 2; ++ks) {
-      uint32_t aL[4], aM[4], aLt[4], aLk[4], bg[4], ba[4];
-      ldsm_x4(aL, a_rowmajor_addr(&sm.dG[0][0], kStrG, 16, 16 * ks, lane));
-      ldsm_x4(aM, a_rowmajor_addr(&sm.dG[0][0], kStrG, 0, 16 * ks, lane));
-      ldsm_x4_t(bg, b_kmajor_addr(&cx.GB[0][0], kStr, 16 * ks, j0, lane));
-      const int krow = ks == 0 ? 16 : 0;
-      ldsm_x4_t(aLt, a_kmajor_addr(&sm.dG[0][0], kStrG, krow, 0, lane));
-      ldsm_x4_t(aLk, a_kmajor_addr(&sm.dG[0][0], kStrG, krow, 16, lane));
-      ldsm_x4_t(ba, b_kmajor_addr(&cx.GA[0][0], kStr, ks == 0 ? 0 : 16, j0, lane));
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        mma16816(dA[nt], aL, bg[2 * nt], bg[2 * nt + 1]);
-        mma16816(dR[nt], aM, bg[2 * nt], bg[2 * nt + 1]);
-        mma16816(dB[nt], aLt, ba[2 * nt], ba[2 * nt + 1]);
-        mma16816(dK[nt], aLk, ba[2 * nt], ba[2 * nt + 1]);
-      }
+    for (int e = 0; e < 8; ++e) {
+      const float mine = ((ls_bits >> (tb + e)) & 1u ? g1b[e] : 0.f) + g2b[e];
+      const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
+      dsa[e] = half ? other : mine;
+      dsa[8 + e] = half ? mine : other;
+      du[e] = 0.f;
+      dv[e] = ((ls_bits >> (tb + e)) & 1u ? g1k[e] : 0.f) + g2k[e];
     }
-    T* gda = static_cast<T*>(p.da);
-    T* gdr = static_cast<T*>(p.dr);
-    T* gdb = static_cast<T*>(p.db);
-    T* gdk = static_cast<T*>(p.dk);
-    float2 e2v[2][2];   // [nt][hh], columns j, j+1
-    float2 e1v[2][2];
-    float2 e3p[2] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
-    const float2 zero2 = make_float2(0.f, 0.f);
+    // dU^T[i][tau] = sum_t dSA^T[i][t] T[t][tau] (T is stored with zeros above its diagonal)
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
-      const int t = g + 8 * hh;
-      const bool m0t = t < fr;
-      const bool ls = (ls_bits >> t) & 1u;
-      const int64_t orow = tok_off(b, t0 + t, h, p.T, p.H);
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        const int j = j0 + 8 * nt + 2 * c4;
-        const int e = 2 * hh;
-        const float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[t][j]);
-        const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
-        const float2 L15 = *reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]);
-        const float2 at = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[t][j]));
-        const float2 rt = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GA[16 + t][j]));
-        const float2 bh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[t][j]));
-        const float2 kh = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&cx.GB[16 + t][j]));
-        const float2 xb2 = ls ? make_float2(xb[nt][e], xb[nt][e + 1]) : zero2;
-        const float2 xk2 = ls ? make_float2(xk[nt][e], xk[nt][e + 1]) : zero2;
-        const float2 dAt = add2(make_float2(dA[nt][e], dA[nt][e + 1]), m0t ? make_float2(xa[nt][e], xa[nt][e + 1]) : zero2);
-        const float2 dRt = add2(make_float2(dR[nt][e], dR[nt][e + 1]), m0t ? make_float2(xr[nt][e], xr[nt][e + 1]) : zero2);
-        const float2 dBt = fma2(L15, xb2, make_float2(dB[nt][e], dB[nt][e + 1]));
-        const float2 dKt = fma2(L15, xk2, make_float2(dK[nt][e], dK[nt][e + 1]));
-        const float2 inv = make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y));
-        e1v[nt][hh] = sub2(mul2(dRt, rt), fma2(dBt, bh, mul2(dKt, kh)));
-        e2v[nt][hh] = mul2(dAt, at);
-        e3p[nt] = fma2(fma2(xb2, bh, mul2(xk2, kh)), L15, e3p[nt]);
-        if constexpr (std::is_same<T, bf16>::value) {   // staged, written coalesced after the barrier
-          store2(&gst[0][t][j], mul2(dAt, Lp));
-          store2(&gst[1][t][j], mul2(dRt, Lt));
-          store2(&gst[2][t][j], mul2(dBt, inv));
-          store2(&gst[3][t][j], mul2(dKt, inv));
-        } else if (t < len) {
-          store2(gda + orow + j, mul2(dAt, Lp));
-          store2(gdr + orow + j, mul2(dRt, Lt));
-          store2(gdb + orow + j, mul2(dBt, inv));
-          store2(gdk + orow + j, mul2(dKt, inv));
-        }
-      }
+    for (int t = 0; t < kChunk; ++t) {
+      const float4 a = *reinterpret_cast<const float4*>(&cx.Tp[t][tb]);
+      const float4 c = *reinterpret_cast<const float4*>(&cx.Tp[t][tb + 4]);
+      du[0] = fmaf(dsa[t], a.x, du[0]); du[1] = fmaf(dsa[t], a.y, du[1]);
+      du[2] = fmaf(dsa[t], a.z, du[2]); du[3] = fmaf(dsa[t], a.w, du[3]);
+      du[4] = fmaf(dsa[t], c.x, du[4]); du[5] = fmaf(dsa[t], c.y, du[5]);
+      du[6] = fmaf(dsa[t], c.z, du[6]); du[7] = fmaf(dsa[t], c.w, du[7]);
     }
-    // d log L_t = E1_t + E2_{t+1}: E2 of row t+1 lives in lane+4 (same half) or, for row 7, in lane c4 (upper half)
+    // dV^T[i][tau] += sum_t dU^T[i][t] Lak[t][tau] (Lak is zero on and above its diagonal)
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
-      float2 dn0, up0, dn1;
-      dn0.x = __shfl_down_sync(0xffffffffu, e2v[nt][0].x, 4);
-      dn0.y = __shfl_down_sync(0xffffffffu, e2v[nt][0].y, 4);
-      up0.x = __shfl_sync(0xffffffffu, e2v[nt][1].x, c4);
-      up0.y = __shfl_sync(0xffffffffu, e2v[nt][1].y, c4);
-      dn1.x = __shfl_down_sync(0xffffffffu, e2v[nt][1].x, 4);
-      dn1.y = __shfl_down_sync(0xffffffffu, e2v[nt][1].y, 4);
-      const int j = j0 + 8 * nt + 2 * c4;
-      *reinterpret_cast<float2*>(&sm.DL[g][j]) = add2(e1v[nt][0], g < 7 ? dn0 : up0);
-      *reinterpret_cast<float2*>(&sm.DL[g + 8][j]) = add2(e1v[nt][1], g < 7 ? dn1 : make_float2(0.f, 0.f));
-      float2 v = e3p[nt];
+    for (int t = 0; t < kChunk; ++t) {
+      const float mine = du[t & 7], other = __shfl_xor_sync(0xffffffffu, mine, 16);
+      const float dut = ((t >> 3) == half) ? mine : other;
+      const float4 a = *reinterpret_cast<const float4*>(&cx.LakP[t][tb]);
+      const float4 c = *reinterpret_cast<const float4*>(&cx.LakP[t][tb + 4]);
+      dv[0] = fmaf(dut, a.x, dv[0]); dv[1] = fmaf(dut, a.y, dv[1]);
+      dv[2] = fmaf(dut, a.z, dv[2]); dv[3] = fmaf(dut, a.w, dv[3]);
+      dv[4] = fmaf(dut, c.x, dv[4]); dv[5] = fmaf(dut, c.y, dv[5]);
+      dv[6] = fmaf(dut, c.z, dv[6]); dv[7] = fmaf(dut, c.w, dv[7]);
+    }
+    // dU: rows 16 + t of DYU (column i) and, masked to the tokens before the first reset, DUY
+    float v[8];
 #pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        v.x += __shfl_xor_sync(0xffffffffu, v.x, o);
-        v.y += __shfl_xor_sync(0xffffffffu, v.y, o);
-      }
-      if (g == 0) *reinterpret_cast<float2*>(&sm.e3[j]) = v;
+    for (int e = 0; e < 8; ++e) {
+      put1(cx.DYU, cb(16 + tb + e, i, 64), du[e]);
+      v[e] = tb + e < fr ? du[e] : 0.f;
     }
-  }
-  named_bar(2, 128);   // DL, e3, staged gradients complete
-
-  if constexpr (std::is_same<T, bf16>::value) {
-    T* const outs[4] = {static_cast<T*>(p.da), static_cast<T*>(p.dr), static_cast<T*>(p.db), static_cast<T*>(p.dk)};
-    const int tt = tid >> 3, part = tid & 7;
-    if (tt < len) {
-      const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + part * 8;
-#pragma unroll
-      for (int q = 0; q < 4; ++q)
-        *reinterpret_cast<uint4*>(outs[q] + o) = *reinterpret_cast<const uint4*>(&gst[q][tt][part * 8]);
-    }
-  }
-
-  // ---- M11: dw = (reverse cumulative sum of d log L) / w.  Thread = (column pair, token quarter
-  // q = warp): each thread first adds the rows of the later quarters itself, then walks its four.
-  {
-    const int j = 2 * lane, q = warp, thi = 4 * q + 3;
-    float2 cum = *reinterpret_cast<const float2*>(&sm.e3[j]);
-    if (keep) {
-      const float2 d01 = add2(*reinterpret_cast<const float2*>(&sm.dlam[0][j]), *reinterpret_cast<const float2*>(&sm.dlam[1][j]));
-      const float2 d23 = add2(*reinterpret_cast<const float2*>(&sm.dlam[2][j]), *reinterpret_cast<const float2*>(&sm.dlam[3][j]));
-      cum = fma2(*reinterpret_cast<const float2*>(&cx.lam[kChunk - 1][j]), add2(d01, d23), cum);
-    }
-    for (int t = kChunk - 1; t > thi; --t) cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
-    T* gdw = static_cast<T*>(p.dw) + tok_off(b, t0, h, p.T, p.H) + j;
+    put8(cx.DUY, cb(i, tb, 32), v);
+    T* dvp = static_cast<T*>(p.dv) + tok_off(b, t0 + tb, h, p.T, p.H) + i;
     const int64_t rs = p.H * kN;
-    float2 Lt = *reinterpret_cast<const float2*>(&cx.lam[thi][j]);
 #pragma unroll
-    for (int u = 3; u >= 0; --u) {
-      const int t = 4 * q + u;
-      cum = add2(cum, *reinterpret_cast<const float2*>(&sm.DL[t][j]));
-      const float2 Lp = t > 0 ? *reinterpret_cast<const float2*>(&cx.lam[t - 1][j]) : make_float2(1.f, 1.f);
-      if (t < len) store2(gdw + t * rs, mul2(cum, mul2(Lp, make_float2(rcp_approx(Lt.x), rcp_approx(Lt.y)))));
-      Lt = Lp;
+    for (int e = 0; e < 8; ++e) {
+      if (tb + e < len) *dvp = Elt<T>::from_f32(dv[e]);
+      dvp += rs;
     }
   }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  named_bar(2, 128);
+
+  // ---- M4: rest of dS0^T; gradient Gram; the S0 and dSl parts of the key-space products
+  if (threadIdx.x == 0) {
+    tc::fence_after_sync();
+    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR, false, 16), op<32, false>(cx.DUY, kExactIn, 0, 16), true);
+    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR), op<32, false>(cx.DUY), true);   // dS0^T += Rt^T m0.dy + At^T m0.dU
+    tc::commit(&sm.chain_bar);
+    const auto SV_M = op<32, true>(cx.SV);
+    mma3<32, 4>(tmem + kColGG, op<64, false>(cx.DYU), SV_M, false);   // [dY; dU] [SA^T | v^T]   (rows t, 16 + t)
+    mma3<32, 4>(tmem + kColE, op<64, false>(cx.S0T), op<32, true>(cx.DUY), false);   // S0^T [m0.dU^T | m0.dy^T] (rows j)
+    mma3<32, 4>(tmem + kColE + 64, op<64, false>(sm.dSlT), SV_M, false);       // dSl^T [SA^T | v^T]
+    tc::commit(&sm.gg_bar);
+  }
+  mma_wait(p, &sm.gg_bar, phase & 1u);
+
+  // ---- M5: masked gradient Gram into the B operand of the key-space products.  Warp 0 holds rows
+  // t of [dMrb | dMrk] (causal), warp 1 rows t of [dLab | dLak] (strictly causal).
+  if (warp < 2) {   // this thread: row t = lane % 16, columns 16 half .. 16 half + 15 (the b or the k block)
+    float g[16];
+    tc::ld_16x32bx2_x16(tmem + tlane + kColGG, g);
+    tc::wait_ld();
+    const int t = lane & 15;
+    const bool strict = warp == 1;
+#pragma unroll
+    for (int tau = 0; tau < kChunk; ++tau) g[tau] = pair_ok(mask, t, tau, strict) ? g[tau] : 0.f;
+    const int r = strict ? t : 16 + t;   // G4 rows t: [dLab | dLak]; rows 16 + t: [dMrb | dMrk]
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float v[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = g[8 * q + e];
+      put8(sm.G4, cb(r, 16 * half + 8 * q, 32), v);
+    }
+  }
+  tc::fence_smem_to_async();
+  tc::fence_before_sync();
+  named_bar(2, 128);
+  if (threadIdx.x == 0) {
+    tc::fence_after_sync();
+    const auto BK_M = op<64, true>(cx.BK), AR_M = op<64, true>(cx.AR);
+    mma3<32, 2>(tmem + kColE, BK_M, op<32, false>(sm.G4), true);        // += [Bh^T|Kh^T] [dLab^T dMrb^T; dLak^T dMrk^T]
+    mma3<32, 2>(tmem + kColE + 32, AR_M, op<32, true>(sm.G4), false);   // [At^T|Rt^T] [dLab dLak; dMrb dMrk]
+    tc::commit(&sm.e_bar);
+  }
+  mma_wait(p, &sm.e_bar, phase & 1u);
+
+  // ---- M6: per key channel j = row: da, dr, db, dk and dw over the chunk's tokens; this thread
+  // holds tokens tb .. tb + 7 of its channel (tb = 8 half)
+  {
+    const int j = row, tb = 8 * half;
+    float eA[8], eR[8], eB[8], eK[8], xb[8], xk[8];
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE, eA);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE + 16, eR);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE + 32, eB);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE + 48, eK);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE + 64, xb);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColE + 80, xk);
+    float Lr[9];   // L_{tb-1} .. L_{tb+7}
+    {
+      const float4 a = *reinterpret_cast<const float4*>(&cx.lamT[j][tb]);
+      const float4 c = *reinterpret_cast<const float4*>(&cx.lamT[j][tb + 4]);
+      Lr[1] = a.x; Lr[2] = a.y; Lr[3] = a.z; Lr[4] = a.w; Lr[5] = c.x; Lr[6] = c.y; Lr[7] = c.z; Lr[8] = c.w;
+      Lr[0] = half ? cx.lamT[j][tb - 1] : 1.f;
+    }
+    float rr[8], ar[8], br[8], kr[8];
+    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[0][j][tb]), rr);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[1][j][tb]), ar);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[2][j][tb]), br);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[3][j][tb]), kr);
+    tc::wait_ld();
+    float DL[8], il[8], e3 = 0.f, sumDL = 0.f, firstA = 0.f;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const bool ls = (ls_bits >> (tb + e)) & 1u;
+      il[e] = rcp_approx(Lr[e + 1]);
+      const float at = ar[e] * Lr[e], rt = rr[e] * Lr[e + 1], bh = br[e] * il[e], kh = kr[e] * il[e];
+      const float xbt = ls ? xb[e] : 0.f, xkt = ls ? xk[e] : 0.f;
+      eB[e] += xbt;   // dBh
+      eK[e] += xkt;   // dKh
+      e3 = fmaf(xbt, bh, fmaf(xkt, kh, e3));
+      DL[e] = fmaf(eR[e], rt, -fmaf(eB[e], bh, eK[e] * kh));
+      const float a_t = eA[e] * at;    // dAt_t At_t, which belongs to d log L_{t-1}
+      if (e > 0) DL[e - 1] += a_t; else firstA = a_t;
+    }
+    // token tb + 7 takes dAt At of token tb + 8 from the other half (none after token 15)
+    const float nextA = __shfl_xor_sync(0xffffffffu, firstA, 16);
+    if (!half) DL[7] += nextA;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) sumDL += DL[e];
+    e3 += __shfl_xor_sync(0xffffffffu, e3, 16);
+    const float upper = __shfl_xor_sync(0xffffffffu, sumDL, 16);   // sum over tokens 8..15, for half 0
+    float cum = dl15 + e3 + (half ? 0.f : upper);
+    const int64_t rs = p.H * kN, o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
+    T* const gda = static_cast<T*>(p.da);
+    T* const gdr = static_cast<T*>(p.dr);
+    T* const gdb = static_cast<T*>(p.db);
+    T* const gdk = static_cast<T*>(p.dk);
+    T* const gdw = static_cast<T*>(p.dw);
+#pragma unroll
+    for (int e = 7; e >= 0; --e) {
+      cum += DL[e];
+      if (tb + e < len) {
+        const int64_t o = o0 + e * rs;
+        gda[o] = Elt<T>::from_f32(eA[e] * Lr[e]);
+        gdr[o] = Elt<T>::from_f32(eR[e] * Lr[e + 1]);
+        gdb[o] = Elt<T>::from_f32(eB[e] * il[e]);
+        gdk[o] = Elt<T>::from_f32(eK[e] * il[e]);
+        gdw[o] = Elt<T>::from_f32(cum * (Lr[e] * il[e]));
+      }
+    }
+  }
+  tc::fence_before_sync();
 }
 
 template <typename T>
-__global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p, const __grid_constant__ InputMaps tm) {
+__global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
-  BwdSmem2<T>& sm = *reinterpret_cast<BwdSmem2<T>*>(smem_raw);
+  BwdSmem<T>& sm = *reinterpret_cast<BwdSmem<T>*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const bool is_main = warp < 4;
   const int ktid = tid - 128;
-  const int g = lane >> 2, c4 = lane & 3;
-  const int row0 = 16 * warp;
   const int64_t nc = (p.T + kChunk - 1) / kChunk;
 
-  if (tid == 0) sm.stop = 0;
+  if (tid == 0) {
+    sm.stop = 0;
+    mbar_init(&sm.in_bar, 1);
+    mbar_init(&sm.gram_bar, 1);
+    mbar_init(&sm.sa_bar, 1);
+    mbar_init(&sm.u_bar, 1);
+    mbar_init(&sm.chain_bar, 1);
+    mbar_init(&sm.gg_bar, 1);
+    mbar_init(&sm.e_bar, 1);
+  }
+  if (warp == 0) {   // 512 TMEM columns: this kernel runs one CTA per SM (its shared memory)
+    tc::alloc(&sm.tmem_base, kTmemCols);
+    tc::relinquish();
+  }
+  tc::fence_before_sync();
+  cta_sync();
+  tc::fence_after_sync();
+  const uint32_t tmem = sm.tmem_base;
 
-  // The two roles run separate loops so that their register sets never overlap; both meet
-  // at one CTA barrier per iteration (bar.sync 0, executed by all 256 threads).
+  // The two roles run separate loops so that their register sets never overlap; both meet at
+  // one CTA barrier per iteration (bar.sync 0, executed by all 256 threads).
   if (is_main) {
-    float dS[8][4];
+    // dS^T entering the last chunk: dsT transposed (row j = TMEM row 16 warp + lane), or zero
+    {
+      const int j = 16 * warp + lane;
 #pragma unroll
-    for (int nt = 0; nt < 8; ++nt)
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float d[16];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        float2 v = make_float2(0.f, 0.f);
-        if (p.dsT) v = *reinterpret_cast<const float2*>(p.dsT + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4);
-        dS[nt][2 * hh] = v.x;
-        dS[nt][2 * hh + 1] = v.y;
+        for (int e = 0; e < 16; ++e) d[e] = (p.dsT && lane < 16) ? p.dsT[(unit * kN + 16 * q4 + e) * kN + j] : 0.f;
+        tc::st_32x32b_x16(tmem + (uint32_t(32 * warp) << 16) + kColDS + 16 * q4, d);
       }
+      tc::wait_st();
+    }
+    tc::fence_before_sync();
     cta_sync();   // prologue staged by the context warps
     bool flagged = false;
+    unsigned phase = 0;
     for (int64_t it = 0; it <= nc; ++it) {
       if (it >= 1) {
         const int64_t c = nc - it;   // chunk whose gradients are computed now
-        const BCtx& cx = sm.ctx[c & 1];
+        Ctx<T>& cx = sm.ctx[c & 1];   // the main warps own this buffer until the next CTA barrier
         if (cx.unsafe) {
           if (tid == 0) sm.stop = 1;
         } else {
+          tc::fence_after_sync();
           const int64_t t0 = c * kChunk;
-          main_chunk<T>(p, sm, cx, dS, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane);
+          main_chunk<T>(p, sm, cx, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane, tmem, phase);
+          ++phase;
         }
       }
       cta_sync();
@@ -718,55 +800,54 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p,
       }
     }
     if (tid == 0 && p.unit_flags) p.unit_flags[unit] = flagged ? 1 : 0;
-    if (!flagged && p.ds0) {
+    if (!flagged && p.ds0) {   // every MMA of the last chunk completed before its e_bar phase
+      tc::fence_after_sync();
+      const int j = 16 * warp + lane;
 #pragma unroll
-      for (int nt = 0; nt < 8; ++nt)
+      for (int q4 = 0; q4 < 4; ++q4) {
+        float d[16];
+        tc::ld_32x32b_x16(tmem + (uint32_t(32 * warp) << 16) + kColDS + 16 * q4, d);
+        tc::wait_ld();
+        if (lane < 16) {
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-          *reinterpret_cast<float2*>(p.ds0 + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-              make_float2(dS[nt][2 * hh], dS[nt][2 * hh + 1]);
+          for (int e = 0; e < 16; ++e) p.ds0[(unit * kN + 16 * q4 + e) * kN + j] = d[e];
+        }
+      }
     }
   } else {
-    // prologue: stage the last chunk, its entering state and reset flags
-    float4 s0rows[8];
     unsigned mask_next;
-    unsigned phase = 0;        // barrier phase of the next staging to wait for
+    unsigned phase = 0;        // staging phase of the next wait
+    unsigned cphase = 0;       // context MMA phase
     bool pending = true;       // a staging was issued and not yet waited for
     bool timed_out = false;
-    {
-      if (ktid == 0) mbar_init(&sm.in_bar, 1);
-      named_bar(1, 128);
-      const int64_t c = nc - 1;
-      const int64_t t0 = c * kChunk;
-      stage7<T>(p, tm, sm, b, h, t0, ktid);
-      load_entry_rows(p, unit, nc, c, ktid, s0rows);
-      mask_next = __ballot_sync(0xffffffffu, reset_flag(p, b, c, lane)) & 0xffffu;
-    }
-    // the flag of the chunk staged next is loaded one iteration before its ballot, off the critical path
+    // prologue: stage the last chunk and fetch its reset flags
+    stage<T>(p, tm, sm, unit, b, h, nc - 1, nc, ktid);
+    mask_next = __ballot_sync(0xffffffffu, reset_flag(p, b, nc - 1, lane)) & 0xffffu;
     bool f_prev = reset_flag(p, b, nc - 2, lane);
     cta_sync();
     for (int64_t it = 0; it <= nc; ++it) {
       const int64_t c = nc - 1 - it;   // chunk whose context is built now
       if (c >= 0 && pending && !timed_out) {   // (an unsafe chunk stages nothing more: the unit stops)
-        BCtx& cx = sm.ctx[c & 1];
+        Ctx<T>& cx = sm.ctx[c & 1];
         const unsigned mask = mask_next;
         bool unsafe = false;
-        build_context<T>(p, sm, cx, mask, s0rows, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, unsafe,
-                         timed_out);
+        context_operands<T>(p, sm, cx, mask, unit, c, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, tmem,
+                            unsafe, timed_out);
         if (!timed_out) {
           pending = false;
           ++phase;
         }
-        // the staged inputs and entering state are consumed: prefetch the previous chunk
+        // the staged inputs and checkpoint are consumed: prefetch the previous chunk
         if (c > 0 && !unsafe) {
-          const int64_t tp = (c - 1) * kChunk;
-          stage7<T>(p, tm, sm, b, h, tp, ktid);
+          stage<T>(p, tm, sm, unit, b, h, c - 1, nc, ktid);
           pending = true;
-          load_entry_rows(p, unit, nc, c - 1, ktid, s0rows);
           mask_next = __ballot_sync(0xffffffffu, f_prev) & 0xffffu;   // chunk c-1
           f_prev = reset_flag(p, b, c - 2, lane);
         }
-        if (!unsafe) finish_context<T>(sm, cx, mask, ktid);
+        if (!unsafe) {
+          context_products<T>(p, sm, cx, mask, ktid, tmem, cphase);
+          ++cphase;
+        }
       }
       cta_sync();
       if (sm.stop) break;
@@ -774,11 +855,16 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_bwd_kernel(const BwdArgs p,
     // copies issued but never waited for (the unit stopped early) must land before the CTA exits
     if (pending) mbar_wait_bounded(&sm.in_bar, phase & 1u, timed_out ? kWaitLimitNs / 100 : kWaitLimitNs);
   }
+  // every MMA was waited for and every TMEM load is complete: release TMEM
+  tc::fence_before_sync();
+  cta_sync();
+  tc::fence_after_sync();
+  if (warp == 0) tc::dealloc(tmem, kTmemCols);
 }
 
 template <typename T>
 cudaError_t launch(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
-  const size_t smem = sizeof(BwdSmem2<T>);
+  const size_t smem = sizeof(BwdSmem<T>);
   cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
   chunk_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
@@ -789,10 +875,9 @@ cudaError_t launch(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
 
 cudaError_t launch_chunk_bwd(const BwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream) {
   switch (dtype) {
-    case 0: return launch<float>(p, tm, stream);
     case 1: return launch<__nv_bfloat16>(p, tm, stream);
     case 2: return launch<__half>(p, tm, stream);
-    default: return cudaErrorInvalidValue;
+    default: return cudaErrorInvalidValue;   // f32 inputs run the exact scan backward
   }
 }
 

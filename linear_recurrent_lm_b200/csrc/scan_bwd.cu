@@ -16,10 +16,13 @@
 //      s0, or zero after a reset), keeping sa_t for every token in shared
 //      memory and ending with the segment's last state; then
 //   B) walked backwards, rebuilding P_t = (S_t - sa_t b^T - v k^T) diag(1/w)
-//      one token at a time.  When the decay product over the segment is so
-//      small that this division would amplify rounding by more than 2^16,
-//      P_t is instead recomputed forward from the entering state with the
-//      stored sa (exact, quadratic in the segment length).
+//      one token at a time.  Step A also keeps the states entering tokens
+//      4, 8 and 12 of the segment in shared memory, and the walk restarts from
+//      them, so no chain of divisions is longer than three tokens (rounding
+//      grows by at most prod(1/w) over three tokens).  When the decay product
+//      over the segment is so small that the divisions could amplify rounding
+//      by more than 2^16, P_t is instead recomputed forward from the entering
+//      state with the stored sa (exact, quadratic in the segment length).
 //
 // One CTA per (b,h), 256 threads: thread (q, j) holds rows 16q..16q+15 of
 // column j of S, P and D, so the five column reductions of the backward
@@ -38,9 +41,12 @@ constexpr int kThreads = 256;
 constexpr int kIn = 7;               // r, w, k, v, a, b, dy
 constexpr float kMaxGrowth = 65536.f;  // largest tolerated prod(1/w) over a segment
 
+constexpr int kSub = 4;               // tokens between the states kept by step A
+
 struct BwdSmem {
   float x[kIn][kChunk][kN];
   float sa[kChunk][kN];
+  float sub[kChunk / kSub - 1][kN][kN];   // states entering tokens 4, 8, 12 of a segment [row][column]
   float row_red[2][2][kN];     // [column half][quantity][row]
   float col_red[5][4][kN];     // [quantity][row quarter][column]
   int flags[kChunk];
@@ -158,6 +164,11 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
           S[ii] = fmaf(S[ii], wj, fmaf(sa, bj, sm.x[3][tt][row] * kj));
         }
         if (tt > seg_start) growth *= 1.f / wj;
+        const int next = tt + 1 - seg_start;   // the state in S enters token tt + 1
+        if (next % kSub == 0 && tt + 1 < seg_end) {
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) sm.sub[next / kSub - 1][q * 16 + ii][j] = S[ii];
+        }
         __syncthreads();
       }
       // prod(1/w) over the tokens whose entering state is rebuilt by division
@@ -172,6 +183,9 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
         if (tt == seg_start) {
 #pragma unroll
           for (int ii = 0; ii < 16; ++ii) P[ii] = zero_entry ? 0.f : E[ii];
+        } else if (!unstable && (tt - seg_start) % kSub == 0) {   // kept by step A
+#pragma unroll
+          for (int ii = 0; ii < 16; ++ii) P[ii] = sm.sub[(tt - seg_start) / kSub - 1][q * 16 + ii][j];
         } else if (!unstable) {
           const float iw = 1.f / wj;
 #pragma unroll

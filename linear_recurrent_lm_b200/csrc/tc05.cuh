@@ -93,6 +93,86 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
          | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
+// Shared-memory matrix descriptor with explicit leading and stride byte offsets (no swizzle).  For a
+// K-major operand LBO is the distance between K-adjacent core matrices and SBO between M/N-adjacent
+// 8-row groups; for an MN-major one (16-bit types only: tf32 operands must be K-major) SBO is the
+// distance between M/N-adjacent core matrices and LBO between K-adjacent 8-row groups.
+__device__ __forceinline__ uint64_t smem_desc2(const void* start, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  const uint64_t addr = smem_u32addr(start);
+  return ((addr >> 4) & 0x3FFFull) | ((uint64_t(lbo_bytes >> 4) & 0x3FFFull) << 16) |
+         ((uint64_t(sbo_bytes >> 4) & 0x3FFFull) << 32) | (uint64_t(1) << 46);
+}
+
+// Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulate, and the major-ness of A
+// and B (0 = K-major, 1 = MN-major).
+__host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, int a_mn, int b_mn) {
+  return (1u << 4)                      // D format: f32
+         | (1u << 7)                    // A format: bf16
+         | (1u << 10)                   // B format: bf16
+         | (uint32_t(a_mn) << 15) | (uint32_t(b_mn) << 16)
+         | (uint32_t(N >> 3) << 17)     // N / 8
+         | (uint32_t(M >> 4) << 24);    // M / 16
+}
+// D[tmem] (+)= A[smem desc] * B[smem desc], kind::f16 (K = 16 per MMA)
+__device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         bool accumulate) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, {%5, %5, %5, %5}, p;\n}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate ? 1u : 0u), "r"(0u)
+      : "memory");
+}
+
+// ---- 32x32b register <-> TMEM moves: thread l of warp w reaches lane 32 (w % 4) + l; register r is
+// column base + r.
+__device__ __forceinline__ void ld_32x32b_x16(uint32_t taddr, float (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16];"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+        "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void st_32x32b_x16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15, %16};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+      : "memory");
+}
+
+// ---- 16x32bx2 register <-> TMEM moves for M = 64 accumulators (rows in lanes 0-15 of the warp's
+// quadrant): thread l < 16 reaches row l, columns base .. base+15; thread l >= 16 reaches row l - 16,
+// columns base+16 .. base+31, so that all 32 threads of the warp share the 16 rows.
+__device__ __forceinline__ void ld_16x32bx2_x16(uint32_t taddr, float (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+      "%15}, [%16], 16;"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7]), "=f"(v[8]),
+        "=f"(v[9]), "=f"(v[10]), "=f"(v[11]), "=f"(v[12]), "=f"(v[13]), "=f"(v[14]), "=f"(v[15])
+      : "r"(taddr)
+      : "memory");
+}
+__device__ __forceinline__ void st_16x32bx2_x16(uint32_t taddr, const float (&v)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.16x32bx2.x16.b32 [%0], 16, {%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, "
+      "%14, %15, %16};" ::"r"(taddr),
+      "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]), "f"(v[8]), "f"(v[9]),
+      "f"(v[10]), "f"(v[11]), "f"(v[12]), "f"(v[13]), "f"(v[14]), "f"(v[15])
+      : "memory");
+}
+// Same with 8 columns per half: thread l < 16 reaches columns base .. base+7 of row l, thread l >= 16
+// columns base+8 .. base+15 of row l - 16.
+__device__ __forceinline__ void ld_16x32bx2_x8(uint32_t taddr, float (&v)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.16x32bx2.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8], 8;"
+      : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3]), "=f"(v[4]), "=f"(v[5]), "=f"(v[6]), "=f"(v[7])
+      : "r"(taddr)
+      : "memory");
+}
+
 // ---- MMA issue (one thread) and completion
 // D[tmem] (+)= A[smem desc] * B[smem desc]; no output lane is disabled
 __device__ __forceinline__ void mma_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,

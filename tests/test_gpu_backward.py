@@ -1,4 +1,10 @@
-"""GPU backward parity against the CPU oracle's hand-derived reverse mode."""
+"""GPU backward parity against the CPU oracle's hand-derived reverse mode.
+
+Every gradient and dS0 is held element by element: max|gpu - oracle| / RMS(oracle) after the
+half-ulp that storing the result in the output dtype costs (``err_rms_excess``) must stay within the
+bound of the input dtype (f32 1e-4, bf16 2e-2, f16 5e-3), and the fp64 cosine of each whole tensor
+must reach 0.999.  The full-size packed batch is compared on all of its (b,h) units.
+"""
 from __future__ import annotations
 
 import numpy as np
@@ -6,12 +12,13 @@ import pytest
 
 import oracle
 from linear_recurrent_lm_b200 import inputs as I
-from tests.gpu_util import f64, inputs_dev, inputs_f64, sample_units, to_dev
-from tests.metrics import cosine
+from tests.gpu_util import f64, inputs_dev, inputs_f64, to_dev
+from tests.metrics import cosine, err_rms, err_rms_excess
 
 pytestmark = pytest.mark.gpu
 
 GRADS = ("dr", "dw", "dk", "dv", "da", "db")
+TOL = {"f32": 1e-4, "bf16": 2e-2, "f16": 5e-3}
 COS = 0.999
 
 
@@ -32,15 +39,23 @@ def fwd_bwd(W, d, dy, s0=None, reset=None, dsT=None, algo="auto"):
     return y, s, g
 
 
-def check_grads(g, go, sl=slice(None)):
+def grad_errors(g, go, dtype):
+    """{name: (err_rms_excess, cosine)} for the six gradients (output dtype) and dS0 (fp32)."""
     out = {}
     for n in GRADS:
-        out[n] = cosine(f64(g[n])[sl], go[n])
-    if "ds0" in go and g.get("ds0") is not None:
-        out["ds0"] = cosine(f64(g["ds0"])[sl[:1] + sl[2:3] if isinstance(sl, tuple) else sl], go["ds0"])
-    bad = {k: v for k, v in out.items() if not v >= COS}
-    assert not bad, bad
+        x = f64(g[n])
+        out[n] = (err_rms_excess(x, go[n], dtype), cosine(x, go[n]))
+    if g.get("ds0") is not None and "ds0" in go:
+        x = f64(g["ds0"])
+        out["ds0"] = (err_rms(x, go["ds0"]), cosine(x, go["ds0"]))
     return out
+
+
+def check_grads(g, go, dtype, where=""):
+    errs = grad_errors(g, go, dtype)
+    bad = {n: e for n, e in errs.items() if not (e[0] <= TOL[dtype] and e[1] >= COS)}
+    assert not bad, (where, bad)
+    return errs
 
 
 @pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
@@ -49,25 +64,32 @@ def test_config1_fwd_bwd(W, algo):
     wl = I.make_workload(1)
     _, _, g = fwd_bwd(W, wl.inputs, wl.dy, algo=algo)
     go, _ = oracle.backward(*inputs_f64(wl.inputs), I.to_f64(wl.dy))
-    check_grads(g, go)
+    check_grads(g, go, "bf16", algo)
 
 
-@pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
-def test_config3_full_size_sampled_units(W, algo):
-    """B=8, T=4096, H=32 packed documents with resets, gradients of sampled units."""
+@pytest.fixture(scope="module")
+def config3_oracle():
+    """Workload 3 (B=8, T=4096, H=32, packed documents): the oracle's gradients of every unit."""
     wl = I.make_workload(3)
+    go, _ = oracle.backward(*inputs_f64(wl.inputs), I.to_f64(wl.dy), reset=wl.reset)
+    return wl, go
+
+
+@pytest.mark.parametrize("algo", ("chunked_fused", "chunked_split", "scan"))
+def test_config3_full_size_all_units(W, config3_oracle, algo):
+    """B=8, T=4096, H=32 packed documents with resets: all 256 (b,h) units, every element."""
+    wl, go = config3_oracle
     _, _, g = fwd_bwd(W, wl.inputs, wl.dy, reset=wl.reset, algo=algo)
-    gg = {n: f64(g[n]) for n in GRADS}
-    for (b, h) in sample_units(8, 32, 6, seed=4):
-        part = {n: wl.inputs[n][b:b + 1, :, h:h + 1] for n in I.NAMES}
-        go, _ = oracle.backward(*inputs_f64(part), I.to_f64(wl.dy[b:b + 1, :, h:h + 1]), reset=wl.reset[b:b + 1])
-        for n in GRADS:
-            c = cosine(gg[n][b:b + 1, :, h:h + 1], go[n])
-            assert c >= COS, ((b, h), n, c)
+    errs = check_grads(g, go, "bf16", algo)
+    print(f"config3 {algo}: " + ", ".join(f"{n} {e[0]:.4f}/{e[1]:.6f}" for n, e in errs.items()))
 
 
-@pytest.mark.parametrize("algo,dtype", [(a, dt) for a in ("scan", "chunked_fused", "chunked_split")
-                                         for dt in ("f32", "bf16", "f16") if not (dt == "f32" and a != "scan")])
+def _ragged_cases():
+    return [(a, dt) for a in ("scan", "chunked_fused", "chunked_split")
+            for dt in ("f32", "bf16", "f16") if not (dt == "f32" and a != "scan")]
+
+
+@pytest.mark.parametrize("algo,dtype", _ragged_cases())
 @pytest.mark.parametrize("T", [1, 15, 17, 40, 100])
 def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
     rng = np.random.default_rng(100 + T)
@@ -83,16 +105,15 @@ def test_ragged_with_state_resets_and_dsT(W, algo, dtype, T):
             reset[0, t] = 1
     _, _, g = fwd_bwd(W, d, dy, s0=s0, reset=reset, dsT=dsT, algo=algo)
     go, _ = oracle.backward(*inputs_f64(d), I.to_f64(dy), s0=s0, reset=reset, dsT=dsT)
-    for n in GRADS + ("ds0",):
-        c = cosine(f64(g[n]), go[n])
-        assert c >= COS, (n, c)
+    check_grads(g, go, dtype, (algo, dtype, T))
     # row 1 is reset at t=0: nothing reaches s0
     assert np.all(f64(g["ds0"])[1] == 0.0)
 
 
 @pytest.mark.parametrize("algo", ("scan", "chunked_fused", "chunked_split"))
 def test_small_decay_segments(W, algo):
-    """Decays far below the generator's range (prod w < 2^-16 over a chunk) and w = 0."""
+    """Decays far below the generator's range (prod w < 2^-16 over a chunk) and w = 0: the chunked
+    backward hands those heads to the exact scan, whose results must still hold the bound."""
     rng = np.random.default_rng(7)
     dt = "f32" if algo == "scan" else "bf16"
     d = I.draw_inputs(rng, (1, 64, 2, 64), dt)
@@ -103,9 +124,7 @@ def test_small_decay_segments(W, algo):
     dy = I.to_storage(rng.standard_normal((1, 64, 2, 64)), dt)
     _, _, g = fwd_bwd(W, d, dy, algo=algo)
     go, _ = oracle.backward(*inputs_f64(d), I.to_f64(dy))
-    for n in GRADS + ("ds0",):
-        c = cosine(f64(g[n]), go[n])
-        assert c >= COS, (n, c)
+    check_grads(g, go, dt, algo)
 
 
 def test_flagged_and_chunked_heads_in_one_batch(W):
@@ -127,17 +146,18 @@ def test_flagged_and_chunked_heads_in_one_batch(W):
     _, _, g = fwd_bwd(W, d, dy, s0=s0, reset=reset, dsT=dsT)
     go, _ = oracle.backward(*inputs_f64(d), I.to_f64(dy), s0=s0.astype(np.float64), reset=reset,
                             dsT=dsT.astype(np.float64))
+    check_grads(g, go, "bf16")
     for b in range(B):
         for h in range(H):
             for n in GRADS:
-                c = cosine(f64(g[n])[b, :, h], go[n][b, :, h])
-                assert c >= COS, (b, h, n, c)
-            c = cosine(f64(g["ds0"])[b, h], go["ds0"][b, h])
-            assert c >= COS, (b, h, "ds0", c)
+                assert cosine(f64(g[n])[b, :, h], go[n][b, :, h]) >= COS, (b, h, n)
+            assert cosine(f64(g["ds0"])[b, h], go["ds0"][b, h]) >= COS, (b, h, "ds0")
 
 
 def test_backward_chaining(W):
-    """dS0 of the second half fed as dS_T of the first equals one backward over the whole row."""
+    """dS0 of the second half fed as dS_T of the first equals one backward over the whole row, bit for
+    bit: the split falls on a chunk boundary, so both run the same arithmetic on the same fp32 state
+    and carried gradient."""
     import torch
     wl = I.make_workload(1, B=1, T=96, H=2)
     xs = inputs_dev(wl.inputs)
@@ -152,7 +172,7 @@ def test_backward_chaining(W):
     g1 = W.backward(*first, dy[:, :48].contiguous(), ws1, dsT=g2["ds0"])
     for n in GRADS:
         joined = torch.cat([g1[n], g2[n]], dim=1)
-        assert cosine(f64(joined), f64(g[n])) >= 0.99999, n
+        assert torch.equal(joined, g[n]), n
 
 
 def test_backward_is_deterministic(W):

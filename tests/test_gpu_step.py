@@ -21,11 +21,12 @@ def W():
 
 
 def test_config4_ragged_decode(W):
+    """All 256 rows x 32 heads, 128 ragged steps: y of every step and the final states against the
+    oracle stepped alongside; padded rows keep their state bit for bit and get y = 0."""
     import torch
     wl = I.make_workload(4)
     state = to_dev(wl.state0)
-    sample = np.array(sorted({0, 1, 77, 128, 200, 255}))
-    st_o = wl.state0[sample].astype(np.float64)
+    st_o = wl.state0.astype(np.float64)
     max_ey = 0.0
     for s, step_in in enumerate(wl.steps):
         act = wl.active(s)
@@ -35,10 +36,12 @@ def test_config4_ragged_decode(W):
         # padded rows: state bitwise unchanged, y = 0
         assert torch.equal(state[inactive], before[inactive])
         assert torch.count_nonzero(y[inactive]) == 0
-        yo, st_o = oracle.step(*(I.to_f64(step_in[n][sample]) for n in I.NAMES), st_o, act[sample])
-        max_ey = max(max_ey, err_rms_excess(f64(y)[sample], yo, "bf16"))
+        yo, st_o = oracle.step(*(I.to_f64(step_in[n]) for n in I.NAMES), st_o, act)
+        max_ey = max(max_ey, err_rms_excess(f64(y), yo, "bf16"))
+    es = err_rms(f64(state), st_o)
+    print(f"decode: y {max_ey:.5f}, state {es:.2e}")
     assert max_ey <= 2e-2
-    assert err_rms(f64(state)[sample], st_o) <= 2e-2
+    assert es <= 2e-2
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16", "f16"])
