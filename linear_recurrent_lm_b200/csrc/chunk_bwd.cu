@@ -71,8 +71,6 @@ using bf16 = __nv_bfloat16;
 
 // TMEM columns (512 allocated: one CTA per SM).  Every accumulator has M = 64 rows.
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColGram = 0;    // context: [At; Rt] [Bh; Kh]^T  (32; rows t)
-constexpr uint32_t kColSA = 32;     // context: SA^T                  (16; rows i)
 constexpr uint32_t kColDS = 64;     // main: dS^T                     (64; rows j)
 constexpr uint32_t kColG1 = 128;    // main: dSl [Bh|Kh]^T            (32; rows i)
 constexpr uint32_t kColG2 = 160;    // main: dY^T [Mrb|Mrk]           (32; rows i)
@@ -115,6 +113,55 @@ __device__ __forceinline__ void get8(const Split<P, Q>& m, int e, float (&x)[8])
     const float2 c = __bfloat1622float2(*reinterpret_cast<const __nv_bfloat162*>(&lw[u]));
     x[2 * u] = a.x + c.x;
     x[2 * u + 1] = a.y + c.y;
+  }
+}
+
+// ---- warp-level products (mma.sync m16n8k16, bf16 in, fp32 accumulate) on split core arrays.
+// ldmatrix reads one 8x8 tile of a core array as 8 rows of 16 bytes; lane l supplies the row address
+// of tile l / 8.
+// A fragment (16 rows x 16 k) of a K-major core array (rows = M, columns = K) at (m0, k0).
+template <int Q>
+__device__ __forceinline__ uint32_t afrag_k(const bf16* a, int m0, int k0, int lane) {
+  const int mi = lane >> 3, r = lane & 7;
+  return smem_u32(a + cb(m0 + (mi & 1) * 8 + r, k0 + (mi >> 1) * 8, Q));
+}
+// A fragment of a matrix stored transposed (rows = K, columns = M), read with ldmatrix.trans.
+template <int Q>
+__device__ __forceinline__ uint32_t afrag_mn(const bf16* a, int m0, int k0, int lane) {
+  const int mi = lane >> 3, r = lane & 7;
+  return smem_u32(a + cb(k0 + (mi >> 1) * 8 + r, m0 + (mi & 1) * 8, Q));
+}
+// B fragments of two n-tiles (n0..n0+15) x 16 k from a core array with rows = N, columns = K.
+template <int Q>
+__device__ __forceinline__ uint32_t bfrag_k(const bf16* b, int n0, int k0, int lane) {
+  const int mi = lane >> 3, r = lane & 7;
+  return smem_u32(b + cb(n0 + (mi >> 1) * 8 + r, k0 + (mi & 1) * 8, Q));
+}
+__device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+__device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
+}
+// acc[nt] (+)= A B over one K step of 16 for two n-tiles, with split operands: hi.hi + hi.lo + lo.hi.
+// The lo addresses are the hi ones plus a fixed byte distance; a_exact skips the A lo half.
+__device__ __forceinline__ void mma_split2(float (&acc)[2][4], uint32_t a_hi, uint32_t a_lo_off, bool a_mn,
+                                           bool a_exact, uint32_t b_hi, uint32_t b_lo_off) {
+  uint32_t ah[4], al[4], bh[4], bl[4];
+  if (a_mn) ldsm4t(ah, a_hi); else ldsm4(ah, a_hi);
+  ldsm4(bh, b_hi);
+  ldsm4(bl, b_hi + b_lo_off);
+#pragma unroll
+  for (int nt = 0; nt < 2; ++nt) {
+    mma16816(acc[nt], ah, bh[2 * nt], bh[2 * nt + 1]);
+    mma16816(acc[nt], ah, bl[2 * nt], bl[2 * nt + 1]);
+  }
+  if (!a_exact) {
+    if (a_mn) ldsm4t(al, a_hi + a_lo_off); else ldsm4(al, a_hi + a_lo_off);
+#pragma unroll
+    for (int nt = 0; nt < 2; ++nt) mma16816(acc[nt], al, bh[2 * nt], bh[2 * nt + 1]);
   }
 }
 
@@ -191,7 +238,6 @@ struct __align__(128) BwdSmem {
   __align__(128) float ck[kN * kN];         // checkpoint entering the chunk being built (tiled order)
   __align__(128) T stg[kIn][kChunk][kN];    // staged inputs of the chunk being built (TMA boxes)
   unsigned long long in_bar;                // staged inputs and checkpoint landed (one phase per staged chunk)
-  unsigned long long gram_bar, sa_bar;      // context MMAs complete (one phase per chunk each)
   unsigned long long u_bar, chain_bar, gg_bar, e_bar;   // main MMAs complete (one phase per chunk each)
   uint32_t tmem_base;
   int kbad[4];
@@ -250,7 +296,7 @@ __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, Bwd
 template <typename T>
 __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
                                                  int64_t unit, int64_t c, int ktid, int len, unsigned parity,
-                                                 uint32_t tmem, bool& unsafe, bool& timed_out) {
+                                                 bool& unsafe, bool& timed_out) {
   const int kw = ktid >> 5, lane = ktid & 31;
   const bool to = !mbar_wait_bounded(&sm.in_bar, parity, kWaitLimitNs);
   const T (*X)[kChunk][kN] = sm.stg;
@@ -328,13 +374,6 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
   const int kb = sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3];
   unsafe = kb != 0;
   timed_out = (kb & 2) != 0;
-  // ---- the Gram [At; Rt] [Bh; Kh]^T runs on the tensor core while S0^T is built (M = 64: rows
-  // 32-63 read the arrays that follow and are unused)
-  if (!unsafe && ktid == 0) {
-    tc::fence_after_sync();
-    mma3<32, 4>(tmem + kColGram, op<64, false>(cx.AR), op<64, false>(cx.BK), false);
-    tc::commit(&sm.gram_bar);
-  }
   // ---- pass C: S0^T [j][i] from the checkpoint (tiled order), s0 or zero; thread = 4 x (j, 8 i)
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -365,47 +404,44 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
 
 // The rest of the context: Gram, T, W, X and SA^T (safe chunks only).
 template <typename T>
-__device__ __forceinline__ void context_products(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
-                                                 int ktid, uint32_t tmem, unsigned phase) {
+__device__ __forceinline__ void context_products(BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask, int ktid) {
   constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
   const int kw = ktid >> 5, lane = ktid & 31;
-  const uint32_t tlane = uint32_t(32 * kw) << 16;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
 
-  // ---- the masked Gram (issued with the operands)
-  mma_wait(p, &sm.gram_bar, phase & 1u);
-  if (kw < 2) {   // warp 0: rows t of [Lab | Lak]; warp 1: rows t of [Mrb | Mrk] (lanes 0-15)
-    float g0[16], g1[16];
-    tc::ld_32x32b_x16(tmem + tlane + kColGram, g0);
-    tc::ld_32x32b_x16(tmem + tlane + kColGram + 16, g1);
-    tc::wait_ld();
-    const int t = lane;
-    if (t < kChunk) {
-      const bool strict = kw == 0;
+  // ---- the masked Gram [At; Rt] [Bh; Kh]^T: warp kw computes block (kw / 2, kw % 2) of 16 x 16
+  // (Lab, Lak, Mrb, Mrk), rows t, columns tau
+  {
+    const int mb = kw >> 1, nb = kw & 1, g = lane >> 2, c4 = lane & 3;
+    float acc[2][4] = {};
+    const uint32_t a_lo = uint32_t(sizeof(cx.AR.hi)), b_lo = uint32_t(sizeof(cx.BK.hi));
 #pragma unroll
-      for (int tau = 0; tau < kChunk; ++tau) {
-        const bool ok = pair_ok(mask, t, tau, strict);
-        g0[tau] = ok ? g0[tau] : 0.f;
-        g1[tau] = ok ? g1[tau] : 0.f;
-      }
-      if (kw == 0) {
+    for (int ks = 0; ks < 4; ++ks)
+      mma_split2(acc, afrag_k<64>(cx.AR.hi, 16 * mb, 16 * ks, lane), a_lo, false, false,
+                 bfrag_k<64>(cx.BK.hi, 16 * nb, 16 * ks, lane), b_lo);
+    const bool strict = mb == 0;
 #pragma unroll
-        for (int tau = 0; tau < kChunk; ++tau) {
-          sm.LabT[tau][t] = g0[tau];
-          cx.LakP[t][tau] = g1[tau];
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int t = g + 8 * hh, tau = 8 * nt + 2 * c4;
+        const float v0 = pair_ok(mask, t, tau, strict) ? acc[nt][2 * hh] : 0.f;
+        const float v1 = pair_ok(mask, t, tau + 1, strict) ? acc[nt][2 * hh + 1] : 0.f;
+        if (kw == 0) {
+          sm.LabT[tau][t] = v0;
+          sm.LabT[tau + 1][t] = v1;
+        } else if (kw == 1) {
+          cx.LakP[t][tau] = v0;
+          cx.LakP[t][tau + 1] = v1;
+        } else {   // [Mrb | Mrk] row t: a split pair
+          const int e = cb(t, 16 * nb + tau, 32);
+          const __nv_bfloat162 hh2 = __floats2bfloat162_rn(v0, v1);
+          const float2 hf = __bfloat1622float2(hh2);
+          *reinterpret_cast<__nv_bfloat162*>(&cx.MM.hi[e]) = hh2;
+          *reinterpret_cast<__nv_bfloat162*>(&cx.MM.lo[e]) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
         }
-      } else {   // [Mrb | Mrk] row t: four 16-byte core rows
-        float v[8];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) v[e] = q < 2 ? g0[8 * q + e] : g1[8 * (q - 2) + e];
-          put8(cx.MM, cb(t, 8 * q, 32), v);
-        }
       }
-    }
   }
-  tc::fence_before_sync();
   named_bar(1, 128);
 
   // ---- T = (I - Lab)^-1 by forward substitution, one column per thread (threads 0-15)
@@ -454,31 +490,30 @@ __device__ __forceinline__ void context_products(const BwdArgs& p, BwdSmem<T>& s
   tc::fence_before_sync();
   named_bar(1, 128);
 
-  // ---- SA^T = S0 W^T + V^T X^T  (A: S0^T and v read MN-major, rows i)
-  if (ktid == 0) {
-    tc::fence_after_sync();
-    mma3<16, 4>(tmem + kColSA, op<64, true>(cx.S0T), op<64, false>(sm.WC), false);
-    mma3<16, 1>(tmem + kColSA, op<32, false>(cx.SV, kExactIn, 0, 16), op<16, false>(sm.XC), true);   // v^T half of SV
-    tc::commit(&sm.sa_bar);
-  }
-  mma_wait(p, &sm.sa_bar, phase & 1u);
+  // ---- SA^T = S0 W^T + V^T X^T: warp kw computes rows i = 16 kw .. 16 kw + 15, columns tau
   {
-    float sa[16];
-    tc::ld_32x32b_x16(tmem + tlane + kColSA, sa);
-    tc::wait_ld();
-    if (lane < 16) {
-      const int i = 16 * kw + lane;
-      float v[8];
+    const int g = lane >> 2, c4 = lane & 3;
+    float acc[2][4] = {};
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
+    for (int ks = 0; ks < 4; ++ks)   // S0 (stored as S0^T) times W^T, K = j
+      mma_split2(acc, afrag_mn<64>(cx.S0T.hi, 16 * kw, 16 * ks, lane), uint32_t(sizeof(cx.S0T.hi)), true, false,
+                 bfrag_k<64>(sm.WC.hi, 0, 16 * ks, lane), uint32_t(sizeof(sm.WC.hi)));
+    mma_split2(acc, afrag_k<32>(cx.SV.hi, 16 * kw, 16, lane), uint32_t(sizeof(cx.SV.hi)), false, kExactIn,   // v^T X^T, K = t
+               bfrag_k<16>(sm.XC.hi, 0, 0, lane), uint32_t(sizeof(sm.XC.hi)));
 #pragma unroll
-        for (int e = 0; e < 8; ++e) v[e] = sa[8 * q + e];
-        put8(cx.SV, cb(i, 8 * q, 32), v);
+    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        const int i = 16 * kw + g + 8 * hh, tau = 8 * nt + 2 * c4;
+        const int e = cb(i, tau, 32);
+        const float v0 = acc[nt][2 * hh], v1 = acc[nt][2 * hh + 1];
+        const __nv_bfloat162 hh2 = __floats2bfloat162_rn(v0, v1);
+        const float2 hf = __bfloat1622float2(hh2);
+        *reinterpret_cast<__nv_bfloat162*>(&cx.SV.hi[e]) = hh2;
+        *reinterpret_cast<__nv_bfloat162*>(&cx.SV.lo[e]) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
       }
-    }
   }
   tc::fence_smem_to_async();
-  tc::fence_before_sync();
 }
 
 // ------------------------------------------------------------------ main warps
@@ -745,8 +780,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   if (tid == 0) {
     sm.stop = 0;
     mbar_init(&sm.in_bar, 1);
-    mbar_init(&sm.gram_bar, 1);
-    mbar_init(&sm.sa_bar, 1);
     mbar_init(&sm.u_bar, 1);
     mbar_init(&sm.chain_bar, 1);
     mbar_init(&sm.gg_bar, 1);
@@ -817,7 +850,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   } else {
     unsigned mask_next;
     unsigned phase = 0;        // staging phase of the next wait
-    unsigned cphase = 0;       // context MMA phase
     bool pending = true;       // a staging was issued and not yet waited for
     bool timed_out = false;
     // prologue: stage the last chunk and fetch its reset flags
@@ -831,8 +863,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         Ctx<T>& cx = sm.ctx[c & 1];
         const unsigned mask = mask_next;
         bool unsafe = false;
-        context_operands<T>(p, sm, cx, mask, unit, c, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, tmem,
-                            unsafe, timed_out);
+        context_operands<T>(p, sm, cx, mask, unit, c, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, unsafe,
+                            timed_out);
         if (!timed_out) {
           pending = false;
           ++phase;
@@ -845,8 +877,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
           f_prev = reset_flag(p, b, c - 2, lane);
         }
         if (!unsafe) {
-          context_products<T>(p, sm, cx, mask, ktid, tmem, cphase);
-          ++cphase;
+          context_products<T>(sm, cx, mask, ktid);
         }
       }
       cta_sync();
