@@ -67,7 +67,8 @@ typedef enum {
   WKV7_ERR_CUDA = 7,        /* the launch failed; cudaGetLastError() was not cudaSuccess      */
   WKV7_ERR_TIMEOUT = 8,     /* reserved for device-side bounded waits                          */
   WKV7_ERR_SCRATCH_LIMIT = 9, /* the problem needs more than WKV7_NOALLOC_SCRATCH_BYTES of scratch */
-  WKV7_ERR_NONFINITE = 10    /* WKV7_FLAG_CHECK_FINITE found a NaN or infinity in an output       */
+  WKV7_ERR_NONFINITE = 10,   /* WKV7_FLAG_CHECK_FINITE found a NaN or infinity in an output       */
+  WKV7_ERR_BOUNDS = 11       /* debug build only: a kernel index failed its bounds check          */
 } wkv7_status_t;
 
 typedef enum { WKV7_F32 = 0, WKV7_BF16 = 1, WKV7_F16 = 2 } wkv7_dtype_t;
@@ -134,15 +135,30 @@ typedef struct {
 /*
  * Device status word (the device-side error channel of the boundary).
  * Kernels record errors they cannot return from an asynchronous launch --
- * a bounded wait that ran out, or a non-finite output found under
- * WKV7_FLAG_CHECK_FINITE -- in one word per device.  This call synchronises
- * the current device, reads the word and, if `clear` is non-zero, resets
- * it.  Returns WKV7_OK, WKV7_ERR_TIMEOUT if a wait ran out since the last
- * clear (this takes precedence), WKV7_ERR_NONFINITE if a checked output
- * held a NaN or infinity, or WKV7_ERR_CUDA if synchronising or reading
- * failed (e.g. no device).
+ * a bounded wait that ran out, a non-finite output found under
+ * WKV7_FLAG_CHECK_FINITE, or (debug build) an index that failed its bounds
+ * check -- in one word per device.  This call synchronises the current
+ * device, reads the word and, if `clear` is non-zero, resets it.  Returns
+ * WKV7_OK; else, in this order of precedence, WKV7_ERR_TIMEOUT if a wait ran
+ * out since the last clear, WKV7_ERR_BOUNDS if a checked index fell outside
+ * its buffer (the access was skipped), WKV7_ERR_NONFINITE if a checked
+ * output held a NaN or infinity; or WKV7_ERR_CUDA if synchronising or
+ * reading failed (e.g. no device).
  */
 wkv7_status_t wkv7_get_device_status(int clear);
+
+/*
+ * 1 in the debug build of this library (libwkv7_debug.so, compiled with
+ * WKV7_DEBUG), 0 in the release build (libwkv7.so).  The debug build is the
+ * same ABI and the same arithmetic; its kernels also check every index they
+ * compute -- global offsets of activations, states, checkpoints and
+ * workspace marks, TMA box coordinates, bulk-copy ranges and shared-memory
+ * operand indices -- against the extent of its buffer, skip an access that
+ * fails and set WKV7_ERR_BOUNDS in the device status word instead of
+ * faulting.  Results of a run with no failed check are bit-identical to the
+ * release build's.
+ */
+int wkv7_debug_checks(void);
 
 /* Library version, major*10000 + minor*100 + patch. */
 int wkv7_version(void);

@@ -80,6 +80,15 @@ constexpr uint32_t kColE = 256;     // main: dAt^T | dRt^T | dBg^T | dKg^T | (SA
 // bf16 index of element (p, q) of a core array with Q columns.
 __device__ __forceinline__ int cb(int p, int q, int Q) { return (p >> 3) * (Q * 8) + (q >> 3) * 64 + (p & 7) * 8 + (q & 7); }
 
+// Device status word of the running launch, for the debug-build bounds checks in helpers that do not
+// see the kernel arguments (set by thread 0 before the first CTA barrier).
+#ifdef WKV7_DEBUG
+__shared__ int* s_dbg_status;
+__device__ __forceinline__ int* debug_status() { return s_dbg_status; }
+#else
+__device__ __forceinline__ int* debug_status() { return nullptr; }
+#endif
+
 // A matrix split in two bf16 core arrays (hi, then lo).
 template <int P, int Q>
 struct Split {
@@ -90,6 +99,10 @@ struct Split {
 // Split 8 fp32 values into one 16-byte row of hi and one of lo at element index e.
 template <int P, int Q>
 __device__ __forceinline__ void put8(Split<P, Q>& m, int e, const float (&x)[8]) {
+  if (kDebugChecks && !(e >= 0 && e + 8 <= P * Q && (e & 7) == 0)) {   // debug build: one whole 16-byte row
+    in_bounds(false, debug_status());
+    return;
+  }
   uint32_t h[4], l[4];
 #pragma unroll
   for (int u = 0; u < 4; ++u) {
@@ -189,6 +202,7 @@ __device__ __forceinline__ Op<Q, MN> op(const Split<P, Q>& m, bool exact = false
 // Store one value as its hi and lo halves at element index e (a single element of a core row).
 template <int P, int Q>
 __device__ __forceinline__ void put1(Split<P, Q>& m, int e, float x) {
+  if (!in_bounds(e >= 0 && e < P * Q, debug_status())) return;
   const bf16 h = __float2bfloat16_rn(x);
   m.hi[e] = h;
   m.lo[e] = __float2bfloat16_rn(x - __bfloat162float(h));
@@ -279,12 +293,14 @@ template <typename T>
 __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, int64_t unit, int64_t b,
                                       int64_t h, int64_t c, int64_t nc, int ktid) {
   if (ktid == 0) {
+    if (!in_bounds(h < p.H && b < p.B && c >= 0 && c < nc && c * kChunk < p.T, p.status)) return;
     const unsigned ck_bytes = c > 0 ? unsigned(kN * kN * sizeof(float)) : 0u;
     mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + ck_bytes + p.extra_tx);
 #pragma unroll
     for (int m = 0; m < kIn; ++m)
       tma_load_4d(&sm.stg[m][0][0], &tm.m[m], 0, int(h), int(c * kChunk), int(b), &sm.in_bar);
-    if (c > 0) bulk_g2s(sm.ck, p.ckpt + (unit * nc + (c - 1)) * kN * kN, ck_bytes, &sm.in_bar);
+    if (c > 0 && range_ok((unit * nc + (c - 1)) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status))
+      bulk_g2s(sm.ck, p.ckpt + (unit * nc + (c - 1)) * kN * kN, ck_bytes, &sm.in_bar);
   }
 }
 
@@ -384,7 +400,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
       const float* src = sm.ck + ckpt_off(i0, j);
 #pragma unroll
       for (int e = 0; e < 8; ++e) s[e] = src[16 * e];
-    } else if (p.s0) {
+    } else if (p.s0 && range_ok((unit * kN + i0) * kN + j, 7 * kN + 1, p.B * p.H * kN * kN, p.status)) {
 #pragma unroll
       for (int e = 0; e < 8; ++e) s[e] = p.s0[(unit * kN + i0 + e) * kN + j];
     } else {
@@ -641,10 +657,11 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
     }
     put8(cx.DUY, cb(i, tb, 32), v);
     T* dvp = static_cast<T*>(p.dv) + tok_off(b, t0 + tb, h, p.T, p.H) + i;
-    const int64_t rs = p.H * kN;
+    const int64_t rs = p.H * kN, total = p.B * p.T * p.H * kN;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
-      if (tb + e < len) *dvp = Elt<T>::from_f32(dv[e]);
+      if (tb + e < len && range_ok(tok_off(b, t0 + tb + e, h, p.T, p.H) + i, 1, total, p.status))
+        *dvp = Elt<T>::from_f32(dv[e]);
       dvp += rs;
     }
   }
@@ -752,7 +769,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
 #pragma unroll
     for (int e = 7; e >= 0; --e) {
       cum += DL[e];
-      if (tb + e < len) {
+      if (tb + e < len && range_ok(o0 + e * rs, 1, p.B * p.T * p.H * kN, p.status)) {
         const int64_t o = o0 + e * rs;
         gda[o] = Elt<T>::from_f32(eA[e] * Lr[e]);
         gdr[o] = Elt<T>::from_f32(eR[e] * Lr[e + 1]);
@@ -778,6 +795,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   const int64_t nc = (p.T + kChunk - 1) / kChunk;
 
   if (tid == 0) {
+#ifdef WKV7_DEBUG
+    s_dbg_status = p.status;
+#endif
     sm.stop = 0;
     mbar_init(&sm.in_bar, 1);
     mbar_init(&sm.u_bar, 1);
@@ -804,7 +824,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
       for (int q4 = 0; q4 < 4; ++q4) {
         float d[16];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) d[e] = (p.dsT && lane < 16) ? p.dsT[(unit * kN + 16 * q4 + e) * kN + j] : 0.f;
+        for (int e = 0; e < 16; ++e)
+          d[e] = (p.dsT && lane < 16 && range_ok((unit * kN + 16 * q4 + e) * kN + j, 1, p.B * p.H * kN * kN, p.status))
+                     ? p.dsT[(unit * kN + 16 * q4 + e) * kN + j] : 0.f;
         tc::st_32x32b_x16(tmem + (uint32_t(32 * warp) << 16) + kColDS + 16 * q4, d);
       }
       tc::wait_st();
@@ -832,7 +854,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         break;
       }
     }
-    if (tid == 0 && p.unit_flags) p.unit_flags[unit] = flagged ? 1 : 0;
+    if (tid == 0 && p.unit_flags && range_ok(unit, 1, p.B * p.H, p.status)) p.unit_flags[unit] = flagged ? 1 : 0;
     if (!flagged && p.ds0) {   // every MMA of the last chunk completed before its e_bar phase
       tc::fence_after_sync();
       const int j = 16 * warp + lane;
@@ -841,7 +863,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         float d[16];
         tc::ld_32x32b_x16(tmem + (uint32_t(32 * warp) << 16) + kColDS + 16 * q4, d);
         tc::wait_ld();
-        if (lane < 16) {
+        if (lane < 16 && range_ok((unit * kN + 16 * q4) * kN + j, 15 * kN + 1, p.B * p.H * kN * kN, p.status)) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) p.ds0[(unit * kN + 16 * q4 + e) * kN + j] = d[e];
         }
@@ -892,6 +914,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   tc::fence_after_sync();
   if (warp == 0) tc::dealloc(tmem, kTmemCols);
 }
+
+// One CTA per SM: the whole shared memory of an SM (227 KB per CTA at most, static part included).
+static_assert(sizeof(BwdSmem<__nv_bfloat16>) + 1024 <= 227 * 1024, "backward shared memory exceeds one SM");
 
 template <typename T>
 cudaError_t launch(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {

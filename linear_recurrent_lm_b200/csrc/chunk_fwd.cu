@@ -143,6 +143,7 @@ template <typename T>
 __device__ __forceinline__ void stage_chunk(const FwdArgs& p, const InputMaps& tm, FwdSmem3<T>& sm, int64_t b,
                                             int64_t h, int64_t t0, int ktid) {
   if (ktid == 0) {
+    if (!in_bounds(h < p.H && b < p.B && t0 >= 0 && t0 < p.T, p.status)) return;   // (debug build)
     mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + p.extra_tx);
 #pragma unroll
     for (int m = 0; m < kIn; ++m) tma_load_4d(&sm.in[m][0][0], &tm.m[m], 0, int(h), int(t0), int(b), &sm.in_bar);
@@ -495,7 +496,8 @@ __device__ __forceinline__ void state_chunk(const FwdArgs& p, FwdSmem3<T>& sm, c
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int t = 8 * nt + 2 * c4 + (e & 1);
-        if (t < len) y[tok_off(b, t0 + t, h, p.T, p.H) + row0 + g + 8 * (e >> 1)] = Elt<T>::from_f32(yy[nt][e]);
+        const int64_t o = tok_off(b, t0 + t, h, p.T, p.H) + row0 + g + 8 * (e >> 1);
+        if (t < len && range_ok(o, 1, p.B * p.T * p.H * kN, p.status)) y[o] = Elt<T>::from_f32(yy[nt][e]);
       }
   }
 
@@ -546,7 +548,8 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         float2 v2 = make_float2(0.f, 0.f);
-        if (p.s0) v2 = *reinterpret_cast<const float2*>(p.s0 + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4);
+        const int64_t so = (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4;
+        if (p.s0 && range_ok(so, 2, p.B * p.H * kN * kN, p.status)) v2 = *reinterpret_cast<const float2*>(p.s0 + so);
         acc[nt][2 * hh] = v2.x;
         acc[nt][2 * hh + 1] = v2.y;
       }
@@ -579,13 +582,16 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         const int len = int(min64(kChunk, p.T - t0));
         if (!cx.unsafe) {
           state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane, tmem, mma_phase, ck);
-          if (sizeof(T) == 2 && ytt < len) ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
+          if (sizeof(T) == 2 && ytt < len &&
+              range_ok(tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8, 8, p.B * p.T * p.H * kN, p.status))
+            ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
         } else {
           store_ck(ck, acc);
           state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
         }
         // this chunk's end state is checkpointed during the next chunk (or after the loop)
-        ck = p.ckpt ? p.ckpt + (unit * nc + c) * kN * kN + warp * 1024 + lane * 4 : nullptr;
+        ck = p.ckpt && range_ok((unit * nc + c) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status)
+                 ? p.ckpt + (unit * nc + c) * kN * kN + warp * 1024 + lane * 4 : nullptr;
       }
       cta_sync();   // context of chunk it handed over; Ys complete
     }
@@ -599,9 +605,11 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh)
-          *reinterpret_cast<float2*>(p.s_out + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-              make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+        for (int hh = 0; hh < 2; ++hh) {
+          const int64_t so = (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4;
+          if (range_ok(so, 2, p.B * p.H * kN * kN, p.status))
+            *reinterpret_cast<float2*>(p.s_out + so) = make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+        }
     }
   } else {
     // prologue: stage chunk 0 and fetch its reset flags

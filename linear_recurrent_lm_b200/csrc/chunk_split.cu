@@ -98,6 +98,8 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(const FwdArgs p, i
   const int64_t t0 = c * kChunk;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c4 = lane & 3;
+  if (!in_bounds(unit < p.B * p.H && c < nfull && t0 + kChunk <= p.T, p.status)) return;   // (debug build)
+  const int64_t act_total = p.B * p.T * p.H * kN;
 
   // ---- stage the six inputs of the chunk (16 rows of 64 elements each)
   {
@@ -106,8 +108,9 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(const FwdArgs p, i
     for (int idx = tid; idx < kIn * kChunk * kPieces; idx += kThreads) {
       const int m = idx / (kChunk * kPieces), rem = idx - m * (kChunk * kPieces);
       const int t = rem / kPieces, piece = rem - t * kPieces;
-      const T* g0 = static_cast<const T*>(src[m]) + tok_off(b, t0 + t, h, p.T, p.H) + piece * (16 / int(sizeof(T)));
-      cp_async16(&sm.in[m][t][piece * (16 / int(sizeof(T)))], g0);
+      const int64_t o = tok_off(b, t0 + t, h, p.T, p.H) + piece * (16 / int(sizeof(T)));
+      if (range_ok(o, 16 / int(sizeof(T)), act_total, p.status))
+        cp_async16(&sm.in[m][t][piece * (16 / int(sizeof(T)))], static_cast<const T*>(src[m]) + o);
     }
     cp_async_commit();
   }
@@ -371,8 +374,9 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(const FwdArgs p, i
   {
     float4* slot = reinterpret_cast<float4*>(p.ckpt + (unit * nc + c) * (kN * kN));
     const float4* src = reinterpret_cast<const float4*>(sm.out);
+    if (range_ok((unit * nc + c) * (kN * kN), kN * kN, p.B * p.H * nc * (kN * kN), p.status))
 #pragma unroll
-    for (int u = 0; u < 4096 / 4 / kThreads; ++u) slot[tid + u * kThreads] = src[tid + u * kThreads];
+      for (int u = 0; u < 4096 / 4 / kThreads; ++u) slot[tid + u * kThreads] = src[tid + u * kThreads];
     const int t = tid >> 3, part = tid & 7;   // y row t, 16-byte piece `part` of its first 128 bytes
     float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
     if (part < 4) {
@@ -383,7 +387,9 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(const FwdArgs p, i
       v.x = __uint_as_float(kMarker);
     }
     float* yrow = reinterpret_cast<float*>(static_cast<T*>(p.y) + tok_off(b, t0 + t, h, p.T, p.H));
-    *reinterpret_cast<float4*>(yrow + 4 * part) = v;
+    if (range_ok(tok_off(b, t0 + t, h, p.T, p.H) * int64_t(sizeof(T)) + 16 * part, 16, act_total * int64_t(sizeof(T)),
+                 p.status))
+      *reinterpret_cast<float4*>(yrow + 4 * part) = v;
   }
 }
 
@@ -415,6 +421,11 @@ struct StagePlan {
   const T* yrow0;            // y row (token tid/8) of chunk 0
   const T* vrow0[kVPer];     // v rows of this thread's pieces, chunk 0
   int64_t chunk_elems;       // elements from a row to the same row of the next chunk
+  // debug build: the buffers' starts and extents the copies are checked against
+  const float* ckpt;
+  const T *ybuf, *vbuf;
+  int64_t ck_total, act_total;
+  int* status;
 };
 
 // Issue the copies of chunk c's operands into `bf` (full chunks only; always one commit group).  The
@@ -436,17 +447,20 @@ __device__ __forceinline__ void chain_stage(const StagePlan<T>& sp, ChainBuf<T>&
         const int q = (i >> 8) - 2, j = (i >> 2) & 63, piece = i & 3;
         dst = &bf.BlT[0][0] + q * (kN * S24) + j * S24 + 4 * piece;
       }
-      cp_async16(dst, slot + 4 * i);
+      if (range_ok(slot + 4 * i - sp.ckpt, 4, sp.ck_total, sp.status)) cp_async16(dst, slot + 4 * i);
     }
     const int64_t off = c * sp.chunk_elems;
     const int part = tid & 7;
     const float* yrow = reinterpret_cast<const float*>(sp.yrow0 + off);
-    cp_async16(part < 4 ? &bf.Z[tid >> 3][4 * part] : &bf.ext[tid >> 3][4 * (part - 4)], yrow + 4 * part);
+    if (range_ok((sp.yrow0 + off - sp.ybuf) + 16 * part / int(sizeof(T)), 16 / int(sizeof(T)), sp.act_total, sp.status))
+      cp_async16(part < 4 ? &bf.Z[tid >> 3][4 * part] : &bf.ext[tid >> 3][4 * (part - 4)], yrow + 4 * part);
 #pragma unroll
     for (int k = 0; k < StagePlan<T>::kVPer; ++k) {
       const int idx = tid + k * kThreads;
       const int t = idx / StagePlan<T>::kPieces, piece = idx - t * StagePlan<T>::kPieces;
-      cp_async16(&bf.v[t][piece * (16 / int(sizeof(T)))], sp.vrow0[k] + off + piece * (16 / int(sizeof(T))));
+      const T* src = sp.vrow0[k] + off + piece * (16 / int(sizeof(T)));
+      if (range_ok(src - sp.vbuf, 16 / int(sizeof(T)), sp.act_total, sp.status))
+        cp_async16(&bf.v[t][piece * (16 / int(sizeof(T)))], src);
     }
   }
   cp_async_commit();
@@ -469,6 +483,8 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
+  if (!in_bounds(unit < p.B * p.H && nfull * kChunk <= p.T, p.status)) return;   // (debug build)
+  const int64_t act_total = p.B * p.T * p.H * kN, st_total = p.B * p.H * kN * kN;
 
   // state fragments: acc[nt][e] = S[16*warp + g + 8*(e>>1)][8*nt + 2*c4 + (e&1)]
   float acc[8][4];
@@ -477,7 +493,8 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
       float2 v2 = make_float2(0.f, 0.f);
-      if (p.s0) v2 = *reinterpret_cast<const float2*>(p.s0 + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4);
+      const int64_t so = (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4;
+      if (p.s0 && range_ok(so, 2, st_total, p.status)) v2 = *reinterpret_cast<const float2*>(p.s0 + so);
       acc[nt][2 * hh] = v2.x;
       acc[nt][2 * hh + 1] = v2.y;
     }
@@ -485,6 +502,12 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
   StagePlan<T> sp;
   sp.slot0 = p.ckpt + unit * nc * (kN * kN);
   sp.chunk_elems = int64_t(kChunk) * p.H * kN;
+  sp.ckpt = p.ckpt;
+  sp.ybuf = static_cast<const T*>(p.y);
+  sp.vbuf = static_cast<const T*>(p.v);
+  sp.ck_total = p.B * p.H * nc * (kN * kN);
+  sp.act_total = act_total;
+  sp.status = p.status;
   sp.yrow0 = static_cast<const T*>(p.y) + tok_off(b, tid >> 3, h, p.T, p.H);
 #pragma unroll
   for (int k = 0; k < StagePlan<T>::kVPer; ++k)
@@ -505,12 +528,13 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
     const int len = int(min64(kChunk, p.T - t0));
     const unsigned mask = chunk_mask(p, b, t0, len, lane);
     const bool ready = c < nfull && __float_as_uint(bf.ext[0][0]) == kMarker;
-    float* ck = p.ckpt + (unit * nc + c) * (kN * kN) + warp * 1024 + lane * 4;
+    float* ck = range_ok((unit * nc + c) * (kN * kN), kN * kN, sp.ck_total, p.status)
+                    ? p.ckpt + (unit * nc + c) * (kN * kN) + warp * 1024 + lane * 4 : nullptr;
 
     if (!ready) {
       state_chunk_tokens<T>(p, mask, acc, b, h, t0, len, warp, lane);
       __syncthreads();   // every thread's reads of this chunk's operand slot (none) and y rows are done
-      store_ck(ck, acc);
+      if (ck) store_ck(ck, acc);
       continue;
     }
 
@@ -599,20 +623,23 @@ __global__ void __launch_bounds__(kThreads) chunk_chain_kernel(const FwdArgs p, 
 #pragma unroll
       for (int idx = tid; idx < kChunk * kPieces; idx += kThreads) {
         const int t = idx / kPieces, piece = idx - t * kPieces;
-        *reinterpret_cast<uint4*>(ybase + (t0 + t) * tok_stride + piece * (16 / int(sizeof(T)))) =
-            *reinterpret_cast<const uint4*>(&sm.Ys[t][piece * (16 / int(sizeof(T)))]);
+        T* dst = ybase + (t0 + t) * tok_stride + piece * (16 / int(sizeof(T)));
+        if (range_ok(dst - static_cast<T*>(p.y), 16 / int(sizeof(T)), act_total, p.status))
+          *reinterpret_cast<uint4*>(dst) = *reinterpret_cast<const uint4*>(&sm.Ys[t][piece * (16 / int(sizeof(T)))]);
       }
     }
-    store_ck(ck, acc);
+    if (ck) store_ck(ck, acc);
   }
   cp_async_wait_all();   // the empty groups past the last chunk
   if (p.s_out) {
 #pragma unroll
     for (int nt = 0; nt < 8; ++nt)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh)
-        *reinterpret_cast<float2*>(p.s_out + (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4) =
-            make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+      for (int hh = 0; hh < 2; ++hh) {
+        const int64_t so = (unit * kN + row0 + g + 8 * hh) * kN + 8 * nt + 2 * c4;
+        if (range_ok(so, 2, st_total, p.status))
+          *reinterpret_cast<float2*>(p.s_out + so) = make_float2(acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+      }
   }
 }
 

@@ -1,5 +1,6 @@
 // Device status word: kernels record device-side errors in it (a bounded wait on staged inputs
-// that ran out); wkv7_get_device_status() reads it after synchronising.  One word per device.
+// that ran out, a non-finite checked output, a failed debug-build bounds check);
+// wkv7_get_device_status() reads it after synchronising.  One word per device.
 #include <cuda_runtime.h>
 
 #include "kernels.h"
@@ -33,5 +34,8 @@ extern "C" wkv7_status_t wkv7_get_device_status(int clear) {
     if (cudaMemcpyToSymbol(g_device_status, &zero, sizeof(int)) != cudaSuccess) return WKV7_ERR_CUDA;
   }
   if (v & wkv7::kStatusWaitTimeout) return WKV7_ERR_TIMEOUT;
+  if (v & wkv7::kStatusBounds) return WKV7_ERR_BOUNDS;
   return (v & wkv7::kStatusNonFinite) ? WKV7_ERR_NONFINITE : WKV7_OK;
 }
+
+extern "C" int wkv7_debug_checks(void) { return wkv7::kDebugChecks ? 1 : 0; }

@@ -18,13 +18,34 @@ struct FwdArgs {
   void* y;                // [B,T,H,64]
   float* s_out;           // [B,H,64,64] or null
   float* ckpt;            // [B,H,ceil(T/16),64,64] or null
-  int* status;            // device status word: bits of wkv7 device errors (bounded waits that ran out)
+  int* status;            // device status word: bits of wkv7 device errors (kStatus* below)
   unsigned extra_tx;      // test hook: bytes a staging expects beyond what it copies (0 in normal use)
 };
 
 // Bits of the device status word.
 constexpr int kStatusWaitTimeout = 1;
 constexpr int kStatusNonFinite = 2;
+constexpr int kStatusBounds = 4;   // debug build: an index failed its bounds check
+
+// Debug build (compiled with -DWKV7_DEBUG, libwkv7_debug.so): the kernels check the indices they
+// compute -- every global-memory access to activations, states, checkpoints and workspace marks,
+// every TMA box coordinate and bulk-copy range, every shared-memory operand index -- against the
+// extent of the buffer.  A failed check sets kStatusBounds in the device status word and the access
+// is skipped; nothing traps.  In the release build the checks compile to nothing.
+#ifdef WKV7_DEBUG
+constexpr bool kDebugChecks = true;
+#else
+constexpr bool kDebugChecks = false;
+#endif
+__device__ __forceinline__ bool in_bounds(bool ok, int* status) {
+  if (!kDebugChecks) return true;
+  if (!ok && status) atomicOr(status, kStatusBounds);
+  return ok;
+}
+// Elements [off, off + n) inside [0, total).
+__device__ __forceinline__ bool range_ok(int64_t off, int64_t n, int64_t total, int* status) {
+  return in_bounds(off >= 0 && n >= 0 && off + n <= total, status);
+}
 
 // Wall-clock limit of one bounded wait on a staging barrier (the copies it waits for take microseconds).
 constexpr unsigned long long kWaitLimitNs = 1000ull * 1000ull * 1000ull;
@@ -50,6 +71,7 @@ struct StepArgs {
   float* state;
   const uint8_t* active;
   void* y;
+  int* status;   // device status word (debug-build bounds checks)
 };
 
 // Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).
@@ -63,7 +85,7 @@ cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
 // Set kStatusNonFinite in *status if any of the n elements at x (dtype as above; 16-byte aligned)
 // is NaN or infinite.  x == nullptr or n == 0: nothing is launched.
 cudaError_t launch_finite_scan(const void* x, int64_t n, int dtype, int* status, cudaStream_t stream);
-// Device address of this device's status word (looked up once per device).
+// Device address of the current device's status word (looked up on every call).
 cudaError_t device_status_ptr(int** out);
 
 // Tensor maps of the token inputs for the chunked kernels' TMA staging.  Each [B,T,H,64] input is

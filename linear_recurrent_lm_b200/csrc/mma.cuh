@@ -33,59 +33,9 @@ __device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* row_ptr) {
                : "r"(smem_u32(row_ptr)));
 }
 
-__device__ __forceinline__ void ldsm_x4_t(uint32_t (&r)[4], const void* row_ptr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];\n"
-               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
-               : "r"(smem_u32(row_ptr)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16(float lo_elem, float hi_elem) {
   __nv_bfloat162 v = __floats2bfloat162_rn(lo_elem, hi_elem);
   return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// Split two fp32 values into packed bf16 hi and lo words.
-__device__ __forceinline__ void split2(float x0, float x1, uint32_t& hi, uint32_t& lo) {
-  __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
-  const float2 hf = __bfloat1622float2(h);
-  __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
-  hi = *reinterpret_cast<uint32_t*>(&h);
-  lo = *reinterpret_cast<uint32_t*>(&l);
-}
-
-__device__ __forceinline__ void split1(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
-  hi = __float2bfloat16_rn(x);
-  lo = __float2bfloat16_rn(x - __bfloat162float(hi));
-}
-
-// Per-lane row address for ldmatrix.x4 of an A fragment (16 rows x 16 k) stored
-// row-major [row][k] with `stride` elements per row, at (row0, k0).
-template <typename E>
-__device__ __forceinline__ const E* a_rowmajor_addr(const E* base, int stride, int row0, int k0, int lane) {
-  const int m = lane >> 3, r = lane & 7;
-  return base + (row0 + (m & 1) * 8 + r) * stride + k0 + (m >> 1) * 8;
-}
-
-// A fragment (16 m x 16 k) stored transposed as [k][m]: use with ldsm_x4_t.
-template <typename E>
-__device__ __forceinline__ const E* a_kmajor_addr(const E* base, int stride, int k0, int m0, int lane) {
-  const int mat = lane >> 3, r = lane & 7;
-  return base + (k0 + (mat >> 1) * 8 + r) * stride + m0 + (mat & 1) * 8;
-}
-
-// Two adjacent B fragments (n0..n0+15, k0..k0+15) stored as [n][k]: ldsm_x4 gives
-// {b0,b1} of n-tile n0 and {b0,b1} of n-tile n0+8.
-template <typename E>
-__device__ __forceinline__ const E* b_nmajor_addr(const E* base, int stride, int n0, int k0, int lane) {
-  const int m = lane >> 3, r = lane & 7;
-  return base + (n0 + (m >> 1) * 8 + r) * stride + k0 + (m & 1) * 8;
-}
-
-// Same two B fragments stored as [k][n]: use with ldsm_x4_t.
-template <typename E>
-__device__ __forceinline__ const E* b_kmajor_addr(const E* base, int stride, int k0, int n0, int lane) {
-  const int m = lane >> 3, r = lane & 7;
-  return base + (k0 + (m & 1) * 8 + r) * stride + n0 + (m >> 1) * 8;
 }
 
 }  // namespace wkv7

@@ -91,7 +91,9 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
   BwdSmem& sm = *reinterpret_cast<BwdSmem*>(smem_raw);
 
   const int64_t unit = blockIdx.x;
+  if (!in_bounds(unit < p.B * p.H, p.status)) return;   // (debug build; block-uniform)
   if (only_flagged && p.unit_flags[unit] == 0) return;
+  const int64_t act_total = p.B * p.T * p.H * kN, st_total = p.B * p.H * kN * kN;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
   const int tid = threadIdx.x, lane = tid & 31;
   const int q = tid >> 6;          // row quarter
@@ -107,7 +109,9 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
 
   float D[16];
 #pragma unroll
-  for (int ii = 0; ii < 16; ++ii) D[ii] = p.dsT ? p.dsT[(unit * kN + q * 16 + ii) * kN + j] : 0.f;
+  for (int ii = 0; ii < 16; ++ii)
+    D[ii] = p.dsT && range_ok((unit * kN + q * 16 + ii) * kN + j, 1, st_total, p.status)
+                ? p.dsT[(unit * kN + q * 16 + ii) * kN + j] : 0.f;
 
   for (int64_t c = nc - 1; c >= 0; --c) {
     const int64_t t0 = c * kChunk;
@@ -117,16 +121,21 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
       const int m = e / (len * kN);
       const int rem = e - m * len * kN;
       const int tt = rem / kN, jj = rem - (rem / kN) * kN;
-      sm.x[m][tt][jj] = Elt<T>::to_f32(src[m][tok_off(b, t0 + tt, h, p.T, p.H) + jj]);
+      const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + jj;
+      if (range_ok(o, 1, act_total, p.status) && in_bounds(tt < kChunk, p.status))
+        sm.x[m][tt][jj] = Elt<T>::to_f32(src[m][o]);
     }
-    if (tid < kChunk) sm.flags[tid] = (tid < len && p.reset) ? (p.reset[b * p.T + t0 + tid] != 0) : 0;
+    if (tid < kChunk)
+      sm.flags[tid] = (tid < len && p.reset && range_ok(b * p.T + t0 + tid, 1, p.B * p.T, p.status))
+                          ? (p.reset[b * p.T + t0 + tid] != 0) : 0;
     __syncthreads();
 
     // state entering the chunk (before the reset of its first token applies)
     float E[16];
     {
       if (c > 0) {   // checkpoint c-1, in the tiled checkpoint order
-        const float* es = p.ckpt + (unit * nc + (c - 1)) * kN * kN;
+        const bool ok = range_ok((unit * nc + (c - 1)) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status);
+        const float* es = p.ckpt + (ok ? (unit * nc + (c - 1)) * kN * kN : 0);
 #pragma unroll
         for (int ii = 0; ii < 16; ++ii) E[ii] = es[ckpt_off(q * 16 + ii, j)];
       } else {       // the caller's s0, row-major
@@ -227,7 +236,7 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
           sm.row_red[half][1][myrow] = dsa_part;
         }
         __syncthreads();
-        if (tid < kN)
+        if (tid < kN && range_ok(tok_off(b, t, h, p.T, p.H) + tid, 1, act_total, p.status))
           dst[5][tok_off(b, t, h, p.T, p.H) + tid] = Elt<T>::from_f32(sm.row_red[0][0][tid] + sm.row_red[1][0][tid]);
         float da_p = 0.f;
         const bool rst = sm.flags[tt] != 0;
@@ -248,7 +257,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
         for (int o = tid; o < 5 * kN; o += kThreads) {
           const int m = o >> 6, jj = o & 63;
           const float s = (sm.col_red[m][0][jj] + sm.col_red[m][1][jj]) + (sm.col_red[m][2][jj] + sm.col_red[m][3][jj]);
-          dst[m][tok_off(b, t, h, p.T, p.H) + jj] = Elt<T>::from_f32(s);
+          if (range_ok(tok_off(b, t, h, p.T, p.H) + jj, 1, act_total, p.status))
+            dst[m][tok_off(b, t, h, p.T, p.H) + jj] = Elt<T>::from_f32(s);
         }
       }
       seg_end = seg_start;
@@ -256,7 +266,9 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
   }
   if (p.ds0) {
 #pragma unroll
-    for (int ii = 0; ii < 16; ++ii) p.ds0[(unit * kN + q * 16 + ii) * kN + j] = D[ii];
+    for (int ii = 0; ii < 16; ++ii)
+      if (range_ok((unit * kN + q * 16 + ii) * kN + j, 1, st_total, p.status))
+        p.ds0[(unit * kN + q * 16 + ii) * kN + j] = D[ii];
   }
 }
 

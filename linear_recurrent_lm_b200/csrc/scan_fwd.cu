@@ -34,9 +34,10 @@ __device__ __forceinline__ void stage_slab(const FwdArgs& p, const T* const* src
     const int rem = idx - in * len * VPT;
     const int tt = rem / VPT;
     const int vec = rem - tt * VPT;
-    const T* g = src[in] + tok_off(b, t0 + tt, h, p.T, p.H) + vec * Vec16<T>::n;
+    const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + vec * Vec16<T>::n;
     unsigned char* s = raw + ((size_t(in) * kChunk + tt) * kN + vec * Vec16<T>::n) * sizeof(T);
-    cp_async16(s, g);
+    if (range_ok(o, Vec16<T>::n, p.B * p.T * p.H * kN, p.status) && in_bounds(tt < kChunk, p.status))
+      cp_async16(s, src[in] + o);
   }
   cp_async_commit();
 }
@@ -63,7 +64,8 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
                            static_cast<const T*>(p.v), static_cast<const T*>(p.a), static_cast<const T*>(p.b)};
 
   float S[kN];
-  if (p.s0) {
+  const int64_t st_total = p.B * p.H * kN * kN;
+  if (p.s0 && range_ok((unit * kN + i) * kN, kN, st_total, p.status)) {
     const float4* row = reinterpret_cast<const float4*>(p.s0 + (unit * kN + i) * kN);
 #pragma unroll
     for (int q = 0; q < kN / 4; ++q) {
@@ -91,7 +93,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
 
     for (int tt = 0; tt < len; ++tt) {
       const int64_t t = t0 + tt;
-      if (p.reset && p.reset[b * p.T + t]) {
+      if (p.reset && range_ok(b * p.T + t, 1, p.B * p.T, p.status) && p.reset[b * p.T + t]) {
 #pragma unroll
         for (int j = 0; j < kN; ++j) S[j] = 0.f;
       }
@@ -124,10 +126,11 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
         y2 = fmaf(S[4 * q + 2], rv.z, y2);
         y3 = fmaf(S[4 * q + 3], rv.w, y3);
       }
-      y[tok_off(b, t, h, p.T, p.H) + i] = Elt<T>::from_f32((y0 + y1) + (y2 + y3));
+      if (range_ok(tok_off(b, t, h, p.T, p.H) + i, 1, p.B * p.T * p.H * kN, p.status))
+        y[tok_off(b, t, h, p.T, p.H) + i] = Elt<T>::from_f32((y0 + y1) + (y2 + y3));
     }
 
-    if (p.ckpt) {
+    if (p.ckpt && range_ok((unit * nc + c) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status)) {
       float* dst = p.ckpt + (unit * nc + c) * kN * kN;
 #pragma unroll
       for (int q = 0; q < kN / 2; ++q) *reinterpret_cast<float2*>(dst + ckpt_off(i, 2 * q)) = make_float2(S[2 * q], S[2 * q + 1]);
@@ -140,7 +143,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
     }
   }
 
-  if (p.s_out) {
+  if (p.s_out && range_ok((unit * kN + i) * kN, kN, st_total, p.status)) {
     float4* dst = reinterpret_cast<float4*>(p.s_out + (unit * kN + i) * kN);
 #pragma unroll
     for (int q = 0; q < kN / 4; ++q) dst[q] = make_float4(S[4 * q], S[4 * q + 1], S[4 * q + 2], S[4 * q + 3]);

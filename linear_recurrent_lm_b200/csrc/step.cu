@@ -53,6 +53,9 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) 
   const int i = t >> 3, q = t & 7;   // row i, columns 8q..8q+7
   const int64_t units = p.B * p.H;
   for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
+    // (debug build: the row of y, the state row and the input rows of this unit)
+    if (!range_ok(unit * kN, kN, units * kN, p.status) || !range_ok((unit * kN + i) * kN + q * 8, 8, units * kN * kN, p.status))
+      continue;
     T* y = static_cast<T*>(p.y) + unit * kN;
     if (p.active && !p.active[unit / p.H]) {   // padded row: its state is not even read
       if (q == 0) y[i] = Elt<T>::from_f32(0.f);

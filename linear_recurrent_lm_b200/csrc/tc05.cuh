@@ -93,15 +93,11 @@ __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
          | (uint32_t(M >> 4) << 24);    // M / 16
 }
 
-// Shared-memory matrix descriptor with explicit leading and stride byte offsets (no swizzle).  For a
-// K-major operand LBO is the distance between K-adjacent core matrices and SBO between M/N-adjacent
-// 8-row groups; for an MN-major one (16-bit types only: tf32 operands must be K-major) SBO is the
-// distance between M/N-adjacent core matrices and LBO between K-adjacent 8-row groups.
-__device__ __forceinline__ uint64_t smem_desc2(const void* start, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  const uint64_t addr = smem_u32addr(start);
-  return ((addr >> 4) & 0x3FFFull) | ((uint64_t(lbo_bytes >> 4) & 0x3FFFull) << 16) |
-         ((uint64_t(sbo_bytes >> 4) & 0x3FFFull) << 32) | (uint64_t(1) << 46);
-}
+// Shared-memory matrix descriptors without swizzle (the backward builds its own at compile time with
+// these rules): for a K-major operand the leading byte offset (LBO) is the distance between
+// K-adjacent core matrices and the stride byte offset (SBO) the distance between M/N-adjacent 8-row
+// groups; for an MN-major one (16-bit types only: tf32 operands must be K-major) SBO is the distance
+// between M/N-adjacent core matrices and LBO the distance between K-adjacent 8-row groups.
 
 // Instruction descriptor of kind::f16 with bf16 A and B, fp32 accumulate, and the major-ness of A
 // and B (0 = K-major, 1 = MN-major).

@@ -24,6 +24,7 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned ma
   T* y = static_cast<T*>(p.y);
   for (int tt = 0; tt < len; ++tt) {
     const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H);
+    if (!range_ok(o, kN, p.B * p.T * p.H * kN, p.status)) continue;   // (debug build)
     if ((mask >> tt) & 1u) {
 #pragma unroll
       for (int nt = 0; nt < 8; ++nt)

@@ -178,6 +178,7 @@ const char* wkv7_status_string(wkv7_status_t s) {
     case WKV7_ERR_TIMEOUT: return "device-side wait timed out";
     case WKV7_ERR_SCRATCH_LIMIT: return "problem exceeds the fixed scratch of wkv7_train_step_noalloc";
     case WKV7_ERR_NONFINITE: return "an output checked under WKV7_FLAG_CHECK_FINITE holds a NaN or infinity";
+    case WKV7_ERR_BOUNDS: return "a kernel index failed its bounds check (debug build)";
   }
   return "unknown status";
 }
@@ -278,8 +279,8 @@ wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, cons
   if (st != WKV7_OK) return st;
   if (units == 0) return WKV7_OK;
   int* status = nullptr;
-  if ((d->flags & WKV7_FLAG_CHECK_FINITE) && wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
-  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y};
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y, status};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return check_outputs(d, wkv7::launch_step(p, d->dtype, s), {{y, units * 64, d->dtype}, {state, units * 64 * 64, WKV7_F32}},
                        status, s);

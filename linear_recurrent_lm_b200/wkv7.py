@@ -9,7 +9,10 @@ stream.  The same entry points as the C ABI:
   -> dict(dr, dw, dk, dv, da, db, ds0)
 * ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
 * ``workspace_bytes(B, T, H, dtype)``
-* ``device_status(clear=True)`` -> OK, ERR_TIMEOUT or ERR_NONFINITE (synchronises the device)
+* ``device_status(clear=True)`` -> OK, ERR_TIMEOUT, ERR_BOUNDS or ERR_NONFINITE (synchronises the device)
+* ``use_build("release" | "debug")``: route every call through ``libwkv7.so`` (default) or its
+  bounds-checked twin ``libwkv7_debug.so`` (same ABI; ``WKV7_BUILD=debug`` in the environment
+  selects it at import)
 
 Tensors are [B,T,H,64] (token inputs), [B,H,64,64] fp32 (states), [B,T] uint8
 (reset), [B] uint8 (active), all on one CUDA device and contiguous.  If the
@@ -24,10 +27,11 @@ from typing import Dict, Optional
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libwkv7.so")
+LIB_PATHS = {"release": os.path.join(_HERE, "libwkv7.so"), "debug": os.path.join(_HERE, "libwkv7_debug.so")}
+LIB_PATH = LIB_PATHS["release"]
 
 (OK, ERR_NULL, ERR_SHAPE, ERR_DTYPE, ERR_ALIGN, ERR_WORKSPACE, ERR_UNSUPPORTED, ERR_CUDA, ERR_TIMEOUT,
- ERR_SCRATCH_LIMIT, ERR_NONFINITE) = range(11)
+ ERR_SCRATCH_LIMIT, ERR_NONFINITE, ERR_BOUNDS) = range(12)
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
 FLAG_CHECK_FINITE = 0x1                    # WKV7_FLAG_CHECK_FINITE: scan outputs for NaN / Inf
@@ -48,36 +52,67 @@ class WKV7Error(RuntimeError):
         self.status = status
 
 
-_lib = None
+_loaded: Dict[str, ctypes.CDLL] = {}
+_active = os.environ.get("WKV7_BUILD", "release")
+if _active not in LIB_PATHS:
+    raise ValueError(f"WKV7_BUILD must be one of {sorted(LIB_PATHS)}, got {_active!r}")
+
+
+def _load(variant: str) -> ctypes.CDLL:
+    path = LIB_PATHS[variant]
+    if not os.path.exists(path):
+        raise ImportError(f"{path} is missing: build it with `python -m linear_recurrent_lm_b200.build` "
+                          "(or __graft_entry__.build()); the WKV-7 path has no CPU fallback")
+    L = ctypes.CDLL(path)
+    vp = ctypes.c_void_p
+    dp = ctypes.POINTER(Desc)
+    L.wkv7_version.restype = ctypes.c_int
+    L.wkv7_status_string.restype = ctypes.c_char_p
+    L.wkv7_status_string.argtypes = [ctypes.c_int]
+    L.wkv7_workspace_bytes.restype = ctypes.c_size_t
+    L.wkv7_workspace_bytes.argtypes = [dp]
+    L.wkv7_forward.restype = ctypes.c_int
+    L.wkv7_forward.argtypes = [dp] + [vp] * 12
+    L.wkv7_backward.restype = ctypes.c_int
+    L.wkv7_backward.argtypes = [dp] + [vp] * 19
+    L.wkv7_step.restype = ctypes.c_int
+    L.wkv7_step.argtypes = [dp] + [vp] * 10
+    L.wkv7_train_step_noalloc.restype = ctypes.c_int
+    L.wkv7_train_step_noalloc.argtypes = [dp] + [vp] * 20
+    L.wkv7_get_device_status.restype = ctypes.c_int
+    L.wkv7_get_device_status.argtypes = [ctypes.c_int]
+    L.wkv7_debug_checks.restype = ctypes.c_int
+    L.wkv7_debug_checks.argtypes = []
+    return L
 
 
 def lib() -> ctypes.CDLL:
-    """The loaded libwkv7.so (raises if it has not been built)."""
-    global _lib
-    if _lib is None:
-        if not os.path.exists(LIB_PATH):
-            raise ImportError(f"{LIB_PATH} is missing: build it with `python -m linear_recurrent_lm_b200.build` "
-                              "(or __graft_entry__.build()); the WKV-7 path has no CPU fallback")
-        L = ctypes.CDLL(LIB_PATH)
-        vp = ctypes.c_void_p
-        dp = ctypes.POINTER(Desc)
-        L.wkv7_version.restype = ctypes.c_int
-        L.wkv7_status_string.restype = ctypes.c_char_p
-        L.wkv7_status_string.argtypes = [ctypes.c_int]
-        L.wkv7_workspace_bytes.restype = ctypes.c_size_t
-        L.wkv7_workspace_bytes.argtypes = [dp]
-        L.wkv7_forward.restype = ctypes.c_int
-        L.wkv7_forward.argtypes = [dp] + [vp] * 12
-        L.wkv7_backward.restype = ctypes.c_int
-        L.wkv7_backward.argtypes = [dp] + [vp] * 19
-        L.wkv7_step.restype = ctypes.c_int
-        L.wkv7_step.argtypes = [dp] + [vp] * 10
-        L.wkv7_train_step_noalloc.restype = ctypes.c_int
-        L.wkv7_train_step_noalloc.argtypes = [dp] + [vp] * 20
-        L.wkv7_get_device_status.restype = ctypes.c_int
-        L.wkv7_get_device_status.argtypes = [ctypes.c_int]
-        _lib = L
-    return _lib
+    """The library every call goes through (raises if it has not been built)."""
+    if _active not in _loaded:
+        _loaded[_active] = _load(_active)
+    return _loaded[_active]
+
+
+def use_build(variant: str) -> str:
+    """Route every later call through ``variant`` ("release" or "debug"); return the previous one.
+
+    The two builds are separate CUDA modules: each has its own device status word, which
+    ``device_status`` reads from the build in use."""
+    global _active
+    if variant not in LIB_PATHS:
+        raise ValueError(f"unknown build {variant!r}; expected one of {sorted(LIB_PATHS)}")
+    prev = _active
+    _active = variant
+    try:
+        lib()
+    except ImportError:
+        _active = prev
+        raise
+    return prev
+
+
+def active_build() -> str:
+    return _active
 
 
 lib()   # fail at import time if the CUDA library is absent
@@ -93,7 +128,8 @@ def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16) -> int:
 
 
 def device_status(clear: bool = True) -> int:
-    """The device status word of the current device (synchronises it): OK, ERR_TIMEOUT or ERR_NONFINITE."""
+    """The device status word of the current device (synchronises it): OK, ERR_TIMEOUT, ERR_BOUNDS or
+    ERR_NONFINITE (in that order of precedence)."""
     return int(lib().wkv7_get_device_status(1 if clear else 0))
 
 

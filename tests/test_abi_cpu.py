@@ -15,7 +15,7 @@ HEADER = os.path.join(ROOT, "include", "wkv7.h")
 @pytest.fixture(scope="module")
 def L():
     from linear_recurrent_lm_b200 import build
-    build.build()
+    build.build_all()
     from linear_recurrent_lm_b200 import wkv7
     return wkv7
 
@@ -26,18 +26,35 @@ def declared_functions():
     return sorted(set(re.findall(r"\b(wkv7_[a-z_0-9]+)\s*\(", text)))
 
 
-def test_exports_every_declared_symbol(L):
+@pytest.mark.parametrize("variant", ("release", "debug"))
+def test_exports_every_declared_symbol(L, variant):
     names = declared_functions()
-    assert {"wkv7_forward", "wkv7_backward", "wkv7_step", "wkv7_workspace_bytes"} <= set(names)
-    lib = ctypes.CDLL(L.LIB_PATH)
+    assert {"wkv7_forward", "wkv7_backward", "wkv7_step", "wkv7_workspace_bytes", "wkv7_debug_checks"} <= set(names)
+    lib = ctypes.CDLL(L.LIB_PATHS[variant])
     for n in names:
-        assert hasattr(lib, n), n
+        assert hasattr(lib, n), (variant, n)
+    assert lib.wkv7_debug_checks() == (1 if variant == "debug" else 0)
+
+
+def test_use_build_switches_library(L):
+    assert L.active_build() == "release"
+    prev = L.use_build("debug")
+    try:
+        assert prev == "release" and L.lib().wkv7_debug_checks() == 1
+        d = L.make_desc(1, 16, 1, 1)
+        d.N = 32
+        assert call_fwd(L, d) == L.ERR_UNSUPPORTED     # same host-side validation in both builds
+    finally:
+        L.use_build(prev)
+    assert L.lib().wkv7_debug_checks() == 0
+    with pytest.raises(ValueError):
+        L.use_build("fast")
 
 
 def test_version_and_status_strings(L):
     lib = L.lib()
     assert lib.wkv7_version() >= 100
-    strings = [lib.wkv7_status_string(s) for s in range(L.ERR_NONFINITE + 1)]
+    strings = [lib.wkv7_status_string(s) for s in range(L.ERR_BOUNDS + 1)]
     assert all(strings) and b"unknown status" not in strings and len(set(strings)) == len(strings)
     assert lib.wkv7_status_string(12345) == b"unknown status"
 
