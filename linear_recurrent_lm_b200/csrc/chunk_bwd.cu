@@ -21,11 +21,14 @@
 // chunk from its checkpoint).
 //
 // Everything runs transposed so that the tensor core's 64-row side is a state dimension: the
-// carried gradient is dS^T (TMEM rows = key channel j), G1 = dSl [Bh|Kh]^T and G2 = dY^T [Mrb|Mrk]
-// have rows = value channel i (dSA^T = ls o G1b + G2b, dU^T = dSA^T T, dV^T = ls o G1k + G2k +
-// dU^T Lak follow on the FP32 cores, one thread per i), and the key-space gradients dAt^T, dRt^T,
+// carried gradient is dS^T (TMEM rows = key channel j), and the key-space gradients dAt^T, dRt^T,
 // dBh^T, dKh^T have rows = j, so that one thread owns one key channel over all 16 tokens of the
-// chunk and keeps the reverse sum for dw in its registers.
+// chunk and keeps the reverse sum for dw in its registers.  dU and dV come straight out of one
+// product, GU = dSl BKx^T + dY^T [Qm | Vq] (rows = value channel i), because the chunk's small
+// factors are folded into its operands beforehand: with Tl = ls.T and X = T Lak,
+//   BKx = [Tl^T 0; (ls.X)^T diag(ls)] [Bh; Kh],   Qm = Mrb T,   Vq = Mrk + Mrb X,
+// so that dU^T = dSA^T T = dSl (Tl^T Bh)^T + dY^T Qm and dV^T = ls.(dSl Kh^T) + dY^T Mrk + dU^T Lak
+// = GU's second half.
 //
 // Precision: the tensor-core products take bf16 operands split in two, x = hi + lo with
 // hi = bf16(x), lo = bf16(x - hi), and accumulate hi.hi + hi.lo + lo.hi in fp32 (lo.lo, about
@@ -43,16 +46,18 @@
 // Products with fewer than 64 useful rows read 64 anyway; the extra rows come from the arrays
 // that follow (always inside the CTA's shared memory) and their results are never read.
 //
-// Work split: one CTA of 8 warps per (b,h) (about 200 KB of shared memory and 512 TMEM columns,
-// so one CTA per SM), chunks in reverse, pipelined:
+// Work split: one CTA of 9 warps per (b,h) (about 200 KB of shared memory, so one CTA per SM),
+// chunks in reverse, pipelined:
 //   warps 4-7 ("context") for chunk c-1: stage its inputs (one TMA box per input) and its
 //     checkpoint (one bulk copy) on an mbarrier with bounded waits, build the decay-scaled
-//     operands, the masked Gram (tcgen05), T by substitution, W, X, and SA^T = S0 W^T + V^T X^T
-//     (tcgen05) into one half of a double buffer;
-//   warps 0-3 ("main") for chunk c: scale the carried dS^T, then one thread issues the products
-//     in three batches (chain: G1, G2, Rt^T m0.dY; then At^T m0.dU, the gradient Gram and the S0
-//     and dSl parts of the key-space products; then their Gram parts), while the warps write dv
-//     and, per key channel, da, dr, db, dk and dw.
+//     operands, the masked Gram, T by substitution, the folded operands BKx, Qm, Vq, W and X, and
+//     SA^T = S0 W^T + V^T X^T (warp-level split products) into one half of a double buffer;
+//   warps 0-3 ("main") for chunk c: scale the carried dS^T, then read GU (dU, dV), mask the
+//     gradient Gram and, per key channel, write da, dr, db, dk and dw;
+//   warp 8 ("issue") for chunk c: one thread issues the tensor-core products as the main warps
+//     hand their operands over (named barriers): GU; then the gradient Gram, dSl [SA^T|v^T], the
+//     rest of dS0^T and S0^T [m0.dU^T | m0.dy^T]; then the Gram parts of the key-space products,
+//     each batch committed to an mbarrier the main warps wait on.
 // One CTA barrier per chunk hands the context over.
 #include <type_traits>
 
@@ -64,18 +69,18 @@
 namespace wkv7 {
 namespace {
 
-constexpr int kThreads = 256;
+constexpr int kThreads = 288;   // warps 0-3 main, 4-7 context, 8 issue
+constexpr int kIssueTid = 256;  // the thread that issues every tensor-core product
 constexpr int kIn = 7;   // r, w, k, v, a, b, dy
 constexpr int S20 = 20;
 using bf16 = __nv_bfloat16;
 
-// TMEM columns (512 allocated: one CTA per SM).  Every accumulator has M = 64 rows.
-constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColDS = 64;     // main: dS^T                     (64; rows j)
-constexpr uint32_t kColG1 = 128;    // main: dSl [Bh|Kh]^T            (32; rows i)
-constexpr uint32_t kColG2 = 160;    // main: dY^T [Mrb|Mrk]           (32; rows i)
-constexpr uint32_t kColGG = 192;    // main: [dY; dU] [SA^T | v^T]     (32; rows t and 16 + t)
-constexpr uint32_t kColE = 256;     // main: dAt^T | dRt^T | dBg^T | dKg^T | (SA dSl)^T | (V dSl)^T  (96; rows j)
+// TMEM columns (256 allocated; one CTA per SM).  Every accumulator has M = 64 rows.
+constexpr uint32_t kTmemCols = 256;
+constexpr uint32_t kColDS = 0;      // dS^T                               (64; rows j)
+constexpr uint32_t kColGU = 64;     // [dU^T | dV^T]                       (32; rows i)
+constexpr uint32_t kColGG = 96;     // [dU; dY] [SA^T | v^T]               (32; rows t and 16 + t)
+constexpr uint32_t kColE = 128;     // dAt^T | dRt^T | dBg^T | dKg^T | (SA dSl)^T | (V dSl)^T  (96; rows j)
 
 // bf16 index of element (p, q) of a core array with Q columns.
 __device__ __forceinline__ int cb(int p, int q, int Q) { return (p >> 3) * (Q * 8) + (q >> 3) * 64 + (p & 7) * 8 + (q & 7); }
@@ -150,6 +155,12 @@ __device__ __forceinline__ uint32_t bfrag_k(const bf16* b, int n0, int k0, int l
   const int mi = lane >> 3, r = lane & 7;
   return smem_u32(b + cb(n0 + (mi >> 1) * 8 + r, k0 + (mi & 1) * 8, Q));
 }
+// The same B fragments from a core array with rows = K, columns = N (read with ldmatrix.trans).
+template <int Q>
+__device__ __forceinline__ uint32_t bfrag_mn(const bf16* b, int n0, int k0, int lane) {
+  const int mi = lane >> 3, r = lane & 7;
+  return smem_u32(b + cb(k0 + (mi & 1) * 8 + r, n0 + (mi >> 1) * 8, Q));
+}
 __device__ __forceinline__ void ldsm4(uint32_t (&r)[4], uint32_t addr) {
   asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
@@ -159,13 +170,19 @@ __device__ __forceinline__ void ldsm4t(uint32_t (&r)[4], uint32_t addr) {
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]) : "r"(addr));
 }
 // acc[nt] (+)= A B over one K step of 16 for two n-tiles, with split operands: hi.hi + hi.lo + lo.hi.
-// The lo addresses are the hi ones plus a fixed byte distance; a_exact skips the A lo half.
+// The lo addresses are the hi ones plus a fixed byte distance; a_exact skips the A lo half; a_mn and
+// b_mn select the transposed (ldmatrix.trans) reads of the fragment helpers above.
 __device__ __forceinline__ void mma_split2(float (&acc)[2][4], uint32_t a_hi, uint32_t a_lo_off, bool a_mn,
-                                           bool a_exact, uint32_t b_hi, uint32_t b_lo_off) {
+                                           bool a_exact, uint32_t b_hi, uint32_t b_lo_off, bool b_mn = false) {
   uint32_t ah[4], al[4], bh[4], bl[4];
   if (a_mn) ldsm4t(ah, a_hi); else ldsm4(ah, a_hi);
-  ldsm4(bh, b_hi);
-  ldsm4(bl, b_hi + b_lo_off);
+  if (b_mn) {
+    ldsm4t(bh, b_hi);
+    ldsm4t(bl, b_hi + b_lo_off);
+  } else {
+    ldsm4(bh, b_hi);
+    ldsm4(bl, b_hi + b_lo_off);
+  }
 #pragma unroll
   for (int nt = 0; nt < 2; ++nt) {
     mma16816(acc[nt], ah, bh[2 * nt], bh[2 * nt + 1]);
@@ -220,22 +237,30 @@ __device__ __forceinline__ void mma3(uint32_t d, const Op<QA, MA>& a, const Op<Q
   }
 }
 
-// Produced by the context warps for one chunk, read by the main warps one iteration later.  The
-// order of the arrays matters: 64-row reads of AR and DY run on into the arrays after them.
+// Store two adjacent values (elements e and e + 1 of one core row) as their hi and lo halves.
+template <int P, int Q>
+__device__ __forceinline__ void put2(Split<P, Q>& m, int e, float v0, float v1) {
+  if (!in_bounds(e >= 0 && e + 2 <= P * Q && (e & 1) == 0, debug_status())) return;
+  const __nv_bfloat162 hh = __floats2bfloat162_rn(v0, v1);
+  const float2 hf = __bfloat1622float2(hh);
+  *reinterpret_cast<__nv_bfloat162*>(&m.hi[e]) = hh;
+  *reinterpret_cast<__nv_bfloat162*>(&m.lo[e]) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+}
+
+// Produced by the context warps for one chunk, read by the main and issue warps one iteration
+// later.  The order of the arrays matters: the 64-column read of UYT (32 columns) runs on into the
+// arrays after it.
 template <typename T>
 struct __align__(128) Ctx {
   Split<32, 64> AR;      // rows 0-15 At [t][j], rows 16-31 Rt [t][j]
   Split<32, 64> BK;      // rows 0-15 Bh [tau][j], rows 16-31 Kh [tau][j]
-  Split<32, 64> DYU;     // rows 0-15 dy [t][i]; rows 16-31 dU [t][i], written by the main warps
+  Split<64, 32> UYT;     // [i][dU^T (t) | dy^T (t)]: the dU half is written by the main warps
   Split<64, 32> DUY;     // [i][m0.dU^T (t) | m0.dy^T (t)]: the dU half is written by the main warps
   Split<64, 32> SV;      // [i][SA^T (tau) | v^T (tau)]
   Split<64, 64> S0T;     // S0^T [j][i]
-  Split<16, 32> MM;      // [t][Mrb[t][0..15] | Mrk[t][0..15]]
-  __align__(16) float Tp[kChunk][kChunk];     // T [t][tau]
-  __align__(16) float LakP[kChunk][kChunk];   // Lak [t][tau]
+  Split<32, 64> BKx;     // rows 0-15 (Tl^T Bh) [tau][j], rows 16-31 ((ls.X)^T Bh + ls.Kh) [tau][j]
+  Split<16, 32> MMx;     // [t][Qm[t][0..15] | Vq[t][0..15]]
   __align__(16) float lam[kChunk][kN];        // L_t [t][j]
-  __align__(16) float lamT[kN][kChunk + 4];   // L_t [j][t] (rows padded against bank conflicts)
-  __align__(16) T rabkT[4][kN][kChunk + 8];   // r, a, b, k of the chunk [j][t]
   int mask;                     // reset bits of the chunk
   int unsafe;                   // decay out of range (or staging timed out): the unit is re-run exactly
 };
@@ -245,14 +270,20 @@ struct __align__(128) BwdSmem {
   Ctx<T> ctx[2];
   Split<64, 64> dSlT;    // dSl^T [j][i]                                        (main)
   Split<32, 32> G4;      // rows t: [dLab[t] | dLak[t]], rows 16 + t: [dMrb[t] | dMrk[t]]   (main)
-  Split<16, 64> WC;      // W [tau][j]                         (context)
-  Split<16, 16> XC;      // X [tau][t]                         (context)
-  __align__(16) float Atf[kChunk][kN];      // At [t][j] in fp32     (context)
-  __align__(16) float LabT[kChunk][S20];    // Lab^T [tau][t]   (context)
+  Split<16, 64> WC;      // W [tau][j]                                (context)
+  Split<16, 16> XC;      // X [tau][t]                                (context)
+  Split<32, 32> AC;      // [Tl^T 0; (ls.X)^T diag(ls)] [tau'][t']    (context)
+  Split<16, 16> TmT;     // (T m0)^T [t][tau]                         (context)
+  __align__(16) float LabT[kChunk][S20];     // Lab^T [tau][t]        (context)
+  __align__(16) float Tp[kChunk][kChunk];    // T [t][tau]            (context)
+  __align__(16) float LakP[kChunk][kChunk];  // Lak [t][tau]          (context)
+  __align__(16) float MrbP[kChunk][kChunk];  // Mrb [t][tau]          (context)
+  __align__(16) float MrkP[kChunk][kChunk];  // Mrk [t][tau]          (context)
+  __align__(16) float Xp[kChunk][kChunk];    // X [t][tau]            (context)
   __align__(128) float ck[kN * kN];         // checkpoint entering the chunk being built (tiled order)
   __align__(128) T stg[kIn][kChunk][kN];    // staged inputs of the chunk being built (TMA boxes)
   unsigned long long in_bar;                // staged inputs and checkpoint landed (one phase per staged chunk)
-  unsigned long long u_bar, chain_bar, gg_bar, e_bar;   // main MMAs complete (one phase per chunk each)
+  unsigned long long u_bar, gg_bar, e_bar;  // tensor-core batches complete (one phase per chunk each)
   uint32_t tmem_base;
   int kbad[4];
   int stop;
@@ -261,7 +292,14 @@ struct __align__(128) BwdSmem {
 __device__ __forceinline__ void named_bar(int id, int n) {
   asm volatile("bar.sync %0, %1;\n" ::"r"(id), "r"(n) : "memory");
 }
+__device__ __forceinline__ void named_arrive(int id, int n) {
+  asm volatile("bar.arrive %0, %1;\n" ::"r"(id), "r"(n) : "memory");
+}
 __device__ __forceinline__ void cta_sync() { asm volatile("bar.sync 0;\n" ::: "memory"); }
+
+// Named barriers: 1 context warps; 3-5 main warps hand operands to the issue warp.
+constexpr int kBarCtx = 1, kBarDsl = 3, kBarDu = 4, kBarG4 = 5;
+constexpr int kHandOff = 128 + 32;   // main warps arrive, the issue warp waits
 
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
@@ -305,10 +343,9 @@ __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, Bwd
 }
 
 // ------------------------------------------------------------------ context warps
-// Decay products, decay-scaled operands, v, dy, S0^T, L_t and the raw r, a, b, k for the main
-// warps' per-token outputs.  A wait for the staged data that runs out marks the chunk unsafe (the
-// unit is then recomputed by the exact scan) and sets `timed_out`, after which nothing more is
-// staged.
+// Decay products, decay-scaled operands, v, dy, S0^T and L_t.  A wait for the staged data that runs
+// out marks the chunk unsafe (the unit is then recomputed by the exact scan) and sets `timed_out`,
+// after which nothing more is staged.
 template <typename T>
 __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
                                                  int64_t unit, int64_t c, int ktid, int len, unsigned parity,
@@ -318,75 +355,79 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
   const T (*X)[kChunk][kN] = sm.stg;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
 
-  // ---- pass B: thread = (token t, 8 channels from j0); one 16-byte core row per array
+  // ---- pass B: thread = (token t, 8 channels from j0), the 16 tokens of a channel group in one
+  // half-warp; one 16-byte core row per array
   bool bad = false;
   {
-    const int t = (lane & 7) + 8 * (kw & 1), j0 = 8 * ((lane >> 3) + 4 * (kw >> 1));
-    // L_{t-1} and L_t: products of the staged decays (rows past T count as w = 1)
+    const int t = lane & 15, j0 = 8 * ((lane >> 4) + 2 * kw);
+    // L_t by a product scan over the half-warp (rows past T count as w = 1); L_{t-1} one lane up
     float L[8], Lp[8];
-#pragma unroll
-    for (int u = 0; u < 8; ++u) Lp[u] = 1.f;
-    for (int s2 = 0; s2 < t; ++s2) {
-      float w[8];
-      unpack16<T>(*reinterpret_cast<const uint4*>(&X[1][s2][j0]), w);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) Lp[u] *= s2 < len ? w[u] : 1.f;
-    }
     {
       float w[8];
       unpack16<T>(*reinterpret_cast<const uint4*>(&X[1][t][j0]), w);
-      float wmin = 1.f, lmin = 1.f, lmax = 1.f;
+      float wmin = 1.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const float wu = t < len ? w[u] : 1.f;
-        L[u] = Lp[u] * wu;
-        wmin = fminf(wmin, wu);
+        L[u] = t < len ? w[u] : 1.f;
+        wmin = fminf(wmin, L[u]);
+      }
+#pragma unroll
+      for (int d = 1; d < kChunk; d *= 2)
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float o = __shfl_up_sync(0xffffffffu, L[u], d, 16);
+          if (t >= d) L[u] *= o;
+        }
+      float lmin = 1.f, lmax = 1.f;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const float o = __shfl_up_sync(0xffffffffu, L[u], 1, 16);
+        Lp[u] = t >= 1 ? o : 1.f;
         lmin = fminf(lmin, L[u]);
         lmax = fmaxf(lmax, L[u]);
       }
       bad = !(wmin >= 0.0625f && lmin >= 0x1p-40f && lmax <= 0x1p40f);
     }
-    *reinterpret_cast<float4*>(&cx.lam[t][j0]) = make_float4(L[0], L[1], L[2], L[3]);
-    *reinterpret_cast<float4*>(&cx.lam[t][j0 + 4]) = make_float4(L[4], L[5], L[6], L[7]);
-    float in[kIn][8];
-#pragma unroll
-    for (int m = 0; m < kIn; ++m) unpack16<T>(*reinterpret_cast<const uint4*>(&X[m][t][j0]), in[m]);
+    float r8[8], k8[8], a8[8], b8[8];
+    unpack16<T>(*reinterpret_cast<const uint4*>(&X[0][t][j0]), r8);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&X[2][t][j0]), k8);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&X[4][t][j0]), a8);
+    unpack16<T>(*reinterpret_cast<const uint4*>(&X[5][t][j0]), b8);
     float at[8], rt[8], bh[8], kh[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const float il = rcp_approx(L[u]);
-      at[u] = in[4][u] * Lp[u];
-      rt[u] = in[0][u] * L[u];
-      bh[u] = in[5][u] * il;
-      kh[u] = in[2][u] * il;
+      at[u] = a8[u] * Lp[u];
+      rt[u] = r8[u] * L[u];
+      bh[u] = b8[u] * il;
+      kh[u] = k8[u] * il;
     }
-    *reinterpret_cast<float4*>(&sm.Atf[t][j0]) = make_float4(at[0], at[1], at[2], at[3]);
-    *reinterpret_cast<float4*>(&sm.Atf[t][j0 + 4]) = make_float4(at[4], at[5], at[6], at[7]);
-#pragma unroll
-    for (int u = 0; u < 8; ++u) {   // transposed copies for the per-key-channel outputs (exact)
-      cx.lamT[j0 + u][t] = L[u];
-      cx.rabkT[0][j0 + u][t] = Elt<T>::from_f32(in[0][u]);
-      cx.rabkT[1][j0 + u][t] = Elt<T>::from_f32(in[4][u]);
-      cx.rabkT[2][j0 + u][t] = Elt<T>::from_f32(in[5][u]);
-      cx.rabkT[3][j0 + u][t] = Elt<T>::from_f32(in[2][u]);
-    }
+    *reinterpret_cast<float4*>(&cx.lam[t][j0]) = make_float4(L[0], L[1], L[2], L[3]);
+    *reinterpret_cast<float4*>(&cx.lam[t][j0 + 4]) = make_float4(L[4], L[5], L[6], L[7]);
     put8(cx.AR, cb(t, j0, 64), at);
     put8(cx.AR, cb(16 + t, j0, 64), rt);
     put8(cx.BK, cb(t, j0, 64), bh);
     put8(cx.BK, cb(16 + t, j0, 64), kh);
-    put8(cx.DYU, cb(t, j0, 64), in[6]);
-    const bool m0t = t < fr;
+  }
+  // ---- v^T, dy^T and m0.dy^T: thread = (channel i, tokens 8 th .. 8 th + 7), one core row each
+  {
+    const int i = ktid & 63, th = ktid >> 6;
+    float v8[8], y8[8], m8[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {   // v^T and m0.dy^T: column t of rows j0..j0+7
-      put1(cx.SV, cb(j0 + u, 16 + t, 32), in[3][u]);
-      put1(cx.DUY, cb(j0 + u, 16 + t, 32), m0t ? in[6][u] : 0.f);
+    for (int e = 0; e < 8; ++e) {
+      const int t = 8 * th + e;
+      v8[e] = Elt<T>::to_f32(X[3][t][i]);
+      y8[e] = Elt<T>::to_f32(X[6][t][i]);
+      m8[e] = t < fr ? y8[e] : 0.f;
     }
+    put8(cx.SV, cb(i, 16 + 8 * th, 32), v8);
+    put8(cx.UYT, cb(i, 16 + 8 * th, 32), y8);
+    put8(cx.DUY, cb(i, 16 + 8 * th, 32), m8);
   }
   const unsigned any_bad = __ballot_sync(0xffffffffu, bad), any_to = __ballot_sync(0xffffffffu, to);
   if (lane == 0) sm.kbad[kw] = (any_bad ? 1 : 0) | (any_to ? 2 : 0);
   tc::fence_smem_to_async();
-  tc::fence_before_sync();
-  named_bar(1, 128);
+  named_bar(kBarCtx, 128);
   const int kb = sm.kbad[0] | sm.kbad[1] | sm.kbad[2] | sm.kbad[3];
   unsafe = kb != 0;
   timed_out = (kb & 2) != 0;
@@ -410,7 +451,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
     put8(cx.S0T, cb(j, i0, 64), s);
   }
   tc::fence_smem_to_async();
-  named_bar(1, 128);
+  named_bar(kBarCtx, 128);
   if (timed_out && ktid == 0 && p.status) atomicOr(p.status, kStatusWaitTimeout);
   if (ktid == 0) {
     cx.mask = int(mask);
@@ -418,12 +459,16 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
   }
 }
 
-// The rest of the context: Gram, T, W, X and SA^T (safe chunks only).
+// The rest of the context (safe chunks only): the masked Gram, T, X, the folded operands BKx, Qm,
+// Vq and W, and SA^T.
 template <typename T>
-__device__ __forceinline__ void context_products(BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask, int ktid) {
+__device__ __forceinline__ void context_products(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, Ctx<T>& cx,
+                                                 unsigned mask, int ktid, int64_t unit, int64_t b, int64_t h,
+                                                 int64_t c_stage, int64_t nc) {
   constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
   const int kw = ktid >> 5, lane = ktid & 31;
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
+  const unsigned ls_bits = last_segment_bits(mask);
 
   // ---- the masked Gram [At; Rt] [Bh; Kh]^T: warp kw computes block (kw / 2, kw % 2) of 16 x 16
   // (Lab, Lak, Mrb, Mrk), rows t, columns tau
@@ -436,6 +481,7 @@ __device__ __forceinline__ void context_products(BwdSmem<T>& sm, Ctx<T>& cx, uns
       mma_split2(acc, afrag_k<64>(cx.AR.hi, 16 * mb, 16 * ks, lane), a_lo, false, false,
                  bfrag_k<64>(cx.BK.hi, 16 * nb, 16 * ks, lane), b_lo);
     const bool strict = mb == 0;
+    float (*dst)[kChunk] = kw == 1 ? sm.LakP : kw == 2 ? sm.MrbP : sm.MrkP;
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
@@ -446,65 +492,151 @@ __device__ __forceinline__ void context_products(BwdSmem<T>& sm, Ctx<T>& cx, uns
         if (kw == 0) {
           sm.LabT[tau][t] = v0;
           sm.LabT[tau + 1][t] = v1;
-        } else if (kw == 1) {
-          cx.LakP[t][tau] = v0;
-          cx.LakP[t][tau + 1] = v1;
-        } else {   // [Mrb | Mrk] row t: a split pair
-          const int e = cb(t, 16 * nb + tau, 32);
-          const __nv_bfloat162 hh2 = __floats2bfloat162_rn(v0, v1);
-          const float2 hf = __bfloat1622float2(hh2);
-          *reinterpret_cast<__nv_bfloat162*>(&cx.MM.hi[e]) = hh2;
-          *reinterpret_cast<__nv_bfloat162*>(&cx.MM.lo[e]) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
+        } else {
+          *reinterpret_cast<float2*>(&dst[t][tau]) = make_float2(v0, v1);
         }
       }
   }
-  named_bar(1, 128);
+  named_bar(kBarCtx, 128);
 
-  // ---- T = (I - Lab)^-1 by forward substitution, one column per thread (threads 0-15)
+  // ---- T = (I - Lab)^-1 by forward substitution, one column cc per thread (threads 0-15), which
+  // also writes row cc of Tl^T (the top-left block of AC) and of (T m0)^T; threads 16-31 write the
+  // right-hand blocks of AC (zero above, diag(ls) below); thread 32 stages the next chunk (the
+  // staged inputs and checkpoint of this one are consumed)
   if (ktid < kChunk) {
     const int cc = ktid;
     float u[kChunk];
 #pragma unroll
     for (int t = 0; t < kChunk; ++t) u[t] = t == cc ? 1.f : 0.f;
+    // whole rows of Lab^T: its entries on and left of the diagonal are zero, so they add nothing
 #pragma unroll
     for (int tau = 0; tau < kChunk - 1; ++tau) {
+      float l[kChunk];
 #pragma unroll
-      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(sm.LabT[tau][t], u[tau], u[t]);
-    }
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) cx.Tp[t][cc] = u[t];
-  }
-  named_bar(1, 128);
-
-  // ---- X = T Lak: thread -> (tau, two t); W = T m0.At: thread -> (tau, 8 j)
-  {
-    const int tau = ktid >> 3;
-    if ((ktid & 7) < 2) {   // X row tau, columns 8 (ktid & 7) .. +7
-      const int t0 = 8 * (ktid & 7);
-      float x[8] = {};
-#pragma unroll
-      for (int s = 0; s < kChunk; ++s) {
-        const float tv = cx.Tp[tau][s];
-#pragma unroll
-        for (int e = 0; e < 8; ++e) x[e] = fmaf(tv, cx.LakP[s][t0 + e], x[e]);
+      for (int q = 0; q < 4; ++q) {
+        const float4 v = *reinterpret_cast<const float4*>(&sm.LabT[tau][4 * q]);
+        l[4 * q] = v.x; l[4 * q + 1] = v.y; l[4 * q + 2] = v.z; l[4 * q + 3] = v.w;
       }
-      put8(sm.XC, cb(tau, t0, 16), x);
-    }
-    const int j0 = 8 * (ktid & 7);
-    float w[8] = {};
 #pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float tv = t < fr ? cx.Tp[tau][t] : 0.f;
-      const float4 a0 = *reinterpret_cast<const float4*>(&sm.Atf[t][j0]);
-      const float4 a1 = *reinterpret_cast<const float4*>(&sm.Atf[t][j0 + 4]);
-      w[0] = fmaf(tv, a0.x, w[0]); w[1] = fmaf(tv, a0.y, w[1]); w[2] = fmaf(tv, a0.z, w[2]); w[3] = fmaf(tv, a0.w, w[3]);
-      w[4] = fmaf(tv, a1.x, w[4]); w[5] = fmaf(tv, a1.y, w[5]); w[6] = fmaf(tv, a1.z, w[6]); w[7] = fmaf(tv, a1.w, w[7]);
+      for (int t = tau + 1; t < kChunk; ++t) u[t] = fmaf(l[t], u[tau], u[t]);
     }
-    put8(sm.WC, cb(tau, j0, 64), w);
+#pragma unroll
+    for (int t = 0; t < kChunk; ++t) sm.Tp[t][cc] = u[t];
+    const float m0c = cc < fr ? 1.f : 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float tl[8], tm[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const int t = 8 * q + e;
+        tl[e] = (ls_bits >> t) & 1u ? u[t] : 0.f;   // Tl^T[cc][t] = ls_t T[t][cc]
+        tm[e] = m0c * u[t];                         // (T m0)^T[cc][tau] = T[tau][cc] m0_cc
+      }
+      put8(sm.AC, cb(cc, 8 * q, 32), tl);
+      put8(sm.TmT, cb(cc, 8 * q, 16), tm);
+    }
+  } else if (ktid < 2 * kChunk) {
+    const int tau = ktid - kChunk;
+    const float lt = (ls_bits >> tau) & 1u ? 1.f : 0.f;
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      float z[8], d[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        z[e] = 0.f;
+        d[e] = 8 * q + e == tau ? lt : 0.f;
+      }
+      put8(sm.AC, cb(tau, 16 + 8 * q, 32), z);
+      put8(sm.AC, cb(16 + tau, 16 + 8 * q, 32), d);
+    }
+  } else if (c_stage >= 0) {
+    stage<T>(p, tm, sm, unit, b, h, c_stage, nc, ktid - 2 * kChunk);
   }
-  tc::fence_smem_to_async();
-  tc::fence_before_sync();
-  named_bar(1, 128);
+  named_bar(kBarCtx, 128);
+
+  // ---- X = T Lak (threads 0-31) and Qm = Mrb T (threads 32-63): thread -> (row r, 8 columns)
+  if (ktid < 4 * kChunk) {
+    const int r = (ktid >> 1) & 15, c0 = 8 * (ktid & 1);
+    const bool isx = ktid < 2 * kChunk;
+    const float (*A)[kChunk] = isx ? sm.Tp : sm.MrbP;
+    const float (*B)[kChunk] = isx ? sm.LakP : sm.Tp;
+    float x[8] = {};
+#pragma unroll
+    for (int s = 0; s < kChunk; ++s) {
+      const float av = A[r][s];
+      const float4 b0 = *reinterpret_cast<const float4*>(&B[s][c0]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&B[s][c0 + 4]);
+      x[0] = fmaf(av, b0.x, x[0]); x[1] = fmaf(av, b0.y, x[1]); x[2] = fmaf(av, b0.z, x[2]); x[3] = fmaf(av, b0.w, x[3]);
+      x[4] = fmaf(av, b1.x, x[4]); x[5] = fmaf(av, b1.y, x[5]); x[6] = fmaf(av, b1.z, x[6]); x[7] = fmaf(av, b1.w, x[7]);
+    }
+    if (isx) {
+      put8(sm.XC, cb(r, c0, 16), x);
+      *reinterpret_cast<float4*>(&sm.Xp[r][c0]) = make_float4(x[0], x[1], x[2], x[3]);
+      *reinterpret_cast<float4*>(&sm.Xp[r][c0 + 4]) = make_float4(x[4], x[5], x[6], x[7]);
+    } else {
+      put8(cx.MMx, cb(r, c0, 32), x);
+    }
+  }
+  named_bar(kBarCtx, 128);
+
+  // ---- Vq = Mrk + Mrb X (threads 0-31) and the (ls.X)^T block of AC (threads 32-63)
+  if (ktid < 2 * kChunk) {
+    const int r = ktid >> 1, c0 = 8 * (ktid & 1);
+    float x[8];
+    {
+      const float4 m0v = *reinterpret_cast<const float4*>(&sm.MrkP[r][c0]);
+      const float4 m1v = *reinterpret_cast<const float4*>(&sm.MrkP[r][c0 + 4]);
+      x[0] = m0v.x; x[1] = m0v.y; x[2] = m0v.z; x[3] = m0v.w; x[4] = m1v.x; x[5] = m1v.y; x[6] = m1v.z; x[7] = m1v.w;
+    }
+#pragma unroll
+    for (int s = 0; s < kChunk; ++s) {
+      const float av = sm.MrbP[r][s];
+      const float4 b0 = *reinterpret_cast<const float4*>(&sm.Xp[s][c0]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&sm.Xp[s][c0 + 4]);
+      x[0] = fmaf(av, b0.x, x[0]); x[1] = fmaf(av, b0.y, x[1]); x[2] = fmaf(av, b0.z, x[2]); x[3] = fmaf(av, b0.w, x[3]);
+      x[4] = fmaf(av, b1.x, x[4]); x[5] = fmaf(av, b1.y, x[5]); x[6] = fmaf(av, b1.z, x[6]); x[7] = fmaf(av, b1.w, x[7]);
+    }
+    put8(cx.MMx, cb(r, 16 + c0, 32), x);
+  } else if (ktid < 4 * kChunk) {   // AC[16 + tau][t] = ls_t X[t][tau]
+    const int tau = (ktid - 2 * kChunk) >> 1, t0 = 8 * (ktid & 1);
+    float z[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) z[e] = (ls_bits >> (t0 + e)) & 1u ? sm.Xp[t0 + e][tau] : 0.f;
+    put8(sm.AC, cb(16 + tau, t0, 32), z);
+  }
+  named_bar(kBarCtx, 128);
+
+  // ---- W = (T m0) At (warp kw: columns 16 kw .. 16 kw + 15) and BKx = AC [Bh; Kh] (warp kw: rows
+  // 16 (kw % 2) .., columns 32 (kw / 2) ..), warp-level split products
+  {
+    const int g = lane >> 2, c4 = lane & 3;
+    {
+      float acc[2][4] = {};
+      mma_split2(acc, afrag_mn<16>(sm.TmT.hi, 0, 0, lane), uint32_t(sizeof(sm.TmT.hi)), true, false,
+                 bfrag_mn<64>(cx.AR.hi, 16 * kw, 0, lane), uint32_t(sizeof(cx.AR.hi)), true);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          put2(sm.WC, cb(g + 8 * hh, 16 * kw + 8 * nt + 2 * c4, 64), acc[nt][2 * hh], acc[nt][2 * hh + 1]);
+    }
+    const int mb = kw & 1, n0 = 32 * (kw >> 1);
+#pragma unroll
+    for (int np = 0; np < 2; ++np) {
+      float acc[2][4] = {};
+#pragma unroll
+      for (int ks = 0; ks < 2; ++ks)
+        mma_split2(acc, afrag_k<32>(sm.AC.hi, 16 * mb, 16 * ks, lane), uint32_t(sizeof(sm.AC.hi)), false, false,
+                   bfrag_mn<64>(cx.BK.hi, n0 + 16 * np, 16 * ks, lane), uint32_t(sizeof(cx.BK.hi)), true);
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+          put2(cx.BKx, cb(16 * mb + g + 8 * hh, n0 + 16 * np + 8 * nt + 2 * c4, 64), acc[nt][2 * hh],
+               acc[nt][2 * hh + 1]);
+    }
+  }
+  named_bar(kBarCtx, 128);
 
   // ---- SA^T = S0 W^T + V^T X^T: warp kw computes rows i = 16 kw .. 16 kw + 15, columns tau
   {
@@ -519,24 +651,50 @@ __device__ __forceinline__ void context_products(BwdSmem<T>& sm, Ctx<T>& cx, uns
 #pragma unroll
     for (int nt = 0; nt < 2; ++nt)
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        const int i = 16 * kw + g + 8 * hh, tau = 8 * nt + 2 * c4;
-        const int e = cb(i, tau, 32);
-        const float v0 = acc[nt][2 * hh], v1 = acc[nt][2 * hh + 1];
-        const __nv_bfloat162 hh2 = __floats2bfloat162_rn(v0, v1);
-        const float2 hf = __bfloat1622float2(hh2);
-        *reinterpret_cast<__nv_bfloat162*>(&cx.SV.hi[e]) = hh2;
-        *reinterpret_cast<__nv_bfloat162*>(&cx.SV.lo[e]) = __floats2bfloat162_rn(v0 - hf.x, v1 - hf.y);
-      }
+      for (int hh = 0; hh < 2; ++hh)
+        put2(cx.SV, cb(16 * kw + g + 8 * hh, 8 * nt + 2 * c4, 32), acc[nt][2 * hh], acc[nt][2 * hh + 1]);
   }
   tc::fence_smem_to_async();
+}
+
+// ------------------------------------------------------------------ issue warp
+// One thread issues every tensor-core product of chunk c, in three batches, each as soon as the
+// main warps have handed over its operands (named barriers kBarDsl, kBarDu, kBarG4).
+template <typename T>
+__device__ __forceinline__ void issue_chunk(BwdSmem<T>& sm, Ctx<T>& cx, uint32_t tmem, bool leader) {
+  constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
+  named_bar(kBarDsl, kHandOff);
+  if (leader) {
+    tc::fence_after_sync();
+    // GU = dSl BKx^T + dY^T [Qm | Vq]                          (rows i: dU^T | dV^T)
+    mma3<32, 4>(tmem + kColGU, op<64, true>(sm.dSlT), op<64, false>(cx.BKx), false);
+    mma3<32, 1>(tmem + kColGU, op<32, false>(cx.UYT, kExactIn, 0, 16), op<32, true>(cx.MMx), true);   // dy^T
+    tc::commit(&sm.u_bar);
+  }
+  named_bar(kBarDu, kHandOff);
+  if (leader) {
+    tc::fence_after_sync();
+    mma3<32, 4>(tmem + kColGG, op<32, true>(cx.UYT), op<32, true>(cx.SV), false);   // [dU; dY] [SA^T | v^T]
+    tc::commit(&sm.gg_bar);
+    mma3<32, 4>(tmem + kColE + 64, op<64, false>(sm.dSlT), op<32, true>(cx.SV), false);   // dSl^T [SA^T | v^T]
+    // dS0^T += Rt^T m0.dy + At^T m0.dU (the carried gradient of the chunk before)
+    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR, false, 16), op<32, false>(cx.DUY, kExactIn, 0, 16), true);
+    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR), op<32, false>(cx.DUY), true);
+    mma3<32, 4>(tmem + kColE, op<64, false>(cx.S0T), op<32, true>(cx.DUY), false);   // S0^T [m0.dU^T | m0.dy^T]
+  }
+  named_bar(kBarG4, kHandOff);
+  if (leader) {
+    tc::fence_after_sync();
+    mma3<32, 2>(tmem + kColE, op<64, true>(cx.BK), op<32, false>(sm.G4), true);        // += [Bh^T|Kh^T] [dLab^T dMrb^T; dLak^T dMrk^T]
+    mma3<32, 2>(tmem + kColE + 32, op<64, true>(cx.AR), op<32, true>(sm.G4), false);   // [At^T|Rt^T] [dLab dLak; dMrb dMrk]
+    tc::commit(&sm.e_bar);
+  }
 }
 
 // ------------------------------------------------------------------ main warps
 template <typename T>
 __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, int64_t b, int64_t h,
                                            int64_t t0, int len, int warp, int lane, uint32_t tmem, unsigned phase) {
-  constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
   const uint32_t tlane = uint32_t(32 * warp) << 16;
   const unsigned mask = unsigned(cx.mask);
   const int fr = mask ? __ffs(int(mask)) - 1 : kChunk;
@@ -544,6 +702,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   const bool keep = mask == 0u;
   const int row = 16 * warp + (lane & 15);   // TMEM row of this thread (both halves of the warp)
   const int half = lane >> 4;                // which half of a row's columns this thread holds
+  const int tb = 8 * half;                   // first token of this thread in per-token phases
+  const int64_t rs = p.H * kN, total = p.B * p.T * p.H * kN;
 
   // ---- M1: dSl^T = L_15 dS^T (row j = row) into shared memory for the chain products.  This
   // thread holds columns 16 half + (0..15) and 32 + 16 half + (0..15) of its row.
@@ -572,15 +732,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  named_bar(2, 128);
+  named_arrive(kBarDsl, kHandOff);
 
-  // ---- M2: G1 = dSl [Bh|Kh]^T, G2 = dY^T [Mrb|Mrk]
-  if (threadIdx.x == 0) {
-    tc::fence_after_sync();
-    mma3<32, 4>(tmem + kColG1, op<64, true>(sm.dSlT), op<64, false>(cx.BK), false);
-    mma3<32, 1>(tmem + kColG2, op<64, true>(cx.DYU, kExactIn), op<32, true>(cx.MM), false);   // dy rows of DYU
-    tc::commit(&sm.u_bar);
-  }
   // while the tensor core works: keep.dSl^T back into TMEM (the start of dS0^T) and the L_15 term
   // keep.sum_i dSl o S0 of this key channel (each half of the row, then both halves added)
   float dl15 = 0.f;
@@ -606,58 +759,20 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   }
   mma_wait(p, &sm.u_bar, phase & 1u);
 
-  // ---- M3: dSA^T, dU^T = dSA^T T and dV^T per value channel i = row (FP32 cores); this thread holds
-  // tokens 8 half .. 8 half + 7 of its row; dv out, dU into shared memory
+  // ---- M3: dU^T and dV^T of value channel i = row for tokens tb .. tb + 7, straight from GU; dU
+  // into shared memory (UYT, and DUY masked to the tokens before the first reset), dv out
   {
-    float g1b[8], g1k[8], g2b[8], g2k[8];
-    tc::ld_16x32bx2_x8(tmem + tlane + kColG1, g1b);
-    tc::ld_16x32bx2_x8(tmem + tlane + kColG1 + 16, g1k);
-    tc::ld_16x32bx2_x8(tmem + tlane + kColG2, g2b);
-    tc::ld_16x32bx2_x8(tmem + tlane + kColG2 + 16, g2k);
+    float du[8], dv[8];
+    tc::ld_16x32bx2_x8(tmem + tlane + kColGU, du);
+    tc::ld_16x32bx2_x8(tmem + tlane + kColGU + 16, dv);
     tc::wait_ld();
-    const int i = row, tb = 8 * half;
-    float dsa[16], du[8], dv[8];
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      const float mine = ((ls_bits >> (tb + e)) & 1u ? g1b[e] : 0.f) + g2b[e];
-      const float other = __shfl_xor_sync(0xffffffffu, mine, 16);
-      dsa[e] = half ? other : mine;
-      dsa[8 + e] = half ? mine : other;
-      du[e] = 0.f;
-      dv[e] = ((ls_bits >> (tb + e)) & 1u ? g1k[e] : 0.f) + g2k[e];
-    }
-    // dU^T[i][tau] = sum_t dSA^T[i][t] T[t][tau] (T is stored with zeros above its diagonal)
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float4 a = *reinterpret_cast<const float4*>(&cx.Tp[t][tb]);
-      const float4 c = *reinterpret_cast<const float4*>(&cx.Tp[t][tb + 4]);
-      du[0] = fmaf(dsa[t], a.x, du[0]); du[1] = fmaf(dsa[t], a.y, du[1]);
-      du[2] = fmaf(dsa[t], a.z, du[2]); du[3] = fmaf(dsa[t], a.w, du[3]);
-      du[4] = fmaf(dsa[t], c.x, du[4]); du[5] = fmaf(dsa[t], c.y, du[5]);
-      du[6] = fmaf(dsa[t], c.z, du[6]); du[7] = fmaf(dsa[t], c.w, du[7]);
-    }
-    // dV^T[i][tau] += sum_t dU^T[i][t] Lak[t][tau] (Lak is zero on and above its diagonal)
-#pragma unroll
-    for (int t = 0; t < kChunk; ++t) {
-      const float mine = du[t & 7], other = __shfl_xor_sync(0xffffffffu, mine, 16);
-      const float dut = ((t >> 3) == half) ? mine : other;
-      const float4 a = *reinterpret_cast<const float4*>(&cx.LakP[t][tb]);
-      const float4 c = *reinterpret_cast<const float4*>(&cx.LakP[t][tb + 4]);
-      dv[0] = fmaf(dut, a.x, dv[0]); dv[1] = fmaf(dut, a.y, dv[1]);
-      dv[2] = fmaf(dut, a.z, dv[2]); dv[3] = fmaf(dut, a.w, dv[3]);
-      dv[4] = fmaf(dut, c.x, dv[4]); dv[5] = fmaf(dut, c.y, dv[5]);
-      dv[6] = fmaf(dut, c.z, dv[6]); dv[7] = fmaf(dut, c.w, dv[7]);
-    }
-    // dU: rows 16 + t of DYU (column i) and, masked to the tokens before the first reset, DUY
+    const int i = row;
     float v[8];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      put1(cx.DYU, cb(16 + tb + e, i, 64), du[e]);
-      v[e] = tb + e < fr ? du[e] : 0.f;
-    }
+    for (int e = 0; e < 8; ++e) v[e] = tb + e < fr ? du[e] : 0.f;
+    put8(cx.UYT, cb(i, tb, 32), du);
     put8(cx.DUY, cb(i, tb, 32), v);
     T* dvp = static_cast<T*>(p.dv) + tok_off(b, t0 + tb, h, p.T, p.H) + i;
-    const int64_t rs = p.H * kN, total = p.B * p.T * p.H * kN;
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       if (tb + e < len && range_ok(tok_off(b, t0 + tb + e, h, p.T, p.H) + i, 1, total, p.status))
@@ -667,30 +782,38 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  named_bar(2, 128);
+  named_arrive(kBarDu, kHandOff);
 
-  // ---- M4: rest of dS0^T; gradient Gram; the S0 and dSl parts of the key-space products
-  if (threadIdx.x == 0) {
-    tc::fence_after_sync();
-    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR, false, 16), op<32, false>(cx.DUY, kExactIn, 0, 16), true);
-    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR), op<32, false>(cx.DUY), true);   // dS0^T += Rt^T m0.dy + At^T m0.dU
-    tc::commit(&sm.chain_bar);
-    const auto SV_M = op<32, true>(cx.SV);
-    mma3<32, 4>(tmem + kColGG, op<64, false>(cx.DYU), SV_M, false);   // [dY; dU] [SA^T | v^T]   (rows t, 16 + t)
-    mma3<32, 4>(tmem + kColE, op<64, false>(cx.S0T), op<32, true>(cx.DUY), false);   // S0^T [m0.dU^T | m0.dy^T] (rows j)
-    mma3<32, 4>(tmem + kColE + 64, op<64, false>(sm.dSlT), SV_M, false);       // dSl^T [SA^T | v^T]
-    tc::commit(&sm.gg_bar);
+  // r, a, b, k of this thread's key channel and tokens for the last phase (cache hits: the context
+  // staged the same rows one chunk earlier), loaded while the tensor core works
+  const int j = row;
+  const int64_t o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
+  float rr[8], ar[8], br[8], kr[8];
+  {
+    const T* const gr = static_cast<const T*>(p.r);
+    const T* const ga = static_cast<const T*>(p.a);
+    const T* const gb = static_cast<const T*>(p.b);
+    const T* const gk = static_cast<const T*>(p.k);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      const int64_t o = o0 + e * rs;
+      const bool ok = tb + e < len && range_ok(o, 1, total, p.status);
+      rr[e] = ok ? Elt<T>::to_f32(gr[o]) : 0.f;
+      ar[e] = ok ? Elt<T>::to_f32(ga[o]) : 0.f;
+      br[e] = ok ? Elt<T>::to_f32(gb[o]) : 0.f;
+      kr[e] = ok ? Elt<T>::to_f32(gk[o]) : 0.f;
+    }
   }
   mma_wait(p, &sm.gg_bar, phase & 1u);
 
   // ---- M5: masked gradient Gram into the B operand of the key-space products.  Warp 0 holds rows
-  // t of [dMrb | dMrk] (causal), warp 1 rows t of [dLab | dLak] (strictly causal).
+  // t of [dLab | dLak] (strictly causal), warp 1 rows t of [dMrb | dMrk] (causal).
   if (warp < 2) {   // this thread: row t = lane % 16, columns 16 half .. 16 half + 15 (the b or the k block)
     float g[16];
     tc::ld_16x32bx2_x16(tmem + tlane + kColGG, g);
     tc::wait_ld();
     const int t = lane & 15;
-    const bool strict = warp == 1;
+    const bool strict = warp == 0;
 #pragma unroll
     for (int tau = 0; tau < kChunk; ++tau) g[tau] = pair_ok(mask, t, tau, strict) ? g[tau] : 0.f;
     const int r = strict ? t : 16 + t;   // G4 rows t: [dLab | dLak]; rows 16 + t: [dMrb | dMrk]
@@ -704,20 +827,12 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   }
   tc::fence_smem_to_async();
   tc::fence_before_sync();
-  named_bar(2, 128);
-  if (threadIdx.x == 0) {
-    tc::fence_after_sync();
-    const auto BK_M = op<64, true>(cx.BK), AR_M = op<64, true>(cx.AR);
-    mma3<32, 2>(tmem + kColE, BK_M, op<32, false>(sm.G4), true);        // += [Bh^T|Kh^T] [dLab^T dMrb^T; dLak^T dMrk^T]
-    mma3<32, 2>(tmem + kColE + 32, AR_M, op<32, true>(sm.G4), false);   // [At^T|Rt^T] [dLab dLak; dMrb dMrk]
-    tc::commit(&sm.e_bar);
-  }
+  named_arrive(kBarG4, kHandOff);
   mma_wait(p, &sm.e_bar, phase & 1u);
 
   // ---- M6: per key channel j = row: da, dr, db, dk and dw over the chunk's tokens; this thread
-  // holds tokens tb .. tb + 7 of its channel (tb = 8 half)
+  // holds tokens tb .. tb + 7 of its channel
   {
-    const int j = row, tb = 8 * half;
     float eA[8], eR[8], eB[8], eK[8], xb[8], xk[8];
     tc::ld_16x32bx2_x8(tmem + tlane + kColE, eA);
     tc::ld_16x32bx2_x8(tmem + tlane + kColE + 16, eR);
@@ -726,17 +841,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
     tc::ld_16x32bx2_x8(tmem + tlane + kColE + 64, xb);
     tc::ld_16x32bx2_x8(tmem + tlane + kColE + 80, xk);
     float Lr[9];   // L_{tb-1} .. L_{tb+7}
-    {
-      const float4 a = *reinterpret_cast<const float4*>(&cx.lamT[j][tb]);
-      const float4 c = *reinterpret_cast<const float4*>(&cx.lamT[j][tb + 4]);
-      Lr[1] = a.x; Lr[2] = a.y; Lr[3] = a.z; Lr[4] = a.w; Lr[5] = c.x; Lr[6] = c.y; Lr[7] = c.z; Lr[8] = c.w;
-      Lr[0] = half ? cx.lamT[j][tb - 1] : 1.f;
-    }
-    float rr[8], ar[8], br[8], kr[8];
-    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[0][j][tb]), rr);
-    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[1][j][tb]), ar);
-    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[2][j][tb]), br);
-    unpack16<T>(*reinterpret_cast<const uint4*>(&cx.rabkT[3][j][tb]), kr);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) Lr[e + 1] = cx.lam[tb + e][j];
+    Lr[0] = half ? cx.lam[tb - 1][j] : 1.f;
     tc::wait_ld();
     float DL[8], il[8], e3 = 0.f, sumDL = 0.f, firstA = 0.f;
 #pragma unroll
@@ -760,7 +867,6 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
     e3 += __shfl_xor_sync(0xffffffffu, e3, 16);
     const float upper = __shfl_xor_sync(0xffffffffu, sumDL, 16);   // sum over tokens 8..15, for half 0
     float cum = dl15 + e3 + (half ? 0.f : upper);
-    const int64_t rs = p.H * kN, o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
     T* const gda = static_cast<T*>(p.da);
     T* const gdr = static_cast<T*>(p.dr);
     T* const gdb = static_cast<T*>(p.db);
@@ -769,7 +875,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
 #pragma unroll
     for (int e = 7; e >= 0; --e) {
       cum += DL[e];
-      if (tb + e < len && range_ok(o0 + e * rs, 1, p.B * p.T * p.H * kN, p.status)) {
+      if (tb + e < len && range_ok(o0 + e * rs, 1, total, p.status)) {
         const int64_t o = o0 + e * rs;
         gda[o] = Elt<T>::from_f32(eA[e] * Lr[e]);
         gdr[o] = Elt<T>::from_f32(eR[e] * Lr[e + 1]);
@@ -790,7 +896,6 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   const int64_t unit = blockIdx.x;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const bool is_main = warp < 4;
   const int ktid = tid - 128;
   const int64_t nc = (p.T + kChunk - 1) / kChunk;
 
@@ -801,11 +906,10 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
     sm.stop = 0;
     mbar_init(&sm.in_bar, 1);
     mbar_init(&sm.u_bar, 1);
-    mbar_init(&sm.chain_bar, 1);
     mbar_init(&sm.gg_bar, 1);
     mbar_init(&sm.e_bar, 1);
   }
-  if (warp == 0) {   // 512 TMEM columns: this kernel runs one CTA per SM (its shared memory)
+  if (warp == 0) {   // this kernel runs one CTA per SM (its shared memory)
     tc::alloc(&sm.tmem_base, kTmemCols);
     tc::relinquish();
   }
@@ -814,9 +918,9 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
   tc::fence_after_sync();
   const uint32_t tmem = sm.tmem_base;
 
-  // The two roles run separate loops so that their register sets never overlap; both meet at
-  // one CTA barrier per iteration (bar.sync 0, executed by all 256 threads).
-  if (is_main) {
+  // The three roles run separate loops so that their register sets never overlap; all meet at one
+  // CTA barrier per iteration (bar.sync 0, executed by all 288 threads).
+  if (warp < 4) {
     // dS^T entering the last chunk: dsT transposed (row j = TMEM row 16 warp + lane), or zero
     {
       const int j = 16 * warp + lane;
@@ -838,7 +942,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
     for (int64_t it = 0; it <= nc; ++it) {
       if (it >= 1) {
         const int64_t c = nc - it;   // chunk whose gradients are computed now
-        Ctx<T>& cx = sm.ctx[c & 1];   // the main warps own this buffer until the next CTA barrier
+        Ctx<T>& cx = sm.ctx[c & 1];   // the main and issue warps own this buffer until the next CTA barrier
         if (cx.unsafe) {
           if (tid == 0) sm.stop = 1;
         } else {
@@ -869,7 +973,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     unsigned mask_next;
     unsigned phase = 0;        // staging phase of the next wait
     bool pending = true;       // a staging was issued and not yet waited for
@@ -891,15 +995,15 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
           pending = false;
           ++phase;
         }
-        // the staged inputs and checkpoint are consumed: prefetch the previous chunk
+        // the staged inputs and checkpoint are consumed: the previous chunk is staged during the
+        // products (by a thread idle there)
         if (c > 0 && !unsafe) {
-          stage<T>(p, tm, sm, unit, b, h, c - 1, nc, ktid);
           pending = true;
           mask_next = __ballot_sync(0xffffffffu, f_prev) & 0xffffu;   // chunk c-1
           f_prev = reset_flag(p, b, c - 2, lane);
         }
         if (!unsafe) {
-          context_products<T>(sm, cx, mask, ktid);
+          context_products<T>(p, tm, sm, cx, mask, ktid, unit, b, h, c > 0 ? c - 1 : -1, nc);
         }
       }
       cta_sync();
@@ -907,6 +1011,17 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
     }
     // copies issued but never waited for (the unit stopped early) must land before the CTA exits
     if (pending) mbar_wait_bounded(&sm.in_bar, phase & 1u, timed_out ? kWaitLimitNs / 100 : kWaitLimitNs);
+  } else {
+    cta_sync();   // prologue
+    for (int64_t it = 0; it <= nc; ++it) {
+      if (it >= 1) {
+        const int64_t c = nc - it;
+        Ctx<T>& cx = sm.ctx[c & 1];
+        if (!cx.unsafe) issue_chunk<T>(sm, cx, tmem, tid == kIssueTid);
+      }
+      cta_sync();
+      if (sm.stop) break;
+    }
   }
   // every MMA was waited for and every TMEM load is complete: release TMEM
   tc::fence_before_sync();

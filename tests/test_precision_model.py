@@ -134,8 +134,10 @@ def split_bf16(x):
 
 def bwd_model(x, dy, reset, rd):
     """One (b,h) unit through the chunked backward's dataflow: state checkpoints every 16 tokens from
-    an fp64 forward (rounded to fp32), then per chunk in reverse the transposed products of the
-    kernel with operands rounded by ``rd``; the carried dS^T, the 16x16 solves and the per-token
+    an fp64 forward (rounded to fp32), then per chunk in reverse the kernel's products with operands
+    rounded by ``rd`` -- the Gram, W = (T m0) At, the folded BKx = [Tl^T 0; (ls.X)^T diag(ls)] [Bh; Kh],
+    SA^T, GU = dSl BKx^T + dY^T [Qm | Vq] (dU^T | dV^T), the rest of dS0^T, the gradient Gram and the
+    key-space products; the carried dS^T, the 16x16 solve and products (X, Qm, Vq) and the per-token
     outputs in fp32.  Returns the six gradients [T, 64]."""
     T_, N = x["r"].shape
     C = 16
@@ -150,6 +152,7 @@ def bwd_model(x, dy, reset, rd):
             sa = S @ x["a"][t]
             S = S * x["w"][t][None] + np.outer(sa, x["b"][t]) + np.outer(x["v"][t], x["k"][t])
     mm = lambda a, b: (rd(a).astype(np.float64) @ rd(b).astype(np.float64)).astype(F32)   # noqa: E731
+    f32mm = lambda a, b: (a.astype(F32) @ b.astype(F32)).astype(F32)                      # noqa: E731
     g = {n: np.zeros((T_, N), F32) for n in ("dr", "dw", "dk", "dv", "da", "db")}
     dST = np.zeros((N, N), F32)
     for c in reversed(range(nc)):
@@ -176,20 +179,24 @@ def bwd_model(x, dy, reset, rd):
         Tm = np.eye(C, dtype=F32)
         for t in range(1, C):
             Tm[t, :t] = Lab[t, :t] @ Tm[:t, :t]
-        W = (Tm @ (m0 * At)).astype(F32)
-        X = (Tm @ Lak).astype(F32)
+        X = f32mm(Tm, Lak)
+        W = mm(Tm * m0.T, At)
+        AC = np.zeros((2 * C, 2 * C), F32)
+        AC[:C, :C] = (ls[:, None] * Tm).T
+        AC[C:, :C] = (ls[:, None] * X).T
+        AC[C:, C:] = np.diag(ls)
+        BKx = mm(AC, np.vstack([Bh, Kh]))
+        Qm = f32mm(Mrb, Tm)
+        Vq = (Mrk + f32mm(Mrb, X)).astype(F32)
         SAT = mm(S0, W.T) + mm(v.T, X.T)                       # SA^T [i][tau]
         dSlT = dST * lam[-1][:, None]                          # dSl^T [j][i]
-        G1 = mm(dSlT.T, np.vstack([Bh, Kh]).T)                 # [i][32]
-        G2 = mm(DY.T, np.hstack([Mrb, Mrk]))
-        dsaT = G1[:, :C] * ls[None] + G2[:, :C]
-        duT = (dsaT @ Tm).astype(F32)                          # dU^T [i][tau] (fp32 cores)
-        dvT = G1[:, C:] * ls[None] + G2[:, C:] + (duT @ Lak).astype(F32)
+        GU = mm(dSlT.T, BKx.T) + mm(DY.T, np.hstack([Qm, Vq]))
+        duT, dvT = GU[:, :C], GU[:, C:]                        # dU^T, dV^T [i][tau]
         m0dU, m0dY = m0 * duT.T, m0 * DY
         dST = (keep * dSlT + mm(Rt.T, m0dY) + mm(At.T, m0dU)).astype(F32)
-        GG = mm(np.vstack([DY, duT.T]), np.hstack([SAT, v.T]))
-        dMrb, dMrk = GG[:C, :C] * lower, GG[:C, C:] * lower
-        dLab, dLak = GG[C:, :C] * strict, GG[C:, C:] * strict
+        GG = mm(np.vstack([duT.T, DY]), np.hstack([SAT, v.T]))
+        dLab, dLak = GG[:C, :C] * strict, GG[:C, C:] * strict
+        dMrb, dMrk = GG[C:, :C] * lower, GG[C:, C:] * lower
         E01 = mm(S0.T, np.hstack([m0dU.T, m0dY.T])) + mm(np.hstack([Bh.T, Kh.T]),
                                                         np.block([[dLab.T, dMrb.T], [dLak.T, dMrk.T]]))
         E23 = mm(np.hstack([At.T, Rt.T]), np.vstack([np.hstack([dLab, dLak]), np.hstack([dMrb, dMrk])]))
