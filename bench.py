@@ -526,7 +526,8 @@ def main():
 
 
 def measure_secondary(wkv7, dev, algo):
-    """Stateful prefill (B=1, T=1024, H=32) and the 128-step ragged decode (256 x 32 states)."""
+    """Stateful prefill (B=1, T=1024, H=32), the backward's exact fallback for a flagged head, and the
+    128-step ragged decode (256 x 32 states)."""
     import torch
     out = {}
     peak, _ = measured_peaks()
@@ -563,6 +564,33 @@ def measure_secondary(wkv7, dev, algo):
         gbs = BYTES_PREFILL * units / (ms / 1e3) / 1e9
         out[key] = {"tokens_per_s": wl.B * wl.T / (ms / 1e3), "ms": ms, "achieved_gbs": gbs,
                     "frac": gbs / peak, "workspace": workspace is not None,
+                    "l2": "flushed (512 MB write) before each rep"}
+
+    # The exact fallback of the chunked backward: a head whose decay the 1/L scaling cannot take
+    # (some w < 1/16 in a chunk) is marked and recomputed by the token-order scan backward.  One such
+    # head among the 32 of one packed row (B=1, T=4096), timed against the same row without it.
+    wl = I.make_workload(3, B=1)
+    xs = [d(wl.inputs[n]) for n in I.NAMES]
+    dyt, rst = d(wl.dy), d(wl.reset)
+    w_flag = I.to_f64(wl.inputs["w"]).copy()
+    w_flag[0, 2000, 5, :4] = 0.03
+    xs_flag = list(xs)
+    xs_flag[I.NAMES.index("w")] = d(I.to_storage(w_flag, "bf16"))
+    for key, xx in (("bwd_B1_T4096_H32", xs), ("bwd_B1_T4096_H32_one_flagged_head", xs_flag)):
+        _, _, wsb = wkv7.forward(*xx, reset=rst, algo=algo)
+        times = []
+        for rep in range(8):
+            flush.fill_(float(rep))
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            wkv7.backward(*xx, dyt, wsb, reset=rst, want_ds0=False, algo=algo)
+            e1.record()
+            torch.cuda.synchronize()
+            if rep >= 2:
+                times.append(e0.elapsed_time(e1))
+        ms = statistics.median(times)
+        out[key] = {"ms": ms, "tokens_per_s": wl.B * wl.T / (ms / 1e3),
+                    "flagged_heads": 1 if "flagged" in key else 0,
                     "l2": "flushed (512 MB write) before each rep"}
 
     wl = I.make_workload(4)
