@@ -78,8 +78,10 @@ def _sigmoid(u: np.ndarray) -> np.ndarray:
     return 0.5 * (1.0 + np.tanh(0.5 * u))
 
 
-def draw_inputs(rng: np.random.Generator, shape, dtype: str) -> Dict[str, np.ndarray]:
-    """Draw r,w,k,v,a,b of ``shape`` (last axis = N) in storage dtype."""
+def draw_inputs(rng: np.random.Generator, shape, dtype: str, log_decay: bool = False) -> Dict[str, np.ndarray]:
+    """Draw r,w,k,v,a,b of ``shape`` (last axis = N) in storage dtype.  With ``log_decay`` the "w"
+    entry holds the decay's log-space parameter x (w = exp(-exp(x))) instead of w; the random draws
+    are the same either way."""
     shape = tuple(int(s) for s in shape)
     r = rng.standard_normal(shape)
     k = rng.standard_normal(shape)
@@ -93,7 +95,7 @@ def draw_inputs(rng: np.random.Generator, shape, dtype: str) -> Dict[str, np.nda
     a = -kk
     b = kk * _sigmoid(z_iclr)
     out = {}
-    for name, val in zip(NAMES, (r, w, k, v, a, b)):
+    for name, val in zip(NAMES, (r, x if log_decay else w, k, v, a, b)):
         out[name] = to_storage(val, dtype)
     return out
 

@@ -21,6 +21,11 @@ sequences reset the state at each boundary).  The backward is hand-derived
 
 Arrays: r,w,k,v,a,b,y,dy and gradients [B,T,H,N] float64; states
 [B,H,N,N] float64 (S[i][j] at [..., i, j]); reset [B,T] uint8.
+
+Log-space decay (``log_decay=True``): the ``w`` argument then holds x and the decay is
+w = exp(-exp(x)), i.e. log w = -exp(x) (the rwkv-lab page, "Highlight result -- GDN in RWKV-7",
+hands the wkv7 kernel its decay in log space; this is the RWKV-7 parametrisation of the decay),
+and the backward's ``dw`` entry is dL/dx = dL/dw * (-w exp(x)), by the chain rule.
 """
 from __future__ import annotations
 
@@ -75,8 +80,16 @@ def _shape(r: np.ndarray):
     return int(B), int(T), int(H), int(N)
 
 
-def forward(r, w, k, v, a, b, s0=None, reset=None, nthreads: int = 0):
-    """Token-order forward.  Returns (y [B,T,H,N], s_out [B,H,N,N], threads used)."""
+def decay_of_log(x) -> np.ndarray:
+    """w = exp(-exp(x)) in fp64 (the log-space decay input)."""
+    return np.exp(-np.exp(_f64(x)))
+
+
+def forward(r, w, k, v, a, b, s0=None, reset=None, nthreads: int = 0, log_decay: bool = False):
+    """Token-order forward.  Returns (y [B,T,H,N], s_out [B,H,N,N], threads used).  With
+    ``log_decay`` the ``w`` argument holds x and the decay is exp(-exp(x))."""
+    if log_decay:
+        w = decay_of_log(w)
     r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
     B, T, H, N = _shape(r)
     s0 = None if s0 is None else _f64(s0)
@@ -90,8 +103,12 @@ def forward(r, w, k, v, a, b, s0=None, reset=None, nthreads: int = 0):
     return y, s_out, used
 
 
-def backward(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, nthreads: int = 0):
-    """Hand-derived reverse mode.  Returns (dict of dr..db [B,T,H,N] and ds0 [B,H,N,N], threads)."""
+def backward(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, nthreads: int = 0, log_decay: bool = False):
+    """Hand-derived reverse mode.  Returns (dict of dr..db [B,T,H,N] and ds0 [B,H,N,N], threads).
+    With ``log_decay`` the ``w`` argument holds x and ``dw`` is returned as dL/dx."""
+    x_log = _f64(w) if log_decay else None
+    if log_decay:
+        w = decay_of_log(x_log)
     r, w, k, v, a, b, dy = (_f64(x) for x in (r, w, k, v, a, b, dy))
     B, T, H, N = _shape(r)
     s0 = None if s0 is None else _f64(s0)
@@ -104,11 +121,15 @@ def backward(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, nthreads: int 
                                       int(nthreads))
     if used < 0:
         raise MemoryError("oracle backward: allocation failed")
+    if log_decay:   # chain rule through w = exp(-exp(x)): dw/dx = -w exp(x)
+        g["dw"] = g["dw"] * (-w * np.exp(x_log))
     return g, used
 
 
-def step(r, w, k, v, a, b, state, active=None):
+def step(r, w, k, v, a, b, state, active=None, log_decay: bool = False):
     """One decode token on ``state`` [B,H,N,N] (returned updated copy) -> (y [B,H,N], state)."""
+    if log_decay:
+        w = decay_of_log(w)
     r, w, k, v, a, b = (_f64(x) for x in (r, w, k, v, a, b))
     B, H, N = (int(s) for s in r.shape)
     st = np.array(state, dtype=np.float64, copy=True, order="C")
