@@ -526,8 +526,8 @@ def main():
 
 
 def measure_secondary(wkv7, dev, algo):
-    """Stateful prefill (B=1, T=1024, H=32), the backward's exact fallback for a flagged head, and the
-    128-step ragged decode (256 x 32 states)."""
+    """Stateful prefill (B=1, T=1024, H=32), the backward's exact fallback for a flagged head, the
+    packed batch with the log-space decay input, and the 128-step ragged decode (256 x 32 states)."""
     import torch
     out = {}
     peak, _ = measured_peaks()
@@ -592,6 +592,30 @@ def measure_secondary(wkv7, dev, algo):
         out[key] = {"ms": ms, "tokens_per_s": wl.B * wl.T / (ms / 1e3),
                     "flagged_heads": 1 if "flagged" in key else 0,
                     "l2": "flushed (512 MB write) before each rep"}
+
+    # The packed training batch with the log-space decay input (x in place of w, w = exp(-exp(x))
+    # computed in the kernels, dL/dx out): the cost of the transform on the full step.
+    wl = I.make_workload(3, log_decay=True)
+    xs = [d(wl.inputs[n]) for n in I.NAMES]
+    dyt, rst = d(wl.dy), d(wl.reset)
+    _, _, wsl = wkv7.forward(*xs, reset=rst, algo=algo, log_decay=True)
+    f_ms, b_ms = [], []
+    for rep in range(6):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        wkv7.forward(*xs, reset=rst, workspace=wsl, algo=algo, log_decay=True)
+        e1.record()
+        wkv7.backward(*xs, dyt, wsl, reset=rst, want_ds0=False, algo=algo, log_decay=True)
+        e2.record()
+        torch.cuda.synchronize()
+        if rep >= 2:
+            f_ms.append(e0.elapsed_time(e1))
+            b_ms.append(e1.elapsed_time(e2))
+    fm, bm = statistics.median(f_ms), statistics.median(b_ms)
+    out["packed_train_B8_T4096_H32_log_decay"] = {
+        "fwd_ms": fm, "bwd_ms": bm, "fwd_bwd_tokens_per_s": wl.B * wl.T / ((fm + bm) / 1e3),
+        "l2": "inputs larger than L2 (no flush)"}
+    del xs, dyt, rst, wsl
 
     wl = I.make_workload(4)
     state = d(wl.state0)

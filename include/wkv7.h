@@ -133,6 +133,19 @@ typedef struct {
 #define WKV7_FLAG_CHECK_FINITE 0x1u
 
 /*
+ * Log-space decay input (rwkv-lab page, "Highlight result -- GDN in RWKV-7":
+ * the wkv7 kernel there takes its decay in log space).  With this flag the
+ * `w` argument of wkv7_forward, wkv7_backward, wkv7_step and
+ * wkv7_train_step_noalloc holds x, same dtype and layout, and the kernels use
+ * the decay w = exp(-exp(x)) (log w = -exp(x)), computed in fp32 from the
+ * stored x -- so a bf16 input no longer rounds w itself, whose spacing near 1
+ * is 2^-8.  wkv7_backward then writes dL/dx into its `dw` output.  Every
+ * algorithm accepts it; the chunked forms apply their decay-range test
+ * (below) to the computed w.
+ */
+#define WKV7_FLAG_LOG_DECAY 0x2u
+
+/*
  * Device status word (the device-side error channel of the boundary).
  * Kernels record errors they cannot return from an asynchronous launch --
  * a bounded wait that ran out, a non-finite output found under

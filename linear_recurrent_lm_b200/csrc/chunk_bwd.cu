@@ -368,7 +368,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
       float wmin = 1.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        L[u] = t < len ? w[u] : 1.f;
+        L[u] = t < len ? decay_of(w[u], p.log_decay) : 1.f;
         wmin = fminf(wmin, L[u]);
       }
 #pragma unroll
@@ -788,8 +788,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   // staged the same rows one chunk earlier), loaded while the tensor core works
   const int j = row;
   const int64_t o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
-  float rr[8], ar[8], br[8], kr[8];
+  float rr[8], ar[8], br[8], kr[8], xw[8];
   {
+    const T* const gw = static_cast<const T*>(p.w);
     const T* const gr = static_cast<const T*>(p.r);
     const T* const ga = static_cast<const T*>(p.a);
     const T* const gb = static_cast<const T*>(p.b);
@@ -802,6 +803,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
       ar[e] = ok ? Elt<T>::to_f32(ga[o]) : 0.f;
       br[e] = ok ? Elt<T>::to_f32(gb[o]) : 0.f;
       kr[e] = ok ? Elt<T>::to_f32(gk[o]) : 0.f;
+      xw[e] = ok && p.log_decay ? Elt<T>::to_f32(gw[o]) : 0.f;   // x, for dL/dx
     }
   }
   mma_wait(p, &sm.gg_bar, phase & 1u);
@@ -881,7 +883,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
         gdr[o] = Elt<T>::from_f32(eR[e] * Lr[e + 1]);
         gdb[o] = Elt<T>::from_f32(eB[e] * il[e]);
         gdk[o] = Elt<T>::from_f32(eK[e] * il[e]);
-        gdw[o] = Elt<T>::from_f32(cum * (Lr[e] * il[e]));
+        // cum = dL/d(log w_t): dw = cum / w_t = cum L_{t-1} / L_t, or dL/dx = -cum exp(x)
+        gdw[o] = Elt<T>::from_f32(p.log_decay ? dx_of_dlogw(cum, xw[e]) : cum * (Lr[e] * il[e]));
       }
     }
   }

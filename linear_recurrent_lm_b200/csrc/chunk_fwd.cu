@@ -171,7 +171,11 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
   {
     const int tq = 4 * kw, ja = lane, jb = lane + 32;
     auto ld2 = [&](int m, int t) { return make_float2(Elt<T>::to_f32(X[m][t][ja]), Elt<T>::to_f32(X[m][t][jb])); };
-    auto ldw = [&](int t) { return t < len ? ld2(1, t) : make_float2(1.f, 1.f); };   // padding: w = 1
+    auto ldw = [&](int t) {   // padding: w = 1
+      if (t >= len) return make_float2(1.f, 1.f);
+      const float2 x = ld2(1, t);
+      return make_float2(decay_of(x.x, p.log_decay), decay_of(x.y, p.log_decay));
+    };
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
     for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
     float at[2][4], bh[2][4], kh[2][4], vv[2][4];

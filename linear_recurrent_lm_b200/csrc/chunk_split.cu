@@ -129,14 +129,18 @@ __global__ void __launch_bounds__(kThreads) chunk_prep_kernel(const FwdArgs p, i
     auto ld2 = [&](int m, int t) {
       return make_float2(Elt<T>::to_f32(sm.in[m][t][ja]), Elt<T>::to_f32(sm.in[m][t][jb]));
     };
+    auto ldw = [&](int t) {
+      const float2 x = ld2(1, t);
+      return make_float2(decay_of(x.x, p.log_decay), decay_of(x.y, p.log_decay));
+    };
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}
-    for (int t = 0; t < tq; ++t) lam = mul2(lam, ld2(1, t));
+    for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
     float bl[2][4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = tq + u;
       const float2 lp = lam;
-      lam = mul2(lam, ld2(1, t));
+      lam = mul2(lam, ldw(t));
       bad |= !(lam.x >= 0x1p-40f && lam.x <= 0x1p40f) || !(lam.y >= 0x1p-40f && lam.y <= 0x1p40f);
       const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
       const float2 a2 = mul2(ld2(4, t), lp), r2 = mul2(ld2(0, t), lam);

@@ -113,6 +113,12 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
   return f2_unpack(d);
 }
 
+// The decay from its stored input: w itself, or, under the log-space convention, x with
+// w = exp(-exp(x)) (log w = -exp(x)).
+__device__ __forceinline__ float decay_of(float x, bool log_decay) { return log_decay ? expf(-expf(x)) : x; }
+// dL/dx from dL/d(log w) under the log-space convention: d(log w)/dx = -exp(x).
+__device__ __forceinline__ float dx_of_dlogw(float dlogw, float x) { return -dlogw * expf(x); }
+
 // Segment index of token t inside a chunk: number of resets among tokens 1..t.
 __device__ __forceinline__ int seg_of(unsigned mask, int t) { return __popc(mask & ((2u << t) - 2u)); }
 

@@ -20,6 +20,7 @@ struct FwdArgs {
   float* ckpt;            // [B,H,ceil(T/16),64,64] or null
   int* status;            // device status word: bits of wkv7 device errors (kStatus* below)
   unsigned extra_tx;      // test hook: bytes a staging expects beyond what it copies (0 in normal use)
+  bool log_decay;         // w holds x and the decay is exp(-exp(x)) (WKV7_FLAG_LOG_DECAY)
 };
 
 // Bits of the device status word.
@@ -63,6 +64,7 @@ struct BwdArgs {
   int* unit_flags;   // [B*H] in the workspace tail: the chunked backward marks units it could not handle
   int* status;       // device status word (see FwdArgs)
   unsigned extra_tx; // test hook (see FwdArgs)
+  bool log_decay;    // w holds x (see FwdArgs); dw receives dL/dx
 };
 
 struct StepArgs {
@@ -72,6 +74,7 @@ struct StepArgs {
   const uint8_t* active;
   void* y;
   int* status;   // device status word (debug-build bounds checks)
+  bool log_decay;  // w holds x (see FwdArgs)
 };
 
 // Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).

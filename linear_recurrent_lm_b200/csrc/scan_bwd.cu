@@ -122,8 +122,10 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
       const int rem = e - m * len * kN;
       const int tt = rem / kN, jj = rem - (rem / kN) * kN;
       const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + jj;
-      if (range_ok(o, 1, act_total, p.status) && in_bounds(tt < kChunk, p.status))
-        sm.x[m][tt][jj] = Elt<T>::to_f32(src[m][o]);
+      if (range_ok(o, 1, act_total, p.status) && in_bounds(tt < kChunk, p.status)) {
+        const float x = Elt<T>::to_f32(src[m][o]);
+        sm.x[m][tt][jj] = m == 1 ? decay_of(x, p.log_decay) : x;   // input 1 is the decay
+      }
     }
     if (tid < kChunk)
       sm.flags[tid] = (tid < len && p.reset && range_ok(b * p.T + t0 + tid, 1, p.B * p.T, p.status))
@@ -257,8 +259,12 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
         for (int o = tid; o < 5 * kN; o += kThreads) {
           const int m = o >> 6, jj = o & 63;
           const float s = (sm.col_red[m][0][jj] + sm.col_red[m][1][jj]) + (sm.col_red[m][2][jj] + sm.col_red[m][3][jj]);
-          if (range_ok(tok_off(b, t, h, p.T, p.H) + jj, 1, act_total, p.status))
-            dst[m][tok_off(b, t, h, p.T, p.H) + jj] = Elt<T>::from_f32(s);
+          if (range_ok(tok_off(b, t, h, p.T, p.H) + jj, 1, act_total, p.status)) {
+            float g = s;
+            if (m == 3 && p.log_decay)   // dL/dx = dL/dw . w . (-exp(x)) = dL/d(log w) . (-exp(x))
+              g = dx_of_dlogw(s * sm.x[1][t - t0][jj], Elt<T>::to_f32(src[1][tok_off(b, t, h, p.T, p.H) + jj]));
+            dst[m][tok_off(b, t, h, p.T, p.H) + jj] = Elt<T>::from_f32(g);
+          }
         }
       }
       seg_end = seg_start;

@@ -43,11 +43,13 @@ __device__ __forceinline__ void stage_slab(const FwdArgs& p, const T* const* src
 }
 
 template <typename T>
-__device__ __forceinline__ void widen_slab(const unsigned char* raw, float* f32, int len) {
+__device__ __forceinline__ void widen_slab(const unsigned char* raw, float* f32, int len, bool log_decay) {
   const T* src = reinterpret_cast<const T*>(raw);
   for (int in = 0; in < kInputs; ++in)
-    for (int e = threadIdx.x; e < len * kN; e += kThreads)
-      f32[in * kChunk * kN + e] = Elt<T>::to_f32(src[in * kChunk * kN + e]);
+    for (int e = threadIdx.x; e < len * kN; e += kThreads) {
+      const float x = Elt<T>::to_f32(src[in * kChunk * kN + e]);
+      f32[in * kChunk * kN + e] = in == 1 ? decay_of(x, log_decay) : x;   // input 1 is the decay
+    }
 }
 
 template <typename T>
@@ -81,7 +83,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
     stage_slab<T>(p, src, raw, b, h, 0, int(min64(kChunk, p.T)));
     cp_async_wait_all();
     __syncthreads();
-    widen_slab<T>(raw, f32, int(min64(kChunk, p.T)));
+    widen_slab<T>(raw, f32, int(min64(kChunk, p.T)), p.log_decay);
     __syncthreads();
   }
 
@@ -138,7 +140,7 @@ __global__ void __launch_bounds__(kThreads) scan_fwd_kernel(FwdArgs p) {
     cp_async_wait_all();
     __syncthreads();
     if (c + 1 < nc) {
-      widen_slab<T>(raw, f32, int(min64(kChunk, p.T - t0 - kChunk)));
+      widen_slab<T>(raw, f32, int(min64(kChunk, p.T - t0 - kChunk)), p.log_decay);
       __syncthreads();
     }
   }

@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) 
     float wv[8], kv[8], av[8], bv[8], rv[8];
     load8<T>(static_cast<const T*>(p.a) + o, av);
     load8<T>(static_cast<const T*>(p.w) + o, wv);
+#pragma unroll
+    for (int j = 0; j < 8; ++j) wv[j] = decay_of(wv[j], p.log_decay);
     load8<T>(static_cast<const T*>(p.b) + o, bv);
     load8<T>(static_cast<const T*>(p.k) + o, kv);
     load8<T>(static_cast<const T*>(p.r) + o, rv);

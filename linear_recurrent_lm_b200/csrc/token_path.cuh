@@ -51,7 +51,7 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned ma
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int col = 8 * nt + 2 * c4 + (e & 1);
-        const float wv = Elt<T>::to_f32(Wd[o + col]), bv = Elt<T>::to_f32(Bb[o + col]);
+        const float wv = decay_of(Elt<T>::to_f32(Wd[o + col]), p.log_decay), bv = Elt<T>::to_f32(Bb[o + col]);
         const float kv = Elt<T>::to_f32(K[o + col]), rv = Elt<T>::to_f32(R[o + col]);
         const bool lo = e < 2;
         acc[nt][e] = fmaf(acc[nt][e], wv, fmaf(lo ? s_lo : s_hi, bv, (lo ? v_lo : v_hi) * kv));

@@ -28,7 +28,7 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
 // Common descriptor checks.  On success fills the element counts.
 wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
   if (!d) return WKV7_ERR_NULL;
-  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE)) != 0u)
+  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE | WKV7_FLAG_LOG_DECAY)) != 0u)
     return WKV7_ERR_UNSUPPORTED;
   if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
   if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
@@ -218,7 +218,7 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   int* status = nullptr;
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
-                  status, test_extra_tx(d)};
+                  status, test_extra_tx(d), (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const std::initializer_list<Output> outs = {{y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}};
   if (d->T == 0 || !use_chunked(d)) return check_outputs(d, wkv7::launch_scan_fwd(p, d->dtype, s), outs, status, s);
@@ -253,7 +253,8 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   int* status = nullptr;
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
-                  dr, dw, dk, dv, da, db, ds0, flags, status, test_extra_tx(d)};
+                  dr, dw, dk, dv, da, db, ds0, flags, status, test_extra_tx(d),
+                  (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const std::initializer_list<Output> outs = {{dr, te, d->dtype}, {dw, te, d->dtype}, {dk, te, d->dtype},
                                               {dv, te, d->dtype}, {da, te, d->dtype}, {db, te, d->dtype},
@@ -280,7 +281,7 @@ wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, cons
   if (units == 0) return WKV7_OK;
   int* status = nullptr;
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
-  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y, status};
+  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y, status, (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return check_outputs(d, wkv7::launch_step(p, d->dtype, s), {{y, units * 64, d->dtype}, {state, units * 64 * 64, WKV7_F32}},
                        status, s);

@@ -157,8 +157,9 @@ DOC_MEAN = 512
 
 def make_workload(idx: int, seed: Optional[int] = None, *, B: Optional[int] = None,
                   T: Optional[int] = None, H: Optional[int] = None, N: int = N_HEAD,
-                  dtype: Optional[str] = None) -> Workload:
-    """Build workload ``idx`` (0..4); size overrides give scaled-down copies."""
+                  dtype: Optional[str] = None, log_decay: bool = False) -> Workload:
+    """Build workload ``idx`` (0..4); size overrides give scaled-down copies.  ``log_decay`` hands
+    out the decays' log-space parameter x in the "w" entries (same draws)."""
     spec = dict(SPECS[idx])
     seed = 1000 + idx if seed is None else int(seed)
     B = spec["B"] if B is None else B
@@ -170,15 +171,15 @@ def make_workload(idx: int, seed: Optional[int] = None, *, B: Optional[int] = No
         steps = DECODE_STEPS if T in (None, 1) else T
         state0 = rng.normal(0.0, 0.1, size=(B, H, N, N)).astype(np.float32)
         lengths = rng.integers(1, steps + 1, size=B)
-        step_inputs = [draw_inputs(rng, (B, H, N), dtype) for _ in range(steps)]
+        step_inputs = [draw_inputs(rng, (B, H, N), dtype, log_decay) for _ in range(steps)]
         return Workload(spec["name"], B, 1, H, N, dtype, seed, inputs={}, state0=state0,
                         steps=step_inputs, lengths=lengths)
-    inputs = draw_inputs(rng, (B, T, H, N), dtype)
+    inputs = draw_inputs(rng, (B, T, H, N), dtype, log_decay)
     wl = Workload(spec["name"], B, T, H, N, dtype, seed, inputs)
     if idx in (1, 3):
         wl.dy = to_storage(rng.standard_normal((B, T, H, N)), dtype)
     if idx == 3:
         wl.reset = geometric_resets(rng, B, T, DOC_MEAN)
     if idx == 2:
-        wl.prior = draw_inputs(rng, (B, PRIOR_TOKENS, H, N), dtype)
+        wl.prior = draw_inputs(rng, (B, PRIOR_TOKENS, H, N), dtype, log_decay)
     return wl

@@ -35,6 +35,7 @@ LIB_PATH = LIB_PATHS["release"]
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
 FLAG_CHECK_FINITE = 0x1                    # WKV7_FLAG_CHECK_FINITE: scan outputs for NaN / Inf
+FLAG_LOG_DECAY = 0x2                       # WKV7_FLAG_LOG_DECAY: w holds x, decay = exp(-exp(x))
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2, "chunked_fused": 3, "chunked_split": 4}
 N_HEAD = 64
@@ -160,9 +161,15 @@ def _token_shape(x: torch.Tensor):
     return tuple(int(s) for s in x.shape[:3])
 
 
+def _flags(flags: int, log_decay: bool) -> int:
+    return int(flags) | (FLAG_LOG_DECAY if log_decay else 0)
+
+
 def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, workspace=None,
-            need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None, flags: int = 0):
-    """WKV-7 forward over [B,T,H,64] inputs.  Returns (y, s_out, workspace)."""
+            need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None, flags: int = 0,
+            log_decay: bool = False):
+    """WKV-7 forward over [B,T,H,64] inputs.  Returns (y, s_out, workspace).  With ``log_decay`` the
+    ``w`` tensor holds x and the decay is exp(-exp(x))."""
     B, T, H = _token_shape(r)
     dev = r.device
     if y is None:
@@ -171,7 +178,7 @@ def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, worksp
         s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=dev, dtype=torch.float32)
     if workspace is None and need_workspace:
         workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype), 16), device=dev, dtype=torch.uint8)
-    d = make_desc(B, T, H, r.dtype, algo, flags=flags)
+    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(flags, log_decay))
     st = lib().wkv7_forward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, workspace)),
                             _stream(stream))
     _check(st, "wkv7_forward")
@@ -179,8 +186,10 @@ def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, worksp
 
 
 def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, grads=None,
-             want_ds0: bool = True, algo: str = "auto", stream=None, flags: int = 0) -> Dict[str, torch.Tensor]:
-    """WKV-7 backward from the checkpoints written by ``forward``."""
+             want_ds0: bool = True, algo: str = "auto", stream=None, flags: int = 0,
+             log_decay: bool = False) -> Dict[str, torch.Tensor]:
+    """WKV-7 backward from the checkpoints written by ``forward``.  With ``log_decay`` (as in the
+    forward) ``w`` holds x and the "dw" entry receives dL/dx."""
     B, T, H = _token_shape(r)
     g = dict(grads) if grads is not None else {}
     for n in ("dr", "dw", "dk", "dv", "da", "db"):
@@ -188,7 +197,7 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
             g[n] = torch.empty_like(r)
     if g.get("ds0") is None and want_ds0:
         g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
-    d = make_desc(B, T, H, r.dtype, algo, flags=flags)
+    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(flags, log_decay))
     st = lib().wkv7_backward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, dy, dsT, workspace)),
                              *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
                              _stream(stream))
@@ -196,21 +205,21 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
     return g
 
 
-def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None, flags: int = 0):
+def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None, flags: int = 0, log_decay: bool = False):
     """One decode token on ``state`` [B,H,64,64] (in place).  Inputs [B,H,64].  Returns y."""
     if r.dim() != 3 or r.shape[-1] != N_HEAD:
         raise ValueError(f"expected [B,H,{N_HEAD}], got {tuple(r.shape)}")
     B, H = int(r.shape[0]), int(r.shape[1])
     if y is None:
         y = torch.empty_like(r)
-    d = make_desc(B, 1, H, r.dtype, flags=flags)
+    d = make_desc(B, 1, H, r.dtype, flags=_flags(flags, log_decay))
     st = lib().wkv7_step(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, state, active, y)), _stream(stream))
     _check(st, "wkv7_step")
     return y
 
 
 def train_step_noalloc(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, *, y=None, s_out=None, grads=None,
-                       want_ds0: bool = True, algo: str = "auto", stream=None):
+                       want_ds0: bool = True, algo: str = "auto", stream=None, log_decay: bool = False):
     """Forward + backward with the library's fixed scratch instead of a workspace (nothing is
     allocated by the library; outputs not given are allocated here by torch).  For callers that
     cannot allocate device memory themselves: pass every output.  Returns (y, s_out, grads)."""
@@ -225,7 +234,7 @@ def train_step_noalloc(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, *, y
             g[n] = torch.empty_like(r)
     if g.get("ds0") is None and want_ds0:
         g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
-    d = make_desc(B, T, H, r.dtype, algo)
+    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(0, log_decay))
     st = lib().wkv7_train_step_noalloc(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, dy, dsT)),
                                        *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
                                        _stream(stream))

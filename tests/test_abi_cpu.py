@@ -88,11 +88,11 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, None) == L.ERR_NULL
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.N = 32
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
-    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 2                 # no such flag bit
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 4                 # no such flag bit
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 17, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT)   # the test hook needs T <= 16
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
-    bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 2)
+    bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 4)
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     for algo in ("chunked", "chunked_fused", "chunked_split"):      # tf32 products cannot meet the f32 bound
         assert call_fwd(L, L.make_desc(1, 16, 1, torch.float32, algo), ws=FAKE) == L.ERR_UNSUPPORTED
@@ -178,3 +178,13 @@ def test_binding_rejects_host_and_strided_tensors_before_any_call(L):
     with pytest.raises(ValueError, match="CUDA"):
         L._ptr(torch.zeros(4))
 
+
+
+def test_log_decay_flag_is_accepted_by_validation(L):
+    """WKV7_FLAG_LOG_DECAY passes the descriptor checks (on this host the call then fails to launch
+    with WKV7_ERR_CUDA instead of being refused as an unknown flag)."""
+    import torch
+    d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_LOG_DECAY)
+    assert call_fwd(L, d) != L.ERR_UNSUPPORTED
+    d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_LOG_DECAY | L.FLAG_CHECK_FINITE)
+    assert call_fwd(L, d) != L.ERR_UNSUPPORTED

@@ -45,11 +45,12 @@ def _host_case(B, T, H, dtype, seed):
     return d, dy, s0, dsT, reset
 
 
-def _fwd_bwd(W, host, algo):
+def _fwd_bwd(W, host, algo, log_decay=False):
     d, dy, s0, dsT, reset = host
     xs = [to_dev(d[n]) for n in I.NAMES]
-    y, s, ws = W.forward(*xs, s0=to_dev(s0), reset=to_dev(reset), algo=algo)
-    g = W.backward(*xs, to_dev(dy), ws, s0=to_dev(s0), reset=to_dev(reset), dsT=to_dev(dsT), algo=algo)
+    y, s, ws = W.forward(*xs, s0=to_dev(s0), reset=to_dev(reset), algo=algo, log_decay=log_decay)
+    g = W.backward(*xs, to_dev(dy), ws, s0=to_dev(s0), reset=to_dev(reset), dsT=to_dev(dsT), algo=algo,
+                   log_decay=log_decay)
     out = {"y": y, "s_out": s, **g}
     B, T, H = y.shape[:3]
     if T > 0:   # the checkpoints themselves (the backward's input) must match too
@@ -88,6 +89,7 @@ def _cases():
                 if B * H > 64 and dt != "bf16":
                     continue
                 out.append(("fwd_bwd", algo, dt, (B, T, H)))
+    out += [("fwd_bwd_log_decay", algo, "bf16", (2, 40, 3)) for algo in ("scan", "chunked_fused", "chunked_split")]
     out += [("step", None, dt, None) for dt in ("f32", "bf16", "f16")]
     out += [("noalloc", None, "bf16", (2, 40, 3))]
     return out
@@ -97,6 +99,10 @@ def _run(W, case, seed):
     kind, algo, dt, shape = case
     if kind == "fwd_bwd":
         return _fwd_bwd(W, _host_case(*shape, dt, seed), algo)
+    if kind == "fwd_bwd_log_decay":   # x in place of w (values of a decay parameter, not of a decay)
+        d, dy, s0, dsT, reset = _host_case(*shape, dt, seed)
+        d["w"] = I.to_storage(-np.abs(I.to_f64(d["r"])) - 0.5, dt)
+        return _fwd_bwd(W, (d, dy, s0, dsT, reset), algo, log_decay=True)
     if kind == "step":
         return _step(W, dt, seed)
     return _noalloc(W, _host_case(*shape, dt, seed))

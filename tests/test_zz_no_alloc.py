@@ -96,3 +96,26 @@ def test_noalloc_rejects_problems_beyond_its_scratch():
     st = W.lib().wkv7_train_step_noalloc(ctypes.byref(desc), *([fake] * 6), None, None, fake, None, fake, None,
                                          *([fake] * 6), None, None)
     assert st == W.ERR_SCRATCH_LIMIT
+
+
+def test_noalloc_with_log_decay_equals_the_pair():
+    """With the log-space decay input the no-allocation call equals forward + backward bit for bit."""
+    import torch
+    from linear_recurrent_lm_b200 import wkv7 as W
+    torch.cuda.set_device(0)
+    rng = np.random.default_rng(901)
+    B, T, H = 2, 40, 3
+    d = I.draw_inputs(rng, (B, T, H, 64), "bf16", log_decay=True)
+    xs = [to_dev(d[n]) for n in I.NAMES]
+    dy = to_dev(I.to_storage(rng.standard_normal((B, T, H, 64)), "bf16"))
+    s0 = to_dev(rng.standard_normal((B, H, 64, 64)).astype(np.float32))
+    dsT = to_dev(rng.standard_normal((B, H, 64, 64)).astype(np.float32))
+    reset = np.zeros((B, T), np.uint8)
+    reset[0, 13] = 1
+    rd = to_dev(reset)
+    y, s, ws = W.forward(*xs, s0=s0, reset=rd, log_decay=True)
+    g = W.backward(*xs, dy, ws, s0=s0, reset=rd, dsT=dsT, log_decay=True)
+    y2, s2, g2 = W.train_step_noalloc(*xs, dy, s0=s0, reset=rd, dsT=dsT, log_decay=True)
+    assert torch.equal(y, y2) and torch.equal(s, s2)
+    for n in GRADS + ("ds0",):
+        assert torch.equal(g[n], g2[n]), n
