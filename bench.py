@@ -40,6 +40,8 @@ BYTES_FWD_TRAIN = 768 + 128 + 1024
 BYTES_BWD = 768 + 128 + 1024 + 768
 BYTES_PREFILL = 768 + 128
 BYTES_DECODE = 64 * 64 * 4 * 2 + 768 + 128
+BYTES_EPI_FWD = 5 * 128 + 128                # y, r, k, v, g in; out (bf16)
+BYTES_EPI_BWD = 6 * 128 + 128 + 4 * 256      # y, r, k, v, g, dout in; dg, and dy, dr, dk, dv parts (fp32) out
 
 
 def rank_seed(rank: int) -> int:
@@ -527,7 +529,8 @@ def main():
 
 def measure_secondary(wkv7, dev, algo):
     """Stateful prefill (B=1, T=1024, H=32), the backward's exact fallback for a flagged head, the
-    packed batch with the log-space decay input, and the 128-step ragged decode (256 x 32 states)."""
+    packed batch with the log-space decay input, the WKV epilogue, and the 128-step ragged decode
+    (256 x 32 states)."""
     import torch
     out = {}
     peak, _ = measured_peaks()
@@ -616,6 +619,39 @@ def measure_secondary(wkv7, dev, algo):
         "fwd_ms": fm, "bwd_ms": bm, "fwd_bwd_tokens_per_s": wl.B * wl.T / ((fm + bm) / 1e3),
         "l2": "inputs larger than L2 (no flush)"}
     del xs, dyt, rst, wsl
+
+    # The WKV epilogue (GroupNorm per head, bonus, gating) on the packed batch's shape, each way one
+    # streaming kernel: forward reads y, r, k, v, g and writes out (768 B per token-head); backward
+    # reads those and dout and writes dg and an fp32 block of dy and the bonus parts of dr, dk, dv (1920 B).
+    B3, T3, H3 = 8, 4096, 32
+    gen = torch.Generator(device=dev).manual_seed(5)
+    tens = [torch.randn((B3, T3, H3, 64), device=dev, generator=gen).to(torch.bfloat16) for _ in range(6)]
+    ln_w = 1.0 + 0.3 * torch.randn((H3, 64), device=dev, generator=gen)
+    ln_b = 0.2 * torch.randn((H3, 64), device=dev, generator=gen)
+    r_k = 0.5 * torch.randn((H3, 64), device=dev, generator=gen)
+    yb, rb, kb, vb, gb, dob = tens
+    outb = torch.empty_like(yb)
+    eg = {"eg": torch.empty((4, B3, T3, H3, 64), device=dev, dtype=torch.float32), "dg": torch.empty_like(yb)}
+    f_ms, b_ms = [], []
+    for rep in range(12):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        wkv7.epilogue_forward(yb, rb, kb, vb, gb, ln_w, ln_b, r_k, 64e-5, out=outb)
+        e1.record()
+        wkv7.epilogue_backward(yb, rb, kb, vb, gb, dob, ln_w, ln_b, r_k, 64e-5, grads=eg)
+        e2.record()
+        torch.cuda.synchronize()
+        if rep >= 2:
+            f_ms.append(e0.elapsed_time(e1))
+            b_ms.append(e1.elapsed_time(e2))
+    fm, bm = statistics.median(f_ms), statistics.median(b_ms)
+    units3 = B3 * T3 * H3
+    out["epilogue_B8_T4096_H32"] = {
+        "fwd_ms": fm, "bwd_ms": bm,
+        "fwd_frac": BYTES_EPI_FWD * units3 / (fm / 1e3) / 1e9 / peak,
+        "bwd_frac": BYTES_EPI_BWD * units3 / (bm / 1e3) / 1e9 / peak,
+        "l2": "inputs larger than L2 (no flush)"}
+    del tens, yb, rb, kb, vb, gb, dob, outb, eg
 
     wl = I.make_workload(4)
     state = d(wl.state0)

@@ -146,6 +146,19 @@ typedef struct {
 #define WKV7_FLAG_LOG_DECAY 0x2u
 
 /*
+ * wkv7_backward (and wkv7_train_step_noalloc) desc->flags bit: `dy` points at
+ * the fp32 block that wkv7_epilogue_backward writes, [4][B,T,H,64], 16-byte
+ * aligned: dy itself, then the epilogue's (bonus) parts of dr, dk and dv,
+ * which the recurrence's backward adds to its own before the one rounding to
+ * the output dtype.  Both stay in fp32 on purpose: the GroupNorm's gradient
+ * is large on tokens whose y has a small spread (right after a reset, for
+ * instance) and, rounded to bf16 first, costs the gradients ~10 % of their
+ * RMS there; and rounding the bonus parts before the sum would round dr, dk,
+ * dv twice (~2 % of their RMS).
+ */
+#define WKV7_FLAG_EPILOGUE_GRADS 0x4u
+
+/*
  * Device status word (the device-side error channel of the boundary).
  * Kernels record errors they cannot return from an asynchronous launch --
  * a bounded wait that ran out, a non-finite output found under
@@ -285,6 +298,52 @@ wkv7_status_t wkv7_train_step_noalloc(const wkv7_desc_t* desc, const void* r, co
                                       const uint8_t* reset, void* y, float* s_out, const void* dy,
                                       const float* dsT, void* dr, void* dw, void* dk, void* dv, void* da,
                                       void* db, float* ds0, void* stream);
+
+/*
+ * ------------------------------------------------------------------ WKV epilogue
+ * The step after the recurrence in an RWKV-7 time-mix block, one streaming
+ * kernel each way (rwkv-metal page, architecture table: "ln_x ... GroupNorm
+ * (per head)"; rwkv-lab page, "Native RWKV megakernel backend": the state
+ * update fused "through GroupNorm, the RWKV bonus, and output gating").  Per
+ * (b, t, h), channels i, j = 0..63:
+ *   mu, var = mean and variance of y over the head's 64 channels,
+ *   yn_i = (y_i - mu) / sqrt(var + eps)                 (GroupNorm, one group per head)
+ *   s    = sum_j r_j k_j r_k[h][j]                      (the bonus weight)
+ *   out_i = (yn_i ln_w[h][i] + ln_b[h][i] + s v_i) g_i  (bonus, then gating)
+ * with r, k, v the recurrence's own inputs and g the gate.  All token
+ * tensors [B,T,H,64] in desc->dtype, 16-byte aligned; the parameters
+ * ln_w, ln_b, r_k are fp32 [H,64] (4-byte aligned) and eps > 0.  desc->algo
+ * is ignored; desc->flags may hold WKV7_FLAG_CHECK_FINITE only (else
+ * WKV7_ERR_UNSUPPORTED).  Errors as for wkv7_forward; eps <= 0 or not
+ * finite -> WKV7_ERR_UNSUPPORTED.
+ */
+typedef struct {
+  const float* ln_w; /* [H, 64] GroupNorm weight */
+  const float* ln_b; /* [H, 64] GroupNorm bias */
+  const float* r_k;  /* [H, 64] bonus weights */
+  float eps;         /* GroupNorm epsilon, > 0 */
+} wkv7_epilogue_t;
+
+/* out = the epilogue of y (formula above).  One launch on `stream`. */
+wkv7_status_t wkv7_epilogue_forward(const wkv7_desc_t* desc, const wkv7_epilogue_t* ep, const void* y,
+                                    const void* r, const void* k, const void* v, const void* g, void* out,
+                                    void* stream);
+
+/*
+ * Reverse mode of the epilogue from dout = dL/dout.  Writes `eg`, an fp32
+ * block [4][B,T,H,64] (16-byte aligned): dy (the gradient reaching the
+ * recurrence), then the bonus parts of dr, dk and dv -- hand it to
+ * wkv7_backward as its dy with WKV7_FLAG_EPILOGUE_GRADS, which adds those
+ * parts to the recurrence's own; writes dg (desc->dtype); adds the parameter
+ * gradients, summed over b and t, to dln_w, dln_b and dr_k (fp32 [H,64];
+ * each may be NULL; the caller zeroes them first -- they are summed with
+ * float atomics, so their last bits depend on the order of the adds).  One
+ * launch on `stream`.
+ */
+wkv7_status_t wkv7_epilogue_backward(const wkv7_desc_t* desc, const wkv7_epilogue_t* ep, const void* y,
+                                     const void* r, const void* k, const void* v, const void* g,
+                                     const void* dout, float* eg, void* dg, float* dln_w, float* dln_b,
+                                     float* dr_k, void* stream);
 
 #ifdef __cplusplus
 }

@@ -282,6 +282,7 @@ struct __align__(128) BwdSmem {
   __align__(16) float Xp[kChunk][kChunk];    // X [t][tau]            (context)
   __align__(128) float ck[kN * kN];         // checkpoint entering the chunk being built (tiled order)
   __align__(128) T stg[kIn][kChunk][kN];    // staged inputs of the chunk being built (TMA boxes)
+  __align__(128) float dyf[kChunk][kN];     // dy of that chunk when it comes from the epilogue's fp32 block
   unsigned long long in_bar;                // staged inputs and checkpoint landed (one phase per staged chunk)
   unsigned long long u_bar, gg_bar, e_bar;  // tensor-core batches complete (one phase per chunk each)
   uint32_t tmem_base;
@@ -324,8 +325,9 @@ __device__ __forceinline__ bool reset_flag(const BwdArgs& p, int64_t b, int64_t 
   return p.reset && c >= 0 && lane < kChunk && t < p.T && p.reset[b * p.T + t] != 0;
 }
 
-// Stage chunk c: the seven inputs of its tokens (one TMA box each; rows past T arrive as zeros, K1
-// reads w there as 1) and, for c > 0, the checkpoint entering it (one bulk copy), issued by one
+// Stage chunk c: the seven inputs of its tokens (one TMA box each, dy in fp32 when it comes from the
+// epilogue's block; rows past T arrive as zeros, K1 reads w there as 1) and, for c > 0, the
+// checkpoint entering it (one bulk copy), issued by one
 // thread on in_bar.
 template <typename T>
 __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, int64_t unit, int64_t b,
@@ -333,10 +335,13 @@ __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, Bwd
   if (ktid == 0) {
     if (!in_bounds(h < p.H && b < p.B && c >= 0 && c < nc && c * kChunk < p.T, p.status)) return;
     const unsigned ck_bytes = c > 0 ? unsigned(kN * kN * sizeof(float)) : 0u;
-    mbar_arrive_expect_tx(&sm.in_bar, unsigned(kIn * kChunk * kN * sizeof(T)) + ck_bytes + p.extra_tx);
+    const unsigned dy_bytes = unsigned(kChunk * kN * (p.epi ? sizeof(float) : sizeof(T)));
+    mbar_arrive_expect_tx(&sm.in_bar, unsigned((kIn - 1) * kChunk * kN * sizeof(T)) + dy_bytes + ck_bytes + p.extra_tx);
 #pragma unroll
-    for (int m = 0; m < kIn; ++m)
-      tma_load_4d(&sm.stg[m][0][0], &tm.m[m], 0, int(h), int(c * kChunk), int(b), &sm.in_bar);
+    for (int m = 0; m < kIn; ++m) {
+      void* dst = (m == kIn - 1 && p.epi) ? static_cast<void*>(&sm.dyf[0][0]) : static_cast<void*>(&sm.stg[m][0][0]);
+      tma_load_4d(dst, &tm.m[m], 0, int(h), int(c * kChunk), int(b), &sm.in_bar);
+    }
     if (c > 0 && range_ok((unit * nc + (c - 1)) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status))
       bulk_g2s(sm.ck, p.ckpt + (unit * nc + (c - 1)) * kN * kN, ck_bytes, &sm.in_bar);
   }
@@ -417,7 +422,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
     for (int e = 0; e < 8; ++e) {
       const int t = 8 * th + e;
       v8[e] = Elt<T>::to_f32(X[3][t][i]);
-      y8[e] = Elt<T>::to_f32(X[6][t][i]);
+      y8[e] = p.epi ? sm.dyf[t][i] : Elt<T>::to_f32(X[6][t][i]);
       m8[e] = t < fr ? y8[e] : 0.f;
     }
     put8(cx.SV, cb(i, 16 + 8 * th, 32), v8);
@@ -661,14 +666,13 @@ __device__ __forceinline__ void context_products(const BwdArgs& p, const InputMa
 // One thread issues every tensor-core product of chunk c, in three batches, each as soon as the
 // main warps have handed over its operands (named barriers kBarDsl, kBarDu, kBarG4).
 template <typename T>
-__device__ __forceinline__ void issue_chunk(BwdSmem<T>& sm, Ctx<T>& cx, uint32_t tmem, bool leader) {
-  constexpr bool kExactIn = std::is_same<T, bf16>::value;   // v and dy have no lo half
+__device__ __forceinline__ void issue_chunk(BwdSmem<T>& sm, Ctx<T>& cx, uint32_t tmem, bool leader, bool dy_exact) {
   named_bar(kBarDsl, kHandOff);
   if (leader) {
     tc::fence_after_sync();
     // GU = dSl BKx^T + dY^T [Qm | Vq]                          (rows i: dU^T | dV^T)
     mma3<32, 4>(tmem + kColGU, op<64, true>(sm.dSlT), op<64, false>(cx.BKx), false);
-    mma3<32, 1>(tmem + kColGU, op<32, false>(cx.UYT, kExactIn, 0, 16), op<32, true>(cx.MMx), true);   // dy^T
+    mma3<32, 1>(tmem + kColGU, op<32, false>(cx.UYT, dy_exact, 0, 16), op<32, true>(cx.MMx), true);   // dy^T
     tc::commit(&sm.u_bar);
   }
   named_bar(kBarDu, kHandOff);
@@ -678,7 +682,7 @@ __device__ __forceinline__ void issue_chunk(BwdSmem<T>& sm, Ctx<T>& cx, uint32_t
     tc::commit(&sm.gg_bar);
     mma3<32, 4>(tmem + kColE + 64, op<64, false>(sm.dSlT), op<32, true>(cx.SV), false);   // dSl^T [SA^T | v^T]
     // dS0^T += Rt^T m0.dy + At^T m0.dU (the carried gradient of the chunk before)
-    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR, false, 16), op<32, false>(cx.DUY, kExactIn, 0, 16), true);
+    mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR, false, 16), op<32, false>(cx.DUY, dy_exact, 0, 16), true);
     mma3<64, 1>(tmem + kColDS, op<64, true>(cx.AR), op<32, false>(cx.DUY), true);
     mma3<32, 4>(tmem + kColE, op<64, false>(cx.S0T), op<32, true>(cx.DUY), false);   // S0^T [m0.dU^T | m0.dy^T]
   }
@@ -776,7 +780,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       if (tb + e < len && range_ok(tok_off(b, t0 + tb + e, h, p.T, p.H) + i, 1, total, p.status))
-        *dvp = Elt<T>::from_f32(dv[e]);
+        *dvp = Elt<T>::from_f32(p.epi ? dv[e] + static_cast<const float*>(p.dy)[3 * total + tok_off(b, t0 + tb + e, h, p.T, p.H) + i]
+                                      : dv[e]);   // + the epilogue's bonus part
       dvp += rs;
     }
   }
@@ -788,8 +793,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   // staged the same rows one chunk earlier), loaded while the tensor core works
   const int j = row;
   const int64_t o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
-  float rr[8], ar[8], br[8], kr[8], xw[8];
+  float rr[8], ar[8], br[8], kr[8], xw[8], er[8], ek[8];
   {
+    const float* const eg = static_cast<const float*>(p.dy);   // the epilogue's block, under p.epi
     const T* const gw = static_cast<const T*>(p.w);
     const T* const gr = static_cast<const T*>(p.r);
     const T* const ga = static_cast<const T*>(p.a);
@@ -804,6 +810,8 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
       br[e] = ok ? Elt<T>::to_f32(gb[o]) : 0.f;
       kr[e] = ok ? Elt<T>::to_f32(gk[o]) : 0.f;
       xw[e] = ok && p.log_decay ? Elt<T>::to_f32(gw[o]) : 0.f;   // x, for dL/dx
+      er[e] = ok && p.epi ? eg[total + o] : 0.f;                 // bonus parts of dr, dk
+      ek[e] = ok && p.epi ? eg[2 * total + o] : 0.f;
     }
   }
   mma_wait(p, &sm.gg_bar, phase & 1u);
@@ -880,9 +888,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
       if (tb + e < len && range_ok(o0 + e * rs, 1, total, p.status)) {
         const int64_t o = o0 + e * rs;
         gda[o] = Elt<T>::from_f32(eA[e] * Lr[e]);
-        gdr[o] = Elt<T>::from_f32(eR[e] * Lr[e + 1]);
+        gdr[o] = Elt<T>::from_f32(fmaf(eR[e], Lr[e + 1], er[e]));
         gdb[o] = Elt<T>::from_f32(eB[e] * il[e]);
-        gdk[o] = Elt<T>::from_f32(eK[e] * il[e]);
+        gdk[o] = Elt<T>::from_f32(fmaf(eK[e], il[e], ek[e]));
         // cum = dL/d(log w_t): dw = cum / w_t = cum L_{t-1} / L_t, or dL/dx = -cum exp(x)
         gdw[o] = Elt<T>::from_f32(p.log_decay ? dx_of_dlogw(cum, xw[e]) : cum * (Lr[e] * il[e]));
       }
@@ -942,12 +950,14 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
     cta_sync();   // prologue staged by the context warps
     bool flagged = false;
     unsigned phase = 0;
+    int64_t first_done = nc;   // first chunk whose gradients were written
     for (int64_t it = 0; it <= nc; ++it) {
       if (it >= 1) {
         const int64_t c = nc - it;   // chunk whose gradients are computed now
         Ctx<T>& cx = sm.ctx[c & 1];   // the main and issue warps own this buffer until the next CTA barrier
         if (cx.unsafe) {
           if (tid == 0) sm.stop = 1;
+          first_done = c + 1;
         } else {
           tc::fence_after_sync();
           const int64_t t0 = c * kChunk;
@@ -961,7 +971,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         break;
       }
     }
-    if (tid == 0 && p.unit_flags && range_ok(unit, 1, p.B * p.H, p.status)) p.unit_flags[unit] = flagged ? 1 : 0;
+    if (tid == 0 && p.unit_flags && range_ok(unit, 1, p.B * p.H, p.status))
+      p.unit_flags[unit] = flagged ? int(first_done + 1) : 0;
     if (!flagged && p.ds0) {   // every MMA of the last chunk completed before its e_bar phase
       tc::fence_after_sync();
       const int j = 16 * warp + lane;
@@ -1020,7 +1031,8 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
       if (it >= 1) {
         const int64_t c = nc - it;
         Ctx<T>& cx = sm.ctx[c & 1];
-        if (!cx.unsafe) issue_chunk<T>(sm, cx, tmem, tid == kIssueTid);
+        // dy has no lo half when it arrives in bf16 (exact); the epilogue's fp32 dy has one
+        if (!cx.unsafe) issue_chunk<T>(sm, cx, tmem, tid == kIssueTid, std::is_same<T, bf16>::value && !p.epi);
       }
       cta_sync();
       if (sm.stop) break;

@@ -62,9 +62,13 @@ struct BwdArgs {
   void *dr, *dw, *dk, *dv, *da, *db;
   float* ds0;
   int* unit_flags;   // [B*H] in the workspace tail: the chunked backward marks units it could not handle
+                     // (0: complete; else 1 + the first chunk whose gradients it did write -- those of
+                     // that chunk and every later one are final)
   int* status;       // device status word (see FwdArgs)
   unsigned extra_tx; // test hook (see FwdArgs)
   bool log_decay;    // w holds x (see FwdArgs); dw receives dL/dx
+  bool epi;          // WKV7_FLAG_EPILOGUE_GRADS: dy points at the epilogue's fp32 block [4][B,T,H,64]
+                     // (dy, then the bonus parts of dr, dk, dv, which are added before rounding)
 };
 
 struct StepArgs {
@@ -77,6 +81,20 @@ struct StepArgs {
   bool log_decay;  // w holds x (see FwdArgs)
 };
 
+// The WKV epilogue (GroupNorm per head, bonus, gating): forward writes `out`; backward writes the
+// fp32 block `eg` [4][B,T,H,64] (dy, then the bonus parts of dr, dk, dv) and dg, and adds the
+// parameter gradients to dln_w, dln_b, dr_k (each may be null).
+struct EpiArgs {
+  int64_t B, T, H;
+  const void *y, *r, *k, *v, *g, *dout;
+  const float *ln_w, *ln_b, *r_k;
+  float eps;
+  void *out, *dg;
+  float* eg;
+  float *dln_w, *dln_b, *dr_k;
+  int* status;
+};
+
 // Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).
 wkv7_status_t validate_desc(const wkv7_desc_t* d);
 
@@ -85,6 +103,7 @@ cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 // only_flagged: run only the (b,h) units whose unit_flags entry is non-zero (others exit at once).
 cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
+cudaError_t launch_epilogue(const EpiArgs& p, int dtype, bool backward, cudaStream_t stream);
 // Set kStatusNonFinite in *status if any of the n elements at x (dtype as above; 16-byte aligned)
 // is NaN or infinite.  x == nullptr or n == 0: nothing is launched.
 cudaError_t launch_finite_scan(const void* x, int64_t n, int dtype, int* status, cudaStream_t stream);

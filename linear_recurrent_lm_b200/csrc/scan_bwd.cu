@@ -93,6 +93,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
   const int64_t unit = blockIdx.x;
   if (!in_bounds(unit < p.B * p.H, p.status)) return;   // (debug build; block-uniform)
   if (only_flagged && p.unit_flags[unit] == 0) return;
+  // the epilogue's block: dy, then the bonus parts of dr, dk, dv (fp32), each B*T*H*64 floats
+  const float* const eg = p.epi ? static_cast<const float*>(p.dy) : nullptr;
   const int64_t act_total = p.B * p.T * p.H * kN, st_total = p.B * p.H * kN * kN;
   const int64_t b = unit / p.H, h = unit - (unit / p.H) * p.H;
   const int tid = threadIdx.x, lane = tid & 31;
@@ -123,8 +125,8 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
       const int tt = rem / kN, jj = rem - (rem / kN) * kN;
       const int64_t o = tok_off(b, t0 + tt, h, p.T, p.H) + jj;
       if (range_ok(o, 1, act_total, p.status) && in_bounds(tt < kChunk, p.status)) {
-        const float x = Elt<T>::to_f32(src[m][o]);
-        sm.x[m][tt][jj] = m == 1 ? decay_of(x, p.log_decay) : x;   // input 1 is the decay
+        const float x = (m == 6 && eg) ? eg[o] : Elt<T>::to_f32(src[m][o]);
+        sm.x[m][tt][jj] = m == 1 ? decay_of(x, p.log_decay) : x;   // input 1 is the decay; 6 is dy
       }
     }
     if (tid < kChunk)
@@ -238,8 +240,11 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
           sm.row_red[half][1][myrow] = dsa_part;
         }
         __syncthreads();
-        if (tid < kN && range_ok(tok_off(b, t, h, p.T, p.H) + tid, 1, act_total, p.status))
-          dst[5][tok_off(b, t, h, p.T, p.H) + tid] = Elt<T>::from_f32(sm.row_red[0][0][tid] + sm.row_red[1][0][tid]);
+        if (tid < kN && range_ok(tok_off(b, t, h, p.T, p.H) + tid, 1, act_total, p.status)) {
+          const int64_t o = tok_off(b, t, h, p.T, p.H) + tid;
+          const float dvv = sm.row_red[0][0][tid] + sm.row_red[1][0][tid];
+          dst[5][o] = Elt<T>::from_f32(eg ? dvv + eg[3 * act_total + o] : dvv);
+        }
         float da_p = 0.f;
         const bool rst = sm.flags[tt] != 0;
 #pragma unroll
@@ -260,10 +265,12 @@ __global__ void __launch_bounds__(kThreads) scan_bwd_kernel(BwdArgs p, bool only
           const int m = o >> 6, jj = o & 63;
           const float s = (sm.col_red[m][0][jj] + sm.col_red[m][1][jj]) + (sm.col_red[m][2][jj] + sm.col_red[m][3][jj]);
           if (range_ok(tok_off(b, t, h, p.T, p.H) + jj, 1, act_total, p.status)) {
+            const int64_t o = tok_off(b, t, h, p.T, p.H) + jj;
             float g = s;
             if (m == 3 && p.log_decay)   // dL/dx = dL/dw . w . (-exp(x)) = dL/d(log w) . (-exp(x))
-              g = dx_of_dlogw(s * sm.x[1][t - t0][jj], Elt<T>::to_f32(src[1][tok_off(b, t, h, p.T, p.H) + jj]));
-            dst[m][tok_off(b, t, h, p.T, p.H) + jj] = Elt<T>::from_f32(g);
+              g = dx_of_dlogw(s * sm.x[1][t - t0][jj], Elt<T>::to_f32(src[1][o]));
+            if (eg && m <= 1) g += eg[(m + 1) * act_total + o];   // dr, dk: the epilogue's bonus parts
+            dst[m][o] = Elt<T>::from_f32(g);
           }
         }
       }

@@ -28,7 +28,8 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
 // Common descriptor checks.  On success fills the element counts.
 wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
   if (!d) return WKV7_ERR_NULL;
-  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE | WKV7_FLAG_LOG_DECAY)) != 0u)
+  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE | WKV7_FLAG_LOG_DECAY |
+                                  WKV7_FLAG_EPILOGUE_GRADS)) != 0u)
     return WKV7_ERR_UNSUPPORTED;
   if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
   if (d->dtype != WKV7_F32 && d->dtype != WKV7_BF16 && d->dtype != WKV7_F16) return WKV7_ERR_DTYPE;
@@ -102,7 +103,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_tiled() {
 
 // Tensor maps of up to seven [B,T,H,64] inputs as {64, H, T, B} with a {64, 1, 16, 1} box (the
 // chunked kernels' staging).  Unused slots stay zero.
-wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const void*> ptrs, wkv7::InputMaps* tm) {
+// `last_f32`: the last map describes an fp32 tensor whatever desc->dtype (dy under
+// WKV7_FLAG_EPILOGUE_GRADS: the first quarter of the epilogue's block).
+wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const void*> ptrs, wkv7::InputMaps* tm,
+                            bool last_f32 = false) {
   *tm = wkv7::InputMaps{};
   if (d->T > INT32_MAX || d->H > INT32_MAX || d->B > INT32_MAX) return WKV7_ERR_SHAPE;   // 32-bit box coordinates
   PFN_cuTensorMapEncodeTiled_v12000 enc = encode_tiled();
@@ -115,11 +119,14 @@ wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const vo
   const cuuint64_t strides[3] = {64 * es, cuuint64_t(d->H) * 64 * es, cuuint64_t(d->T) * cuuint64_t(d->H) * 64 * es};
   const cuuint32_t box[4] = {64, 1, 16, 1};
   const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const cuuint64_t strides32[3] = {64 * 4, cuuint64_t(d->H) * 64 * 4, cuuint64_t(d->T) * cuuint64_t(d->H) * 64 * 4};
   int i = 0;
+  const int n = int(ptrs.size());
   for (const void* ptr : ptrs) {
-    if (enc(&tm->m[i++], dt, 4, const_cast<void*>(ptr), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-            CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+    const bool f32 = last_f32 && i == n - 1;
+    if (enc(&tm->m[i++], f32 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT32 : dt, 4, const_cast<void*>(ptr), dims,
+            f32 ? strides32 : strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+            CU_TENSOR_MAP_L2_PROMOTION_L2_128B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
       return WKV7_ERR_CUDA;
   }
   return WKV7_OK;
@@ -254,7 +261,7 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::BwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, dy, dsT, static_cast<const float*>(workspace),
                   dr, dw, dk, dv, da, db, ds0, flags, status, test_extra_tx(d),
-                  (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
+                  (d->flags & WKV7_FLAG_LOG_DECAY) != 0u, (d->flags & WKV7_FLAG_EPILOGUE_GRADS) != 0u};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const std::initializer_list<Output> outs = {{dr, te, d->dtype}, {dw, te, d->dtype}, {dk, te, d->dtype},
                                               {dv, te, d->dtype}, {da, te, d->dtype}, {db, te, d->dtype},
@@ -263,11 +270,62 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
     return check_outputs(d, wkv7::launch_scan_bwd(p, d->dtype, false, s), outs, status, s);
   // Chunked pass, then the exact scan for the units it marked (decays too small for 1/L scaling).
   wkv7::InputMaps tm;
-  st = encode_inputs(d, {r, w, k, v, a, b, dy}, &tm);
+  st = encode_inputs(d, {r, w, k, v, a, b, dy}, &tm, (d->flags & WKV7_FLAG_EPILOGUE_GRADS) != 0u);
   if (st != WKV7_OK) return st;
   cudaError_t e = wkv7::launch_chunk_bwd(p, tm, d->dtype, s);
   if (e != cudaSuccess) return WKV7_ERR_CUDA;
   return check_outputs(d, wkv7::launch_scan_bwd(p, d->dtype, true, s), outs, status, s);
+}
+
+// The epilogue's descriptor: the token tensors as everywhere; flags other than CHECK_FINITE refused.
+static wkv7_status_t check_epilogue(const wkv7_desc_t* d, const wkv7_epilogue_t* ep, int64_t* units, int64_t* te) {
+  wkv7_status_t st = check_desc(d, units, te);
+  if (st != WKV7_OK) return st;
+  if ((d->flags & ~WKV7_FLAG_CHECK_FINITE) != 0u) return WKV7_ERR_UNSUPPORTED;
+  if (!ep || !ep->ln_w || !ep->ln_b || !ep->r_k) return WKV7_ERR_NULL;
+  if (!(ep->eps > 0.f) || !(ep->eps < 1e30f)) return WKV7_ERR_UNSUPPORTED;   // also refuses NaN
+  for (const void* q : {static_cast<const void*>(ep->ln_w), static_cast<const void*>(ep->ln_b),
+                        static_cast<const void*>(ep->r_k)})
+    if (reinterpret_cast<uintptr_t>(q) % 4u != 0u) return WKV7_ERR_ALIGN;
+  return WKV7_OK;
+}
+
+wkv7_status_t wkv7_epilogue_forward(const wkv7_desc_t* d, const wkv7_epilogue_t* ep, const void* y, const void* r,
+                                    const void* k, const void* v, const void* g, void* out, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_epilogue(d, ep, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(te > 0, {y, r, k, v, g, out});
+  if (st != WKV7_OK) return st;
+  if (te == 0) return WKV7_OK;
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::EpiArgs p{d->B, d->T, d->H, y, r, k, v, g, nullptr, ep->ln_w, ep->ln_b, ep->r_k, ep->eps,
+                  out, nullptr, nullptr, nullptr, nullptr, nullptr, status};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return check_outputs(d, wkv7::launch_epilogue(p, d->dtype, false, s), {{out, te, d->dtype}}, status, s);
+}
+
+wkv7_status_t wkv7_epilogue_backward(const wkv7_desc_t* d, const wkv7_epilogue_t* ep, const void* y, const void* r,
+                                     const void* k, const void* v, const void* g, const void* dout, float* eg,
+                                     void* dg, float* dln_w, float* dln_b, float* dr_k, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_epilogue(d, ep, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(te > 0, {y, r, k, v, g, dout, eg, dg});
+  if (st != WKV7_OK) return st;
+  for (const float* q : {dln_w, dln_b, dr_k})
+    if (q && reinterpret_cast<uintptr_t>(q) % 4u != 0u) return WKV7_ERR_ALIGN;
+  if (te == 0) return WKV7_OK;
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::EpiArgs p{d->B, d->T, d->H, y, r, k, v, g, dout, ep->ln_w, ep->ln_b, ep->r_k, ep->eps,
+                  nullptr, dg, eg, dln_w, dln_b, dr_k, status};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return check_outputs(d, wkv7::launch_epilogue(p, d->dtype, true, s),
+                       {{eg, 4 * te, WKV7_F32}, {dg, te, d->dtype}, {dln_w, d->H * 64, WKV7_F32}, {dln_b, d->H * 64, WKV7_F32},
+                        {dr_k, d->H * 64, WKV7_F32}},
+                       status, s);
 }
 
 wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,

@@ -36,6 +36,7 @@ NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # WKV7_NOALLOC_SCRATCH_BYTES
 FLAG_TEST_WAIT_TIMEOUT = 0x80000000        # WKV7_FLAG_TEST_WAIT_TIMEOUT (test hook, T <= 16)
 FLAG_CHECK_FINITE = 0x1                    # WKV7_FLAG_CHECK_FINITE: scan outputs for NaN / Inf
 FLAG_LOG_DECAY = 0x2                       # WKV7_FLAG_LOG_DECAY: w holds x, decay = exp(-exp(x))
+FLAG_EPILOGUE_GRADS = 0x4                  # WKV7_FLAG_EPILOGUE_GRADS: dy is the epilogue's fp32 block
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2, "chunked_fused": 3, "chunked_split": 4}
 N_HEAD = 64
@@ -45,6 +46,12 @@ CHUNK = 16
 class Desc(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int64), ("T", ctypes.c_int64), ("H", ctypes.c_int64), ("N", ctypes.c_int32),
                 ("dtype", ctypes.c_int32), ("algo", ctypes.c_int32), ("flags", ctypes.c_uint32)]
+
+
+class Epilogue(ctypes.Structure):
+    """wkv7_epilogue_t: fp32 [H,64] GroupNorm weight and bias, bonus weights, and eps."""
+    _fields_ = [("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("r_k", ctypes.c_void_p),
+                ("eps", ctypes.c_float)]
 
 
 class WKV7Error(RuntimeError):
@@ -84,6 +91,11 @@ def _load(variant: str) -> ctypes.CDLL:
     L.wkv7_get_device_status.argtypes = [ctypes.c_int]
     L.wkv7_debug_checks.restype = ctypes.c_int
     L.wkv7_debug_checks.argtypes = []
+    ep = ctypes.POINTER(Epilogue)
+    L.wkv7_epilogue_forward.restype = ctypes.c_int
+    L.wkv7_epilogue_forward.argtypes = [dp, ep] + [vp] * 7
+    L.wkv7_epilogue_backward.restype = ctypes.c_int
+    L.wkv7_epilogue_backward.argtypes = [dp, ep] + [vp] * 12
     return L
 
 
@@ -189,7 +201,13 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
              want_ds0: bool = True, algo: str = "auto", stream=None, flags: int = 0,
              log_decay: bool = False) -> Dict[str, torch.Tensor]:
     """WKV-7 backward from the checkpoints written by ``forward``.  With ``log_decay`` (as in the
-    forward) ``w`` holds x and the "dw" entry receives dL/dx."""
+    forward) ``w`` holds x and the "dw" entry receives dL/dx.  ``dy`` may be the fp32 block
+    [4,B,T,H,64] that ``epilogue_backward`` returns as "eg" (dy, then the epilogue's parts of dr, dk,
+    dv, which are added in)."""
+    if dy.dim() == 5:
+        if dy.dtype != torch.float32 or tuple(dy.shape) != (4,) + tuple(r.shape):
+            raise ValueError(f"the epilogue's gradient block must be fp32 [4,B,T,H,64], got {tuple(dy.shape)}")
+        flags = int(flags) | FLAG_EPILOGUE_GRADS
     B, T, H = _token_shape(r)
     g = dict(grads) if grads is not None else {}
     for n in ("dr", "dw", "dk", "dv", "da", "db"):
@@ -234,9 +252,54 @@ def train_step_noalloc(r, w, k, v, a, b, dy, s0=None, reset=None, dsT=None, *, y
             g[n] = torch.empty_like(r)
     if g.get("ds0") is None and want_ds0:
         g["ds0"] = torch.empty((B, H, N_HEAD, N_HEAD), device=r.device, dtype=torch.float32)
-    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(0, log_decay))
+    flags = FLAG_EPILOGUE_GRADS if dy.dim() == 5 else 0   # the epilogue's fp32 block (see backward)
+    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(flags, log_decay))
     st = lib().wkv7_train_step_noalloc(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, dy, dsT)),
                                        *(_ptr(g[n]) for n in ("dr", "dw", "dk", "dv", "da", "db")), _ptr(g.get("ds0")),
                                        _stream(stream))
     _check(st, "wkv7_train_step_noalloc")
     return y, s_out, g
+
+
+def _epi(ln_w, ln_b, r_k, eps) -> Epilogue:
+    for t in (ln_w, ln_b, r_k):
+        if t.dtype != torch.float32 or not t.is_cuda or not t.is_contiguous():
+            raise ValueError("epilogue parameters must be contiguous fp32 CUDA tensors [H,64]")
+    return Epilogue(ln_w.data_ptr(), ln_b.data_ptr(), r_k.data_ptr(), float(eps))
+
+
+def epilogue_forward(y, r, k, v, g, ln_w, ln_b, r_k, eps: float, *, out=None, stream=None, flags: int = 0):
+    """The WKV epilogue: out = (GroupNorm_h(y) ln_w + ln_b + (sum r k r_k) v) g, per (b,t,h).  Token
+    tensors [B,T,H,64]; ln_w, ln_b, r_k fp32 [H,64]."""
+    B, T, H = _token_shape(y)
+    if out is None:
+        out = torch.empty_like(y)
+    d = make_desc(B, T, H, y.dtype, flags=flags)
+    ep = _epi(ln_w, ln_b, r_k, eps)
+    st = lib().wkv7_epilogue_forward(ctypes.byref(d), ctypes.byref(ep), *(_ptr(x) for x in (y, r, k, v, g, out)),
+                                     _stream(stream))
+    _check(st, "wkv7_epilogue_forward")
+    return out
+
+
+def epilogue_backward(y, r, k, v, g, dout, ln_w, ln_b, r_k, eps: float, *, grads=None, want_params: bool = True,
+                      stream=None, flags: int = 0) -> Dict[str, torch.Tensor]:
+    """Reverse mode of ``epilogue_forward``: dict of "eg" (fp32 [4,B,T,H,64]: dy, then the bonus parts
+    of dr, dk, dv -- pass it to ``backward`` as its dy), "dg" [B,T,H,64], and (zeroed here, then summed
+    over b and t) dln_w, dln_b, dr_k [H,64]."""
+    B, T, H = _token_shape(y)
+    g_ = dict(grads) if grads is not None else {}
+    if g_.get("eg") is None:
+        g_["eg"] = torch.empty((4,) + tuple(y.shape), device=y.device, dtype=torch.float32)
+    if g_.get("dg") is None:
+        g_["dg"] = torch.empty_like(y)
+    if want_params:
+        for n in ("dln_w", "dln_b", "dr_k"):
+            g_[n] = torch.zeros((H, N_HEAD), device=y.device, dtype=torch.float32)
+    d = make_desc(B, T, H, y.dtype, flags=flags)
+    ep = _epi(ln_w, ln_b, r_k, eps)
+    st = lib().wkv7_epilogue_backward(ctypes.byref(d), ctypes.byref(ep), *(_ptr(x) for x in (y, r, k, v, g, dout)),
+                                      _ptr(g_["eg"]), _ptr(g_["dg"]),
+                                      *(_ptr(g_.get(n)) for n in ("dln_w", "dln_b", "dr_k")), _stream(stream))
+    _check(st, "wkv7_epilogue_backward")
+    return g_

@@ -88,11 +88,11 @@ def test_forward_validation_codes(L):
     assert call_fwd(L, None) == L.ERR_NULL
     bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.N = 32
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
-    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 4                 # no such flag bit
+    bad = L.make_desc(1, 16, 1, torch.bfloat16); bad.flags = 8                 # no such flag bit
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     bad = L.make_desc(1, 17, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT)   # the test hook needs T <= 16
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
-    bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 4)
+    bad = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_TEST_WAIT_TIMEOUT | 8)
     assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
     for algo in ("chunked", "chunked_fused", "chunked_split"):      # tf32 products cannot meet the f32 bound
         assert call_fwd(L, L.make_desc(1, 16, 1, torch.float32, algo), ws=FAKE) == L.ERR_UNSUPPORTED
@@ -187,4 +187,38 @@ def test_log_decay_flag_is_accepted_by_validation(L):
     d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_LOG_DECAY)
     assert call_fwd(L, d) != L.ERR_UNSUPPORTED
     d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_LOG_DECAY | L.FLAG_CHECK_FINITE)
+    assert call_fwd(L, d) != L.ERR_UNSUPPORTED
+
+
+def test_epilogue_validation_codes(L):
+    """The epilogue entry points refuse bad arguments before any launch."""
+    import torch
+    lib = L.lib()
+    vp = ctypes.c_void_p
+    P = vp(0x10000)                                   # aligned, never dereferenced
+    ep = L.Epilogue(0x10000, 0x10000, 0x10000, 6.4e-4)
+    d = L.make_desc(1, 16, 1, torch.bfloat16)
+    fwd = lambda desc, e, *p: lib.wkv7_epilogue_forward(desc, e, *p, None)   # noqa: E731
+    assert fwd(None, ctypes.byref(ep), *([P] * 6)) == L.ERR_NULL
+    assert fwd(ctypes.byref(d), None, *([P] * 6)) == L.ERR_NULL
+    assert fwd(ctypes.byref(d), ctypes.byref(ep), None, *([P] * 5)) == L.ERR_NULL
+    bad = L.Epilogue(0x10000, 0x10000, 0x10000, 0.0)
+    assert fwd(ctypes.byref(d), ctypes.byref(bad), *([P] * 6)) == L.ERR_UNSUPPORTED
+    bad = L.Epilogue(0x10002, 0x10000, 0x10000, 6.4e-4)
+    assert fwd(ctypes.byref(d), ctypes.byref(bad), *([P] * 6)) == L.ERR_ALIGN
+    dl = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_LOG_DECAY)
+    assert fwd(ctypes.byref(dl), ctypes.byref(ep), *([P] * 6)) == L.ERR_UNSUPPORTED
+    assert fwd(ctypes.byref(d), ctypes.byref(ep), vp(0x10008), *([P] * 5)) == L.ERR_ALIGN
+    bwd = lambda desc, e, *p: lib.wkv7_epilogue_backward(desc, e, *p, None)   # noqa: E731
+    # y, r, k, v, g, dout, eg, dg, then the three parameter gradients (optional)
+    assert bwd(ctypes.byref(d), ctypes.byref(ep), *([P] * 7), None, None, None, None) == L.ERR_NULL
+    assert bwd(ctypes.byref(d), ctypes.byref(ep), *([P] * 8), vp(0x10002), None, None) == L.ERR_ALIGN
+    # T = 0: nothing to do, and no launch
+    d0 = L.make_desc(1, 0, 1, torch.bfloat16)
+    assert fwd(ctypes.byref(d0), ctypes.byref(ep), *([None] * 6)) == L.OK
+
+
+def test_epilogue_grads_flag_is_accepted_by_validation(L):
+    import torch
+    d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_EPILOGUE_GRADS)
     assert call_fwd(L, d) != L.ERR_UNSUPPORTED

@@ -81,7 +81,7 @@ def test_noalloc_equals_regular_entry_points_call_after_call():
         if zero is not None:                   # the regular call did mark that head for the exact re-run
             n_ck = B * H * ((T + 15) // 16) * 64 * 64 * 4
             marks = ws[n_ck:n_ck + 4 * B * H].view(torch.int32).cpu().numpy()
-            assert marks[zero[0] * H + zero[2]] == 1 and marks.sum() == 1
+            assert marks[zero[0] * H + zero[2]] >= 1 and (marks != 0).sum() == 1
         assert torch.equal(y, y_r) and torch.equal(s_out, s_r), (seed, "forward")
         for n in GRADS + ("ds0",):
             assert torch.equal(g[n], g_r[n]), (seed, n)
