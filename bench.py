@@ -646,7 +646,27 @@ def measure_secondary(wkv7, dev, algo):
             b_ms.append(e1.elapsed_time(e2))
     fm, bm = statistics.median(f_ms), statistics.median(b_ms)
     units3 = B3 * T3 * H3
+    # the forward with the epilogue fused into its y write-out (packed batch, fused chunked form)
+    wl = I.make_workload(3)
+    xs = [d(wl.inputs[n]) for n in I.NAMES]
+    rst = d(wl.reset)
+    ws3 = torch.empty(wkv7.workspace_bytes(wl.B, wl.T, wl.H, xs[0].dtype), device=dev, dtype=torch.uint8)
+    fused = {}
+    for key, want_y in (("with_y", True), ("out_only", False)):
+        ms = []
+        for rep in range(8):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            wkv7.forward_epilogue(*xs, gb, ln_w, ln_b, r_k, 64e-5, reset=rst, out=outb, y=yb if want_y else None,
+                                  want_y=want_y, workspace=ws3, algo=algo)
+            e1.record()
+            torch.cuda.synchronize()
+            if rep >= 2:
+                ms.append(e0.elapsed_time(e1))
+        fused[key] = statistics.median(ms)
+    del xs, rst, ws3
     out["epilogue_B8_T4096_H32"] = {
+        "forward_with_fused_epilogue_ms": fused["with_y"], "forward_with_fused_epilogue_out_only_ms": fused["out_only"],
         "fwd_ms": fm, "bwd_ms": bm,
         "fwd_frac": BYTES_EPI_FWD * units3 / (fm / 1e3) / 1e9 / peak,
         "bwd_frac": BYTES_EPI_BWD * units3 / (bm / 1e3) / 1e9 / peak,

@@ -330,6 +330,23 @@ wkv7_status_t wkv7_epilogue_forward(const wkv7_desc_t* desc, const wkv7_epilogue
                                     void* stream);
 
 /*
+ * The forward with the epilogue: out = epilogue(y) for the y that
+ * wkv7_forward computes from the same arguments (s_out and the checkpoints
+ * in `workspace` as there); y itself is written only when `y` is not NULL
+ * (the epilogue's backward needs it).  In the fused chunked form (16-bit
+ * inputs where wkv7_forward would run that form) the epilogue runs inside
+ * the recurrence's kernel as each chunk's y is written out: one launch, y
+ * never read back from memory.  The other forms run wkv7_forward and then
+ * wkv7_epilogue_forward (with `y` NULL, `out` holds y in between).  Either
+ * way out is bit for bit what wkv7_epilogue_forward gives on the stored y.
+ * desc->flags as for wkv7_forward (WKV7_FLAG_EPILOGUE_GRADS refused).
+ */
+wkv7_status_t wkv7_forward_epilogue(const wkv7_desc_t* desc, const wkv7_epilogue_t* ep, const void* r,
+                                    const void* w, const void* k, const void* v, const void* a, const void* b,
+                                    const float* s0, const uint8_t* reset, const void* g, void* y, void* out,
+                                    float* s_out, void* workspace, void* stream);
+
+/*
  * Reverse mode of the epilogue from dout = dL/dout.  Writes `eg`, an fp32
  * block [4][B,T,H,64] (16-byte aligned): dy (the gradient reaching the
  * recurrence), then the bonus parts of dr, dk and dv -- hand it to

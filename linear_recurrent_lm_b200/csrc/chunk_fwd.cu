@@ -45,6 +45,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "epilogue.cuh"
 #include "mma.cuh"
 #include "tc05.cuh"
 #include "token_path.cuh"
@@ -87,6 +88,7 @@ struct __align__(128) FwdSmem3 {
   float M[kChunk][S20];
   __align__(128) T in[kIn][kChunk][kN];      // staged inputs of the chunk being built (TMA boxes)
   __align__(16) uint16_t Ys[kChunk][kStrY]; // y of the last chunk [t][i] (16-bit outputs), written next iteration
+  __align__(16) float epi_par[3][kN];        // fused epilogue: GroupNorm weight, bias and bonus weights of the head
   unsigned long long in_bar;                 // completion of the bulk copies into `in` (one phase per chunk)
   unsigned long long d1_bar, mma_bar;        // completion of a chunk's D1 MMAs / of all its MMAs (one phase per chunk)
   uint32_t tmem_base;                        // TMEM: S0 (cols 0-63), D1 (64-95), D3 (128-191)
@@ -528,7 +530,7 @@ __device__ __forceinline__ void store_ck(float* ck, const float (&acc)[8][4]) {
   }
 }
 
-template <typename T>
+template <typename T, bool kEpi>
 __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FwdSmem3<T>& sm = *reinterpret_cast<FwdSmem3<T>*>(smem_raw);
@@ -565,20 +567,47 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
       mbar_init(&sm.d1_bar, 1);
       mbar_init(&sm.mma_bar, 1);
     }
+    if constexpr (kEpi) {   // the head's epilogue parameters
+      const float* const par[3] = {p.ln_w, p.ln_b, p.r_k};
+      for (int i = tid; i < 3 * kN; i += 128) sm.epi_par[i / kN][i % kN] = par[i / kN][h * kN + i % kN];
+    }
     tc::fence_before_sync();
-    cta_sync();   // chunk 0 staged; TMEM allocated
+    cta_sync();   // chunk 0 staged; TMEM allocated; the epilogue parameters in place
     tc::fence_after_sync();
     const uint32_t tmem = sm.tmem_base;
     unsigned mma_phase = 0;
-    // y of the previous chunk (16-bit outputs): this thread's 16-byte piece of token row tid/8
-    T* ydst = nullptr;
+    // y of the previous chunk (16-bit outputs): this thread's 16-byte piece of token row tid/8, at
+    // element offset yoff; with the fused epilogue also the r, k, v and g of that piece, loaded before
+    // the CTA barrier and used after it, and the 8 lanes of the row form one GroupNorm group.
+    int64_t yoff = -1;
     const int ytt = tid >> 3, ypart = tid & 7;
+    uint4 er = {}, ek = {}, ev = {}, eg = {};
+    auto flush_y = [&]() {
+      if (yoff < 0) return;
+      const uint4 yv = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+      if constexpr (kEpi) {
+        float y8[8], r8[8], k8[8], v8[8], g8[8], o8[8];
+        unpack16<T>(yv, y8);
+        unpack16<T>(er, r8);
+        unpack16<T>(ek, k8);
+        unpack16<T>(ev, v8);
+        unpack16<T>(eg, g8);
+        epi_forward<8, 8>(y8, r8, k8, v8, g8, &sm.epi_par[0][ypart * 8], &sm.epi_par[1][ypart * 8],
+                          &sm.epi_par[2][ypart * 8], p.eps, 0xffu << (lane & 24), o8);
+        uint4 ov;
+        T* const oq = reinterpret_cast<T*>(&ov);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) oq[e] = Elt<T>::from_f32(o8[e]);
+        *reinterpret_cast<uint4*>(static_cast<T*>(p.out) + yoff) = ov;
+        if (p.y) *reinterpret_cast<uint4*>(static_cast<T*>(p.y) + yoff) = yv;
+      } else {
+        *reinterpret_cast<uint4*>(static_cast<T*>(p.y) + yoff) = yv;
+      }
+      yoff = -1;
+    };
     float* ck = nullptr;   // checkpoint slot of the state in the fragments (tiled order), if still due
     for (int64_t it = 0; it <= nc; ++it) {
-      if (ydst) {
-        *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
-        ydst = nullptr;
-      }
+      flush_y();
       if (it >= 1) {
         const int64_t c = it - 1;
         const Ctx& cx = sm.ctx[c & 1];
@@ -587,8 +616,25 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
         if (!cx.unsafe) {
           state_chunk<T>(p, sm, cx, acc, b, h, t0, len, warp, lane, tmem, mma_phase, ck);
           if (sizeof(T) == 2 && ytt < len &&
-              range_ok(tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8, 8, p.B * p.T * p.H * kN, p.status))
-            ydst = static_cast<T*>(p.y) + tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
+              range_ok(tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8, 8, p.B * p.T * p.H * kN, p.status)) {
+            yoff = tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
+            if constexpr (kEpi) {
+              er = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.r) + yoff);
+              ek = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k) + yoff);
+              ev = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v) + yoff);
+              eg = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.g) + yoff);
+            }
+          }
+        } else if constexpr (kEpi) {   // token by token into the y tile, then out like a safe chunk
+          store_ck(ck, acc);
+          state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane, &sm.Ys[0][0], kStrY);
+          if (ytt < len && range_ok(tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8, 8, p.B * p.T * p.H * kN, p.status)) {
+            yoff = tok_off(b, t0 + ytt, h, p.T, p.H) + ypart * 8;
+            er = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.r) + yoff);
+            ek = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.k) + yoff);
+            ev = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.v) + yoff);
+            eg = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.g) + yoff);
+          }
         } else {
           store_ck(ck, acc);
           state_chunk_tokens<T>(p, unsigned(cx.mask), acc, b, h, t0, len, warp, lane);
@@ -599,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
       }
       cta_sync();   // context of chunk it handed over; Ys complete
     }
-    if (ydst) *reinterpret_cast<uint4*>(ydst) = *reinterpret_cast<const uint4*>(&sm.Ys[ytt][ypart * 8]);
+    flush_y();
     store_ck(ck, acc);
     // every batch was waited for and every TMEM load is complete: release TMEM
     named_bar(2, 128);
@@ -651,22 +697,29 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
   }
 }
 
-template <typename T>
+template <typename T, bool kEpi>
 cudaError_t launch(const FwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
   const size_t smem = sizeof(FwdSmem3<T>);
-  cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<T, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  chunk_fwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
+  chunk_fwd_kernel<T, kEpi><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
 }  // namespace
 
 cudaError_t launch_chunk_fwd(const FwdArgs& p, const InputMaps& tm, int dtype, cudaStream_t stream) {
+  if (p.out) {   // the fused epilogue: 16-bit types only (their y goes out through the staged tile)
+    switch (dtype) {
+      case 1: return launch<__nv_bfloat16, true>(p, tm, stream);
+      case 2: return launch<__half, true>(p, tm, stream);
+      default: return cudaErrorInvalidValue;
+    }
+  }
   switch (dtype) {
-    case 0: return launch<float>(p, tm, stream);
-    case 1: return launch<__nv_bfloat16>(p, tm, stream);
-    case 2: return launch<__half>(p, tm, stream);
+    case 0: return launch<float, false>(p, tm, stream);
+    case 1: return launch<__nv_bfloat16, false>(p, tm, stream);
+    case 2: return launch<__half, false>(p, tm, stream);
     default: return cudaErrorInvalidValue;
   }
 }

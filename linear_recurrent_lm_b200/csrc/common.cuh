@@ -114,8 +114,9 @@ __device__ __forceinline__ float2 sub2(float2 a, float2 b) {
 }
 
 // The decay from its stored input: w itself, or, under the log-space convention, x with
-// w = exp(-exp(x)) (log w = -exp(x)).
-__device__ __forceinline__ float decay_of(float x, bool log_decay) { return log_decay ? expf(-expf(x)) : x; }
+// w = exp(-exp(x)) (log w = -exp(x)).  The fast exponential (a few ulp) keeps the chunked kernels'
+// decay scan, which the context warps sit on, short; it is far inside every tolerance.
+__device__ __forceinline__ float decay_of(float x, bool log_decay) { return log_decay ? __expf(-__expf(x)) : x; }
 // dL/dx from dL/d(log w) under the log-space convention: d(log w)/dx = -exp(x).
 __device__ __forceinline__ float dx_of_dlogw(float dlogw, float x) { return -dlogw * expf(x); }
 

@@ -17,6 +17,7 @@
 // a CTA works on one head, so the backward keeps its parameter gradients in registers across its
 // rows, reduces them over the CTA in shared memory and adds one partial per CTA with atomics.
 #include "common.cuh"
+#include "epilogue.cuh"
 #include "kernels.h"
 
 namespace wkv7 {
@@ -83,21 +84,8 @@ __global__ void __launch_bounds__(kThreads) epilogue_fwd_kernel(const EpiArgs p)
       load_vec<T>(p.v, off, v);
       load_vec<T>(p.g, off, g);
     }
-    float sy = 0.f, srk = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) {
-      sy += y[e];
-      srk = fmaf(r[e] * k[e], rk[e], srk);
-    }
-    const float mu = group_sum<P>(sy) * (1.f / kN);
-    float sq = 0.f;
-#pragma unroll
-    for (int e = 0; e < E; ++e) sq = fmaf(y[e] - mu, y[e] - mu, sq);
-    const float rstd = rsqrtf(group_sum<P>(sq) * (1.f / kN) + p.eps);
-    const float s = group_sum<P>(srk);
     float out[E];
-#pragma unroll
-    for (int e = 0; e < E; ++e) out[e] = fmaf((y[e] - mu) * rstd, gam[e], fmaf(s, v[e], bet[e])) * g[e];
+    epi_forward<P, E>(y, r, k, v, g, gam, bet, rk, p.eps, 0xffffffffu, out);
     if (act) store_vec<T>(p.out, off, out);
   }
 }

@@ -21,6 +21,12 @@ struct FwdArgs {
   int* status;            // device status word: bits of wkv7 device errors (kStatus* below)
   unsigned extra_tx;      // test hook: bytes a staging expects beyond what it copies (0 in normal use)
   bool log_decay;         // w holds x and the decay is exp(-exp(x)) (WKV7_FLAG_LOG_DECAY)
+  // The WKV epilogue fused into the y write-out (chunked fused form, 16-bit types): with `out`
+  // non-null the kernel writes out = epilogue(y) (and y only if `y` is non-null).
+  const void* g;
+  void* out;
+  const float *ln_w, *ln_b, *r_k;
+  float eps;
 };
 
 // Bits of the device status word.

@@ -2,7 +2,8 @@
 // by four warps (warp w: rows 16w..16w+15; acc[nt][e] = S[16w + g + 8(e>>1)][8nt + 2c + (e&1)],
 // g = lane/4, c = lane%4), inputs read from global memory: the recurrence itself, used by the
 // chunked forward kernels for chunks whose decay product leaves the range of the 1/L scaling and,
-// in the split form, for a ragged last chunk.  Writes y of the chunk's len tokens.
+// in the split form, for a ragged last chunk.  Writes y of the chunk's len tokens -- to global memory,
+// or, with `ys` given (a [16][ys_stride] tile of 16-bit y), into that tile for the caller to write out.
 #pragma once
 
 #include "common.cuh"
@@ -12,7 +13,8 @@ namespace wkv7 {
 
 template <typename T>
 __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned mask, float (&acc)[8][4], int64_t b,
-                                                   int64_t h, int64_t t0, int len, int warp, int lane) {
+                                                   int64_t h, int64_t t0, int len, int warp, int lane,
+                                                   uint16_t* ys = nullptr, int ys_stride = 0) {
   const int g = lane >> 2, c4 = lane & 3;
   const int row0 = 16 * warp;
   const T* R = static_cast<const T*>(p.r);
@@ -62,8 +64,14 @@ __device__ __forceinline__ void state_chunk_tokens(const FwdArgs& p, unsigned ma
     y_hi += __shfl_xor_sync(0xffffffffu, y_hi, 1);
     y_hi += __shfl_xor_sync(0xffffffffu, y_hi, 2);
     if (c4 == 0) {
-      y[o + row0 + g] = Elt<T>::from_f32(y_lo);
-      y[o + row0 + g + 8] = Elt<T>::from_f32(y_hi);
+      if (ys) {   // 16-bit T: the tile holds its bits
+        const T lo = Elt<T>::from_f32(y_lo), hi = Elt<T>::from_f32(y_hi);
+        ys[tt * ys_stride + row0 + g] = *reinterpret_cast<const uint16_t*>(&lo);
+        ys[tt * ys_stride + row0 + g + 8] = *reinterpret_cast<const uint16_t*>(&hi);
+      } else {
+        y[o + row0 + g] = Elt<T>::from_f32(y_lo);
+        y[o + row0 + g + 8] = Elt<T>::from_f32(y_hi);
+      }
     }
   }
 }

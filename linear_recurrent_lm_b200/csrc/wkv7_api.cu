@@ -328,6 +328,46 @@ wkv7_status_t wkv7_epilogue_backward(const wkv7_desc_t* d, const wkv7_epilogue_t
                        status, s);
 }
 
+wkv7_status_t wkv7_forward_epilogue(const wkv7_desc_t* d, const wkv7_epilogue_t* ep, const void* r, const void* w,
+                                    const void* k, const void* v, const void* a, const void* b, const float* s0,
+                                    const uint8_t* reset, const void* g, void* y, void* out, float* s_out,
+                                    void* workspace, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_algo_dtype(d);
+  if (st != WKV7_OK) return st;
+  if (d->flags & WKV7_FLAG_EPILOGUE_GRADS) return WKV7_ERR_UNSUPPORTED;
+  wkv7_desc_t de = *d;   // the epilogue's own descriptor: only the finite check carries over
+  de.flags = d->flags & WKV7_FLAG_CHECK_FINITE;
+  st = check_epilogue(&de, ep, &units, &te);
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(te > 0, {r, w, k, v, a, b, g, out});
+  if (st != WKV7_OK) return st;
+  st = check_ptrs(false, {s0, s_out, workspace, y});
+  if (st != WKV7_OK) return st;
+  if (units == 0 || te == 0) return wkv7_forward(d, r, w, k, v, a, b, s0, reset, y ? y : out, s_out, workspace, stream);
+  bool split = false;
+  const bool fused = d->dtype != WKV7_F32 && use_chunked(d) && use_split(d, units, workspace, &split) == WKV7_OK && !split;
+  if (!fused) {   // the recurrence, then the epilogue on its stored y (out holds y in between when y is NULL)
+    void* yb = y ? y : out;
+    st = wkv7_forward(d, r, w, k, v, a, b, s0, reset, yb, s_out, workspace, stream);
+    if (st != WKV7_OK) return st;
+    return wkv7_epilogue_forward(&de, ep, yb, r, k, v, g, out, stream);
+  }
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
+                  status, test_extra_tx(d), (d->flags & WKV7_FLAG_LOG_DECAY) != 0u,
+                  g, out, ep->ln_w, ep->ln_b, ep->r_k, ep->eps};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  wkv7::InputMaps tm;
+  st = encode_inputs(d, {r, w, k, v, a, b}, &tm);
+  if (st != WKV7_OK) return st;
+  return check_outputs(d, wkv7::launch_chunk_fwd(p, tm, d->dtype, s),
+                       {{out, te, d->dtype}, {y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}}, status, s);
+}
+
 wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
                         const void* a, const void* b, float* state, const uint8_t* active, void* y, void* stream) {
   int64_t units = 0, te = 0;

@@ -94,6 +94,8 @@ def _load(variant: str) -> ctypes.CDLL:
     ep = ctypes.POINTER(Epilogue)
     L.wkv7_epilogue_forward.restype = ctypes.c_int
     L.wkv7_epilogue_forward.argtypes = [dp, ep] + [vp] * 7
+    L.wkv7_forward_epilogue.restype = ctypes.c_int
+    L.wkv7_forward_epilogue.argtypes = [dp, ep] + [vp] * 14
     L.wkv7_epilogue_backward.restype = ctypes.c_int
     L.wkv7_epilogue_backward.argtypes = [dp, ep] + [vp] * 12
     return L
@@ -303,3 +305,28 @@ def epilogue_backward(y, r, k, v, g, dout, ln_w, ln_b, r_k, eps: float, *, grads
                                       *(_ptr(g_.get(n)) for n in ("dln_w", "dln_b", "dr_k")), _stream(stream))
     _check(st, "wkv7_epilogue_backward")
     return g_
+
+
+def forward_epilogue(r, w, k, v, a, b, g, ln_w, ln_b, r_k, eps: float, s0=None, reset=None, *, out=None, y=None,
+                     want_y: bool = True, s_out=None, workspace=None, need_workspace: bool = True,
+                     want_state: bool = True, algo: str = "auto", stream=None, flags: int = 0,
+                     log_decay: bool = False):
+    """The forward with the WKV epilogue: out = epilogue(y) (fused into the recurrence's kernel in the
+    fused chunked form).  Returns (out, y or None, s_out, workspace)."""
+    B, T, H = _token_shape(r)
+    dev = r.device
+    if out is None:
+        out = torch.empty_like(r)
+    if y is None and want_y:
+        y = torch.empty_like(r)
+    if s_out is None and want_state:
+        s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=dev, dtype=torch.float32)
+    if workspace is None and need_workspace:
+        workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype), 16), device=dev, dtype=torch.uint8)
+    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(flags, log_decay))
+    ep = _epi(ln_w, ln_b, r_k, eps)
+    st = lib().wkv7_forward_epilogue(ctypes.byref(d), ctypes.byref(ep),
+                                     *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, g, y, out, s_out, workspace)),
+                                     _stream(stream))
+    _check(st, "wkv7_forward_epilogue")
+    return out, y, s_out, workspace

@@ -117,3 +117,37 @@ def test_recurrence_and_epilogue_composed(W, algo, flag_a_head):
         assert e <= 2e-2 and cosine(f64(g[n]), go[n]) >= 0.999, (n, e)
     assert err_rms_excess(f64(ge["dg"]), go["dg"], "bf16") <= 2e-2
     assert err_rms(f64(g["ds0"]), go["ds0"]) <= 2e-2
+
+
+@pytest.mark.parametrize("algo", ("chunked_fused", "chunked_split", "scan", "auto"))
+@pytest.mark.parametrize("want_y", (True, False))
+@pytest.mark.parametrize("T", (40, 333))
+def test_forward_with_fused_epilogue(W, algo, want_y, T):
+    """wkv7_forward_epilogue: out is bit for bit the epilogue of the stored y (fused into the chunked
+    forward's y write-out, or the two kernels back to back), y and s_out equal the plain forward's;
+    a head with a decay out of the 1/L range takes the token path inside the fused kernel."""
+    import torch
+    rng = np.random.default_rng(400 + T)
+    B, H = 2, 5
+    d = I.draw_inputs(rng, (B, T, H, 64), "bf16")
+    w = I.to_f64(d["w"])
+    w[1, T // 2, 3, :4] = 0.0                   # one chunk of one head runs token by token
+    d["w"] = I.to_storage(w, "bf16")
+    gate = to_dev(I.to_storage(rng.standard_normal((B, T, H, 64)), "bf16"))
+    s0 = to_dev(rng.standard_normal((B, H, 64, 64)).astype(np.float32))
+    reset = np.zeros((B, T), np.uint8)
+    reset[0, 21] = 1
+    rd = to_dev(reset)
+    pd = [to_dev(a) for a in _params(rng, H)]
+    xs = inputs_dev(d)
+    y, s, _ = W.forward(*xs, s0=s0, reset=rd, algo=algo)
+    ref = W.epilogue_forward(y, xs[0], xs[2], xs[3], gate, *pd, EPS)
+    out, y2, s2, _ = W.forward_epilogue(*xs, gate, *pd, EPS, s0=s0, reset=rd, algo=algo, want_y=want_y)
+    assert torch.equal(out, ref)
+    assert torch.equal(s2, s)
+    if want_y:
+        assert torch.equal(y2, y)
+    yo, _, _ = oracle.forward(*inputs_f64(d), s0=f64(s0), reset=reset)
+    oo, _, _ = E.forward(f64(y), *(inputs_f64(d)[i] for i in (0, 2, 3)), f64(gate), *(f64(t) for t in pd), EPS)
+    assert err_rms_excess(f64(out), oo, "bf16") <= 2e-2
+    assert err_rms_excess(f64(y), yo, "bf16") <= 2e-2
