@@ -260,7 +260,8 @@ struct __align__(128) Ctx {
   Split<64, 64> S0T;     // S0^T [j][i]
   Split<32, 64> BKx;     // rows 0-15 (Tl^T Bh) [tau][j], rows 16-31 ((ls.X)^T Bh + ls.Kh) [tau][j]
   Split<16, 32> MMx;     // [t][Qm[t][0..15] | Vq[t][0..15]]
-  __align__(16) float lam[kChunk][kN];        // L_t [t][j]
+  __align__(16) float lam[kChunk][kN + 4];    // L_t [t][j] (rows padded: the float4 stores of 16 tokens
+                                              // of one channel group fall in distinct banks)
   int mask;                     // reset bits of the chunk
   int unsafe;                   // decay out of range (or staging timed out): the unit is re-run exactly
 };
@@ -329,17 +330,17 @@ __device__ __forceinline__ bool reset_flag(const BwdArgs& p, int64_t b, int64_t 
 // epilogue's block; rows past T arrive as zeros, K1 reads w there as 1) and, for c > 0, the
 // checkpoint entering it (one bulk copy), issued by one
 // thread on in_bar.
-template <typename T>
+template <typename T, bool kLog, bool kEpi>
 __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, int64_t unit, int64_t b,
                                       int64_t h, int64_t c, int64_t nc, int ktid) {
   if (ktid == 0) {
     if (!in_bounds(h < p.H && b < p.B && c >= 0 && c < nc && c * kChunk < p.T, p.status)) return;
     const unsigned ck_bytes = c > 0 ? unsigned(kN * kN * sizeof(float)) : 0u;
-    const unsigned dy_bytes = unsigned(kChunk * kN * (p.epi ? sizeof(float) : sizeof(T)));
+    const unsigned dy_bytes = unsigned(kChunk * kN * (kEpi ? sizeof(float) : sizeof(T)));
     mbar_arrive_expect_tx(&sm.in_bar, unsigned((kIn - 1) * kChunk * kN * sizeof(T)) + dy_bytes + ck_bytes + p.extra_tx);
 #pragma unroll
     for (int m = 0; m < kIn; ++m) {
-      void* dst = (m == kIn - 1 && p.epi) ? static_cast<void*>(&sm.dyf[0][0]) : static_cast<void*>(&sm.stg[m][0][0]);
+      void* dst = (m == kIn - 1 && kEpi) ? static_cast<void*>(&sm.dyf[0][0]) : static_cast<void*>(&sm.stg[m][0][0]);
       tma_load_4d(dst, &tm.m[m], 0, int(h), int(c * kChunk), int(b), &sm.in_bar);
     }
     if (c > 0 && range_ok((unit * nc + (c - 1)) * kN * kN, kN * kN, p.B * p.H * nc * kN * kN, p.status))
@@ -351,7 +352,7 @@ __device__ __forceinline__ void stage(const BwdArgs& p, const InputMaps& tm, Bwd
 // Decay products, decay-scaled operands, v, dy, S0^T and L_t.  A wait for the staged data that runs
 // out marks the chunk unsafe (the unit is then recomputed by the exact scan) and sets `timed_out`,
 // after which nothing more is staged.
-template <typename T>
+template <typename T, bool kLog, bool kEpi>
 __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, unsigned mask,
                                                  int64_t unit, int64_t c, int ktid, int len, unsigned parity,
                                                  bool& unsafe, bool& timed_out) {
@@ -373,7 +374,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
       float wmin = 1.f;
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        L[u] = t < len ? decay_of(w[u], p.log_decay) : 1.f;
+        L[u] = t < len ? decay_of(w[u], kLog) : 1.f;
         wmin = fminf(wmin, L[u]);
       }
 #pragma unroll
@@ -422,7 +423,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
     for (int e = 0; e < 8; ++e) {
       const int t = 8 * th + e;
       v8[e] = Elt<T>::to_f32(X[3][t][i]);
-      y8[e] = p.epi ? sm.dyf[t][i] : Elt<T>::to_f32(X[6][t][i]);
+      y8[e] = kEpi ? sm.dyf[t][i] : Elt<T>::to_f32(X[6][t][i]);
       m8[e] = t < fr ? y8[e] : 0.f;
     }
     put8(cx.SV, cb(i, 16 + 8 * th, 32), v8);
@@ -466,7 +467,7 @@ __device__ __forceinline__ void context_operands(const BwdArgs& p, BwdSmem<T>& s
 
 // The rest of the context (safe chunks only): the masked Gram, T, X, the folded operands BKx, Qm,
 // Vq and W, and SA^T.
-template <typename T>
+template <typename T, bool kLog, bool kEpi>
 __device__ __forceinline__ void context_products(const BwdArgs& p, const InputMaps& tm, BwdSmem<T>& sm, Ctx<T>& cx,
                                                  unsigned mask, int ktid, int64_t unit, int64_t b, int64_t h,
                                                  int64_t c_stage, int64_t nc) {
@@ -555,7 +556,7 @@ __device__ __forceinline__ void context_products(const BwdArgs& p, const InputMa
       put8(sm.AC, cb(16 + tau, 16 + 8 * q, 32), d);
     }
   } else if (c_stage >= 0) {
-    stage<T>(p, tm, sm, unit, b, h, c_stage, nc, ktid - 2 * kChunk);
+    stage<T, kLog, kEpi>(p, tm, sm, unit, b, h, c_stage, nc, ktid - 2 * kChunk);
   }
   named_bar(kBarCtx, 128);
 
@@ -696,7 +697,7 @@ __device__ __forceinline__ void issue_chunk(BwdSmem<T>& sm, Ctx<T>& cx, uint32_t
 }
 
 // ------------------------------------------------------------------ main warps
-template <typename T>
+template <typename T, bool kLog, bool kEpi>
 __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx<T>& cx, int64_t b, int64_t h,
                                            int64_t t0, int len, int warp, int lane, uint32_t tmem, unsigned phase) {
   const uint32_t tlane = uint32_t(32 * warp) << 16;
@@ -780,7 +781,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
 #pragma unroll
     for (int e = 0; e < 8; ++e) {
       if (tb + e < len && range_ok(tok_off(b, t0 + tb + e, h, p.T, p.H) + i, 1, total, p.status))
-        *dvp = Elt<T>::from_f32(p.epi ? dv[e] + static_cast<const float*>(p.dy)[3 * total + tok_off(b, t0 + tb + e, h, p.T, p.H) + i]
+        *dvp = Elt<T>::from_f32(kEpi ? dv[e] + static_cast<const float*>(p.dy)[3 * total + tok_off(b, t0 + tb + e, h, p.T, p.H) + i]
                                       : dv[e]);   // + the epilogue's bonus part
       dvp += rs;
     }
@@ -795,7 +796,7 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
   const int64_t o0 = tok_off(b, t0 + tb, h, p.T, p.H) + j;
   float rr[8], ar[8], br[8], kr[8], xw[8], er[8], ek[8];
   {
-    const float* const eg = static_cast<const float*>(p.dy);   // the epilogue's block, under p.epi
+    const float* const eg = static_cast<const float*>(p.dy);   // the epilogue's block, under kEpi
     const T* const gw = static_cast<const T*>(p.w);
     const T* const gr = static_cast<const T*>(p.r);
     const T* const ga = static_cast<const T*>(p.a);
@@ -809,9 +810,9 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
       ar[e] = ok ? Elt<T>::to_f32(ga[o]) : 0.f;
       br[e] = ok ? Elt<T>::to_f32(gb[o]) : 0.f;
       kr[e] = ok ? Elt<T>::to_f32(gk[o]) : 0.f;
-      xw[e] = ok && p.log_decay ? Elt<T>::to_f32(gw[o]) : 0.f;   // x, for dL/dx
-      er[e] = ok && p.epi ? eg[total + o] : 0.f;                 // bonus parts of dr, dk
-      ek[e] = ok && p.epi ? eg[2 * total + o] : 0.f;
+      xw[e] = ok && kLog ? Elt<T>::to_f32(gw[o]) : 0.f;   // x, for dL/dx
+      er[e] = ok && kEpi ? eg[total + o] : 0.f;                 // bonus parts of dr, dk
+      ek[e] = ok && kEpi ? eg[2 * total + o] : 0.f;
     }
   }
   mma_wait(p, &sm.gg_bar, phase & 1u);
@@ -888,18 +889,18 @@ __device__ __forceinline__ void main_chunk(const BwdArgs& p, BwdSmem<T>& sm, Ctx
       if (tb + e < len && range_ok(o0 + e * rs, 1, total, p.status)) {
         const int64_t o = o0 + e * rs;
         gda[o] = Elt<T>::from_f32(eA[e] * Lr[e]);
-        gdr[o] = Elt<T>::from_f32(fmaf(eR[e], Lr[e + 1], er[e]));
+        gdr[o] = Elt<T>::from_f32(kEpi ? fmaf(eR[e], Lr[e + 1], er[e]) : eR[e] * Lr[e + 1]);
         gdb[o] = Elt<T>::from_f32(eB[e] * il[e]);
-        gdk[o] = Elt<T>::from_f32(fmaf(eK[e], il[e], ek[e]));
+        gdk[o] = Elt<T>::from_f32(kEpi ? fmaf(eK[e], il[e], ek[e]) : eK[e] * il[e]);
         // cum = dL/d(log w_t): dw = cum / w_t = cum L_{t-1} / L_t, or dL/dx = -cum exp(x)
-        gdw[o] = Elt<T>::from_f32(p.log_decay ? dx_of_dlogw(cum, xw[e]) : cum * (Lr[e] * il[e]));
+        gdw[o] = Elt<T>::from_f32(kLog ? dx_of_dlogw(cum, xw[e]) : cum * (Lr[e] * il[e]));
       }
     }
   }
   tc::fence_before_sync();
 }
 
-template <typename T>
+template <typename T, bool kLog, bool kEpi>
 __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   BwdSmem<T>& sm = *reinterpret_cast<BwdSmem<T>*>(smem_raw);
@@ -961,7 +962,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         } else {
           tc::fence_after_sync();
           const int64_t t0 = c * kChunk;
-          main_chunk<T>(p, sm, cx, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane, tmem, phase);
+          main_chunk<T, kLog, kEpi>(p, sm, cx, b, h, t0, int(min64(kChunk, p.T - t0)), warp, lane, tmem, phase);
           ++phase;
         }
       }
@@ -993,7 +994,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
     bool pending = true;       // a staging was issued and not yet waited for
     bool timed_out = false;
     // prologue: stage the last chunk and fetch its reset flags
-    stage<T>(p, tm, sm, unit, b, h, nc - 1, nc, ktid);
+    stage<T, kLog, kEpi>(p, tm, sm, unit, b, h, nc - 1, nc, ktid);
     mask_next = __ballot_sync(0xffffffffu, reset_flag(p, b, nc - 1, lane)) & 0xffffu;
     bool f_prev = reset_flag(p, b, nc - 2, lane);
     cta_sync();
@@ -1003,7 +1004,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         Ctx<T>& cx = sm.ctx[c & 1];
         const unsigned mask = mask_next;
         bool unsafe = false;
-        context_operands<T>(p, sm, cx, mask, unit, c, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, unsafe,
+        context_operands<T, kLog, kEpi>(p, sm, cx, mask, unit, c, ktid, int(min64(kChunk, p.T - c * kChunk)), phase & 1u, unsafe,
                             timed_out);
         if (!timed_out) {
           pending = false;
@@ -1017,7 +1018,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
           f_prev = reset_flag(p, b, c - 2, lane);
         }
         if (!unsafe) {
-          context_products<T>(p, tm, sm, cx, mask, ktid, unit, b, h, c > 0 ? c - 1 : -1, nc);
+          context_products<T, kLog, kEpi>(p, tm, sm, cx, mask, ktid, unit, b, h, c > 0 ? c - 1 : -1, nc);
         }
       }
       cta_sync();
@@ -1032,7 +1033,7 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
         const int64_t c = nc - it;
         Ctx<T>& cx = sm.ctx[c & 1];
         // dy has no lo half when it arrives in bf16 (exact); the epilogue's fp32 dy has one
-        if (!cx.unsafe) issue_chunk<T>(sm, cx, tmem, tid == kIssueTid, std::is_same<T, bf16>::value && !p.epi);
+        if (!cx.unsafe) issue_chunk<T>(sm, cx, tmem, tid == kIssueTid, std::is_same<T, bf16>::value && !kEpi);
       }
       cta_sync();
       if (sm.stop) break;
@@ -1048,13 +1049,21 @@ __global__ void __launch_bounds__(kThreads, 1) chunk_bwd_kernel(const BwdArgs p,
 // One CTA per SM: the whole shared memory of an SM (227 KB per CTA at most, static part included).
 static_assert(sizeof(BwdSmem<__nv_bfloat16>) + 1024 <= 227 * 1024, "backward shared memory exceeds one SM");
 
+// The log-space decay and the epilogue's gradient block are template parameters: the kernel without
+// them has none of their code in its hot loops.
+template <typename T, bool kLog, bool kEpi>
+cudaError_t launch_t(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
+  const size_t smem = sizeof(BwdSmem<T>);
+  cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<T, kLog, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       int(smem));
+  if (e != cudaSuccess) return e;
+  chunk_bwd_kernel<T, kLog, kEpi><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
+  return cudaGetLastError();
+}
 template <typename T>
 cudaError_t launch(const BwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
-  const size_t smem = sizeof(BwdSmem<T>);
-  cudaError_t e = cudaFuncSetAttribute(chunk_bwd_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
-  if (e != cudaSuccess) return e;
-  chunk_bwd_kernel<T><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
-  return cudaGetLastError();
+  if (p.log_decay) return p.epi ? launch_t<T, true, true>(p, tm, stream) : launch_t<T, true, false>(p, tm, stream);
+  return p.epi ? launch_t<T, false, true>(p, tm, stream) : launch_t<T, false, false>(p, tm, stream);
 }
 
 }  // namespace

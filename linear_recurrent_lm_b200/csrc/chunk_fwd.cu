@@ -155,7 +155,7 @@ __device__ __forceinline__ void stage_chunk(const FwdArgs& p, const InputMaps& t
 // ------------------------------------------------------------------ context warps
 // `degraded` (CTA-uniform, sticky): a wait for staged inputs ran out; from then on nothing more is
 // staged and every chunk takes the token path, which reads its inputs from global memory.
-template <typename T>
+template <typename T, bool kLog>
 __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps& tm, FwdSmem3<T>& sm, Ctx& cx,
                                               unsigned mask, int64_t b, int64_t h, int64_t c, int64_t nc, int ktid,
                                               bool& degraded) {
@@ -176,7 +176,7 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
     auto ldw = [&](int t) {   // padding: w = 1
       if (t >= len) return make_float2(1.f, 1.f);
       const float2 x = ld2(1, t);
-      return make_float2(decay_of(x.x, p.log_decay), decay_of(x.y, p.log_decay));
+      return make_float2(decay_of(x.x, kLog), decay_of(x.y, kLog));
     };
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
     for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
@@ -530,7 +530,7 @@ __device__ __forceinline__ void store_ck(float* ck, const float (&acc)[8][4]) {
   }
 }
 
-template <typename T, bool kEpi>
+template <typename T, bool kEpi, bool kLog>
 __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p, const __grid_constant__ InputMaps tm) {
   extern __shared__ __align__(1024) unsigned char smem_raw[];
   FwdSmem3<T>& sm = *reinterpret_cast<FwdSmem3<T>*>(smem_raw);
@@ -686,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
           reset_bits = __ballot_sync(0xffffffffu, f) & 0xffffu;
         }
         const bool was_degraded = degraded;
-        build_context<T>(p, tm, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid, degraded);
+        build_context<T, kLog>(p, tm, sm, sm.ctx[c & 1], mask, b, h, c, nc, ktid, degraded);
         if (degraded && !was_degraded) stuck = unsigned(c & 1);
         tc::fence_smem_to_async();   // the tcgen05 operands of the context, for the tensor core
       }
@@ -697,12 +697,14 @@ __global__ void __launch_bounds__(kThreads, 2) chunk_fwd_kernel(const FwdArgs p,
   }
 }
 
+// The log-space decay is a template parameter: the kernel without it has none of its code in K1.
 template <typename T, bool kEpi>
 cudaError_t launch(const FwdArgs& p, const InputMaps& tm, cudaStream_t stream) {
   const size_t smem = sizeof(FwdSmem3<T>);
-  cudaError_t e = cudaFuncSetAttribute(chunk_fwd_kernel<T, kEpi>, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
+  auto kern = p.log_decay ? chunk_fwd_kernel<T, kEpi, true> : chunk_fwd_kernel<T, kEpi, false>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem));
   if (e != cudaSuccess) return e;
-  chunk_fwd_kernel<T, kEpi><<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
+  kern<<<dim3(unsigned(p.B * p.H)), dim3(kThreads), smem, stream>>>(p, tm);
   return cudaGetLastError();
 }
 
