@@ -42,6 +42,11 @@ BYTES_PREFILL = 768 + 128
 BYTES_DECODE = 64 * 64 * 4 * 2 + 768 + 128
 BYTES_EPI_FWD = 5 * 128 + 128                # y, r, k, v, g in; out (bf16)
 BYTES_EPI_BWD = 6 * 128 + 128 + 4 * 256      # y, r, k, v, g, dout in; dg, and dy, dr, dk, dv parts (fp32) out
+# GDN map per value token-head at N = 128, bf16, two value heads per key head: q, k read once per key
+# head (512 B / 2), g and beta (8 B), r, x, kw, a, b written (5 x 256 B).
+BYTES_GDN_MAP = 512 // 2 + 8 + 5 * 256
+# Token-order forward at N = 128 without checkpoints: six inputs and y, 256 B each.
+BYTES_SCAN128_FWD = 7 * 256
 
 
 def rank_seed(rank: int) -> int:
@@ -672,6 +677,39 @@ def measure_secondary(wkv7, dev, algo):
         "bwd_frac": BYTES_EPI_BWD * units3 / (bm / 1e3) / 1e9 / peak,
         "l2": "inputs larger than L2 (no flush)"}
     del tens, yb, rb, kb, vb, gb, dob, outb, eg
+
+    # A gated-DeltaNet layer on this recurrence (rwkv-lab page, "Highlight result -- GDN in RWKV-7"):
+    # 32 value heads over 16 key heads of 128 channels, B=8, T=4096, bf16.  The map (q, k, g, beta ->
+    # r, x, kw, a, b; HBM streaming) and then the token-order forward at N = 128 with the log-space
+    # decay, no checkpoints (there is no N = 128 backward).
+    Bg, Tg, Hg, Hkg, Ng = 8, 4096, 32, 16, 128
+    gd = I.draw_gdn_inputs(np.random.default_rng(77), Bg, Tg, Hg, Hkg, Ng, "bf16")
+    gq, gk, gv, gg, gb = (d(gd[n]) for n in ("q", "k", "v", "g", "beta"))
+    del gd
+    mo = {n: torch.empty((Bg, Tg, Hg, Ng), device=dev, dtype=torch.bfloat16) for n in ("r", "x", "kw", "a", "b")}
+    yg = torch.empty_like(gv)
+    sg = torch.empty((Bg, Hg, Ng, Ng), device=dev, dtype=torch.float32)
+    m_ms, f_ms = [], []
+    for rep in range(6):
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        wkv7.gdn_map(gq, gk, gg, gb, Hg, eps=1e-6, out=mo)
+        e1.record()
+        wkv7.forward(mo["r"], mo["x"], mo["kw"], gv, mo["a"], mo["b"], y=yg, s_out=sg, need_workspace=False,
+                     log_decay=True)
+        e2.record()
+        torch.cuda.synchronize()
+        if rep >= 2:
+            m_ms.append(e0.elapsed_time(e1))
+            f_ms.append(e1.elapsed_time(e2))
+    mm, fm = statistics.median(m_ms), statistics.median(f_ms)
+    ug = Bg * Tg * Hg
+    out["gdn_layer_B8_T4096_H32_Hk16_N128"] = {
+        "map_ms": mm, "forward_ms": fm, "tokens_per_s": Bg * Tg / ((mm + fm) / 1e3),
+        "map_frac": BYTES_GDN_MAP * ug / (mm / 1e3) / 1e9 / peak,
+        "forward_gbs": BYTES_SCAN128_FWD * ug / (fm / 1e3) / 1e9,
+        "l2": "inputs larger than L2 (no flush)"}
+    del gq, gk, gv, gg, gb, mo, yg, sg
 
     wl = I.make_workload(4)
     state = d(wl.state0)

@@ -19,8 +19,13 @@
  *
  * Conventions shared by every entry point
  * ---------------------------------------
- * - Head size N must be 64 (the HF model card page limits its kernel to heads
- *   of 64 channels with an fp32 state); anything else -> WKV7_ERR_UNSUPPORTED.
+ * - Head size N is 64 (the HF model card page limits its kernel to heads
+ *   of 64 channels with an fp32 state).  wkv7_forward with the token-order
+ *   scan (algo SCAN, or AUTO, which picks it), wkv7_step and wkv7_gdn_map also
+ *   take N = 128, the head size of the gated-DeltaNet layers that the rwkv-lab
+ *   page maps onto this recurrence; every other entry point and algo returns
+ *   WKV7_ERR_UNSUPPORTED for it, as does any other N.  Below, "64" in a shape
+ *   stands for N where N = 128 is accepted.
  * - Activations r,w,k,v,a,b,y,dy and the gradients dr..db are [B,T,H,64],
  *   contiguous, row-major, all in the one dtype of the descriptor (f32, bf16
  *   or f16, the three activation types the same page lists).  Outputs in a
@@ -105,7 +110,7 @@ typedef struct {
   int64_t B;      /* batch rows                                  */
   int64_t T;      /* tokens per row (for wkv7_step: must be 1)   */
   int64_t H;      /* heads                                       */
-  int32_t N;      /* head size: must be 64                       */
+  int32_t N;      /* head size: 64 (128 where stated)            */
   int32_t dtype;  /* wkv7_dtype_t of every activation/gradient   */
   int32_t algo;   /* wkv7_algo_t                                 */
   uint32_t flags; /* 0, or the WKV7_FLAG_* bits below            */
@@ -201,7 +206,8 @@ const char* wkv7_status_string(wkv7_status_t status);
  * Checkpoint c holds the state after token min(16(c+1), T) - 1, its element
  * (i, j) at offset (i/16)*1024 + (j/8)*128 + (4*(i%8) + (j%8)/2)*4
  * + 2*((i/8)%2) + j%2 (the order of the kernels' mma accumulator fragments, so
- * that every warp moves 512 contiguous bytes per store).  After the
+ * that every warp moves 512 contiguous bytes per store); with N = 128 the
+ * checkpoints are 128x128, row-major (no backward reads them).  After the
  * checkpoints come B*H ints (rounded up to 16 bytes) that wkv7_backward uses
  * to mark heads it must recompute with the exact scan.
  * Returns 0 for an invalid descriptor or T == 0.
@@ -255,7 +261,7 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* desc, const void* r, const void* 
  * one-token step on a carried state, with ragged batches padded on the right
  * without changing the padded rows' results).
  *
- *   desc         B, H, N=64, dtype; T must be 1; algo is ignored
+ *   desc         B, H, N (64 or 128), dtype; T must be 1; algo is ignored
  *   r..b         in      [B,H,64] desc->dtype (one token per row)
  *   state        in/out  [B,H,64,64] fp32
  *   active       in      [B] u8, or NULL for all rows active.  A row with
@@ -361,6 +367,45 @@ wkv7_status_t wkv7_epilogue_backward(const wkv7_desc_t* desc, const wkv7_epilogu
                                      const void* r, const void* k, const void* v, const void* g,
                                      const void* dout, float* eg, void* dg, float* dln_w, float* dln_b,
                                      float* dr_k, void* stream);
+
+/*
+ * ------------------------------------------------------------------ GDN map
+ * The front end that runs a gated DeltaNet (GDN) layer on this recurrence
+ * (rwkv-lab page, "Highlight result -- GDN in RWKV-7": the gated delta rule is
+ * the wkv7 recurrence at matched head sizes, fed through a fixed map of GDN's
+ * inputs).  Per (b, t) and value head h, reading key head kh = h / (H / Hk):
+ *
+ *   q^ = q / sqrt(|q|^2 + eps),  k^ = k / sqrt(|k|^2 + eps)   (over N channels)
+ *   r  = r_scale q^          (1/sqrt(N) gives GDN's output scale: y is linear in r)
+ *   x  = log(-g) on every channel: the log-space decay input, exp(-exp(x)) = exp(g)
+ *   kw = beta k^,   a = -k^,   b = exp(g) beta k^
+ *
+ * after which wkv7_forward / wkv7_step with WKV7_FLAG_LOG_DECAY on (r, x, kw,
+ * v, a, b) -- v is GDN's own, unchanged -- compute GDN's output and state:
+ * S_t = exp(g_t) S_{t-1} (I - beta_t k^ k^T) + beta_t v_t k^T, o_t = S_t r_t.
+ *
+ *   desc         B, T, H (value heads), N (64 or 128), dtype; algo is ignored;
+ *                flags 0 or WKV7_FLAG_CHECK_FINITE (which scans r, kw, a, b:
+ *                x is -inf wherever g = 0, i.e. no decay)
+ *   gd           Hk >= 1 key heads with H % Hk == 0; eps >= 0 and r_scale
+ *                finite (else WKV7_ERR_UNSUPPORTED)
+ *   q, k         in   [B,T,Hk,N] desc->dtype, 16-byte aligned
+ *   g, beta      in   [B,T,H] fp32, 4-byte aligned; g <= 0 (GDN's decay is
+ *                exp(g) <= 1; g > 0 writes NaN into x)
+ *   r, x, kw, a, b  out  [B,T,H,N] desc->dtype, 16-byte aligned, not
+ *                overlapping the inputs
+ * With eps = 0 a zero q or k row gives non-finite outputs.  Errors as for
+ * wkv7_forward.
+ */
+typedef struct {
+  int64_t Hk;    /* key heads: value head h reads key head h / (H / Hk) */
+  float eps;     /* L2-normalisation guard, >= 0 */
+  float r_scale; /* multiplies q^ into r */
+} wkv7_gdn_t;
+
+wkv7_status_t wkv7_gdn_map(const wkv7_desc_t* desc, const wkv7_gdn_t* gd, const void* q, const void* k,
+                           const float* g, const float* beta, void* r, void* x, void* kw, void* a, void* b,
+                           void* stream);
 
 #ifdef __cplusplus
 }

@@ -74,6 +74,11 @@ __host__ __device__ __forceinline__ int ckpt_off(int i, int j) {
 __device__ __forceinline__ int64_t tok_off(int64_t b, int64_t t, int64_t h, int64_t T, int64_t H) {
   return ((b * T + t) * H + h) * kN;
 }
+// The same in a [B,T,H,N] tensor.
+template <int N>
+__device__ __forceinline__ int64_t tok_offn(int64_t b, int64_t t, int64_t h, int64_t T, int64_t H) {
+  return ((b * T + t) * H + h) * N;
+}
 
 }  // namespace wkv7
 

@@ -27,6 +27,7 @@ struct FwdArgs {
   void* out;
   const float *ln_w, *ln_b, *r_k;
   float eps;
+  int N;                  // head size: 64, or 128 (token-order scan only)
 };
 
 // Bits of the device status word.
@@ -85,6 +86,7 @@ struct StepArgs {
   void* y;
   int* status;   // device status word (debug-build bounds checks)
   bool log_decay;  // w holds x (see FwdArgs)
+  int N;           // head size: 64 or 128
 };
 
 // The WKV epilogue (GroupNorm per head, bonus, gating): forward writes `out`; backward writes the
@@ -101,6 +103,17 @@ struct EpiArgs {
   int* status;
 };
 
+// The gated-delta-rule map: q, k [B,T,Hk,N] -> r, x, kw, a, b [B,T,H,N] (all of dtype T); g, beta
+// fp32 [B,T,H].
+struct GdnArgs {
+  int64_t B, T, H, Hk;
+  const void *q, *k;
+  const float *g, *beta;
+  float eps, r_scale;
+  void *r, *x, *kw, *a, *b;
+  int* status;
+};
+
 // Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).
 wkv7_status_t validate_desc(const wkv7_desc_t* d);
 
@@ -110,6 +123,7 @@ cudaError_t launch_scan_fwd(const FwdArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cudaStream_t stream);
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_epilogue(const EpiArgs& p, int dtype, bool backward, cudaStream_t stream);
+cudaError_t launch_gdn_map(const GdnArgs& p, int dtype, int N, cudaStream_t stream);
 // Set kStatusNonFinite in *status if any of the n elements at x (dtype as above; 16-byte aligned)
 // is NaN or infinite.  x == nullptr or n == 0: nothing is launched.
 cudaError_t launch_finite_scan(const void* x, int64_t n, int dtype, int* status, cudaStream_t stream);

@@ -44,6 +44,7 @@ extern "C" wkv7_status_t wkv7_train_step_noalloc(const wkv7_desc_t* d, const voi
                                                  void* db, float* ds0, void* stream) {
   const wkv7_status_t valid = wkv7::validate_desc(d);
   if (valid != WKV7_OK) return valid;
+  if (d->N != 64) return WKV7_ERR_UNSUPPORTED;   // the backward is written for heads of 64
   const size_t need = wkv7_workspace_bytes(d);
   if (need == 0 && d->T != 0) return WKV7_ERR_SHAPE;   // (an accepted descriptor always has a size)
   if (need > size_t(WKV7_NOALLOC_SCRATCH_BYTES)) return WKV7_ERR_SCRATCH_LIMIT;

@@ -29,8 +29,13 @@
 namespace wkv7 {
 namespace {
 
-constexpr int kThreads = 512;
-constexpr int kMinBlocks = 3;
+// N = 64: 512 threads, three CTAs per SM; N = 128 (the gated-delta-rule heads of the rwkv-lab
+// page's GDN map): 1024 threads, 16 columns per thread.
+template <int N> struct StepShape {
+  static constexpr int kThreads = 8 * N;                 // 8 threads per state row
+  static constexpr int kCols = N / 8;                    // columns per thread
+  static constexpr int kMinBlocks = N == 64 ? 3 : 1;
+};
 constexpr int kMaxDevices = 64;
 
 // Eight consecutive elements of T (16-byte aligned) as fp32.
@@ -44,40 +49,50 @@ __device__ __forceinline__ void load8(const T* g, float* out) {
   }
 }
 
-template <typename T>
-__global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) {
+template <typename T, int N>
+__global__ void __launch_bounds__(StepShape<N>::kThreads, StepShape<N>::kMinBlocks) step_kernel(StepArgs p) {
+  constexpr int C = StepShape<N>::kCols;
   // Everything this grid reads or writes may belong to the grid launched before it.
   asm volatile("griddepcontrol.wait;" ::: "memory");
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int t = threadIdx.x;
-  const int i = t >> 3, q = t & 7;   // row i, columns 8q..8q+7
+  const int i = t >> 3, q = t & 7;   // row i, columns C q .. C q + C - 1
   const int64_t units = p.B * p.H;
   for (int64_t unit = blockIdx.x; unit < units; unit += gridDim.x) {
     // (debug build: the row of y, the state row and the input rows of this unit)
-    if (!range_ok(unit * kN, kN, units * kN, p.status) || !range_ok((unit * kN + i) * kN + q * 8, 8, units * kN * kN, p.status))
+    if (!range_ok(unit * N, N, units * N, p.status) || !range_ok((unit * N + i) * N + q * C, C, units * N * N, p.status))
       continue;
-    T* y = static_cast<T*>(p.y) + unit * kN;
+    T* y = static_cast<T*>(p.y) + unit * N;
     if (p.active && !p.active[unit / p.H]) {   // padded row: its state is not even read
       if (q == 0) y[i] = Elt<T>::from_f32(0.f);
       continue;
     }
-    float4* row = reinterpret_cast<float4*>(p.state + (unit * kN + i) * kN + q * 8);
-    const float4 s_lo = row[0], s_hi = row[1];
-    float S[8] = {s_lo.x, s_lo.y, s_lo.z, s_lo.w, s_hi.x, s_hi.y, s_hi.z, s_hi.w};
-    const int64_t o = unit * kN + q * 8;
-    float wv[8], kv[8], av[8], bv[8], rv[8];
-    load8<T>(static_cast<const T*>(p.a) + o, av);
-    load8<T>(static_cast<const T*>(p.w) + o, wv);
+    float4* row = reinterpret_cast<float4*>(p.state + (unit * N + i) * N + q * C);
+    float S[C];
 #pragma unroll
-    for (int j = 0; j < 8; ++j) wv[j] = decay_of(wv[j], p.log_decay);
-    load8<T>(static_cast<const T*>(p.b) + o, bv);
-    load8<T>(static_cast<const T*>(p.k) + o, kv);
-    load8<T>(static_cast<const T*>(p.r) + o, rv);
-    const float vi = Elt<T>::to_f32(static_cast<const T*>(p.v)[unit * kN + i]);
+    for (int u = 0; u < C / 4; ++u) {
+      const float4 s4 = row[u];
+      S[4 * u] = s4.x; S[4 * u + 1] = s4.y; S[4 * u + 2] = s4.z; S[4 * u + 3] = s4.w;
+    }
+    const int64_t o = unit * N + q * C;
+    float wv[C], kv[C], av[C], bv[C], rv[C];
+#pragma unroll
+    for (int u = 0; u < C / 8; ++u) load8<T>(static_cast<const T*>(p.a) + o + 8 * u, av + 8 * u);
+#pragma unroll
+    for (int u = 0; u < C / 8; ++u) load8<T>(static_cast<const T*>(p.w) + o + 8 * u, wv + 8 * u);
+#pragma unroll
+    for (int j = 0; j < C; ++j) wv[j] = decay_of(wv[j], p.log_decay);
+#pragma unroll
+    for (int u = 0; u < C / 8; ++u) {
+      load8<T>(static_cast<const T*>(p.b) + o + 8 * u, bv + 8 * u);
+      load8<T>(static_cast<const T*>(p.k) + o + 8 * u, kv + 8 * u);
+      load8<T>(static_cast<const T*>(p.r) + o + 8 * u, rv + 8 * u);
+    }
+    const float vi = Elt<T>::to_f32(static_cast<const T*>(p.v)[unit * N + i]);
 
     float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; j += 2) {
+    for (int j = 0; j < C; j += 2) {
       s0 = fmaf(S[j], av[j], s0);
       s1 = fmaf(S[j + 1], av[j + 1], s1);
     }
@@ -88,12 +103,12 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) 
 
     float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
+    for (int j = 0; j < C; ++j) {
       S[j] = fmaf(S[j], wv[j], fmaf(sa, bv[j], vi * kv[j]));
       if (j & 1) y1 = fmaf(S[j], rv[j], y1); else y0 = fmaf(S[j], rv[j], y0);
     }
-    row[0] = make_float4(S[0], S[1], S[2], S[3]);
-    row[1] = make_float4(S[4], S[5], S[6], S[7]);
+#pragma unroll
+    for (int u = 0; u < C / 4; ++u) row[u] = make_float4(S[4 * u], S[4 * u + 1], S[4 * u + 2], S[4 * u + 3]);
     float yy = y0 + y1;
     yy += __shfl_xor_sync(0xffffffffu, yy, 1);
     yy += __shfl_xor_sync(0xffffffffu, yy, 2);
@@ -104,7 +119,7 @@ __global__ void __launch_bounds__(kThreads, kMinBlocks) step_kernel(StepArgs p) 
 
 // Resident grid size for this device and element type, looked up once (concurrent first calls
 // may both look it up; they store the same value).
-template <typename T>
+template <typename T, int N>
 cudaError_t grid_size(int64_t units, unsigned* out) {
   static std::atomic<int> cached[kMaxDevices];   // SMs x resident CTAs per SM; 0 = not looked up yet
   int dev = 0;
@@ -115,7 +130,7 @@ cudaError_t grid_size(int64_t units, unsigned* out) {
     int sms = 0, per_sm = 0;
     e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
     if (e != cudaSuccess) return e;
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<T>, kThreads, 0);
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, step_kernel<T, N>, StepShape<N>::kThreads, 0);
     if (e != cudaSuccess) return e;
     slots = sms * (per_sm > 0 ? per_sm : 1);
     if (dev >= 0 && dev < kMaxDevices) cached[dev].store(slots, std::memory_order_relaxed);
@@ -124,14 +139,14 @@ cudaError_t grid_size(int64_t units, unsigned* out) {
   return cudaSuccess;
 }
 
-template <typename T>
+template <typename T, int N>
 cudaError_t launch(const StepArgs& p, cudaStream_t stream) {
   unsigned grid = 0;
-  cudaError_t e = grid_size<T>(p.B * p.H, &grid);
+  cudaError_t e = grid_size<T, N>(p.B * p.H, &grid);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(grid);
-  cfg.blockDim = dim3(kThreads);
+  cfg.blockDim = dim3(StepShape<N>::kThreads);
   cfg.dynamicSmemBytes = 0;
   cfg.stream = stream;
   cudaLaunchAttribute attr[1];
@@ -139,7 +154,7 @@ cudaError_t launch(const StepArgs& p, cudaStream_t stream) {
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, step_kernel<T>, p);
+  e = cudaLaunchKernelEx(&cfg, step_kernel<T, N>, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
@@ -147,10 +162,11 @@ cudaError_t launch(const StepArgs& p, cudaStream_t stream) {
 }  // namespace
 
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream) {
+  const bool n128 = p.N == 128;
   switch (dtype) {
-    case 0: return launch<float>(p, stream);
-    case 1: return launch<__nv_bfloat16>(p, stream);
-    case 2: return launch<__half>(p, stream);
+    case 0: return n128 ? launch<float, 128>(p, stream) : launch<float, 64>(p, stream);
+    case 1: return n128 ? launch<__nv_bfloat16, 128>(p, stream) : launch<__nv_bfloat16, 64>(p, stream);
+    case 2: return n128 ? launch<__half, 128>(p, stream) : launch<__half, 64>(p, stream);
     default: return cudaErrorInvalidValue;
   }
 }

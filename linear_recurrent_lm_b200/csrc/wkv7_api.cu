@@ -28,7 +28,7 @@ bool mul_ok(int64_t a, int64_t b, int64_t* out) {
 // Common descriptor checks.  On success fills the element counts.
 wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elems) {
   if (!d) return WKV7_ERR_NULL;
-  if (d->N != 64 || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE | WKV7_FLAG_LOG_DECAY |
+  if ((d->N != 64 && d->N != 128) || (d->flags & ~(WKV7_FLAG_TEST_WAIT_TIMEOUT | WKV7_FLAG_CHECK_FINITE | WKV7_FLAG_LOG_DECAY |
                                   WKV7_FLAG_EPILOGUE_GRADS)) != 0u)
     return WKV7_ERR_UNSUPPORTED;
   if ((d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) && (d->T > 16 || d->T < 0)) return WKV7_ERR_UNSUPPORTED;
@@ -37,23 +37,26 @@ wkv7_status_t check_desc(const wkv7_desc_t* d, int64_t* units, int64_t* tok_elem
   if (d->B < 0 || d->T < 0 || d->H < 0) return WKV7_ERR_SHAPE;
   int64_t bh, bth, e;
   if (!mul_ok(d->B, d->H, &bh) || bh > kMaxGrid) return WKV7_ERR_SHAPE;
-  if (!mul_ok(bh, d->T, &bth) || !mul_ok(bth, 64 * 4, &e)) return WKV7_ERR_SHAPE;   // byte count fits
+  if (!mul_ok(bh, d->T, &bth) || !mul_ok(bth, d->N * 4, &e)) return WKV7_ERR_SHAPE;   // byte count fits
   int64_t st;
-  if (!mul_ok(bh, 64 * 64 * 4, &st)) return WKV7_ERR_SHAPE;
+  const int64_t n = d->N;
+  if (!mul_ok(bh, n * n * 4, &st)) return WKV7_ERR_SHAPE;
   // the checkpoint workspace (one 16 KiB state per head per 16 tokens, then one int per head) must
   // have a byte count too, so that wkv7_workspace_bytes is non-zero for every accepted T > 0
   int64_t ck;
-  if (!mul_ok(bh, (d->T + 15) / 16, &ck) || !mul_ok(ck, 64 * 64 * 4, &ck) || ck > INT64_MAX - (bh * 4 + 15))
+  if (!mul_ok(bh, (d->T + 15) / 16, &ck) || !mul_ok(ck, n * n * 4, &ck) || ck > INT64_MAX - (bh * 4 + 15))
     return WKV7_ERR_SHAPE;
   *units = bh;
-  *tok_elems = bth * 64;
+  *tok_elems = bth * d->N;
   return WKV7_OK;
 }
 
 // The chunked kernels compute their products in tf32 (11 significant bits): on f32 inputs they
 // cannot hold the 1e-4 bound that f32 results must meet, so only the exact scan takes f32.  (A
 // decode step has no algorithm choice and is not affected.)
+// Heads of 128 (the GDN map's) run the token-order scan only.
 wkv7_status_t check_algo_dtype(const wkv7_desc_t* d) {
+  if (d->N != 64 && d->algo >= WKV7_ALGO_CHUNKED) return WKV7_ERR_UNSUPPORTED;
   return (d->dtype == WKV7_F32 && d->algo >= WKV7_ALGO_CHUNKED) ? WKV7_ERR_UNSUPPORTED : WKV7_OK;
 }
 
@@ -136,7 +139,7 @@ wkv7_status_t encode_inputs(const wkv7_desc_t* d, std::initializer_list<const vo
 unsigned test_extra_tx(const wkv7_desc_t* d) { return (d->flags & WKV7_FLAG_TEST_WAIT_TIMEOUT) ? 16u : 0u; }
 
 bool use_chunked(const wkv7_desc_t* d) {
-  if (d->algo == WKV7_ALGO_SCAN) return false;
+  if (d->algo == WKV7_ALGO_SCAN || d->N != 64) return false;
   if (d->algo == WKV7_ALGO_AUTO) return d->dtype != WKV7_F32;
   return true;
 }
@@ -194,7 +197,7 @@ const char* wkv7_status_string(wkv7_status_t s) {
 int64_t checkpoint_bytes(const wkv7_desc_t* d, int64_t units) {
   const int64_t nc = (d->T + 15) / 16;
   int64_t n1, n2;
-  if (!mul_ok(units, nc, &n1) || !mul_ok(n1, 64 * 64 * 4, &n2)) return -1;
+  if (!mul_ok(units, nc, &n1) || !mul_ok(n1, int64_t(d->N) * d->N * 4, &n2)) return -1;
   return n2;
 }
 
@@ -226,8 +229,9 @@ wkv7_status_t wkv7_forward(const wkv7_desc_t* d, const void* r, const void* w, c
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
                   status, test_extra_tx(d), (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
+  p.N = int(d->N);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  const std::initializer_list<Output> outs = {{y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}};
+  const std::initializer_list<Output> outs = {{y, te, d->dtype}, {s_out, units * d->N * d->N, WKV7_F32}};
   if (d->T == 0 || !use_chunked(d)) return check_outputs(d, wkv7::launch_scan_fwd(p, d->dtype, s), outs, status, s);
   bool split = false;
   st = use_split(d, units, workspace, &split);
@@ -246,6 +250,7 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
   int64_t units = 0, te = 0;
   wkv7_status_t st = check_desc(d, &units, &te);
   if (st != WKV7_OK) return st;
+  if (d->N != 64) return WKV7_ERR_UNSUPPORTED;   // the backward kernels are written for heads of 64
   st = check_algo_dtype(d);
   if (st != WKV7_OK) return st;
   st = check_ptrs(te > 0, {r, w, k, v, a, b, dy, dr, dw, dk, dv, da, db});
@@ -281,7 +286,7 @@ wkv7_status_t wkv7_backward(const wkv7_desc_t* d, const void* r, const void* w, 
 static wkv7_status_t check_epilogue(const wkv7_desc_t* d, const wkv7_epilogue_t* ep, int64_t* units, int64_t* te) {
   wkv7_status_t st = check_desc(d, units, te);
   if (st != WKV7_OK) return st;
-  if ((d->flags & ~WKV7_FLAG_CHECK_FINITE) != 0u) return WKV7_ERR_UNSUPPORTED;
+  if ((d->flags & ~WKV7_FLAG_CHECK_FINITE) != 0u || d->N != 64) return WKV7_ERR_UNSUPPORTED;
   if (!ep || !ep->ln_w || !ep->ln_b || !ep->r_k) return WKV7_ERR_NULL;
   if (!(ep->eps > 0.f) || !(ep->eps < 1e30f)) return WKV7_ERR_UNSUPPORTED;   // also refuses NaN
   for (const void* q : {static_cast<const void*>(ep->ln_w), static_cast<const void*>(ep->ln_b),
@@ -359,13 +364,38 @@ wkv7_status_t wkv7_forward_epilogue(const wkv7_desc_t* d, const wkv7_epilogue_t*
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
   wkv7::FwdArgs p{d->B, d->T, d->H, r, w, k, v, a, b, s0, reset, y, s_out, static_cast<float*>(workspace),
                   status, test_extra_tx(d), (d->flags & WKV7_FLAG_LOG_DECAY) != 0u,
-                  g, out, ep->ln_w, ep->ln_b, ep->r_k, ep->eps};
+                  g, out, ep->ln_w, ep->ln_b, ep->r_k, ep->eps, int(d->N)};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   wkv7::InputMaps tm;
   st = encode_inputs(d, {r, w, k, v, a, b}, &tm);
   if (st != WKV7_OK) return st;
   return check_outputs(d, wkv7::launch_chunk_fwd(p, tm, d->dtype, s),
                        {{out, te, d->dtype}, {y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}}, status, s);
+}
+
+wkv7_status_t wkv7_gdn_map(const wkv7_desc_t* d, const wkv7_gdn_t* gd, const void* q, const void* k,
+                           const float* g, const float* beta, void* r, void* x, void* kw, void* a, void* b,
+                           void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  if ((d->flags & ~WKV7_FLAG_CHECK_FINITE) != 0u) return WKV7_ERR_UNSUPPORTED;
+  if (!gd) return WKV7_ERR_NULL;
+  if (gd->Hk < 1 || d->H % gd->Hk != 0 || !(gd->eps >= 0.f) || !(gd->eps < 1e30f) ||
+      !(gd->r_scale == gd->r_scale) || !(gd->r_scale < 1e30f && gd->r_scale > -1e30f))
+    return WKV7_ERR_UNSUPPORTED;
+  st = check_ptrs(te > 0, {q, k, r, x, kw, a, b});
+  if (st != WKV7_OK) return st;
+  if (te > 0 && (!g || !beta)) return WKV7_ERR_NULL;
+  for (const float* p : {g, beta})
+    if (reinterpret_cast<uintptr_t>(p) % 4u != 0u) return WKV7_ERR_ALIGN;
+  if (te == 0) return WKV7_OK;
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::GdnArgs p{d->B, d->T, d->H, gd->Hk, q, k, g, beta, gd->eps, gd->r_scale, r, x, kw, a, b, status};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return check_outputs(d, wkv7::launch_gdn_map(p, d->dtype, d->N, s),
+                       {{r, te, d->dtype}, {kw, te, d->dtype}, {a, te, d->dtype}, {b, te, d->dtype}}, status, s);
 }
 
 wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, const void* k, const void* v,
@@ -379,9 +409,10 @@ wkv7_status_t wkv7_step(const wkv7_desc_t* d, const void* r, const void* w, cons
   if (units == 0) return WKV7_OK;
   int* status = nullptr;
   if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
-  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y, status, (d->flags & WKV7_FLAG_LOG_DECAY) != 0u};
+  wkv7::StepArgs p{d->B, d->H, r, w, k, v, a, b, state, active, y, status, (d->flags & WKV7_FLAG_LOG_DECAY) != 0u,
+                   d->N};
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return check_outputs(d, wkv7::launch_step(p, d->dtype, s), {{y, units * 64, d->dtype}, {state, units * 64 * 64, WKV7_F32}},
+  return check_outputs(d, wkv7::launch_step(p, d->dtype, s), {{y, units * d->N, d->dtype}, {state, units * d->N * d->N, WKV7_F32}},
                        status, s);
 }
 

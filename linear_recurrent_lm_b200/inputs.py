@@ -100,6 +100,33 @@ def draw_inputs(rng: np.random.Generator, shape, dtype: str, log_decay: bool = F
     return out
 
 
+GDN_NAMES = ("q", "k", "v")
+
+
+def draw_gdn_inputs(rng: np.random.Generator, B: int, T: int, H: int, Hk: int, N: int, dtype: str) -> Dict[str, np.ndarray]:
+    """Gated-DeltaNet layer inputs (the rwkv-lab page's GDN target: 32 value heads and 16 key heads
+    of 128 channels).  Draw order: q, k [B,T,Hk,N], v [B,T,H,N], z_g, z_beta [B,T,H] standard
+    normal, then per value head A ~ U(1, 16) and dt ~ log-uniform on [1e-3, 1e-1].  Returns q, k, v
+    in storage dtype and fp32 g = -A softplus(z_g + softplus^-1(dt)) (a log-decay <= 0 whose
+    typical size is A dt) and beta = sigmoid(z_beta) (the write strength, in (0, 1)).  The pages
+    give no distributions for these inputs; this is the common GDN parametrisation of the decay
+    and the write gate."""
+    q = rng.standard_normal((B, T, Hk, N))
+    k = rng.standard_normal((B, T, Hk, N))
+    v = rng.standard_normal((B, T, H, N))
+    z_g = rng.standard_normal((B, T, H))
+    z_beta = rng.standard_normal((B, T, H))
+    A = rng.uniform(1.0, 16.0, H)
+    dt = np.exp(rng.uniform(np.log(1e-3), np.log(1e-1), H))
+    dt_bias = dt + np.log(-np.expm1(-dt))              # softplus(dt_bias) = dt
+    g = -A * _softplus(z_g + dt_bias)
+    beta = _sigmoid(z_beta)
+    out = {n: to_storage(x, dtype) for n, x in zip(GDN_NAMES, (q, k, v))}
+    out["g"] = g.astype(np.float32)
+    out["beta"] = beta.astype(np.float32)
+    return out
+
+
 def geometric_resets(rng: np.random.Generator, B: int, T: int, mean_len: float) -> np.ndarray:
     """Per-token reset flags [B,T] u8 for packed documents.
 

@@ -8,14 +8,16 @@ stream.  The same entry points as the C ABI:
 * ``backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, ...)``
   -> dict(dr, dw, dk, dv, da, db, ds0)
 * ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
+* ``gdn_map(q, k, g, beta, H, ...)`` -> dict(r, x, kw, a, b)   (gated-DeltaNet inputs -> WKV-7 inputs)
 * ``workspace_bytes(B, T, H, dtype)``
 * ``device_status(clear=True)`` -> OK, ERR_TIMEOUT, ERR_BOUNDS or ERR_NONFINITE (synchronises the device)
 * ``use_build("release" | "debug")``: route every call through ``libwkv7.so`` (default) or its
   bounds-checked twin ``libwkv7_debug.so`` (same ABI; ``WKV7_BUILD=debug`` in the environment
   selects it at import)
 
-Tensors are [B,T,H,64] (token inputs), [B,H,64,64] fp32 (states), [B,T] uint8
-(reset), [B] uint8 (active), all on one CUDA device and contiguous.  If the
+Tensors are [B,T,H,N] (token inputs), [B,H,N,N] fp32 (states), [B,T] uint8
+(reset), [B] uint8 (active), all on one CUDA device and contiguous.  The head size N is 64; the
+token-order forward and the decode step also take N = 128 (the gated-delta-rule map's heads).  If the
 library is missing, importing this module raises: there is no fallback.
 """
 from __future__ import annotations
@@ -40,6 +42,7 @@ FLAG_EPILOGUE_GRADS = 0x4                  # WKV7_FLAG_EPILOGUE_GRADS: dy is the
 DTYPE_CODE = {torch.float32: 0, torch.bfloat16: 1, torch.float16: 2}
 ALGO_CODE = {"auto": 0, "scan": 1, "chunked": 2, "chunked_fused": 3, "chunked_split": 4}
 N_HEAD = 64
+HEAD_SIZES = (64, 128)
 CHUNK = 16
 
 
@@ -52,6 +55,11 @@ class Epilogue(ctypes.Structure):
     """wkv7_epilogue_t: fp32 [H,64] GroupNorm weight and bias, bonus weights, and eps."""
     _fields_ = [("ln_w", ctypes.c_void_p), ("ln_b", ctypes.c_void_p), ("r_k", ctypes.c_void_p),
                 ("eps", ctypes.c_float)]
+
+
+class Gdn(ctypes.Structure):
+    """wkv7_gdn_t: key heads, the L2-normalisation guard and the scale taken into r."""
+    _fields_ = [("Hk", ctypes.c_int64), ("eps", ctypes.c_float), ("r_scale", ctypes.c_float)]
 
 
 class WKV7Error(RuntimeError):
@@ -98,6 +106,8 @@ def _load(variant: str) -> ctypes.CDLL:
     L.wkv7_forward_epilogue.argtypes = [dp, ep] + [vp] * 14
     L.wkv7_epilogue_backward.restype = ctypes.c_int
     L.wkv7_epilogue_backward.argtypes = [dp, ep] + [vp] * 12
+    L.wkv7_gdn_map.restype = ctypes.c_int
+    L.wkv7_gdn_map.argtypes = [dp, ctypes.POINTER(Gdn)] + [vp] * 10
     return L
 
 
@@ -138,8 +148,8 @@ def make_desc(B: int, T: int, H: int, dtype, algo: str = "auto", N: int = N_HEAD
     return Desc(int(B), int(T), int(H), int(N), code, ALGO_CODE[algo] if isinstance(algo, str) else int(algo), int(flags))
 
 
-def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16) -> int:
-    return int(lib().wkv7_workspace_bytes(ctypes.byref(make_desc(B, T, H, dtype))))
+def workspace_bytes(B: int, T: int, H: int, dtype=torch.bfloat16, N: int = N_HEAD) -> int:
+    return int(lib().wkv7_workspace_bytes(ctypes.byref(make_desc(B, T, H, dtype, N=N))))
 
 
 def device_status(clear: bool = True) -> int:
@@ -169,9 +179,9 @@ def _check(status: int, where: str):
         raise WKV7Error(status, where)
 
 
-def _token_shape(x: torch.Tensor):
-    if x.dim() != 4 or x.shape[-1] != N_HEAD:
-        raise ValueError(f"expected [B,T,H,{N_HEAD}], got {tuple(x.shape)}")
+def _token_shape(x: torch.Tensor, sizes=(N_HEAD,)):
+    if x.dim() != 4 or x.shape[-1] not in sizes:
+        raise ValueError(f"expected [B,T,H,N] with N in {sizes}, got {tuple(x.shape)}")
     return tuple(int(s) for s in x.shape[:3])
 
 
@@ -182,17 +192,18 @@ def _flags(flags: int, log_decay: bool) -> int:
 def forward(r, w, k, v, a, b, s0=None, reset=None, *, y=None, s_out=None, workspace=None,
             need_workspace: bool = True, want_state: bool = True, algo: str = "auto", stream=None, flags: int = 0,
             log_decay: bool = False):
-    """WKV-7 forward over [B,T,H,64] inputs.  Returns (y, s_out, workspace).  With ``log_decay`` the
-    ``w`` tensor holds x and the decay is exp(-exp(x))."""
-    B, T, H = _token_shape(r)
+    """WKV-7 forward over [B,T,H,N] inputs (N = 64, or 128 with the token-order scan).  Returns (y,
+    s_out, workspace).  With ``log_decay`` the ``w`` tensor holds x and the decay is exp(-exp(x))."""
+    B, T, H = _token_shape(r, HEAD_SIZES)
+    N = int(r.shape[-1])
     dev = r.device
     if y is None:
         y = torch.empty_like(r)
     if s_out is None and want_state:
-        s_out = torch.empty((B, H, N_HEAD, N_HEAD), device=dev, dtype=torch.float32)
+        s_out = torch.empty((B, H, N, N), device=dev, dtype=torch.float32)
     if workspace is None and need_workspace:
-        workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype), 16), device=dev, dtype=torch.uint8)
-    d = make_desc(B, T, H, r.dtype, algo, flags=_flags(flags, log_decay))
+        workspace = torch.empty(max(workspace_bytes(B, T, H, r.dtype, N), 16), device=dev, dtype=torch.uint8)
+    d = make_desc(B, T, H, r.dtype, algo, N=N, flags=_flags(flags, log_decay))
     st = lib().wkv7_forward(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, s0, reset, y, s_out, workspace)),
                             _stream(stream))
     _check(st, "wkv7_forward")
@@ -226,13 +237,13 @@ def backward(r, w, k, v, a, b, dy, workspace, s0=None, reset=None, dsT=None, *, 
 
 
 def step(r, w, k, v, a, b, state, active=None, *, y=None, stream=None, flags: int = 0, log_decay: bool = False):
-    """One decode token on ``state`` [B,H,64,64] (in place).  Inputs [B,H,64].  Returns y."""
-    if r.dim() != 3 or r.shape[-1] != N_HEAD:
-        raise ValueError(f"expected [B,H,{N_HEAD}], got {tuple(r.shape)}")
+    """One decode token on ``state`` [B,H,N,N] (in place).  Inputs [B,H,N], N = 64 or 128.  Returns y."""
+    if r.dim() != 3 or r.shape[-1] not in HEAD_SIZES:
+        raise ValueError(f"expected [B,H,N] with N in {HEAD_SIZES}, got {tuple(r.shape)}")
     B, H = int(r.shape[0]), int(r.shape[1])
     if y is None:
         y = torch.empty_like(r)
-    d = make_desc(B, 1, H, r.dtype, flags=_flags(flags, log_decay))
+    d = make_desc(B, 1, H, r.dtype, N=int(r.shape[-1]), flags=_flags(flags, log_decay))
     st = lib().wkv7_step(ctypes.byref(d), *(_ptr(x) for x in (r, w, k, v, a, b, state, active, y)), _stream(stream))
     _check(st, "wkv7_step")
     return y
@@ -330,3 +341,27 @@ def forward_epilogue(r, w, k, v, a, b, g, ln_w, ln_b, r_k, eps: float, s0=None, 
                                      _stream(stream))
     _check(st, "wkv7_forward_epilogue")
     return out, y, s_out, workspace
+
+
+def gdn_map(q, k, g, beta, H: int, eps: float = 1e-6, r_scale: Optional[float] = None, *, out=None, stream=None,
+            flags: int = 0) -> Dict[str, torch.Tensor]:
+    """The gated-DeltaNet front end (wkv7_gdn_map): q, k [B,T,Hk,N] and fp32 g, beta [B,T,H] ->
+    dict of r, x, kw, a, b [B,T,H,N] for ``forward`` / ``step`` with ``log_decay=True`` and GDN's
+    own v.  ``r_scale`` defaults to 1/sqrt(N)."""
+    B, T, Hk = _token_shape(q, HEAD_SIZES)
+    N = int(q.shape[-1])
+    if tuple(k.shape) != tuple(q.shape) or k.dtype != q.dtype:
+        raise ValueError(f"q and k must match, got {tuple(q.shape)} {q.dtype} and {tuple(k.shape)} {k.dtype}")
+    for n, t in (("g", g), ("beta", beta)):
+        if t.dtype != torch.float32 or tuple(t.shape) != (B, T, H):
+            raise ValueError(f"{n} must be fp32 [B,T,H] = {(B, T, H)}, got {tuple(t.shape)} {t.dtype}")
+    o = dict(out) if out is not None else {}
+    for n in ("r", "x", "kw", "a", "b"):
+        if o.get(n) is None:
+            o[n] = torch.empty((B, T, H, N), device=q.device, dtype=q.dtype)
+    d = make_desc(B, T, H, q.dtype, N=N, flags=flags)
+    gd = Gdn(int(Hk), float(eps), float(N ** -0.5 if r_scale is None else r_scale))
+    st = lib().wkv7_gdn_map(ctypes.byref(d), ctypes.byref(gd), *(_ptr(x) for x in (q, k, g, beta)),
+                            *(_ptr(o[n]) for n in ("r", "x", "kw", "a", "b")), _stream(stream))
+    _check(st, "wkv7_gdn_map")
+    return o

@@ -222,3 +222,51 @@ def test_epilogue_grads_flag_is_accepted_by_validation(L):
     import torch
     d = L.make_desc(1, 16, 1, torch.bfloat16, flags=L.FLAG_EPILOGUE_GRADS)
     assert call_fwd(L, d) != L.ERR_UNSUPPORTED
+
+
+def test_head_size_128_limits(L):
+    """N = 128 (the gated-DeltaNet heads) runs the token-order forward and the decode step only:
+    every chunked form, the backward, the no-alloc step and the epilogue refuse it before any
+    launch; the workspace counts 128x128 checkpoints."""
+    import torch
+    lib = L.lib()
+    P = ctypes.c_void_p(FAKE)
+    for algo in ("chunked", "chunked_fused", "chunked_split"):
+        d = L.make_desc(1, 16, 1, torch.bfloat16, algo, N=128)
+        assert call_fwd(L, d, ws=FAKE) == L.ERR_UNSUPPORTED
+    d = L.make_desc(1, 16, 1, torch.bfloat16, N=128)
+    assert lib.wkv7_backward(ctypes.byref(d), *([P] * 6), None, None, P, None, P, *([P] * 6), None, None) \
+        == L.ERR_UNSUPPORTED
+    assert lib.wkv7_train_step_noalloc(ctypes.byref(d), *([P] * 6), None, None, P, None, P, None,
+                                       *([P] * 6), None, None) == L.ERR_UNSUPPORTED
+    ep = L.Epilogue(FAKE, FAKE, FAKE, 6.4e-4)
+    assert lib.wkv7_epilogue_forward(ctypes.byref(d), ctypes.byref(ep), *([P] * 6), None) == L.ERR_UNSUPPORTED
+    assert L.workspace_bytes(1, 17, 1, torch.bfloat16, N=128) == 2 * 128 * 128 * 4 + 16
+    bad = L.make_desc(1, 16, 1, torch.bfloat16, N=96)
+    assert call_fwd(L, bad) == L.ERR_UNSUPPORTED
+
+
+def test_gdn_map_validation_codes(L):
+    """wkv7_gdn_map refuses bad arguments before any launch."""
+    import torch
+    lib = L.lib()
+    vp = ctypes.c_void_p
+    P = vp(FAKE)
+    d = L.make_desc(1, 16, 4, torch.bfloat16, N=128)
+    call = lambda desc, gd, *p: lib.wkv7_gdn_map(desc, gd, *p, None)   # noqa: E731
+    gd = L.Gdn(2, 1e-6, 128 ** -0.5)
+    assert call(None, ctypes.byref(gd), *([P] * 9)) == L.ERR_NULL
+    assert call(ctypes.byref(d), None, *([P] * 9)) == L.ERR_NULL
+    for bad in (L.Gdn(3, 1e-6, 1.0), L.Gdn(0, 1e-6, 1.0), L.Gdn(2, -1.0, 1.0), L.Gdn(2, float("nan"), 1.0),
+                L.Gdn(2, 1e-6, float("inf")), L.Gdn(2, 1e-6, float("nan"))):
+        assert call(ctypes.byref(d), ctypes.byref(bad), *([P] * 9)) == L.ERR_UNSUPPORTED
+    assert call(ctypes.byref(d), ctypes.byref(gd), None, *([P] * 8)) == L.ERR_NULL
+    assert call(ctypes.byref(d), ctypes.byref(gd), P, P, None, *([P] * 6)) == L.ERR_NULL     # g
+    assert call(ctypes.byref(d), ctypes.byref(gd), P, P, vp(FAKE + 2), *([P] * 6)) == L.ERR_ALIGN
+    assert call(ctypes.byref(d), ctypes.byref(gd), *([P] * 4), vp(FAKE + 8), *([P] * 4)) == L.ERR_ALIGN
+    dl = L.make_desc(1, 16, 4, torch.bfloat16, N=128, flags=L.FLAG_LOG_DECAY)
+    assert call(ctypes.byref(dl), ctypes.byref(gd), *([P] * 9)) == L.ERR_UNSUPPORTED
+    d96 = L.make_desc(1, 16, 4, torch.bfloat16, N=96)
+    assert call(ctypes.byref(d96), ctypes.byref(gd), *([P] * 9)) == L.ERR_UNSUPPORTED
+    d0 = L.make_desc(1, 0, 4, torch.bfloat16, N=128)                # nothing to do, no launch
+    assert call(ctypes.byref(d0), ctypes.byref(gd), *([None] * 9)) == L.OK
