@@ -711,6 +711,46 @@ def measure_secondary(wkv7, dev, algo):
         "l2": "inputs larger than L2 (no flush)"}
     del gq, gk, gv, gg, gb, mo, yg, sg
 
+    # Context parallelism (the packed batch's rows split into R segments of T/R tokens, one per GPU),
+    # emulated on this one GPU: the compute of one middle rank -- the transition P and zero-state end U
+    # of its segment (two forwards), its entering state composed from R-2 gathered pairs (the most any
+    # rank composes), its real forward; its backward with dsT = 0, the leaving gradient composed
+    # through R-2 transitions, its real backward.  The all-gathers (2 x B*H*64*64*4 bytes per rank in
+    # the forward, half that in the backward) are not timed here.
+    from linear_recurrent_lm_b200 import context_parallel as cp
+    wl = I.make_workload(3)
+    cpo = {}
+    for R in (2, 4, 8):
+        bnd = cp.split_tokens(wl.T, R)
+        t0, t1 = bnd[1], bnd[2]
+        seg = cp.Segment([d(np.ascontiguousarray(wl.inputs[n][:, t0:t1])) for n in I.NAMES],
+                         d(np.ascontiguousarray(wl.reset[:, t0:t1])))
+        dys = d(np.ascontiguousarray(wl.dy[:, t0:t1]))
+        gen = torch.Generator(device=dev).manual_seed(R)
+        pairs = [torch.randn((wl.B, wl.H, 64, 64), device=dev, generator=gen) for _ in range(2 * R)]
+        Ps, Us = pairs[:R], pairs[R:]
+        ms = []
+        for rep in range(5):
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            cp.forward_local(seg, 1, None)
+            s_in = cp.entering_state(R - 1, Ps, Us)
+            _, _, ws = cp.forward_final(seg, 1, s_in)
+            ctx = cp.Context(0, R, seg, s_in, ws, [None] + Ps[1:], "auto", False)
+            cp.backward_local(ctx, dys, None)
+            cp.backward_final(ctx, dys, cp.leaving_gradient(ctx, Us))
+            e1.record()
+            torch.cuda.synchronize()
+            if rep >= 2:
+                ms.append(e0.elapsed_time(e1))
+        m = statistics.median(ms)
+        cpo[f"R{R}"] = {"segment_tokens": t1 - t0, "rank_ms": m,
+                        "job_tokens_per_s_without_exchange": wl.B * wl.T / (m / 1e3),
+                        "exchange_bytes_per_rank": 3 * wl.B * wl.H * 64 * 64 * 4}
+        del seg, dys, pairs, Ps, Us, ws, ctx
+    out["context_parallel_B8_T4096_H32_emulated"] = {
+        **cpo, "note": "one GPU runs one middle rank's compute; all-gathers not timed (one GPU per run)"}
+
     wl = I.make_workload(4)
     state = d(wl.state0)
     steps = [[d(s[n]) for n in I.NAMES] for s in wl.steps]

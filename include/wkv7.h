@@ -407,6 +407,32 @@ wkv7_status_t wkv7_gdn_map(const wkv7_desc_t* desc, const wkv7_gdn_t* gd, const 
                            const float* g, const float* beta, void* r, void* x, void* kw, void* a, void* b,
                            void* stream);
 
+/*
+ * ------------------------------------------------------------------ state composition
+ * For splitting a sequence's tokens across devices (context parallelism;
+ * the pages have no passage on it).  Over a segment of tokens the
+ * recurrence is affine in the state entering it:
+ *
+ *   S_end = S_in P + U,   P = prod_t (diag(w_t) + a_t b_t^T)   (the forward
+ *   from s0 = I with v = 0),   U = the forward's end state from s0 = 0,
+ *
+ * and the state gradient goes back through the same P:
+ * dS_in = dS_end P^T + (the backward's ds0 from dsT = 0).  This call is the
+ * composition step: per (b, h) unit,
+ *
+ *   out = S P + U        (transpose_p == 0)
+ *   out = S P^T + U      (transpose_p != 0)
+ *
+ * in fp32 (plain k order).  desc: B, H, N (64 or 128) give the unit count
+ * and size; T, dtype and algo are validated as usual but not used; flags 0
+ * or WKV7_FLAG_CHECK_FINITE.  S, P, U, out: fp32 [B,H,N,N], 16-byte
+ * aligned; S NULL means zero (then P may be NULL; out = U); U NULL means
+ * zero.  out may be U itself but must not overlap S or P (out == S or
+ * out == P -> WKV7_ERR_UNSUPPORTED).  Errors as for wkv7_forward.
+ */
+wkv7_status_t wkv7_state_compose(const wkv7_desc_t* desc, const float* S, const float* P, const float* U,
+                                 float* out, int transpose_p, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

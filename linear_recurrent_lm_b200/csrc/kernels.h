@@ -114,6 +114,16 @@ struct GdnArgs {
   int* status;
 };
 
+// State composition: out = S P + U (P transposed when transpose_p) per unit of N x N fp32; S or U
+// null means zero (P may then be null too).
+struct ComposeArgs {
+  int64_t units;
+  const float *S, *P, *U;
+  float* out;
+  bool transpose_p;
+  int* status;
+};
+
 // Descriptor checks shared by every entry point (WKV7_OK, or the status the entry points return).
 wkv7_status_t validate_desc(const wkv7_desc_t* d);
 
@@ -124,6 +134,7 @@ cudaError_t launch_scan_bwd(const BwdArgs& p, int dtype, bool only_flagged, cuda
 cudaError_t launch_step(const StepArgs& p, int dtype, cudaStream_t stream);
 cudaError_t launch_epilogue(const EpiArgs& p, int dtype, bool backward, cudaStream_t stream);
 cudaError_t launch_gdn_map(const GdnArgs& p, int dtype, int N, cudaStream_t stream);
+cudaError_t launch_compose(const ComposeArgs& p, int N, cudaStream_t stream);
 // Set kStatusNonFinite in *status if any of the n elements at x (dtype as above; 16-byte aligned)
 // is NaN or infinite.  x == nullptr or n == 0: nothing is launched.
 cudaError_t launch_finite_scan(const void* x, int64_t n, int dtype, int* status, cudaStream_t stream);

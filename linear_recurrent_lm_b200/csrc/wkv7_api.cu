@@ -373,6 +373,26 @@ wkv7_status_t wkv7_forward_epilogue(const wkv7_desc_t* d, const wkv7_epilogue_t*
                        {{out, te, d->dtype}, {y, te, d->dtype}, {s_out, units * 64 * 64, WKV7_F32}}, status, s);
 }
 
+wkv7_status_t wkv7_state_compose(const wkv7_desc_t* d, const float* S, const float* P, const float* U, float* out,
+                                 int transpose_p, void* stream) {
+  int64_t units = 0, te = 0;
+  wkv7_status_t st = check_desc(d, &units, &te);
+  if (st != WKV7_OK) return st;
+  if ((d->flags & ~WKV7_FLAG_CHECK_FINITE) != 0u) return WKV7_ERR_UNSUPPORTED;
+  st = check_ptrs(units > 0, {out});
+  if (st != WKV7_OK) return st;
+  if (units > 0 && S && !P) return WKV7_ERR_NULL;
+  st = check_ptrs(false, {S, P, U});
+  if (st != WKV7_OK) return st;
+  if (out && (static_cast<const void*>(out) == S || static_cast<const void*>(out) == P)) return WKV7_ERR_UNSUPPORTED;
+  if (units == 0) return WKV7_OK;
+  int* status = nullptr;
+  if (wkv7::device_status_ptr(&status) != cudaSuccess) return WKV7_ERR_CUDA;
+  wkv7::ComposeArgs p{units, S, P, U, out, transpose_p != 0, status};
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return check_outputs(d, wkv7::launch_compose(p, d->N, s), {{out, units * d->N * d->N, WKV7_F32}}, status, s);
+}
+
 wkv7_status_t wkv7_gdn_map(const wkv7_desc_t* d, const wkv7_gdn_t* gd, const void* q, const void* k,
                            const float* g, const float* beta, void* r, void* x, void* kw, void* a, void* b,
                            void* stream) {

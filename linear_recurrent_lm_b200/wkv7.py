@@ -9,6 +9,7 @@ stream.  The same entry points as the C ABI:
   -> dict(dr, dw, dk, dv, da, db, ds0)
 * ``step(r, w, k, v, a, b, state, active=None, ...)`` -> y   (state updated in place)
 * ``gdn_map(q, k, g, beta, H, ...)`` -> dict(r, x, kw, a, b)   (gated-DeltaNet inputs -> WKV-7 inputs)
+* ``state_compose(S, P, U, ...)`` -> S P + U (or S P^T + U) per (b, h)   (context parallelism)
 * ``workspace_bytes(B, T, H, dtype)``
 * ``device_status(clear=True)`` -> OK, ERR_TIMEOUT, ERR_BOUNDS or ERR_NONFINITE (synchronises the device)
 * ``use_build("release" | "debug")``: route every call through ``libwkv7.so`` (default) or its
@@ -106,6 +107,8 @@ def _load(variant: str) -> ctypes.CDLL:
     L.wkv7_forward_epilogue.argtypes = [dp, ep] + [vp] * 14
     L.wkv7_epilogue_backward.restype = ctypes.c_int
     L.wkv7_epilogue_backward.argtypes = [dp, ep] + [vp] * 12
+    L.wkv7_state_compose.restype = ctypes.c_int
+    L.wkv7_state_compose.argtypes = [dp, vp, vp, vp, vp, ctypes.c_int, vp]
     L.wkv7_gdn_map.restype = ctypes.c_int
     L.wkv7_gdn_map.argtypes = [dp, ctypes.POINTER(Gdn)] + [vp] * 10
     return L
@@ -365,3 +368,22 @@ def gdn_map(q, k, g, beta, H: int, eps: float = 1e-6, r_scale: Optional[float] =
                             *(_ptr(o[n]) for n in ("r", "x", "kw", "a", "b")), _stream(stream))
     _check(st, "wkv7_gdn_map")
     return o
+
+
+def state_compose(S, P, U, *, out=None, transpose: bool = False, stream=None, flags: int = 0) -> torch.Tensor:
+    """wkv7_state_compose: out = S P + U (S P^T + U with ``transpose``) per (b, h) unit, all fp32
+    [B,H,N,N]; S or U may be None (zero).  ``out`` may be U itself."""
+    ref = next(t for t in (S, P, U, out) if t is not None)
+    if ref.dim() != 4 or ref.shape[-1] != ref.shape[-2] or ref.shape[-1] not in HEAD_SIZES:
+        raise ValueError(f"expected fp32 states [B,H,N,N] with N in {HEAD_SIZES}, got {tuple(ref.shape)}")
+    for t in (S, P, U, out):
+        if t is not None and (t.dtype != torch.float32 or tuple(t.shape) != tuple(ref.shape)):
+            raise ValueError(f"states must all be fp32 {tuple(ref.shape)}, got {tuple(t.shape)} {t.dtype}")
+    B, H, N = int(ref.shape[0]), int(ref.shape[1]), int(ref.shape[-1])
+    if out is None:
+        out = torch.empty_like(ref)
+    d = make_desc(B, 1, H, torch.float32, N=N, flags=flags)
+    st = lib().wkv7_state_compose(ctypes.byref(d), _ptr(S), _ptr(P), _ptr(U), _ptr(out), 1 if transpose else 0,
+                                  _stream(stream))
+    _check(st, "wkv7_state_compose")
+    return out

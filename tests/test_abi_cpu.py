@@ -270,3 +270,24 @@ def test_gdn_map_validation_codes(L):
     assert call(ctypes.byref(d96), ctypes.byref(gd), *([P] * 9)) == L.ERR_UNSUPPORTED
     d0 = L.make_desc(1, 0, 4, torch.bfloat16, N=128)                # nothing to do, no launch
     assert call(ctypes.byref(d0), ctypes.byref(gd), *([None] * 9)) == L.OK
+
+
+def test_state_compose_validation_codes(L):
+    import torch
+    lib = L.lib()
+    vp = ctypes.c_void_p
+    P = vp(FAKE)
+    d = L.make_desc(2, 1, 3, torch.float32)
+    call = lambda desc, S, Pm, U, out, tr=0: lib.wkv7_state_compose(desc, S, Pm, U, out, tr, None)   # noqa: E731
+    assert call(None, P, P, P, vp(FAKE + 4096)) == L.ERR_NULL
+    assert call(ctypes.byref(d), P, P, P, None) == L.ERR_NULL                     # out
+    assert call(ctypes.byref(d), P, None, P, vp(FAKE + 4096)) == L.ERR_NULL       # S without P
+    assert call(ctypes.byref(d), vp(FAKE + 8), P, P, vp(FAKE + 4096)) == L.ERR_ALIGN
+    assert call(ctypes.byref(d), P, vp(FAKE + 4096), P, vp(FAKE + 4096)) == L.ERR_UNSUPPORTED   # out == P
+    assert call(ctypes.byref(d), vp(FAKE + 4096), P, P, vp(FAKE + 4096)) == L.ERR_UNSUPPORTED   # out == S
+    bad = L.make_desc(2, 1, 3, torch.float32, N=96)
+    assert call(ctypes.byref(bad), P, P, P, vp(FAKE + 4096)) == L.ERR_UNSUPPORTED
+    bad = L.make_desc(2, 1, 3, torch.float32, flags=L.FLAG_LOG_DECAY)
+    assert call(ctypes.byref(bad), P, P, P, vp(FAKE + 4096)) == L.ERR_UNSUPPORTED
+    d0 = L.make_desc(0, 1, 3, torch.float32)
+    assert call(ctypes.byref(d0), None, None, None, None) == L.OK               # no units, no launch
