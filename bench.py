@@ -330,7 +330,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-secondary", action="store_true")
-    ap.add_argument("--only", choices=["fwd", "bwd", "prefill", "step"],
+    ap.add_argument("--only", choices=["fwd", "bwd", "prefill", "step", "gdn_map"],
                     help="time one kernel alone (profiling entry point); prints its own JSON line")
     ap.add_argument("--B", type=int, default=None, help="batch override for --only")
     ap.add_argument("--step", type=int, default=0, help="--only step: which of the 128 ragged decode steps")
@@ -791,12 +791,44 @@ def measure_secondary(wkv7, dev, algo):
     return out
 
 
+def run_only_gdn_map(args):
+    """Warm-up + timed launches of the GDN map on the GDN layer shape (B=8 or --B, T=4096, 32 value
+    heads over 16 key heads of 128, bf16)."""
+    import torch
+    from linear_recurrent_lm_b200 import wkv7
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    B = args.B or 8
+    T, H, Hk, N = 4096, 32, 16, 128
+    gd = I.draw_gdn_inputs(np.random.default_rng(77), B, T, H, Hk, N, "bf16")
+    q, k = (torch.from_numpy(gd[n].view(np.int16)).view(torch.bfloat16).to(dev) for n in ("q", "k"))
+    g, beta = (torch.from_numpy(gd[n]).to(dev) for n in ("g", "beta"))
+    out = {n: torch.empty((B, T, H, N), device=dev, dtype=torch.bfloat16) for n in ("r", "x", "kw", "a", "b")}
+    fn = lambda: wkv7.gdn_map(q, k, g, beta, H, eps=1e-6, out=out)   # noqa: E731
+    for _ in range(args.warmup):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(args.steps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1) / max(args.steps, 1)
+    peak, _ = measured_peaks()
+    gbs = BYTES_GDN_MAP * B * T * H / (ms / 1e3) / 1e9
+    print(json.dumps({"only": "gdn_map", "workload": f"gdn_layer_B{B}_T{T}_H{H}_Hk{Hk}_N{N}", "ms": ms,
+                      "achieved_gbs": gbs, "frac": gbs / peak}))
+
+
 def run_only(args):
     """Warm-up + timed launches of a single kernel on the default workload (or a smaller batch)."""
     import torch
     from linear_recurrent_lm_b200 import wkv7
     dev = torch.device("cuda", 0)
     torch.cuda.set_device(dev)
+    if args.only == "gdn_map":
+        return run_only_gdn_map(args)
     idx = {"fwd": 3, "bwd": 3, "prefill": 2, "step": 4}[args.only]
     wl = I.make_workload(idx, B=args.B)
 
