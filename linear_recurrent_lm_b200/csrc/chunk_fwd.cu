@@ -93,6 +93,7 @@ struct __align__(128) FwdSmem3 {
   unsigned long long d1_bar, mma_bar;        // completion of a chunk's D1 MMAs / of all its MMAs (one phase per chunk)
   uint32_t tmem_base;                        // TMEM: S0 (cols 0-63), D1 (64-95), D3 (128-191)
   int kbad[4];
+  float qsum[4][kN];                         // log-space decay: sum of -exp(x) over each token quarter
 };
 
 __device__ __forceinline__ void named_bar(int id, int n) {
@@ -178,15 +179,44 @@ __device__ __forceinline__ void build_context(const FwdArgs& p, const InputMaps&
       const float2 x = ld2(1, t);
       return make_float2(decay_of(x.x, kLog), decay_of(x.y, kLog));
     };
+    // log-space decay: log L_t = sum_{s<=t} -exp(x_s).  Each warp sums its own quarter's terms and
+    // takes the earlier quarters' sums from the other warps (one exponential per input, not a chain
+    // of two per token over every earlier token)
+    auto ldl = [&](int t) {   // -exp(x_t); padding: 0 (w = 1)
+      if (t >= len) return make_float2(0.f, 0.f);
+      const float2 x = ld2(1, t);
+      return make_float2(-__expf(x.x), -__expf(x.y));
+    };
     float2 lam = make_float2(1.f, 1.f);   // L_{tq-1}: product over the earlier quarters (warp-uniform count)
-    for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
+    float2 lsum = make_float2(0.f, 0.f);  // log L_{tq-1} (log-space decay)
+    float2 dl[4];
+    if (kLog) {
+      float2 qs = make_float2(0.f, 0.f);
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        dl[u] = ldl(tq + u);
+        qs = add2(qs, dl[u]);
+      }
+      sm.qsum[kw][ja] = qs.x;
+      sm.qsum[kw][jb] = qs.y;
+      named_bar(1, 128);   // (the next writes come after the barrier below, once every warp has read)
+      for (int w2 = 0; w2 < kw; ++w2) lsum = add2(lsum, make_float2(sm.qsum[w2][ja], sm.qsum[w2][jb]));
+      lam = make_float2(__expf(lsum.x), __expf(lsum.y));
+    } else {
+      for (int t = 0; t < tq; ++t) lam = mul2(lam, ldw(t));
+    }
     float at[2][4], bh[2][4], kh[2][4], vv[2][4];
     const unsigned ls_bits = last_segment_bits(mask);   // S_16 sees only the chunk's last segment
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int t = tq + u;
       const float2 lp = lam;
-      lam = mul2(lam, ldw(t));
+      if (kLog) {
+        lsum = add2(lsum, dl[u]);
+        lam = make_float2(__expf(lsum.x), __expf(lsum.y));
+      } else {
+        lam = mul2(lam, ldw(t));
+      }
       bad |= !(lam.x >= 0x1p-40f && lam.x <= 0x1p40f) || !(lam.y >= 0x1p-40f && lam.y <= 0x1p40f);
       const float2 inv = make_float2(rcp_approx(lam.x), rcp_approx(lam.y));
       const float2 a2 = mul2(ld2(4, t), lp), r2 = mul2(ld2(0, t), lam);
