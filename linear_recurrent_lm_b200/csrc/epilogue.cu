@@ -90,8 +90,10 @@ __global__ void __launch_bounds__(kThreads) epilogue_fwd_kernel(const EpiArgs p)
   }
 }
 
+// Two CTAs per SM (128 registers, no spills): at its natural 153 registers one CTA of 8 warps per SM
+// could not keep enough loads in flight.
 template <typename T>
-__global__ void __launch_bounds__(kThreads) epilogue_bwd_kernel(const EpiArgs p) {
+__global__ void __launch_bounds__(kThreads, 2) epilogue_bwd_kernel(const EpiArgs p) {
   constexpr int P = Lanes<T>::kPer, E = Lanes<T>::kElts, RW = Lanes<T>::kRows;
   __shared__ float red[3][RW][kN];           // per-group partial parameter gradients
   const int h = blockIdx.y;
