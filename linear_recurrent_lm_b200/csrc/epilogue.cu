@@ -194,11 +194,16 @@ __global__ void __launch_bounds__(kThreads, 2) epilogue_bwd_kernel(const EpiArgs
 template <typename T>
 cudaError_t launch(const EpiArgs& p, bool backward, cudaStream_t stream) {
   const int64_t rows = p.B * p.T;
-  int sms = 148;
-  int dev = 0;
+  int sms = 148, dev = 0, per_sm = 1;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  // about four CTAs per SM over all heads, at most one pass of rows per CTA group
-  const int64_t per_head = (int64_t(sms) * 4 + p.H - 1) / p.H;
+  if (backward)
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, epilogue_bwd_kernel<T>, kThreads, 0);
+  else
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, epilogue_fwd_kernel<T>, kThreads, 0);
+  // one wave: the resident CTAs of every SM shared out over the heads (at least one per head), at
+  // most one pass of rows per CTA group
+  const int64_t slots = int64_t(sms) * (per_sm > 0 ? per_sm : 1);
+  const int64_t per_head = slots / p.H > 0 ? slots / p.H : 1;
   const int64_t need = (rows + Lanes<T>::kRows - 1) / Lanes<T>::kRows;
   const unsigned gx = unsigned(need < per_head ? need : per_head);
   if (gx == 0 || p.H > 65535) return p.H > 65535 ? cudaErrorInvalidValue : cudaSuccess;

@@ -103,10 +103,11 @@ __global__ void __launch_bounds__(kThreads) gdn_map_kernel(const GdnArgs p) {
 template <typename T, int N>
 cudaError_t launch(const GdnArgs& p, cudaStream_t stream) {
   const int64_t rows = p.B * p.T * p.Hk;
-  int sms = 148, dev = 0;
+  int sms = 148, dev = 0, per_sm = 1;
   if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, gdn_map_kernel<T, N>, kThreads, 0);
   const int64_t need = (rows + MapLanes<T, N>::kRows - 1) / MapLanes<T, N>::kRows;
-  const int64_t cap = int64_t(sms) * 8;   // eight 256-thread CTAs per SM; a grid-stride loop past that
+  const int64_t cap = int64_t(sms) * (per_sm > 0 ? per_sm : 1);   // one wave; a grid-stride loop past that
   const unsigned grid = unsigned(need < cap ? need : cap);
   if (grid == 0) return cudaSuccess;
   gdn_map_kernel<T, N><<<grid, kThreads, 0, stream>>>(p);
