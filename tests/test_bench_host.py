@@ -43,3 +43,10 @@ def test_profile_headers_are_well_formed(name):
     assert re.search(r"code_sha256:\s*[0-9a-f]{64}", text)
     assert re.search(r"traffic_bytes_per_launch:\s*[0-9]+", text)
     assert "--clock-control none" in text            # every ncu command leaves the clocks alone
+
+
+def test_dominant_kernel_profile_matches_current_code():
+    """The roofline line's traffic comes from the committed capture of the backward kernel: that
+    capture must have been taken on the kernel's current code (else bench.py reports null)."""
+    t = bench.kernel_traffic("chunk_bwd", "packed_train_B8_T4096_H32")
+    assert t is not None and 2.0e9 < t < 3.0e9
