@@ -111,3 +111,28 @@ def test_split_tokens():
     assert cp.split_tokens(20, 3) == [0, 16, 20, 20]
     with pytest.raises(ValueError):
         cp.split_tokens(10, 0)
+
+
+def test_emulated_ranks_equal_one_run():
+    """The single-process driver (every rank's phases in turn, the gathers as lists) with the same
+    oracle steps: 4 segments, the last one ragged."""
+    import oracle
+    from linear_recurrent_lm_b200 import context_parallel as cp
+    T = 61
+    xs, s0, dy, dsT, reset = _problem(T)
+    bounds = cp.split_tokens(T, 4)
+    segs = [cp.Segment([torch.from_numpy(np.ascontiguousarray(x[:, t0:t1])) for x in xs],
+                       torch.from_numpy(np.ascontiguousarray(reset[:, t0:t1])))
+            for t0, t1 in zip(bounds[:-1], bounds[1:])]
+    ys, ends, ctxs = cp.emulate_forward(segs, torch.from_numpy(s0), ops=OracleOps)
+    gs = cp.emulate_backward(ctxs, [torch.from_numpy(np.ascontiguousarray(dy[:, t0:t1]))
+                                    for t0, t1 in zip(bounds[:-1], bounds[1:])],
+                             torch.from_numpy(dsT), ops=OracleOps)
+    y, s, _ = oracle.forward(*xs, s0=s0, reset=reset)
+    g, _ = oracle.backward(*xs, dy, s0=s0, reset=reset, dsT=dsT)
+    rel = lambda a, b: float(np.max(np.abs(a - b)) / np.sqrt(np.mean(b * b)))   # noqa: E731
+    assert rel(torch.cat(ys, dim=1).numpy(), y) < 1e-12
+    assert rel(ends[-1].numpy(), s) < 1e-12
+    for n in ("dr", "dw", "dk", "dv", "da", "db"):
+        assert rel(torch.cat([gp[n] for gp in gs], dim=1).numpy(), g[n]) < 1e-11, n
+    assert rel(gs[0]["ds0"].numpy(), g["ds0"]) < 1e-11

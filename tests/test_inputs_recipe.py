@@ -74,3 +74,22 @@ def test_bf16_storage_round_trip_is_exact_on_representable_values():
     assert bits.dtype == np.uint16
     assert np.array_equal(I.to_f64(bits, "bf16"), I.bf16_bits_to_f32(I.f32_to_bf16_bits(vals.astype(np.float32))))
     assert I.to_f64(I.to_storage(np.array([1.0 + 2.0 ** -9]), "bf16"), "bf16")[0] == 1.0   # round to nearest even
+
+
+def test_gdn_inputs_recipe():
+    """The gated-DeltaNet inputs: seeded, q and k per key head, v per value head, a log-decay
+    g <= 0 per value head whose typical size follows A * dt, and beta in (0, 1)."""
+    import numpy as np
+    from linear_recurrent_lm_b200 import inputs as I
+    a = I.draw_gdn_inputs(np.random.default_rng(3), 2, 64, 8, 4, 128, "bf16")
+    b = I.draw_gdn_inputs(np.random.default_rng(3), 2, 64, 8, 4, 128, "bf16")
+    for n in ("q", "k", "v", "g", "beta"):
+        np.testing.assert_array_equal(a[n], b[n])
+    assert a["q"].shape == a["k"].shape == (2, 64, 4, 128) and a["q"].dtype == np.uint16
+    assert a["v"].shape == (2, 64, 8, 128)
+    assert a["g"].shape == a["beta"].shape == (2, 64, 8) and a["g"].dtype == np.float32
+    assert np.all(a["g"] <= 0.0) and np.all(a["g"] > -1e3)
+    assert np.all((a["beta"] > 0.0) & (a["beta"] < 1.0))
+    # per head the median decay is near -A dt with A in [1, 16], dt in [1e-3, 1e-1]
+    med = np.median(-a["g"], axis=(0, 1))
+    assert np.all(med > 1e-3 * 0.3) and np.all(med < 16 * 0.1 * 3)
