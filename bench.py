@@ -463,8 +463,10 @@ def main():
     e2e_ms = rank_max([e0.elapsed_time(e1)], dev, world)[0] / args.e2e_steps
     e2e_value = job_tokens_per_s(B * T, world, e2e_ms)
 
+    # The secondary lines are single-GPU diagnostics (about a minute of work): under torchrun the
+    # other ranks would sit in the barrier below for all of it, against the process group's timeout.
     secondary = {}
-    if rank == 0 and not args.no_secondary:
+    if rank == 0 and world == 1 and not args.no_secondary:
         secondary = measure_secondary(wkv7, dev, args.algo)
         if args.algo != "scan":   # the token-order scan kernels on the same batch, for comparison
             ev3 = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
