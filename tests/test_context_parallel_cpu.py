@@ -136,3 +136,25 @@ def test_emulated_ranks_equal_one_run():
     for n in ("dr", "dw", "dk", "dv", "da", "db"):
         assert rel(torch.cat([gp[n] for gp in gs], dim=1).numpy(), g[n]) < 1e-11, n
     assert rel(gs[0]["ds0"].numpy(), g["ds0"]) < 1e-11
+
+
+def test_segment_is_affine_in_its_entering_state():
+    """The identity the split rests on, on the oracle alone: with P the end state from s0 = I and
+    v = 0, and U the end state from s0 = 0, the end state from any s0 is s0 P + U (a reset inside
+    the segment included); and the backward's ds0 from a final-state gradient D and dy is
+    D P^T + (its ds0 from dy alone)."""
+    import oracle
+    xs, s0, dy, dsT, reset = _problem(37)
+    B, H, N = s0.shape[0], s0.shape[1], s0.shape[2]
+    eye = np.broadcast_to(np.eye(N), (B, H, N, N)).copy()
+    v0 = np.zeros_like(xs[3])
+    for rs in (np.zeros_like(reset), reset):
+        _, P, _ = oracle.forward(xs[0], xs[1], xs[2], v0, xs[4], xs[5], s0=eye, reset=rs)
+        _, U, _ = oracle.forward(*xs, reset=rs)
+        _, S, _ = oracle.forward(*xs, s0=s0, reset=rs)
+        np.testing.assert_allclose(S, s0 @ P + U, rtol=0, atol=1e-12 * np.abs(S).max())
+        g, _ = oracle.backward(*xs, dy, s0=s0, reset=rs, dsT=dsT)
+        g0, _ = oracle.backward(*xs, dy, s0=s0, reset=rs)
+        ref = dsT @ np.swapaxes(P, -1, -2) + g0["ds0"]
+        np.testing.assert_allclose(g["ds0"], ref, rtol=0, atol=1e-12 * np.abs(ref).max())
+    assert np.abs(P).max() == 0.0        # the reset inside the segment (row 0) and at t = 32 (row 1)
