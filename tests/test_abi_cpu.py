@@ -291,3 +291,39 @@ def test_state_compose_validation_codes(L):
     assert call(ctypes.byref(bad), P, P, P, vp(FAKE + 4096)) == L.ERR_UNSUPPORTED
     d0 = L.make_desc(0, 1, 3, torch.float32)
     assert call(ctypes.byref(d0), None, None, None, None) == L.OK               # no units, no launch
+
+
+def test_plain_c_program_links_and_calls_the_library(L, tmp_path):
+    """The boundary is a C ABI: a C99 program compiles against include/wkv7.h with -pedantic, links
+    libwkv7.so and gets status codes back from it without a GPU (validation runs before anything
+    touches a device)."""
+    import shutil
+    import subprocess
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use.c"
+    src.write_text(r"""
+#include <stdio.h>
+#include <string.h>
+#include "wkv7.h"
+int main(void) {
+  wkv7_desc_t d;
+  memset(&d, 0, sizeof d);
+  d.B = 1; d.T = 16; d.H = 1; d.N = 96; d.dtype = WKV7_BF16; d.algo = WKV7_ALGO_AUTO;
+  if (wkv7_version() < 100) return 2;
+  if (wkv7_forward(&d, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0) != WKV7_ERR_UNSUPPORTED) return 3;
+  d.N = 64;
+  if (wkv7_workspace_bytes(&d) != 64u * 64u * 4u + 16u) return 4;
+  if (wkv7_forward(NULL, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0, 0) != WKV7_ERR_NULL) return 5;
+  printf("%s\n", wkv7_status_string(WKV7_ERR_SHAPE));
+  return 0;
+}
+""")
+    exe = tmp_path / "use"
+    libdir = os.path.dirname(L.LIB_PATHS["release"])
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", f"-I{os.path.join(ROOT, 'include')}",
+                    str(src), f"-L{libdir}", "-lwkv7", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    res = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert res.returncode == 0, (res.returncode, res.stderr)
+    assert res.stdout.strip()
